@@ -1,0 +1,226 @@
+"""CPU oracle for one Mixture-of-Groups Attention (MoGA) layer.
+
+TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only the tests, the package's smoke
+check and the benchmark's CPU-baseline / reference arm may import this module.
+It shares no code with the CUDA library: it is plain numpy in float64, written
+from the method's definitions, and slow on purpose so that a reader can check
+each step against the text by eye.
+
+Source of every definition: "MoGA: Mixture-of-Groups Attention for End-to-End
+Long Video Generation" (arXiv 2510.18692), as summarised on the paper-graph-ui
+page of that title, §3.4 "Detailed, Sentence-Based Technical Breakdown":
+
+* Eq. 1  SA(q, K, V) = softmax(q K^T / sqrt(d)) V         ("Vanilla Self-Attention")
+* Eq. 2  r = Router(x) = x W_r (+ b), W_r in R^{d x M}      ("MoGA Router")
+* Eq. 3  p(i|x) = softmax(r)_i                              ("MoGA Router")
+* Eq. 4  g(x) = argmax_i p(i|x)                             ("MoGA Router")
+* Eq. 5  MoGA(x) = p(g(x)|x) * SA(q, K_g(x), V_g(x))        ("Grouped Attention")
+* Algorithm 1: route, permute Q/K/V into contiguous per-group segments
+  (cu_seqlen, max_seqlen, permute index), attend per segment, un-permute
+  ("MoGA Pseudocode and Kernel Integration").
+* STGA: attention inside fixed local spatio-temporal windows; the block output
+  is the mean of the MoGA and STGA outputs ("Spatial-Temporal Group Attention").
+
+Readings where the pages leave a step open (each one is pinned by a test):
+
+* softmax scale: 1/sqrt(d_h) per head (Algorithm 1 hands each head to
+  FlashAttention, whose default scale is 1/sqrt(head dim)).
+* argmax ties: the lowest group index wins.  softmax is strictly increasing, so
+  argmax p = argmax r; it is taken on r, where rounding cannot create ties.
+* order inside a group: original token index ascending (a stable sort), which
+  makes the permutation unique.  ``perm[j]`` = original index of the token at
+  sorted position j (the inverse of the pages' original-to-permuted index).
+* STGA windows: non-overlapping boxes of (wt, wh, ww) tokens anchored at the
+  grid origin, clipped at the grid edges; token index (t*Hg + h)*Wg + w.
+* combine: out = (MoGA + STGA) / 2 when STGA is on, MoGA alone otherwise.
+
+Every function here is pinned by ``tests/test_oracle_pins.py`` to something
+other than itself (closed forms, a library attention routine, numpy's stable
+argsort, brute force on tiny inputs, invariants).  No function is unpinned.
+"""
+from __future__ import annotations
+
+import math
+from typing import Iterable, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+__all__ = [
+    "route", "counting_sort", "attention_rows", "group_attention",
+    "stga_windows", "stga_attention", "moga_layer",
+]
+
+_ROW_BLOCK = 16384
+
+
+def _f64(a) -> np.ndarray:
+    """Exact upcast to float64 (accepts numpy arrays or torch CPU tensors)."""
+    if hasattr(a, "detach"):
+        a = a.detach()
+        if str(a.dtype) in ("torch.bfloat16", "torch.float16"):
+            a = a.float()
+        a = a.cpu().numpy()
+    return np.asarray(a, dtype=np.float64)
+
+
+def route(x, W_r, b_r=None) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Router, softmax gate and hard assignment (Eqs. 2-4).
+
+    x: [N, d]; W_r: [M, d] (row i is group i's prototype, i.e. the transposed
+    d x M matrix of Eq. 2); b_r: [M] or None.
+    Returns (group_id int32 [N], gate float64 [N], margin float64 [N]) where
+    gate = p(g(x)|x) and margin = r_(1) - r_(2), the gap between the largest
+    and second largest logit (infinite when M == 1).
+    """
+    W = _f64(W_r)
+    M = W.shape[0]
+    b = np.zeros(M) if b_r is None else _f64(b_r)
+    N = x.shape[0]
+    gid = np.empty(N, dtype=np.int32)
+    gate = np.empty(N, dtype=np.float64)
+    margin = np.empty(N, dtype=np.float64)
+    for r0 in range(0, N, _ROW_BLOCK):
+        r1 = min(N, r0 + _ROW_BLOCK)
+        r = _f64(x[r0:r1]) @ W.T + b                      # Eq. 2
+        e = np.exp(r - r.max(axis=1, keepdims=True))
+        p = e / e.sum(axis=1, keepdims=True)              # Eq. 3
+        g = np.argmax(r, axis=1)                          # Eq. 4, first max wins
+        gid[r0:r1] = g
+        gate[r0:r1] = p[np.arange(r1 - r0), g]
+        if M == 1:
+            margin[r0:r1] = np.inf
+        else:
+            top2 = np.sort(r, axis=1)[:, -2:]
+            margin[r0:r1] = top2[:, 1] - top2[:, 0]
+    return gid, gate, margin
+
+
+def counting_sort(group_id, M: int) -> Tuple[np.ndarray, np.ndarray, int]:
+    """Algorithm 1 step 2 index part: group tokens into contiguous segments.
+
+    Returns (perm int32 [N], offsets int32 [M+1], max_seqlen) where
+    offsets is the cu_seqlen array (exclusive prefix sum of the group sizes,
+    offsets[M] = N) and perm lists group 0's tokens in index order, then
+    group 1's, and so on.
+    """
+    g = np.asarray(group_id, dtype=np.int64)
+    counts = np.array([(g == m).sum() for m in range(M)], dtype=np.int64)
+    offsets = np.zeros(M + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    perm = np.concatenate([np.nonzero(g == m)[0] for m in range(M)] + [np.zeros(0, np.int64)])
+    max_seqlen = int(counts.max()) if M > 0 else 0
+    return perm.astype(np.int32), offsets.astype(np.int32), max_seqlen
+
+
+def attention_rows(q_rows: np.ndarray, K: np.ndarray, V: np.ndarray) -> np.ndarray:
+    """Eq. 1 for a block of queries of one head: softmax(q K^T / sqrt(d_h)) V.
+
+    q_rows [r, d_h], K and V [n, d_h]; float64 throughout, max-subtracted
+    softmax over the n keys of each row.
+    """
+    d_h = K.shape[1]
+    s = (q_rows @ K.T) / math.sqrt(d_h)
+    s = s - s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    p = p / p.sum(axis=1, keepdims=True)
+    return p @ V
+
+
+def _attend_sets(q, k, v, sets: Iterable[np.ndarray], rows_mask, heads, scale_rows,
+                 out: np.ndarray, q_block: int = 512):
+    """Attention of each token set's queries to the same set's keys/values."""
+    for idx in sets:
+        if idx.size == 0:
+            continue
+        qi = idx if rows_mask is None else idx[rows_mask[idx]]
+        if qi.size == 0:
+            continue
+        for h in heads:
+            Kh = _f64(k[idx, h])
+            Vh = _f64(v[idx, h])
+            for b0 in range(0, qi.size, q_block):
+                rows = qi[b0:b0 + q_block]
+                o = attention_rows(_f64(q[rows, h]), Kh, Vh)
+                if scale_rows is not None:
+                    o = o * scale_rows[rows][:, None]
+                out[rows, h] = o
+    return out
+
+
+def group_attention(q, k, v, group_id, gate, M: int,
+                    rows: Optional[Sequence[int]] = None,
+                    heads: Optional[Sequence[int]] = None) -> np.ndarray:
+    """MoGA output, Eq. 5, computed directly in original token order.
+
+    out[i, h] = gate[i] * SA(q[i,h], K_{g(i),h}, V_{g(i),h}) where K_g, V_g hold
+    the keys/values of every token routed to g(i).  ``rows`` restricts the
+    queries that are computed (others stay NaN); ``heads`` restricts the heads.
+    q, k, v: [N, H, d_h] arrays (any float type; upcast exactly to float64).
+    """
+    N, H, d_h = q.shape
+    g = np.asarray(group_id, dtype=np.int64)
+    gate = _f64(gate)
+    out = np.full((N, H, d_h), np.nan)
+    mask = None
+    if rows is not None:
+        mask = np.zeros(N, dtype=bool)
+        mask[np.asarray(rows, dtype=np.int64)] = True
+    hs = range(H) if heads is None else heads
+    sets = (np.nonzero(g == m)[0] for m in range(M))
+    return _attend_sets(q, k, v, sets, mask, hs, gate, out)
+
+
+def stga_windows(T: int, Hg: int, Wg: int, window) -> List[np.ndarray]:
+    """Token index sets of the STGA windows (non-overlapping, clipped at edges).
+
+    Windows are enumerated with the temporal block outermost, then rows, then
+    columns; tokens inside a window are listed in index order.
+    """
+    wt, wh, ww = window
+    sets = []
+    for t0 in range(0, T, wt):
+        for h0 in range(0, Hg, wh):
+            for w0 in range(0, Wg, ww):
+                ts = np.arange(t0, min(T, t0 + wt))
+                hs = np.arange(h0, min(Hg, h0 + wh))
+                ws = np.arange(w0, min(Wg, w0 + ww))
+                idx = ((ts[:, None, None] * Hg + hs[None, :, None]) * Wg
+                       + ws[None, None, :]).reshape(-1)
+                sets.append(np.sort(idx))
+    return sets
+
+
+def stga_attention(q, k, v, T: int, Hg: int, Wg: int, window,
+                   rows: Optional[Sequence[int]] = None,
+                   heads: Optional[Sequence[int]] = None) -> np.ndarray:
+    """STGA: full attention inside each spatio-temporal window (no gate)."""
+    N, H, d_h = q.shape
+    assert T * Hg * Wg == N
+    out = np.full((N, H, d_h), np.nan)
+    mask = None
+    if rows is not None:
+        mask = np.zeros(N, dtype=bool)
+        mask[np.asarray(rows, dtype=np.int64)] = True
+    hs = range(H) if heads is None else heads
+    return _attend_sets(q, k, v, stga_windows(T, Hg, Wg, window), mask, hs, None, out)
+
+
+def moga_layer(x, W_r, b_r, q, k, v, M: int, grid=None, window=None,
+               rows=None, heads=None):
+    """One visual attention block: route, group attention, optional STGA, mean.
+
+    Returns a dict with group_id, gate, margin, perm, offsets, max_seqlen,
+    moga (Eq. 5 output), stga (or None) and out (the block output).
+    """
+    gid, gate, margin = route(x, W_r, b_r)
+    perm, offsets, max_seqlen = counting_sort(gid, M)
+    moga = group_attention(q, k, v, gid, gate, M, rows=rows, heads=heads)
+    stga = None
+    out = moga
+    if window is not None:
+        T, Hg, Wg = grid
+        stga = stga_attention(q, k, v, T, Hg, Wg, window, rows=rows, heads=heads)
+        out = 0.5 * (moga + stga)
+    return {"group_id": gid, "gate": gate, "margin": margin, "perm": perm,
+            "offsets": offsets, "max_seqlen": max_seqlen, "moga": moga,
+            "stga": stga, "out": out}

@@ -1,0 +1,381 @@
+"""Pins of the CPU oracle to things other than itself.
+
+Each ``check_*`` function takes the oracle module and raises AssertionError
+when the oracle disagrees with a closed form, a library routine, brute force
+on a tiny input or an invariant of the method.  The plain tests run every
+check on the real oracle; ``test_planted_mistakes_are_caught`` runs them on
+copies of the oracle with one plausible mistake planted (on the CPU) and
+requires that some check fails, so the pins are known to bite.
+
+Method source: "MoGA: Mixture-of-Groups Attention for End-to-End Long Video
+Generation" (paper-graph-ui summary), section 3.4 (Eqs. 1-5, Algorithm 1, STGA).
+"""
+import math
+import os
+import types
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------------------
+# helpers that are independent of the oracle
+# ----------------------------------------------------------------------------
+def _sdpa(q, k, v):
+    """Library attention (torch CPU, float64): q,k,v [L, H, E] -> [L, H, E]."""
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(np.asarray(a, np.float64).transpose(1, 0, 2)))
+    o = torch.nn.functional.scaled_dot_product_attention(t(q)[None], t(k)[None], t(v)[None])[0]
+    return o.numpy().transpose(1, 0, 2)
+
+
+def _brute_route(x, W, b):
+    """Pure-Python loops: logits, softmax, first argmax, gate."""
+    N, d = len(x), len(x[0])
+    M = len(W)
+    gid, gate = [], []
+    for i in range(N):
+        r = [sum(float(x[i][c]) * float(W[m][c]) for c in range(d)) + (float(b[m]) if b is not None else 0.0)
+             for m in range(M)]
+        best = 0
+        for m in range(1, M):
+            if r[m] > r[best]:
+                best = m
+        z = sum(math.exp(rm - r[best]) for rm in r)
+        gid.append(best)
+        gate.append(1.0 / z)
+    return np.array(gid), np.array(gate)
+
+
+def _brute_masked_dense(q, k, v, gid, gate):
+    """Pure-Python masked dense attention: key j is visible to query i iff
+    both tokens carry the same group id; output scaled by the gate."""
+    N, H, E = q.shape
+    out = np.zeros((N, H, E))
+    for i in range(N):
+        for h in range(H):
+            s = []
+            for j in range(N):
+                if gid[j] == gid[i]:
+                    s.append((j, sum(float(q[i, h, c]) * float(k[j, h, c]) for c in range(E)) / math.sqrt(E)))
+            mx = max(val for _, val in s)
+            w = [(j, math.exp(val - mx)) for j, val in s]
+            z = sum(wj for _, wj in w)
+            for c in range(E):
+                out[i, h, c] = gate[i] * sum(wj * float(v[j, h, c]) for j, wj in w) / z
+    return out
+
+
+def _brute_stga(q, k, v, grid, window):
+    """Pure-Python window attention: tokens share a window iff their
+    (t // wt, h // wh, w // ww) coordinates agree."""
+    T, Hg, Wg = grid
+    wt, wh, ww = window
+    N, H, E = q.shape
+    coord = []
+    for i in range(N):
+        t, rem = divmod(i, Hg * Wg)
+        hh, w = divmod(rem, Wg)
+        coord.append((t // wt, hh // wh, w // ww))
+    out = np.zeros((N, H, E))
+    for i in range(N):
+        keys = [j for j in range(N) if coord[j] == coord[i]]
+        for h in range(H):
+            s = [sum(float(q[i, h, c]) * float(k[j, h, c]) for c in range(E)) / math.sqrt(E) for j in keys]
+            mx = max(s)
+            w = [math.exp(a - mx) for a in s]
+            z = sum(w)
+            for c in range(E):
+                out[i, h, c] = sum(wj * float(v[j, h, c]) for j, wj in zip(keys, w)) / z
+    return out
+
+
+def _read_golden(name):
+    sections, cur = {}, None
+    env = {"e": math.e, "log": math.log, "__builtins__": {}}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            if line.startswith("["):
+                cur = sections.setdefault(line.strip("[]"), {})
+                continue
+            key, expr = line.split("=", 1)
+            cur[key.strip()] = eval(expr, env)  # fixture expressions only
+    return sections
+
+
+# ----------------------------------------------------------------------------
+# checks
+# ----------------------------------------------------------------------------
+def check_route_closed_form(o):
+    # W_r = I, x = a * e_k: r = a e_k, so p_k = e^a / (e^a + M - 1).
+    M, a = 5, 2.0
+    x = np.zeros((3 * M, M))
+    for i in range(3 * M):
+        x[i, i % M] = a
+    gid, gate, margin = o.route(x, np.eye(M))
+    assert np.array_equal(gid, np.arange(3 * M) % M)
+    assert np.allclose(gate, math.exp(a) / (math.exp(a) + M - 1), rtol=0, atol=1e-15)
+    assert np.allclose(margin, a)
+
+
+def check_route_ties_and_M1(o):
+    gid, gate, _ = o.route(np.zeros((4, 3)), np.ones((6, 3)))
+    assert np.array_equal(gid, np.zeros(4)) and np.allclose(gate, 1 / 6)
+    # logits (1, 3, 3, 0): the first of the two maxima wins
+    W = np.array([[1.0], [3.0], [3.0], [0.0]])
+    gid, gate, _ = o.route(np.ones((1, 1)), W)
+    assert gid[0] == 1
+    assert abs(gate[0] - math.exp(3) / (math.exp(1) + 2 * math.exp(3) + 1)) < 1e-15
+    rng = np.random.default_rng(1)
+    gid, gate, margin = o.route(rng.normal(size=(7, 4)), rng.normal(size=(1, 4)))
+    assert np.all(gid == 0) and np.all(gate == 1.0) and np.all(np.isinf(margin))
+
+
+def check_route_brute(o):
+    rng = np.random.default_rng(2)
+    x = rng.normal(size=(16, 8))
+    W = rng.normal(size=(3, 8)) / math.sqrt(8)
+    b = rng.normal(size=3)
+    g0, p0 = _brute_route(x.tolist(), W.tolist(), b.tolist())
+    gid, gate, margin = o.route(x, W, b)
+    assert np.array_equal(gid, g0)
+    assert np.allclose(gate, p0, rtol=0, atol=1e-13)
+    assert np.all(gate >= 1 / 3 - 1e-15) and np.all(gate <= 1)
+    r = x @ W.T + b
+    srt = np.sort(r, axis=1)
+    assert np.allclose(margin, srt[:, -1] - srt[:, -2])
+
+
+def check_counting_sort(o):
+    rng = np.random.default_rng(3)
+    for N, M in [(0, 3), (1, 1), (50, 7), (1000, 16), (333, 64)]:
+        g = rng.integers(0, max(1, M // 2), size=N).astype(np.int32)  # upper groups empty
+        perm, offsets, mx = o.counting_sort(g, M)
+        assert np.array_equal(perm, np.argsort(g, kind="stable"))
+        assert np.array_equal(np.sort(perm), np.arange(N))
+        assert offsets[0] == 0 and offsets[-1] == N and np.all(np.diff(offsets) >= 0)
+        assert np.array_equal(np.diff(offsets), np.bincount(g, minlength=M))
+        assert mx == (np.bincount(g, minlength=M).max() if N else 0)
+        for m in range(M):
+            seg = perm[offsets[m]:offsets[m + 1]]
+            assert np.all(g[seg] == m) and np.all(np.diff(seg) > 0)
+
+
+def check_full_attention_when_M1(o):
+    rng = np.random.default_rng(4)
+    q, k, v = (rng.normal(size=(40, 3, 16)) for _ in range(3))
+    x = rng.normal(size=(40, 5))
+    res = o.moga_layer(x, rng.normal(size=(1, 5)), None, q, k, v, 1)
+    assert np.all(res["gate"] == 1.0)
+    assert np.allclose(res["out"], _sdpa(q, k, v), rtol=0, atol=1e-12)
+
+
+def check_group_equals_subset_attention(o):
+    rng = np.random.default_rng(5)
+    N, H, E, M = 60, 2, 8, 4
+    q, k, v = (rng.normal(size=(N, H, E)) for _ in range(3))
+    gid = rng.integers(0, M, size=N)
+    gate = rng.uniform(0.25, 1.0, size=N)
+    out = o.group_attention(q, k, v, gid, gate, M)
+    for m in range(M):
+        idx = np.nonzero(gid == m)[0]
+        if idx.size:
+            ref = _sdpa(q[idx], k[idx], v[idx]) * gate[idx][:, None, None]
+            assert np.allclose(out[idx], ref, rtol=0, atol=1e-12)
+
+
+def check_special_cases(o):
+    rng = np.random.default_rng(6)
+    N, H, E, M = 30, 2, 4, 3
+    q, k = rng.normal(size=(N, H, E)), rng.normal(size=(N, H, E))
+    gid = np.array([0] * 12 + [1] * 17 + [2])           # group 2 is a single token
+    gid = gid[rng.permutation(N)]
+    gate = rng.uniform(1 / M, 1, size=N)
+    v = rng.normal(size=(N, H, E))
+    # constant V inside each group -> out = gate * v
+    vc = np.zeros_like(v)
+    for m in range(M):
+        vc[gid == m] = rng.normal(size=(1, H, E))
+    out = o.group_attention(q, k, vc, gid, gate, M)
+    assert np.allclose(out, gate[:, None, None] * vc, rtol=0, atol=1e-12)
+    # q = 0 -> uniform weights -> out = gate * mean of the group's V
+    out = o.group_attention(np.zeros_like(q), k, v, gid, gate, M)
+    for m in range(M):
+        idx = gid == m
+        assert np.allclose(out[idx], gate[idx][:, None, None] * v[idx].mean(0), rtol=0, atol=1e-12)
+    # singleton group -> out = gate * own v
+    s = np.nonzero(gid == 2)[0][0]
+    out = o.group_attention(q, k, v, gid, gate, M)
+    assert np.allclose(out[s], gate[s] * v[s], rtol=0, atol=1e-14)
+
+
+def check_brute_force_tiny(o):
+    rng = np.random.default_rng(7)
+    N, H, E, M, d = 24, 2, 4, 3, 6
+    x = rng.normal(size=(N, d))
+    W = rng.normal(size=(M, d))
+    q, k, v = (rng.normal(size=(N, H, E)) for _ in range(3))
+    res = o.moga_layer(x, W, None, q, k, v, M)
+    g0, p0 = _brute_route(x.tolist(), W.tolist(), None)
+    ref = _brute_masked_dense(q, k, v, g0, p0)
+    assert np.array_equal(res["group_id"], g0)
+    assert np.allclose(res["out"], ref, rtol=0, atol=1e-12)
+
+
+def check_permutation_equivariance(o):
+    rng = np.random.default_rng(8)
+    N, H, E, M, d = 48, 2, 8, 5, 6
+    x = rng.normal(size=(N, d))
+    W = rng.normal(size=(M, d))
+    q, k, v = (rng.normal(size=(N, H, E)) for _ in range(3))
+    pi = rng.permutation(N)
+    a = o.moga_layer(x, W, None, q, k, v, M)["out"]
+    b = o.moga_layer(x[pi], W, None, q[pi], k[pi], v[pi], M)["out"]
+    assert np.allclose(a[pi], b, rtol=0, atol=1e-12)
+
+
+def check_stga(o):
+    rng = np.random.default_rng(9)
+    grid = (3, 10, 12)
+    N = 360
+    q, k, v = (rng.normal(size=(N, 1, 8)) for _ in range(3))
+    # window = whole grid -> full attention
+    assert np.allclose(o.stga_attention(q, k, v, *grid, grid), _sdpa(q, k, v), rtol=0, atol=1e-12)
+    # window (1,1,1) -> out = v
+    assert np.allclose(o.stga_attention(q, k, v, *grid, (1, 1, 1)), v, rtol=0, atol=1e-14)
+    # clipped edge windows against brute force (10 = 4+4+2, 12 = 8+4)
+    small = (2, 5, 6)
+    n = 60
+    qs, ks, vs = q[:n], k[:n], v[:n]
+    ref = _brute_stga(qs, ks, vs, small, (2, 4, 4))
+    assert np.allclose(o.stga_attention(qs, ks, vs, *small, (2, 4, 4)), ref, rtol=0, atol=1e-12)
+    sets = o.stga_windows(*grid, (3, 8, 8))
+    assert sorted(np.concatenate(sets).tolist()) == list(range(N)) and len(sets) == 4
+
+
+def check_layer_combine(o):
+    rng = np.random.default_rng(10)
+    grid, N = (2, 4, 6), 48
+    x = rng.normal(size=(N, 5))
+    W = rng.normal(size=(3, 5))
+    q, k, v = (rng.normal(size=(N, 2, 8)) for _ in range(3))
+    res = o.moga_layer(x, W, None, q, k, v, 3, grid=grid, window=(1, 2, 3))
+    ref_stga = _brute_stga(q, k, v, grid, (1, 2, 3))
+    g0, p0 = _brute_route(x.tolist(), W.tolist(), None)
+    ref = 0.5 * (_brute_masked_dense(q, k, v, g0, p0) + ref_stga)
+    assert np.allclose(res["out"], ref, rtol=0, atol=1e-12)
+    # M = 1 and a whole-grid window: both branches are full attention
+    res = o.moga_layer(x, W[:1], None, q, k, v, 1, grid=grid, window=grid)
+    assert np.allclose(res["out"], _sdpa(q, k, v), rtol=0, atol=1e-12)
+
+
+def check_golden(o):
+    g = _read_golden("worked_example.txt")
+    inp, exp = g["input"], g["expect"]
+    x = np.array(inp["x"], float)
+    q, k, v = (np.array(inp[n], float).reshape(4, 1, 1) for n in ("q", "k", "v"))
+    res = o.moga_layer(x, np.array(inp["W_r"], float), None, q, k, v, inp["M"])
+    assert res["group_id"].tolist() == exp["group_id"]
+    assert np.allclose(res["gate"], exp["gate"], rtol=0, atol=1e-15)
+    assert res["perm"].tolist() == exp["perm"] and res["offsets"].tolist() == exp["offsets"]
+    assert res["max_seqlen"] == exp["max_seqlen"]
+    assert np.allclose(res["out"][:, 0, 0], exp["moga"], rtol=0, atol=1e-14)
+    s = _read_golden("stga_example.txt")
+    T, Hg, Wg = s["input"]["grid"]
+    v = np.array(s["input"]["v"], float).reshape(6, 1, 1)
+    out = o.stga_attention(np.zeros_like(v), np.ones_like(v), v, T, Hg, Wg, s["input"]["window"])
+    assert np.allclose(out[:, 0, 0], s["expect"]["stga"], rtol=0, atol=1e-14)
+
+
+CHECKS = [check_route_closed_form, check_route_ties_and_M1, check_route_brute, check_counting_sort,
+          check_full_attention_when_M1, check_group_equals_subset_attention, check_special_cases,
+          check_brute_force_tiny, check_permutation_equivariance, check_stga, check_layer_combine,
+          check_golden]
+
+
+@pytest.mark.parametrize("check", CHECKS, ids=[c.__name__ for c in CHECKS])
+def test_oracle_pin(check):
+    check(oracle)
+
+
+# ----------------------------------------------------------------------------
+# planted mistakes: each must be caught by at least one check
+# ----------------------------------------------------------------------------
+def _wrong_scale(q_rows, K, V):
+    s = (q_rows @ K.T) / K.shape[1]
+    p = np.exp(s - s.max(1, keepdims=True))
+    return (p / p.sum(1, keepdims=True)) @ V
+
+
+def _no_max_transpose(q_rows, K, V):                   # softmax over the wrong axis
+    s = (q_rows @ K.T) / math.sqrt(K.shape[1])
+    p = np.exp(s - s.max(0, keepdims=True))
+    return (p / p.sum(0, keepdims=True)) @ V
+
+
+def _route_last_argmax(x, W_r, b_r=None):
+    gid, gate, margin = _ORIG_ROUTE(x, W_r, b_r)
+    W = np.asarray(W_r, float)
+    r = np.asarray(x, float) @ W.T + (0 if b_r is None else np.asarray(b_r, float))
+    last = r.shape[1] - 1 - np.argmax(r[:, ::-1], axis=1)
+    return last.astype(np.int32), gate, margin
+
+
+def _route_gate_of_group0(x, W_r, b_r=None):
+    gid, gate, margin = _ORIG_ROUTE(x, W_r, b_r)
+    W = np.asarray(W_r, float)
+    r = np.asarray(x, float) @ W.T
+    e = np.exp(r - r.max(1, keepdims=True))
+    return gid, (e / e.sum(1, keepdims=True))[:, 0], margin
+
+
+def _unstable_sort(group_id, M):
+    perm, offsets, mx = _ORIG_SORT(group_id, M)
+    out = perm.copy()
+    for m in range(M):
+        out[offsets[m]:offsets[m + 1]] = out[offsets[m]:offsets[m + 1]][::-1]
+    return out, offsets, mx
+
+
+def _no_gate(q, k, v, group_id, gate, M, rows=None, heads=None):
+    return _ORIG_GA(q, k, v, group_id, np.ones(len(group_id)), M, rows, heads)
+
+
+def _windows_off_by_one(T, Hg, Wg, window):
+    return _ORIG_WIN(T, Hg, Wg, (window[0], window[1], window[2] + 1))
+
+
+_ORIG_GA = oracle.group_attention
+_ORIG_WIN = oracle.stga_windows
+_ORIG_ROUTE = oracle.route
+_ORIG_SORT = oracle.counting_sort
+
+MUTANTS = {
+    "scale_1_over_d": ("attention_rows", _wrong_scale),
+    "softmax_wrong_axis": ("attention_rows", _no_max_transpose),
+    "argmax_last_on_ties": ("route", _route_last_argmax),
+    "gate_of_wrong_group": ("route", _route_gate_of_group0),
+    "unstable_group_order": ("counting_sort", _unstable_sort),
+    "gate_dropped": ("group_attention", _no_gate),
+    "window_width_off_by_one": ("stga_windows", _windows_off_by_one),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistakes_are_caught(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(oracle, attr, fn)
+    caught = []
+    for check in CHECKS:
+        try:
+            check(oracle)
+        except AssertionError:
+            caught.append(check.__name__)
+    assert caught, f"planted mistake {name} went unnoticed by every pin"
