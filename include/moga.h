@@ -1,0 +1,160 @@
+/*
+ * moga.h - C ABI of a single-GPU Mixture-of-Groups Attention (MoGA) layer for
+ * NVIDIA B200 (sm_100a).
+ *
+ * Method: "MoGA: Mixture-of-Groups Attention for End-to-End Long Video
+ * Generation" (arXiv 2510.18692), as summarised on the paper-graph-ui page of
+ * that title, section 3.4 "Detailed, Sentence-Based Technical Breakdown":
+ *   Eq. 1  SA(q, K, V) = softmax(q K^T / sqrt(d)) V              (Vanilla Self-Attention)
+ *   Eq. 2  r = x W_r (+ b)                                       (MoGA Router)
+ *   Eq. 3  p(i|x) = softmax(r)_i                                 (MoGA Router)
+ *   Eq. 4  g(x) = argmax_i p(i|x)                                (MoGA Router)
+ *   Eq. 5  MoGA(x) = p(g(x)|x) * SA(q, K_g(x), V_g(x))           (Grouped Attention)
+ *   Algorithm 1: route; permute Q/K/V into per-group segments (cu_seqlen,
+ *   max_seqlen, permute index); attention per segment; un-permute
+ *                                                    (MoGA Pseudocode and Kernel Integration)
+ *   STGA: attention inside fixed spatio-temporal windows; the block output is
+ *   the mean of the MoGA and STGA outputs   (Spatial-Temporal Group Attention)
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All tensor pointers are DEVICE pointers, owned by the caller, 16-byte
+ *   aligned and dense (row-major, no padding).  The library allocates no
+ *   device memory: calls that need scratch take a caller-allocated workspace
+ *   whose size comes from the matching *_workspace_size query.
+ * - q, k, v and out are bf16 in [N, H, d_h] layout (token-major, then head,
+ *   then channel).  d_h must be 64 or 128.
+ * - x is [N, d] (fp32 or bf16), W_r is [M, d] in the same dtype (row i is
+ *   group i's prototype, i.e. the nn.Linear weight layout; the d x M matrix of
+ *   Eq. 2 is its transpose), b_r is an optional fp32 [M] bias.
+ * - Softmax scale: 1/sqrt(d_h) per head.  Argmax ties go to the lowest group.
+ * - perm[j] is the ORIGINAL index of the token at sorted position j; tokens
+ *   are sorted by group, then by original index (stable), so perm is unique.
+ *   offsets ("cu_seqlen") is int32 [M+1], offsets[0] = 0, offsets[M] = N.
+ * - `stream` is a cudaStream_t (NULL = the legacy default stream).  All work
+ *   is enqueued asynchronously on it; a return of MOGA_OK means the work was
+ *   validated and launched.  Errors found on the device (a bounded wait that
+ *   timed out) are recorded in the workspace status word and reported by
+ *   moga_sync_status().
+ * - Arguments are validated before any device work is enqueued; an invalid
+ *   argument returns MOGA_ERR_INVALID_ARG (or MOGA_ERR_UNSUPPORTED /
+ *   MOGA_ERR_WORKSPACE) and touches nothing.
+ * - The library keeps no state between calls apart from cached kernel
+ *   attributes, so distinct workspaces may be used from distinct threads.
+ */
+#ifndef MOGA_H_
+#define MOGA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOGA_OK = 0,
+  MOGA_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad size or shape */
+  MOGA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. d_h not 64/128) */
+  MOGA_ERR_WORKSPACE = 3,     /* ws_bytes smaller than the size query returned */
+  MOGA_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+  MOGA_ERR_TIMEOUT = 5,       /* a device-side bounded wait gave up */
+  MOGA_ERR_DEVICE_CHECK = 6   /* a device-side range check fired */
+} moga_status;
+
+typedef enum { MOGA_F32 = 0, MOGA_BF16 = 1 } moga_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* moga_status_string(int status);
+
+/* ABI version: (major << 16) | minor. */
+int moga_version(void);
+
+/* ---------------------------------------------------------------- routing
+ * moga_route: Eqs. 2-4 plus the index half of Algorithm 1, step 2.
+ *   logits r = x W_r^T + b (fp32 accumulation), p = softmax(r),
+ *   group_id[i] = argmax r (lowest index on ties), gate[i] = p(group_id[i]|x_i),
+ *   offsets = exclusive prefix sum of the group sizes, max_seqlen = largest
+ *   group, perm = stable sort of token indices by group.
+ * In:  x [N, d] (dtype dt), W_r [M, d] (dtype dt), b_r [M] fp32 or NULL.
+ * Out: group_id int32 [N], gate fp32 [N], perm int32 [N], offsets int32 [M+1],
+ *      max_seqlen int32 [1] (device).
+ * Limits: 0 <= N < 2^31, 1 <= M <= 1024, d >= 8 and d % 8 == 0 (bf16) or
+ *         d % 4 == 0 (fp32).  N == 0 writes offsets = 0 and max_seqlen = 0.
+ * Workspace: moga_route_workspace_size(N, M) bytes.
+ */
+size_t moga_route_workspace_size(int64_t N, int M);
+moga_status moga_route(const void* x, const void* W_r, const float* b_r, moga_dtype dt, int64_t N, int d,
+                       int M, int32_t* group_id, float* gate, int32_t* perm, int32_t* offsets,
+                       int32_t* max_seqlen, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- grouped attention
+ * moga_group_attn: Algorithm 1 steps 2 (gather), 3 (attention inside each
+ * group segment) and 4 (un-permute), with the gate of Eq. 5 fused into the
+ * store:   out[perm[j], h, :] = out_scale * gate[perm[j]] *
+ *              SA(q[perm[j],h], K_seg(j),h, V_seg(j),h)
+ * where seg(j) is the segment of offsets that contains j.  gate may be NULL
+ * (gate = 1).  Tokens of empty groups do not exist, so every token's row of
+ * `out` is written exactly once.
+ * In:  q, k, v bf16 [N, H, d_h]; perm int32 [N]; offsets int32 [M+1]
+ *      (non-decreasing, offsets[0] = 0, offsets[M] = N; not checked on the
+ *      device); gate fp32 [N] or NULL.
+ * Out: out bf16 [N, H, d_h].
+ * Limits: d_h in {64, 128}; 1 <= H; N * H < 2^31; 1 <= M <= 1024.
+ * Workspace: moga_group_attn_workspace_size(N, H, d_h, M) bytes.
+ */
+size_t moga_group_attn_workspace_size(int64_t N, int H, int d_h, int M);
+moga_status moga_group_attn(const void* q, const void* k, const void* v, const int32_t* perm,
+                            const int32_t* offsets, const float* gate, int64_t N, int H, int d_h, int M,
+                            float out_scale, void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- STGA windows
+ * stga_window_attn: full attention inside non-overlapping windows of
+ * window[0] x window[1] x window[2] (frames x rows x columns) tokens over the
+ * T x Hg x Wg latent grid, windows anchored at the grid origin and clipped at
+ * the edges; token index = (t * Hg + h) * Wg + w.
+ *   accumulate == 0: out = STGA(q, k, v)
+ *   accumulate == 1: out = out + 0.5 * STGA(q, k, v)   (second half of the
+ *                    two-branch mean; the caller wrote 0.5 * MoGA before)
+ * In:  q, k, v bf16 [N, H, d_h], N = T * Hg * Wg.   Out: out bf16 [N, H, d_h].
+ * Limits: as moga_group_attn; every window extent >= 1.
+ * Workspace: stga_window_attn_workspace_size(...) bytes.
+ */
+size_t stga_window_attn_workspace_size(int T, int Hg, int Wg, const int* window, int H, int d_h);
+moga_status stga_window_attn(const void* q, const void* k, const void* v, int T, int Hg, int Wg,
+                             const int* window, int H, int d_h, int accumulate, void* out, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- full layer
+ * moga_layer: one visual attention block = moga_route, then moga_group_attn,
+ * then (when window != NULL) stga_window_attn, combined as
+ *   out = 0.5 * (MoGA(x) + STGA(x))   (window != NULL)
+ *   out = MoGA(x)                     (window == NULL; T, Hg, Wg ignored)
+ * All outputs (out, group_id, gate, perm, offsets) are caller-owned device
+ * buffers with the shapes given above.
+ * Workspace: moga_layer_workspace_size(...) bytes.
+ */
+size_t moga_layer_workspace_size(int64_t N, int H, int d_h, int M, int T, int Hg, int Wg, const int* window);
+moga_status moga_layer(const void* x, const void* W_r, const float* b_r, moga_dtype x_dt, const void* q,
+                       const void* k, const void* v, int64_t N, int d, int H, int d_h, int M, int T, int Hg,
+                       int Wg, const int* window, void* out, int32_t* group_id, float* gate, int32_t* perm,
+                       int32_t* offsets, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- device status
+ * moga_sync_status: synchronises `stream`, reads the device status word kept
+ * at the start of a workspace `ws` used by the calls above, clears it, and
+ * returns MOGA_OK, MOGA_ERR_TIMEOUT or MOGA_ERR_DEVICE_CHECK (or MOGA_ERR_CUDA
+ * if the synchronisation itself failed).  Workspaces must be zero-filled once
+ * before first use so that the status word starts clear.
+ */
+moga_status moga_sync_status(void* ws, void* stream);
+
+/* moga_set_wait_limit_ns: upper bound, in nanoseconds, on any single
+ * device-side wait of the kernels launched after this call (default 4e9).
+ * Process-wide.  Returns the previous value. */
+uint64_t moga_set_wait_limit_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOGA_H_ */

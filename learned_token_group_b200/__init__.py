@@ -1,0 +1,228 @@
+"""Python binding of the MoGA layer library (``libmoga.so``, C ABI in moga.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch provides device memory and the current CUDA stream.  There
+is no CPU fallback: if the library is missing or a call fails, an exception
+is raised.
+
+Method: "MoGA: Mixture-of-Groups Attention for End-to-End Long Video
+Generation" (paper-graph-ui summary, §3.4: router Eqs. 2-4, grouped attention
+Eq. 5, Algorithm 1, STGA).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional, Sequence
+
+import torch
+
+__all__ = ["MogaError", "get_lib", "LIB_PATH", "HEADER_PATH", "route", "group_attn", "stga_window_attn",
+           "moga_layer", "sync_status", "workspace", "MogaLayer", "exported_names"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoga.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "moga.h")
+
+MOGA_F32, MOGA_BF16 = 0, 1
+STATUS = {0: "MOGA_OK", 1: "MOGA_ERR_INVALID_ARG", 2: "MOGA_ERR_UNSUPPORTED", 3: "MOGA_ERR_WORKSPACE",
+          4: "MOGA_ERR_CUDA", 5: "MOGA_ERR_TIMEOUT", 6: "MOGA_ERR_DEVICE_CHECK"}
+
+
+class MogaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+
+
+_lib = None
+_P, _I64, _I, _F, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+
+
+def get_lib():
+    """Loads libmoga.so (raises ImportError if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m learned_token_group_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "moga_status_string": (ctypes.c_char_p, [_I]),
+        "moga_version": (_I, []),
+        "moga_set_wait_limit_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
+        "moga_route_workspace_size": (_SZ, [_I64, _I]),
+        "moga_route": (_I, [_P, _P, _P, _I, _I64, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+        "moga_group_attn_workspace_size": (_SZ, [_I64, _I, _I, _I]),
+        "moga_group_attn": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I, _I, _I, _F, _P, _P, _SZ, _P]),
+        "stga_window_attn_workspace_size": (_SZ, [_I, _I, _I, _P, _I, _I]),
+        "stga_window_attn": (_I, [_P, _P, _P, _I, _I, _I, _P, _I, _I, _I, _P, _P, _SZ, _P]),
+        "moga_layer_workspace_size": (_SZ, [_I64, _I, _I, _I, _I, _I, _I, _P]),
+        "moga_layer": (_I, [_P, _P, _P, _I, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _I, _P,
+                            _P, _P, _P, _P, _P, _P, _SZ, _P]),
+        "moga_sync_status": (_I, [_P, _P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def exported_names():
+    """Function names declared in include/moga.h."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b((?:moga|stga)_[a-z_0-9]+)\s*\(", text)))
+
+
+# ----------------------------------------------------------------------------- helpers
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(st: int, what: str):
+    if st != 0:
+        raise MogaError(st, what)
+
+
+def _int3(w):
+    return (ctypes.c_int * 3)(*[int(v) for v in w])
+
+
+def _dev_tensor(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """Zero-filled device workspace (the status word must start clear)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def sync_status(ws: torch.Tensor) -> None:
+    """Synchronises the current stream and raises if a kernel flagged an error."""
+    _check(get_lib().moga_sync_status(_ptr(ws), _stream(ws.device)), "device status")
+
+
+# ----------------------------------------------------------------------------- calls
+def route(x: torch.Tensor, W_r: torch.Tensor, b_r: Optional[torch.Tensor], M: int, out=None, ws=None):
+    """moga_route: returns dict(group_id, gate, perm, offsets, max_seqlen) on x's device."""
+    lib = get_lib()
+    _dev_tensor(x, "x")
+    _dev_tensor(W_r, "W_r", x.dtype)
+    if b_r is not None:
+        _dev_tensor(b_r, "b_r", torch.float32)
+    dt = {torch.float32: MOGA_F32, torch.bfloat16: MOGA_BF16}[x.dtype]
+    N, d = x.shape
+    dev = x.device
+    if out is None:
+        out = {"group_id": torch.empty(N, dtype=torch.int32, device=dev),
+               "gate": torch.empty(N, dtype=torch.float32, device=dev),
+               "perm": torch.empty(N, dtype=torch.int32, device=dev),
+               "offsets": torch.empty(M + 1, dtype=torch.int32, device=dev),
+               "max_seqlen": torch.empty(1, dtype=torch.int32, device=dev)}
+    need = lib.moga_route_workspace_size(N, M)
+    if ws is None:
+        ws = workspace(need, dev)
+    st = lib.moga_route(_ptr(x), _ptr(W_r), _ptr(b_r), dt, N, d, M, _ptr(out["group_id"]), _ptr(out["gate"]),
+                        _ptr(out["perm"]), _ptr(out["offsets"]), _ptr(out["max_seqlen"]), _ptr(ws), ws.numel(),
+                        _stream(dev))
+    _check(st, "moga_route")
+    return out
+
+
+def group_attn(q, k, v, perm, offsets, gate, M: int, out_scale: float = 1.0, out=None, ws=None):
+    """moga_group_attn: out[perm[j]] = out_scale * gate * SA within each segment."""
+    lib = get_lib()
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _dev_tensor(t, n, torch.bfloat16)
+    _dev_tensor(perm, "perm", torch.int32)
+    _dev_tensor(offsets, "offsets", torch.int32)
+    if gate is not None:
+        _dev_tensor(gate, "gate", torch.float32)
+    N, H, d_h = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    need = lib.moga_group_attn_workspace_size(N, H, d_h, M)
+    if ws is None:
+        ws = workspace(need, q.device)
+    st = lib.moga_group_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(perm), _ptr(offsets), _ptr(gate), N, H, d_h, M,
+                             float(out_scale), _ptr(out), _ptr(ws), ws.numel(), _stream(q.device))
+    _check(st, "moga_group_attn")
+    return out
+
+
+def stga_window_attn(q, k, v, grid: Sequence[int], window: Sequence[int], accumulate: bool = False,
+                     out=None, ws=None):
+    """stga_window_attn over a (T, Hg, Wg) grid with (wt, wh, ww) windows."""
+    lib = get_lib()
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _dev_tensor(t, n, torch.bfloat16)
+    N, H, d_h = q.shape
+    T, Hg, Wg = (int(g) for g in grid)
+    w3 = _int3(window)
+    if out is None:
+        if accumulate:
+            raise ValueError("accumulate=True needs an existing out tensor")
+        out = torch.empty_like(q)
+    need = lib.stga_window_attn_workspace_size(T, Hg, Wg, w3, H, d_h)
+    if ws is None:
+        ws = workspace(need, q.device)
+    st = lib.stga_window_attn(_ptr(q), _ptr(k), _ptr(v), T, Hg, Wg, w3, H, d_h, int(bool(accumulate)),
+                              _ptr(out), _ptr(ws), ws.numel(), _stream(q.device))
+    _check(st, "stga_window_attn")
+    return out
+
+
+class MogaLayer:
+    """Preallocated outputs + workspace for repeated moga_layer calls."""
+
+    def __init__(self, N, d, H, d_h, M, grid=None, window=None, x_dtype=torch.bfloat16, device="cuda"):
+        lib = get_lib()
+        self.N, self.d, self.H, self.d_h, self.M = N, d, H, d_h, M
+        self.grid = tuple(grid) if grid is not None else (0, 0, 0)
+        self.window = tuple(window) if window is not None else None
+        self.x_dt = {torch.float32: MOGA_F32, torch.bfloat16: MOGA_BF16}[x_dtype]
+        self.device = torch.device(device)
+        self._w3 = _int3(self.window) if self.window else None
+        need = lib.moga_layer_workspace_size(N, H, d_h, M, *self.grid, self._w3)
+        self.ws = workspace(need, self.device)
+        self.out = torch.empty((N, H, d_h), dtype=torch.bfloat16, device=self.device)
+        self.group_id = torch.empty(N, dtype=torch.int32, device=self.device)
+        self.gate = torch.empty(N, dtype=torch.float32, device=self.device)
+        self.perm = torch.empty(N, dtype=torch.int32, device=self.device)
+        self.offsets = torch.empty(M + 1, dtype=torch.int32, device=self.device)
+
+    def __call__(self, x, W_r, b_r, q, k, v):
+        lib = get_lib()
+        st = lib.moga_layer(_ptr(x), _ptr(W_r), _ptr(b_r), self.x_dt, _ptr(q), _ptr(k), _ptr(v), self.N, self.d,
+                            self.H, self.d_h, self.M, *self.grid, self._w3, _ptr(self.out), _ptr(self.group_id),
+                            _ptr(self.gate), _ptr(self.perm), _ptr(self.offsets), _ptr(self.ws), self.ws.numel(),
+                            _stream(self.device))
+        _check(st, "moga_layer")
+        return self.out
+
+
+def moga_layer(x, W_r, b_r, q, k, v, M: int, grid=None, window=None):
+    """One MoGA block: returns dict(out, group_id, gate, perm, offsets)."""
+    N, d = x.shape
+    _, H, d_h = q.shape
+    for n, t in (("x", x), ("q", q), ("k", k), ("v", v)):
+        _dev_tensor(t, n)
+    layer = MogaLayer(N, d, H, d_h, M, grid, window, x.dtype, x.device)
+    layer(x, W_r, b_r, q, k, v)
+    return {"out": layer.out, "group_id": layer.group_id, "gate": layer.gate, "perm": layer.perm,
+            "offsets": layer.offsets, "ws": layer.ws}

@@ -1,0 +1,376 @@
+// C ABI of the MoGA layer library (declarations and contracts in moga.h).
+// Host side only: argument validation, workspace carving, TMA descriptor
+// encoding and kernel sequencing.  No device memory is allocated here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "../../include/moga.h"
+#include "internal.h"
+
+namespace moga {
+
+namespace {
+
+std::atomic<uint64_t> g_wait_ns{4000000000ull};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int num_sms_of(int dev) {
+  static std::atomic<int> cache[64];
+  if (dev < 0 || dev >= 64) return 148;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+  cache[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+constexpr size_t kHeader = 256;  // status word and spare words
+
+// Sequential 256-byte aligned carving of a workspace after its header.
+struct Carve {
+  size_t off = kHeader;
+  size_t take(size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  }
+};
+
+struct RouteWs {
+  size_t hist, base, total;
+};
+RouteWs route_ws(int64_t N, int M) {
+  Carve c;
+  RouteWs w;
+  const size_t cells = (size_t)ceil_div(N, kTile) * (size_t)M;
+  w.hist = c.take(cells * 4);
+  w.base = c.take(cells * 4);
+  w.total = c.off;
+  return w;
+}
+
+struct AttnWs {
+  size_t table, permw, qh, kh, vh, total;
+};
+AttnWs attn_ws(int64_t N, int H, int d_h, int nseg_table, bool window_perm) {
+  Carve c;
+  AttnWs w;
+  w.table = c.take((size_t)(3 * nseg_table + 1) * 4);
+  w.permw = window_perm ? c.take((size_t)N * 4) : 0;
+  const size_t mat = (size_t)N * H * d_h * 2;
+  w.qh = c.take(mat);
+  w.kh = c.take(mat);
+  w.vh = c.take(mat);
+  w.total = c.off;
+  return w;
+}
+
+moga_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MOGA_OK : MOGA_ERR_CUDA; }
+
+bool make_ctx(DevCtx* c, void* ws, void* stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  c->device = dev;
+  c->num_sms = num_sms_of(dev);
+  c->stream = reinterpret_cast<cudaStream_t>(stream);
+  c->status = reinterpret_cast<int*>(ws);
+  c->wait_ns = g_wait_ns.load(std::memory_order_relaxed);
+  return true;
+}
+
+moga_status check_attn_shape(int64_t N, int H, int d_h) {
+  if (N < 0 || H < 1) return MOGA_ERR_INVALID_ARG;
+  if (d_h != 64 && d_h != 128) return MOGA_ERR_UNSUPPORTED;
+  if (N * (int64_t)H >= (int64_t)1 << 31) return MOGA_ERR_UNSUPPORTED;
+  return MOGA_OK;
+}
+
+moga_status check_window(int T, int Hg, int Wg, const int* window, int64_t* N) {
+  if (!window || T < 1 || Hg < 1 || Wg < 1) return MOGA_ERR_INVALID_ARG;
+  if (window[0] < 1 || window[1] < 1 || window[2] < 1) return MOGA_ERR_INVALID_ARG;
+  const int64_t n = (int64_t)T * Hg * Wg;
+  if (n >= (int64_t)1 << 31) return MOGA_ERR_UNSUPPORTED;
+  *N = n;
+  return MOGA_OK;
+}
+
+// ------------------------------------------------------------------ bodies (args already validated)
+moga_status route_body(const DevCtx& c, const void* x, const void* W, const float* b, moga_dtype dt, int64_t N,
+                       int d, int M, int32_t* gid, float* gate, int32_t* perm, int32_t* offsets,
+                       int32_t* max_seqlen, uint8_t* ws) {
+  if (N == 0) {
+    cudaError_t e = cudaMemsetAsync(offsets, 0, (size_t)(M + 1) * 4, c.stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(max_seqlen, 0, 4, c.stream);
+    return from_cuda(e);
+  }
+  const RouteWs w = route_ws(N, M);
+  int32_t* hist = reinterpret_cast<int32_t*>(ws + w.hist);
+  int32_t* base = reinterpret_cast<int32_t*>(ws + w.base);
+  cudaError_t e;
+  if (dt == MOGA_BF16 && M <= 256 && d >= 64)
+    e = launch_route_tc(c, x, W, b, N, d, M, gid, gate, hist);
+  else
+    e = launch_route_simt(c, x, W, b, dt == MOGA_BF16, N, d, M, gid, gate, hist);
+  if (e != cudaSuccess) return MOGA_ERR_CUDA;
+  if ((e = launch_scan(c, hist, ceil_div(N, kTile), M, base, offsets, max_seqlen)) != cudaSuccess)
+    return MOGA_ERR_CUDA;
+  if ((e = launch_scatter(c, gid, base, N, M, perm)) != cudaSuccess) return MOGA_ERR_CUDA;
+  return MOGA_OK;
+}
+
+moga_status group_attn_body(const DevCtx& c, const void* q, const void* k, const void* v, const int32_t* perm,
+                            const int32_t* offsets, const float* gate, int64_t N, int H, int d_h, int M,
+                            float out_scale, void* out, uint8_t* ws) {
+  if (N == 0) return MOGA_OK;
+  const AttnWs w = attn_ws(N, H, d_h, M, false);
+  int32_t* table = reinterpret_cast<int32_t*>(ws + w.table);
+  if (launch_seg_table(c, offsets, M, H, N, table) != cudaSuccess) return MOGA_ERR_CUDA;
+  if (launch_gather(c, q, k, v, perm, N, H, d_h, ws + w.qh, ws + w.kh, ws + w.vh) != cudaSuccess)
+    return MOGA_ERR_CUDA;
+  AttnArgs a{};
+  a.qh = ws + w.qh;
+  a.kh = ws + w.kh;
+  a.vh = ws + w.vh;
+  a.perm = perm;
+  a.gate = gate;
+  a.out = out;
+  a.N = N;
+  a.H = H;
+  a.d_h = d_h;
+  a.out_scale = out_scale;
+  a.accumulate = 0;
+  a.mode = 0;
+  a.table = table;
+  a.nseg = M;
+  return from_cuda(launch_attention(c, a));
+}
+
+moga_status stga_body(const DevCtx& c, const void* q, const void* k, const void* v, int T, int Hg, int Wg,
+                      const int* window, int H, int d_h, int accumulate, void* out, uint8_t* ws) {
+  const int64_t N = (int64_t)T * Hg * Wg;
+  const AttnWs w = attn_ws(N, H, d_h, 0, true);
+  int32_t* permw = reinterpret_cast<int32_t*>(ws + w.permw);
+  if (launch_window_perm(c, T, Hg, Wg, window, permw) != cudaSuccess) return MOGA_ERR_CUDA;
+  if (launch_gather(c, q, k, v, permw, N, H, d_h, ws + w.qh, ws + w.kh, ws + w.vh) != cudaSuccess)
+    return MOGA_ERR_CUDA;
+  AttnArgs a{};
+  a.qh = ws + w.qh;
+  a.kh = ws + w.kh;
+  a.vh = ws + w.vh;
+  a.perm = permw;
+  a.gate = nullptr;
+  a.out = out;
+  a.N = N;
+  a.H = H;
+  a.d_h = d_h;
+  a.out_scale = accumulate ? 0.5f : 1.0f;
+  a.accumulate = accumulate ? 1 : 0;
+  a.mode = 1;
+  a.table = nullptr;
+  a.nseg = (int)stga_num_windows(T, Hg, Wg, window);
+  a.T = T;
+  a.Hg = Hg;
+  a.Wg = Wg;
+  a.wt = window[0];
+  a.wh = window[1];
+  a.ww = window[2];
+  return from_cuda(launch_attention(c, a));
+}
+
+moga_status check_route_args(const void* x, const void* W_r, const float* b_r, moga_dtype dt, int64_t N, int d,
+                             int M, const int32_t* gid, const float* gate, const int32_t* perm,
+                             const int32_t* offsets, const int32_t* max_seqlen) {
+  if (!x || !W_r || !gid || !gate || !perm || !offsets || !max_seqlen) return MOGA_ERR_INVALID_ARG;
+  if (dt != MOGA_F32 && dt != MOGA_BF16) return MOGA_ERR_INVALID_ARG;
+  if (N < 0 || N >= ((int64_t)1 << 31) || M < 1 || M > 1024) return MOGA_ERR_INVALID_ARG;
+  if (d < 1) return MOGA_ERR_INVALID_ARG;
+  if (dt == MOGA_BF16 && (d % 8) != 0) return MOGA_ERR_UNSUPPORTED;
+  if (dt == MOGA_F32 && (d % 4) != 0) return MOGA_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(W_r)) return MOGA_ERR_INVALID_ARG;
+  if ((b_r && !aligned4(b_r)) || !aligned4(gid) || !aligned4(gate) || !aligned4(perm) || !aligned4(offsets) ||
+      !aligned4(max_seqlen))
+    return MOGA_ERR_INVALID_ARG;
+  return MOGA_OK;
+}
+
+moga_status check_qkv(const void* q, const void* k, const void* v, const void* out) {
+  if (!q || !k || !v || !out) return MOGA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return MOGA_ERR_INVALID_ARG;
+  return MOGA_OK;
+}
+
+}  // namespace
+
+bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
+                  uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace moga
+
+using namespace moga;
+
+extern "C" {
+
+const char* moga_status_string(int s) {
+  switch (s) {
+    case MOGA_OK: return "MOGA_OK";
+    case MOGA_ERR_INVALID_ARG: return "MOGA_ERR_INVALID_ARG";
+    case MOGA_ERR_UNSUPPORTED: return "MOGA_ERR_UNSUPPORTED";
+    case MOGA_ERR_WORKSPACE: return "MOGA_ERR_WORKSPACE";
+    case MOGA_ERR_CUDA: return "MOGA_ERR_CUDA";
+    case MOGA_ERR_TIMEOUT: return "MOGA_ERR_TIMEOUT";
+    case MOGA_ERR_DEVICE_CHECK: return "MOGA_ERR_DEVICE_CHECK";
+    default: return "MOGA_ERR_UNKNOWN";
+  }
+}
+
+int moga_version(void) { return (1 << 16) | 0; }
+
+uint64_t moga_set_wait_limit_ns(uint64_t ns) { return g_wait_ns.exchange(ns ? ns : 1); }
+
+size_t moga_route_workspace_size(int64_t N, int M) {
+  if (N < 0 || M < 1) return 0;
+  return route_ws(N, M).total;
+}
+
+moga_status moga_route(const void* x, const void* W_r, const float* b_r, moga_dtype dt, int64_t N, int d, int M,
+                       int32_t* group_id, float* gate, int32_t* perm, int32_t* offsets, int32_t* max_seqlen,
+                       void* ws, size_t ws_bytes, void* stream) {
+  moga_status st = check_route_args(x, W_r, b_r, dt, N, d, M, group_id, gate, perm, offsets, max_seqlen);
+  if (st != MOGA_OK) return st;
+  if (!ws || !aligned16(ws)) return MOGA_ERR_INVALID_ARG;
+  if (ws_bytes < route_ws(N, M).total) return MOGA_ERR_WORKSPACE;
+  DevCtx c;
+  if (!make_ctx(&c, ws, stream)) return MOGA_ERR_CUDA;
+  return route_body(c, x, W_r, b_r, dt, N, d, M, group_id, gate, perm, offsets, max_seqlen, (uint8_t*)ws);
+}
+
+size_t moga_group_attn_workspace_size(int64_t N, int H, int d_h, int M) {
+  if (N < 0 || H < 1 || M < 1) return 0;
+  return attn_ws(N, H, d_h, M, false).total;
+}
+
+moga_status moga_group_attn(const void* q, const void* k, const void* v, const int32_t* perm,
+                            const int32_t* offsets, const float* gate, int64_t N, int H, int d_h, int M,
+                            float out_scale, void* out, void* ws, size_t ws_bytes, void* stream) {
+  moga_status st = check_qkv(q, k, v, out);
+  if (st != MOGA_OK) return st;
+  if (!perm || !offsets || !aligned4(perm) || !aligned4(offsets) || (gate && !aligned4(gate)))
+    return MOGA_ERR_INVALID_ARG;
+  if (M < 1 || M > 1024) return MOGA_ERR_INVALID_ARG;
+  if ((st = check_attn_shape(N, H, d_h)) != MOGA_OK) return st;
+  if (!ws || !aligned16(ws)) return MOGA_ERR_INVALID_ARG;
+  if (ws_bytes < attn_ws(N, H, d_h, M, false).total) return MOGA_ERR_WORKSPACE;
+  DevCtx c;
+  if (!make_ctx(&c, ws, stream)) return MOGA_ERR_CUDA;
+  return group_attn_body(c, q, k, v, perm, offsets, gate, N, H, d_h, M, out_scale, out, (uint8_t*)ws);
+}
+
+size_t stga_window_attn_workspace_size(int T, int Hg, int Wg, const int* window, int H, int d_h) {
+  int64_t N = 0;
+  if (check_window(T, Hg, Wg, window, &N) != MOGA_OK || H < 1) return 0;
+  return attn_ws(N, H, d_h, 0, true).total;
+}
+
+moga_status stga_window_attn(const void* q, const void* k, const void* v, int T, int Hg, int Wg,
+                             const int* window, int H, int d_h, int accumulate, void* out, void* ws,
+                             size_t ws_bytes, void* stream) {
+  moga_status st = check_qkv(q, k, v, out);
+  if (st != MOGA_OK) return st;
+  int64_t N = 0;
+  if ((st = check_window(T, Hg, Wg, window, &N)) != MOGA_OK) return st;
+  if ((st = check_attn_shape(N, H, d_h)) != MOGA_OK) return st;
+  if (accumulate != 0 && accumulate != 1) return MOGA_ERR_INVALID_ARG;
+  if (!ws || !aligned16(ws)) return MOGA_ERR_INVALID_ARG;
+  if (ws_bytes < attn_ws(N, H, d_h, 0, true).total) return MOGA_ERR_WORKSPACE;
+  DevCtx c;
+  if (!make_ctx(&c, ws, stream)) return MOGA_ERR_CUDA;
+  return stga_body(c, q, k, v, T, Hg, Wg, window, H, d_h, accumulate, out, (uint8_t*)ws);
+}
+
+size_t moga_layer_workspace_size(int64_t N, int H, int d_h, int M, int T, int Hg, int Wg, const int* window) {
+  if (N < 0 || H < 1 || M < 1) return 0;
+  size_t need = route_ws(N, M).total;
+  const size_t ga = attn_ws(N, H, d_h, M, false).total;
+  if (ga > need) need = ga;
+  if (window) {
+    const size_t sw = attn_ws(N, H, d_h, 0, true).total;
+    if (sw > need) need = sw;
+  }
+  return need;
+}
+
+moga_status moga_layer(const void* x, const void* W_r, const float* b_r, moga_dtype x_dt, const void* q,
+                       const void* k, const void* v, int64_t N, int d, int H, int d_h, int M, int T, int Hg,
+                       int Wg, const int* window, void* out, int32_t* group_id, float* gate, int32_t* perm,
+                       int32_t* offsets, void* ws, size_t ws_bytes, void* stream) {
+  moga_status st = check_route_args(x, W_r, b_r, x_dt, N, d, M, group_id, gate, perm, offsets, offsets);
+  if (st != MOGA_OK) return st;
+  if ((st = check_qkv(q, k, v, out)) != MOGA_OK) return st;
+  if ((st = check_attn_shape(N, H, d_h)) != MOGA_OK) return st;
+  if (window) {
+    int64_t n = 0;
+    if ((st = check_window(T, Hg, Wg, window, &n)) != MOGA_OK) return st;
+    if (n != N) return MOGA_ERR_INVALID_ARG;
+  }
+  if (!ws || !aligned16(ws)) return MOGA_ERR_INVALID_ARG;
+  if (ws_bytes < moga_layer_workspace_size(N, H, d_h, M, T, Hg, Wg, window)) return MOGA_ERR_WORKSPACE;
+  DevCtx c;
+  if (!make_ctx(&c, ws, stream)) return MOGA_ERR_CUDA;
+  uint8_t* w = (uint8_t*)ws;
+  // max_seqlen has no output slot in the layer call: keep it in the header.
+  int32_t* max_seqlen = reinterpret_cast<int32_t*>(w + 16);
+  if ((st = route_body(c, x, W_r, b_r, x_dt, N, d, M, group_id, gate, perm, offsets, max_seqlen, w)) != MOGA_OK)
+    return st;
+  if (N == 0) return MOGA_OK;
+  const float scale = window ? 0.5f : 1.0f;
+  if ((st = group_attn_body(c, q, k, v, perm, offsets, gate, N, H, d_h, M, scale, out, w)) != MOGA_OK) return st;
+  if (window) return stga_body(c, q, k, v, T, Hg, Wg, window, H, d_h, 1, out, w);
+  return MOGA_OK;
+}
+
+moga_status moga_sync_status(void* ws, void* stream) {
+  if (!ws || !aligned16(ws)) return MOGA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOGA_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOGA_ERR_CUDA;
+  if (word != 0 && cudaMemset(ws, 0, sizeof(int)) != cudaSuccess) return MOGA_ERR_CUDA;
+  if (word & DEV_TIMEOUT) return MOGA_ERR_TIMEOUT;
+  if (word) return MOGA_ERR_DEVICE_CHECK;
+  return MOGA_OK;
+}
+
+}  // extern "C"

@@ -126,16 +126,20 @@ def attention_rows(q_rows: np.ndarray, K: np.ndarray, V: np.ndarray) -> np.ndarr
     return p @ V
 
 
-def _attend_sets(q, k, v, sets: Iterable[np.ndarray], rows_mask, heads, scale_rows,
+def _attend_sets(q, k, v, sets: Iterable[np.ndarray], row_pos, heads, scale_rows,
                  out: np.ndarray, q_block: int = 512):
-    """Attention of each token set's queries to the same set's keys/values."""
+    """Attention of each token set's queries to the same set's keys/values.
+
+    row_pos[i] is the output row of token i (or -1 when token i is not
+    requested); heads lists the heads to compute, in output order.
+    """
     for idx in sets:
         if idx.size == 0:
             continue
-        qi = idx if rows_mask is None else idx[rows_mask[idx]]
+        qi = idx[row_pos[idx] >= 0]
         if qi.size == 0:
             continue
-        for h in heads:
+        for hp, h in enumerate(heads):
             Kh = _f64(k[idx, h])
             Vh = _f64(v[idx, h])
             for b0 in range(0, qi.size, q_block):
@@ -143,8 +147,22 @@ def _attend_sets(q, k, v, sets: Iterable[np.ndarray], rows_mask, heads, scale_ro
                 o = attention_rows(_f64(q[rows, h]), Kh, Vh)
                 if scale_rows is not None:
                     o = o * scale_rows[rows][:, None]
-                out[rows, h] = o
+                out[row_pos[rows], hp] = o
     return out
+
+
+def _row_layout(N, H, d_h, rows, heads):
+    """Output buffer and token -> output-row map for full or sampled runs."""
+    heads = list(range(H)) if heads is None else [int(h) for h in heads]
+    row_pos = np.full(N, -1, dtype=np.int64)
+    if rows is None:
+        row_pos[:] = np.arange(N)
+        n_out = N
+    else:
+        rows = np.asarray(rows, dtype=np.int64)
+        row_pos[rows] = np.arange(rows.size)
+        n_out = rows.size
+    return np.full((n_out, len(heads), d_h), np.nan), row_pos, heads
 
 
 def group_attention(q, k, v, group_id, gate, M: int,
@@ -153,21 +171,18 @@ def group_attention(q, k, v, group_id, gate, M: int,
     """MoGA output, Eq. 5, computed directly in original token order.
 
     out[i, h] = gate[i] * SA(q[i,h], K_{g(i),h}, V_{g(i),h}) where K_g, V_g hold
-    the keys/values of every token routed to g(i).  ``rows`` restricts the
-    queries that are computed (others stay NaN); ``heads`` restricts the heads.
-    q, k, v: [N, H, d_h] arrays (any float type; upcast exactly to float64).
+    the keys/values of every token routed to g(i).  q, k, v: [N, H, d_h]
+    arrays or tensors (any float type; upcast exactly to float64, and only the
+    rows a group needs are read).  Returns [N, H, d_h]; with ``rows`` (distinct
+    token indices) and/or ``heads`` only those are computed and the result is
+    [len(rows), len(heads), d_h] in the given order.
     """
     N, H, d_h = q.shape
     g = np.asarray(group_id, dtype=np.int64)
     gate = _f64(gate)
-    out = np.full((N, H, d_h), np.nan)
-    mask = None
-    if rows is not None:
-        mask = np.zeros(N, dtype=bool)
-        mask[np.asarray(rows, dtype=np.int64)] = True
-    hs = range(H) if heads is None else heads
+    out, row_pos, hs = _row_layout(N, H, d_h, rows, heads)
     sets = (np.nonzero(g == m)[0] for m in range(M))
-    return _attend_sets(q, k, v, sets, mask, hs, gate, out)
+    return _attend_sets(q, k, v, sets, row_pos, hs, gate, out)
 
 
 def stga_windows(T: int, Hg: int, Wg: int, window) -> List[np.ndarray]:
@@ -193,16 +208,14 @@ def stga_windows(T: int, Hg: int, Wg: int, window) -> List[np.ndarray]:
 def stga_attention(q, k, v, T: int, Hg: int, Wg: int, window,
                    rows: Optional[Sequence[int]] = None,
                    heads: Optional[Sequence[int]] = None) -> np.ndarray:
-    """STGA: full attention inside each spatio-temporal window (no gate)."""
+    """STGA: full attention inside each spatio-temporal window (no gate).
+
+    Output layout as for ``group_attention``.
+    """
     N, H, d_h = q.shape
     assert T * Hg * Wg == N
-    out = np.full((N, H, d_h), np.nan)
-    mask = None
-    if rows is not None:
-        mask = np.zeros(N, dtype=bool)
-        mask[np.asarray(rows, dtype=np.int64)] = True
-    hs = range(H) if heads is None else heads
-    return _attend_sets(q, k, v, stga_windows(T, Hg, Wg, window), mask, hs, None, out)
+    out, row_pos, hs = _row_layout(N, H, d_h, rows, heads)
+    return _attend_sets(q, k, v, stga_windows(T, Hg, Wg, window), row_pos, hs, None, out)
 
 
 def moga_layer(x, W_r, b_r, q, k, v, M: int, grid=None, window=None,

@@ -1,0 +1,111 @@
+"""C ABI checks that need no GPU: the library loads, exports every function
+declared in include/moga.h, and rejects invalid arguments before touching the
+device.  Fake pointer values are never dereferenced: validation fails first."""
+import ctypes
+
+import pytest
+
+import learned_token_group_b200 as moga
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+P = 1 << 20          # a 16-byte aligned fake device address (never dereferenced)
+BIG = 1 << 40
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return moga.get_lib()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = moga.exported_names()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in moga.h but not exported"
+
+
+def test_version_and_status_strings(lib):
+    assert lib.moga_version() >> 16 == 1
+    for code, name in moga.STATUS.items():
+        assert lib.moga_status_string(code).decode() == name
+    assert lib.moga_status_string(99).decode() == "MOGA_ERR_UNKNOWN"
+
+
+def test_workspace_sizes(lib):
+    r1 = lib.moga_route_workspace_size(1000, 16)
+    r2 = lib.moga_route_workspace_size(100000, 16)
+    assert 256 < r1 < r2
+    a = lib.moga_group_attn_workspace_size(1000, 2, 128, 4)
+    assert a >= 3 * 1000 * 2 * 128 * 2
+    w3 = (ctypes.c_int * 3)(3, 8, 8)
+    s = lib.stga_window_attn_workspace_size(3, 8, 16, w3, 2, 128)
+    assert s >= 3 * 384 * 2 * 128 * 2 + 384 * 4
+    layer = lib.moga_layer_workspace_size(384, 2, 128, 4, 3, 8, 16, w3)
+    assert layer >= max(s, lib.moga_group_attn_workspace_size(384, 2, 128, 4), lib.moga_route_workspace_size(384, 4))
+    assert lib.moga_route_workspace_size(-1, 4) == 0
+
+
+def _route(lib, x=P, W=P, b=None, dt=1, N=1000, d=64, M=4, out=P, ws=P, wsb=BIG):
+    return lib.moga_route(x, W, b, dt, N, d, M, out, out, out, out, out, ws, wsb, None)
+
+
+def test_route_validation(lib):
+    assert _route(lib, x=None) == INVALID
+    assert _route(lib, W=None) == INVALID
+    assert _route(lib, out=None) == INVALID
+    assert _route(lib, M=0) == INVALID
+    assert _route(lib, M=1025) == INVALID
+    assert _route(lib, dt=7) == INVALID
+    assert _route(lib, N=-1) == INVALID
+    assert _route(lib, d=60) == UNSUPPORTED          # bf16 rows must be 16-byte multiples
+    assert _route(lib, x=P + 2) == INVALID           # misaligned
+    assert _route(lib, ws=None) == INVALID
+    assert _route(lib, wsb=16) == WORKSPACE
+
+
+def _ga(lib, q=P, perm=P, N=1000, H=2, d_h=128, M=4, ws=P, wsb=BIG):
+    return lib.moga_group_attn(q, q, q, perm, perm, None, N, H, d_h, M, 1.0, q, ws, wsb, None)
+
+
+def test_group_attn_validation(lib):
+    assert _ga(lib, q=None) == INVALID
+    assert _ga(lib, perm=None) == INVALID
+    assert _ga(lib, d_h=96) == UNSUPPORTED
+    assert _ga(lib, H=0) == INVALID
+    assert _ga(lib, M=0) == INVALID
+    assert _ga(lib, N=1 << 28, H=16) == UNSUPPORTED  # N*H beyond int32 rows
+    assert _ga(lib, q=P + 8) == INVALID
+    assert _ga(lib, wsb=1024) == WORKSPACE
+
+
+def test_stga_validation(lib):
+    w = (ctypes.c_int * 3)(3, 8, 8)
+    bad = (ctypes.c_int * 3)(3, 0, 8)
+    f = lib.stga_window_attn
+    assert f(P, P, P, 3, 8, 16, None, 2, 128, 0, P, P, BIG, None) == INVALID
+    assert f(P, P, P, 3, 8, 16, bad, 2, 128, 0, P, P, BIG, None) == INVALID
+    assert f(P, P, P, 0, 8, 16, w, 2, 128, 0, P, P, BIG, None) == INVALID
+    assert f(P, P, P, 3, 8, 16, w, 2, 128, 2, P, P, BIG, None) == INVALID
+    assert f(P, P, P, 3, 8, 16, w, 2, 32, 0, P, P, BIG, None) == UNSUPPORTED
+    assert f(P, P, P, 3, 8, 16, w, 2, 128, 0, P, P, 100, None) == WORKSPACE
+
+
+def test_layer_validation(lib):
+    w = (ctypes.c_int * 3)(3, 8, 8)
+    f = lib.moga_layer
+    args = [P, P, None, 1, P, P, P, 384, 256, 2, 128, 4, 3, 8, 16, w, P, P, P, P, P, P, BIG, None]
+    bad_n = list(args)
+    bad_n[7] = 385                                    # N != T*Hg*Wg
+    assert f(*bad_n) == INVALID
+    no_ws = list(args)
+    no_ws[21] = None
+    assert f(*no_ws) == INVALID
+    small = list(args)
+    small[22] = 4096
+    assert f(*small) == WORKSPACE
+    assert lib.moga_sync_status(None, None) == INVALID
+
+
+def test_wait_limit_roundtrip(lib):
+    old = lib.moga_set_wait_limit_ns(123456)
+    assert lib.moga_set_wait_limit_ns(old) == 123456
