@@ -1,0 +1,388 @@
+#!/usr/bin/env python
+"""Benchmark of one MoGA block (router -> grouped attention -> STGA -> mean).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one call of the library's moga_layer over one batch of synthetic
+inputs already resident in HBM (the whole hot path: router, counting sort,
+gather, grouped attention with gate + un-permute, STGA window attention with
+the two-branch mean).  Inputs are larger than L2 (126 MB), so no flush is
+needed between steps.  Multi-GPU runs (torchrun) are independent replicas:
+the layer has no exchange step on one node, every rank runs its own seeded
+batch, and the time is the max over ranks.
+
+Rank 0 prints ONE JSON line.  Besides the contract keys it carries the
+per-stage breakdown (CUDA events recorded by the library on its own stream),
+the roofline of the dominant kernel (grouped attention: useful FLOPs
+4 * sum_g n_g^2 * d_h * H over the kernel's own time), the end-to-end number
+through the C ABI with pinned host buffers, and the CPU oracle baseline on a
+bounded sample.  ``--impl reference`` times the oracle alone (CPU).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "MoGA layer fwd tokens/s & group-attn TFLOPS (% bf16 peak) at 187k/580k ctx"
+UNIT = "tokens/s"
+DEFAULT_CONFIG = "video_187k"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p["bf16_tflops_sustained"]), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = os.path.join("/tmp", f"moga_clocks_{os.getpid()}.csv")
+        ident = str(device_index)
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            pass
+        self.ident = ident
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.ident, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+                except ValueError:
+                    continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        pmax = max(r[2] for r in rows)
+        load = [r for r in rows if r[2] >= 0.5 * pmax] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": pmax, "samples": len(load), "reasons": reasons}
+
+
+# ----------------------------------------------------------------------------- helpers
+def _stga_flops(wl):
+    if wl.window is None:
+        return 0.0
+    import itertools
+    T, Hg, Wg = wl.grid
+    wt, wh, ww = wl.window
+    s = 0
+    for t0, h0, w0 in itertools.product(range(0, T, wt), range(0, Hg, wh), range(0, Wg, ww)):
+        n = min(wt, T - t0) * min(wh, Hg - h0) * min(ww, Wg - w0)
+        s += n * n
+    return 4.0 * s * wl.d_h * wl.H
+
+
+def _cfg(wl, world):
+    return {"workload": wl.name, "N": wl.N, "H": wl.H, "d_h": wl.d_h, "d_model": wl.d, "M": wl.M,
+            "grid": "x".join(map(str, wl.grid)) if wl.grid else None,
+            "stga_window": "x".join(map(str, wl.window)) if wl.window else None,
+            "x": f"{wl.x_kind} {wl.x_dtype}", "l2": "inputs larger than L2 (no flush)",
+            "parallelism": f"replicas x{world}"}
+
+
+def oracle_sample_time(wl, inp_cpu, seed=0, route_rows=16384, attn_rows=256):
+    """Times the CPU oracle on a bounded sample and extrapolates to N tokens.
+
+    route: `route_rows` tokens (per-token independent, scaled by N/route_rows);
+    counting sort: all N tokens; grouped attention and STGA: `attn_rows` query
+    tokens (all heads), scaled by N/attn_rows.  Returns (seconds for N tokens,
+    sample description).
+    """
+    import oracle
+
+    rng = np.random.default_rng(seed)
+    N = wl.N
+    r0 = int(rng.integers(0, max(1, N - route_rows)))
+    t = time.perf_counter()
+    oracle.route(inp_cpu["x"][r0:r0 + route_rows], inp_cpu["W_r"], inp_cpu["b_r"])
+    t_route = (time.perf_counter() - t) * N / min(route_rows, N)
+    # full routing is needed for the groups (not timed beyond the sample above)
+    gid, gate, _ = oracle.route(inp_cpu["x"], inp_cpu["W_r"], inp_cpu["b_r"]) if "gid" not in inp_cpu else \
+        (inp_cpu["gid"], inp_cpu["gate"], None)
+    inp_cpu["gid"], inp_cpu["gate"] = gid, gate
+    t = time.perf_counter()
+    oracle.counting_sort(gid, wl.M)
+    t_sort = time.perf_counter() - t
+    # attention: two sample sizes give the per-(group, head) set-up cost a (the
+    # oracle converts each group's K/V once) and the per-query cost b;
+    # t(N) = a + b * N.
+    sizes = (min(attn_rows // 4, N), min(attn_rows, N))
+    ts = []
+    for S in sizes:
+        rows = np.sort(rng.choice(N, size=S, replace=False))
+        t = time.perf_counter()
+        oracle.group_attention(inp_cpu["q"], inp_cpu["k"], inp_cpu["v"], gid, gate, wl.M, rows=rows)
+        if wl.window is not None:
+            oracle.stga_attention(inp_cpu["q"], inp_cpu["k"], inp_cpu["v"], *wl.grid, wl.window, rows=rows)
+        ts.append(time.perf_counter() - t)
+    b = max(ts[1] - ts[0], 0.0) / max(sizes[1] - sizes[0], 1)
+    a = max(ts[0] - b * sizes[0], 0.0)
+    t_attn = a + b * N
+    total = t_route + t_sort + t_attn
+    desc = (f"router on {min(route_rows, N)} tokens scaled to N; counting sort on all {N}; grouped attention + "
+            f"STGA on {sizes[0]} and {sizes[1]} query tokens (all heads), fitted as fixed + per-token cost and "
+            f"extrapolated to N={N}")
+    return total, desc
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+# ----------------------------------------------------------------------------- arms
+def run_reference(args, wl, rank, world):
+    """The oracle (CPU) as the reference arm: each step is a bounded sample."""
+    if rank != 0:
+        return
+    inp = make_inputs(wl, seed=args.seed, device="cpu")
+    desc = ""
+    for _ in range(args.warmup):
+        _, desc = oracle_sample_time(wl, inp, seed=args.seed)
+    times = []
+    for i in range(args.steps):
+        t_i, desc = oracle_sample_time(wl, inp, seed=args.seed + 1 + i)
+        times.append(t_i)
+    t = statistics.mean(times)
+    value = wl.N / t
+    cores = _blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, CPU)",
+            "config": _cfg(wl, 1),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, wl, rank, world, dist):
+    import learned_token_group_b200 as moga
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = make_inputs(wl, seed=args.seed + rank, device=dev)
+    layer = moga.MogaLayer(wl.N, wl.d, wl.H, wl.d_h, wl.M, wl.grid, wl.window,
+                           torch.float32 if wl.x_dtype == "f32" else torch.bfloat16, dev)
+    step = lambda: layer(inp["x"], inp["W_r"], inp["b_r"], inp["q"], inp["k"], inp["v"])
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    moga.sync_status(layer.ws)
+    counts = np.diff(layer.offsets.cpu().numpy().astype(np.int64))
+    flops_group = 4.0 * float((counts.astype(np.float64) ** 2).sum()) * wl.d_h * wl.H
+    flops_stga = _stga_flops(wl)
+
+    # ---- timed region: K layer steps, device time, max over ranks
+    stream = torch.cuda.current_stream(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        torch.cuda.synchronize()
+        barrier()
+        l0 = moga.kernel_launches()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        launches = moga.kernel_launches() - l0
+    moga.sync_status(layer.ws)
+    ms = ev0.elapsed_time(ev1) / args.steps
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    clocks = clk.summary()
+
+    # ---- per-stage breakdown: events recorded by the library around each stage
+    stages = list(moga.STAGES)
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in stages]
+           for _ in range(args.steps)]
+    for row in evs:                      # create the CUDA events before handing them to the library
+        for b_ev, e_ev in row:
+            b_ev.record(stream)
+            e_ev.record(stream)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        for s, name in enumerate(stages):
+            moga.set_timing_events(name, *evs[i][s])
+        step()
+    for name in stages:
+        moga.set_timing_events(name, None, None)
+    torch.cuda.synchronize()
+    stage_ms = {name: statistics.mean(evs[i][s][0].elapsed_time(evs[i][s][1]) for i in range(args.steps))
+                for s, name in enumerate(stages)}
+
+    # ---- end to end through the C ABI: pinned host inputs in, result out, every step
+    host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in inp.items()}
+    dinp = {k: (torch.empty_like(v) if v is not None else None) for k, v in inp.items()}
+    out_host = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        for k, v in host.items():
+            if v is not None:
+                dinp[k].copy_(v, non_blocking=True)
+        layer(dinp["x"], dinp["W_r"], dinp["b_r"], dinp["q"], dinp["k"], dinp["v"])
+        out_host.copy_(layer.out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    ev0.record(stream)
+    n_e2e = max(1, min(args.steps, 5))
+    for _ in range(n_e2e):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = ev0.elapsed_time(ev1) / n_e2e
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    moga.sync_status(layer.ws)
+
+    if rank != 0:
+        return
+    peaks = _peaks()
+    peak = peaks["bf16_tflops_sustained"]
+    t_attn = stage_ms["group_attn"] * 1e-3
+    attn_tflops = flops_group / t_attn / 1e12
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu_inp = {k: (v.cpu() if v is not None else None) for k, v in inp.items()}
+        t_cpu, desc = oracle_sample_time(wl, cpu_inp, seed=args.seed)
+        cpu = {"value": wl.N / t_cpu, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle", "sample": desc}
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", f"traffic_{wl.name}.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            traffic = json.load(f).get("group_attn_bytes_per_launch")
+    hbm = peaks["hbm_gbs"]
+    Dbytes = wl.N * wl.H * wl.d_h * 2
+    bw = {
+        "router_GBs": (wl.N * wl.d * (2 if wl.x_dtype == "bf16" else 4) + 8 * wl.N) / (stage_ms["router"] * 1e-3) / 1e9,
+        "gather_GBs": (6 * Dbytes + 4 * wl.N) / (stage_ms["gather"] * 1e-3) / 1e9,
+        "stga_prep_GBs": (6 * Dbytes + 8 * wl.N) / (stage_ms["stga_prep"] * 1e-3) / 1e9 if wl.window else None,
+    }
+    line = {
+        "metric": METRIC, "value": wl.N * world / (ms * 1e-3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; random router weights, clustered tokens)",
+        "config": _cfg(wl, world),
+        "group_attn_tflops": attn_tflops,
+        "group_attn_frac_of_peak": attn_tflops / peak,
+        "flops_vs_full_attention": (flops_group + flops_stga) / (4.0 * wl.N * wl.N * wl.d_h * wl.H),
+        "stage_ms": stage_ms,
+        "stage_hbm_GBs": bw,
+        "group_sizes": counts.tolist(),
+        "roofline": {"kernel": "attn_kernel<128> (grouped attention)", "bound": "tensor",
+                     "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s", "frac": attn_tflops / peak,
+                     "peak_kind": f"bf16 dense, sustained, {peaks['source']}", "traffic": traffic},
+        "cpu_baseline": cpu,
+        "e2e": {"value": wl.N * world / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = WORKLOADS[args.config]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, wl, rank, world)
+        return
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist = dist_mod
+    try:
+        run_ours(args, wl, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

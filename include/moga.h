@@ -154,6 +154,27 @@ moga_status moga_sync_status(void* ws, void* stream);
  * Process-wide.  Returns the previous value. */
 uint64_t moga_set_wait_limit_ns(uint64_t ns);
 
+/* ---------------------------------------------------------------- instrumentation
+ * moga_kernel_launches: process-wide count of kernels this library has
+ * launched so far (memsets excluded).
+ *
+ * moga_set_timing_events: when begin/end are non-NULL cudaEvent_t handles,
+ * every later call records `begin` on its stream right before the launches of
+ * `stage` and `end` right after them (so the event pair brackets exactly that
+ * stage's kernels on the stream they run on).  NULL/NULL detaches.  Process-
+ * wide and not synchronised with concurrent calls: meant for benchmarks.
+ * Returns MOGA_ERR_INVALID_ARG for an unknown stage or a half-NULL pair. */
+typedef enum {
+  MOGA_STAGE_ROUTER = 0,      /* router kernel (logits, gate, argmax, tile histogram) */
+  MOGA_STAGE_SORT = 1,        /* scan + stable scatter -> offsets, perm */
+  MOGA_STAGE_GATHER = 2,      /* segment table + gather of Q/K/V into group order */
+  MOGA_STAGE_GROUP_ATTN = 3,  /* grouped attention kernel (incl. gate + un-permute) */
+  MOGA_STAGE_STGA_PREP = 4,   /* window permutation + gather into window order */
+  MOGA_STAGE_STGA_ATTN = 5    /* STGA window attention kernel (incl. the mean) */
+} moga_stage;
+uint64_t moga_kernel_launches(void);
+moga_status moga_set_timing_events(int stage, void* begin, void* end);
+
 #ifdef __cplusplus
 }
 #endif

@@ -19,7 +19,8 @@ from typing import Optional, Sequence
 import torch
 
 __all__ = ["MogaError", "get_lib", "LIB_PATH", "HEADER_PATH", "route", "group_attn", "stga_window_attn",
-           "moga_layer", "sync_status", "workspace", "MogaLayer", "exported_names"]
+           "moga_layer", "sync_status", "workspace", "MogaLayer", "exported_names", "kernel_launches",
+           "set_timing_events", "STAGES"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoga.so")
@@ -62,6 +63,8 @@ def get_lib():
         "moga_layer": (_I, [_P, _P, _P, _I, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _I, _P,
                             _P, _P, _P, _P, _P, _P, _SZ, _P]),
         "moga_sync_status": (_I, [_P, _P]),
+        "moga_kernel_launches": (ctypes.c_uint64, []),
+        "moga_set_timing_events": (_I, [_I, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -110,6 +113,21 @@ def _dev_tensor(t: torch.Tensor, name: str, dtype=None):
 def workspace(nbytes: int, device) -> torch.Tensor:
     """Zero-filled device workspace (the status word must start clear)."""
     return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+STAGES = {"router": 0, "sort": 1, "gather": 2, "group_attn": 3, "stga_prep": 4, "stga_attn": 5}
+
+
+def kernel_launches() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(get_lib().moga_kernel_launches())
+
+
+def set_timing_events(stage: str, begin=None, end=None) -> None:
+    """Attach (or detach, with None) a torch.cuda.Event pair to a stage."""
+    b = None if begin is None else ctypes.c_void_p(begin.cuda_event)
+    e = None if end is None else ctypes.c_void_p(end.cuda_event)
+    _check(get_lib().moga_set_timing_events(STAGES[stage], b, e), "moga_set_timing_events")
 
 
 def sync_status(ws: torch.Tensor) -> None:

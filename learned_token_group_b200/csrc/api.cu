@@ -15,6 +15,17 @@ namespace moga {
 namespace {
 
 std::atomic<uint64_t> g_wait_ns{4000000000ull};
+std::atomic<uint64_t> g_launches{0};
+constexpr int kNumStages = 6;
+std::atomic<void*> g_ev_begin[kNumStages];
+std::atomic<void*> g_ev_end[kNumStages];
+
+// Records the optional timing event of `stage` on the call's stream.
+void mark(int stage, bool begin, cudaStream_t s) {
+  void* ev = (begin ? g_ev_begin : g_ev_end)[stage].load(std::memory_order_relaxed);
+  if (ev) cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev), s);
+}
+void count(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -129,14 +140,19 @@ moga_status route_body(const DevCtx& c, const void* x, const void* W, const floa
   int32_t* hist = reinterpret_cast<int32_t*>(ws + w.hist);
   int32_t* base = reinterpret_cast<int32_t*>(ws + w.base);
   cudaError_t e;
+  mark(MOGA_STAGE_ROUTER, true, c.stream);
   if (dt == MOGA_BF16 && M <= 256 && d >= 64)
     e = launch_route_tc(c, x, W, b, N, d, M, gid, gate, hist);
   else
     e = launch_route_simt(c, x, W, b, dt == MOGA_BF16, N, d, M, gid, gate, hist);
+  mark(MOGA_STAGE_ROUTER, false, c.stream);
   if (e != cudaSuccess) return MOGA_ERR_CUDA;
+  mark(MOGA_STAGE_SORT, true, c.stream);
   if ((e = launch_scan(c, hist, ceil_div(N, kTile), M, base, offsets, max_seqlen)) != cudaSuccess)
     return MOGA_ERR_CUDA;
   if ((e = launch_scatter(c, gid, base, N, M, perm)) != cudaSuccess) return MOGA_ERR_CUDA;
+  mark(MOGA_STAGE_SORT, false, c.stream);
+  count(3);
   return MOGA_OK;
 }
 
@@ -146,9 +162,12 @@ moga_status group_attn_body(const DevCtx& c, const void* q, const void* k, const
   if (N == 0) return MOGA_OK;
   const AttnWs w = attn_ws(N, H, d_h, M, false);
   int32_t* table = reinterpret_cast<int32_t*>(ws + w.table);
+  mark(MOGA_STAGE_GATHER, true, c.stream);
   if (launch_seg_table(c, offsets, M, H, N, table) != cudaSuccess) return MOGA_ERR_CUDA;
   if (launch_gather(c, q, k, v, perm, N, H, d_h, ws + w.qh, ws + w.kh, ws + w.vh) != cudaSuccess)
     return MOGA_ERR_CUDA;
+  mark(MOGA_STAGE_GATHER, false, c.stream);
+  count(2);
   AttnArgs a{};
   a.qh = ws + w.qh;
   a.kh = ws + w.kh;
@@ -164,7 +183,11 @@ moga_status group_attn_body(const DevCtx& c, const void* q, const void* k, const
   a.mode = 0;
   a.table = table;
   a.nseg = M;
-  return from_cuda(launch_attention(c, a));
+  mark(MOGA_STAGE_GROUP_ATTN, true, c.stream);
+  const cudaError_t e = launch_attention(c, a);
+  mark(MOGA_STAGE_GROUP_ATTN, false, c.stream);
+  count(1);
+  return from_cuda(e);
 }
 
 moga_status stga_body(const DevCtx& c, const void* q, const void* k, const void* v, int T, int Hg, int Wg,
@@ -172,9 +195,12 @@ moga_status stga_body(const DevCtx& c, const void* q, const void* k, const void*
   const int64_t N = (int64_t)T * Hg * Wg;
   const AttnWs w = attn_ws(N, H, d_h, 0, true);
   int32_t* permw = reinterpret_cast<int32_t*>(ws + w.permw);
+  mark(MOGA_STAGE_STGA_PREP, true, c.stream);
   if (launch_window_perm(c, T, Hg, Wg, window, permw) != cudaSuccess) return MOGA_ERR_CUDA;
   if (launch_gather(c, q, k, v, permw, N, H, d_h, ws + w.qh, ws + w.kh, ws + w.vh) != cudaSuccess)
     return MOGA_ERR_CUDA;
+  mark(MOGA_STAGE_STGA_PREP, false, c.stream);
+  count(2);
   AttnArgs a{};
   a.qh = ws + w.qh;
   a.kh = ws + w.kh;
@@ -196,15 +222,20 @@ moga_status stga_body(const DevCtx& c, const void* q, const void* k, const void*
   a.wt = window[0];
   a.wh = window[1];
   a.ww = window[2];
-  return from_cuda(launch_attention(c, a));
+  mark(MOGA_STAGE_STGA_ATTN, true, c.stream);
+  const cudaError_t e = launch_attention(c, a);
+  mark(MOGA_STAGE_STGA_ATTN, false, c.stream);
+  count(1);
+  return from_cuda(e);
 }
 
 moga_status check_route_args(const void* x, const void* W_r, const float* b_r, moga_dtype dt, int64_t N, int d,
                              int M, const int32_t* gid, const float* gate, const int32_t* perm,
                              const int32_t* offsets, const int32_t* max_seqlen) {
-  if (!x || !W_r || !gid || !gate || !perm || !offsets || !max_seqlen) return MOGA_ERR_INVALID_ARG;
-  if (dt != MOGA_F32 && dt != MOGA_BF16) return MOGA_ERR_INVALID_ARG;
   if (N < 0 || N >= ((int64_t)1 << 31) || M < 1 || M > 1024) return MOGA_ERR_INVALID_ARG;
+  // per-token buffers may be NULL when there are no tokens
+  if (!W_r || !offsets || !max_seqlen || (N > 0 && (!x || !gid || !gate || !perm))) return MOGA_ERR_INVALID_ARG;
+  if (dt != MOGA_F32 && dt != MOGA_BF16) return MOGA_ERR_INVALID_ARG;
   if (d < 1) return MOGA_ERR_INVALID_ARG;
   if (dt == MOGA_BF16 && (d % 8) != 0) return MOGA_ERR_UNSUPPORTED;
   if (dt == MOGA_F32 && (d % 4) != 0) return MOGA_ERR_UNSUPPORTED;
@@ -259,6 +290,16 @@ const char* moga_status_string(int s) {
 int moga_version(void) { return (1 << 16) | 0; }
 
 uint64_t moga_set_wait_limit_ns(uint64_t ns) { return g_wait_ns.exchange(ns ? ns : 1); }
+
+uint64_t moga_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+moga_status moga_set_timing_events(int stage, void* begin, void* end) {
+  if (stage < 0 || stage >= kNumStages) return MOGA_ERR_INVALID_ARG;
+  if ((begin == nullptr) != (end == nullptr)) return MOGA_ERR_INVALID_ARG;
+  g_ev_begin[stage].store(begin, std::memory_order_relaxed);
+  g_ev_end[stage].store(end, std::memory_order_relaxed);
+  return MOGA_OK;
+}
 
 size_t moga_route_workspace_size(int64_t N, int M) {
   if (N < 0 || M < 1) return 0;
