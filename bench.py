@@ -256,6 +256,12 @@ def run_ours(args, wl, rank, world, dist):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
     clocks = clk.summary()
+    if args.lean:
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": wl.N * world / (ms * 1e-3), "unit": UNIT,
+                              "n_gpus": world, "ms_per_step": ms, "config": _cfg(wl, world), "lean": True,
+                              "gpu_launches": int(launches), "clocks": clocks}), flush=True)
+        return
 
     # ---- per-stage breakdown: events recorded by the library around each stage
     stages = list(moga.STAGES)
@@ -363,6 +369,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--lean", action="store_true",
+                    help="warm-up and timed steps only (for hardware-counter captures)")
     args = ap.parse_args()
     wl = WORKLOADS[args.config]
     world = int(os.environ.get("WORLD_SIZE", "1"))

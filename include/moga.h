@@ -88,6 +88,31 @@ moga_status moga_route(const void* x, const void* W_r, const float* b_r, moga_dt
                        int M, int32_t* group_id, float* gate, int32_t* perm, int32_t* offsets,
                        int32_t* max_seqlen, void* ws, size_t ws_bytes, void* stream);
 
+/* moga_route_noalloc: the same routing as moga_route, for callers that cannot
+ * allocate device memory themselves (for example code running inside a
+ * framework whose allocator owns the GPU, or a pre-recorded launch sequence
+ * that must not call cudaMalloc).  It takes no workspace: its scratch (the
+ * per-tile group histograms and bases, about 2 MiB) is a fixed device array
+ * inside the library that every GPU loading the library keeps until the
+ * process exits.  The method pages have no counterpart to this call; it only
+ * changes where the scratch lives.
+ * - Outputs, limits and results are those of moga_route, plus one more limit:
+ *   ceil(N / 128) * M <= 262144 (e.g. N = 580,320 with M = 32, or N = 187,200
+ *   with M = 64); larger sizes return MOGA_ERR_WORKSPACE and touch nothing.
+ * - It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * - The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture on the device.
+ * - Every call shares the one array and it keeps the last call's contents;
+ *   the call clears what must start at zero.  Calls that overlap on the GPU
+ *   (different streams, or different host threads, on one device) race on
+ *   the array: order them on one stream.
+ * - Device-side wait timeouts of this call are not reported (there is no
+ *   workspace status word to read back). */
+moga_status moga_route_noalloc(const void* x, const void* W_r, const float* b_r, moga_dtype dt, int64_t N, int d,
+                               int M, int32_t* group_id, float* gate, int32_t* perm, int32_t* offsets,
+                               int32_t* max_seqlen, void* stream);
+
 /* ---------------------------------------------------------------- grouped attention
  * moga_group_attn: Algorithm 1 steps 2 (gather), 3 (attention inside each
  * group segment) and 4 (un-permute), with the gate of Eq. 5 fused into the

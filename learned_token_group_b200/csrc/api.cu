@@ -54,6 +54,31 @@ int num_sms_of(int dev) {
   return v;
 }
 
+// ------------------------------------------------------------------ allocation-free routing scratch
+// Scratch of moga_route_noalloc: the routing tile histograms and bases live in
+// this file-scope device array instead of a caller workspace.  Every GPU that
+// loads the library holds it (about 2 MiB) until the process exits.  Host code
+// must not pass the symbol itself to a kernel (on the host it only names a
+// stand-in); its device address comes from cudaGetSymbolAddress below.
+constexpr int64_t kNoAllocCells = (int64_t)1 << 18;  // max ceil(N/128) * M
+constexpr size_t kNoAllocBytes = 256 + 2 * (size_t)kNoAllocCells * 4;
+static __device__ __align__(256) uint8_t g_route_scratch[kNoAllocBytes];
+
+// Device address of g_route_scratch for the current device, looked up once per
+// device (the first call on a device does it; see moga.h).
+uint8_t* noalloc_scratch(int dev) {
+  static std::mutex mu;
+  static uint8_t* addr[64] = {};
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    addr[dev] = static_cast<uint8_t*>(p);
+  }
+  return addr[dev];
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
@@ -316,6 +341,22 @@ moga_status moga_route(const void* x, const void* W_r, const float* b_r, moga_dt
   DevCtx c;
   if (!make_ctx(&c, ws, stream)) return MOGA_ERR_CUDA;
   return route_body(c, x, W_r, b_r, dt, N, d, M, group_id, gate, perm, offsets, max_seqlen, (uint8_t*)ws);
+}
+
+moga_status moga_route_noalloc(const void* x, const void* W_r, const float* b_r, moga_dtype dt, int64_t N, int d,
+                               int M, int32_t* group_id, float* gate, int32_t* perm, int32_t* offsets,
+                               int32_t* max_seqlen, void* stream) {
+  moga_status st = check_route_args(x, W_r, b_r, dt, N, d, M, group_id, gate, perm, offsets, max_seqlen);
+  if (st != MOGA_OK) return st;
+  if (ceil_div(N, kTile) * (int64_t)M > kNoAllocCells) return MOGA_ERR_WORKSPACE;
+  DevCtx c;
+  if (!make_ctx(&c, nullptr, stream)) return MOGA_ERR_CUDA;
+  uint8_t* scratch = noalloc_scratch(c.device);
+  if (!scratch) return MOGA_ERR_CUDA;
+  c.status = reinterpret_cast<int*>(scratch);
+  // route_body writes every scratch word it reads later, except the tile
+  // histogram of the tensor-core router, which its launcher zeroes first.
+  return route_body(c, x, W_r, b_r, dt, N, d, M, group_id, gate, perm, offsets, max_seqlen, scratch);
 }
 
 size_t moga_group_attn_workspace_size(int64_t N, int H, int d_h, int M) {

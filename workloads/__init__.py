@@ -73,6 +73,10 @@ WORKLOADS = {
                             (372, 30, 52), (3, 8, 8)),
     "skew_187k": Workload("skew_187k", 187200, 12, 128, 1536, 64, "bf16", "skew",
                           (120, 30, 52), (3, 8, 8)),
+    # video_187k with 4 heads: q/k/v still exceed L2 (192 MB each) while the
+    # device footprint stays near 2 GB, for hardware-counter captures.
+    "profile_187k_h4": Workload("profile_187k_h4", 187200, 4, 128, 1536, 16, "bf16", "clustered",
+                                (120, 30, 52), (3, 8, 8)),
 }
 
 _FORCED = (1, 2, 3, 5, 8, 13, 21, 34)   # sizes of the forced small groups (skew)
