@@ -122,8 +122,10 @@ moga_status moga_route_noalloc(const void* x, const void* W_r, const float* b_r,
  * (gate = 1).  Tokens of empty groups do not exist, so every token's row of
  * `out` is written exactly once.
  * In:  q, k, v bf16 [N, H, d_h]; perm int32 [N]; offsets int32 [M+1]
- *      (non-decreasing, offsets[0] = 0, offsets[M] = N; not checked on the
- *      device); gate fp32 [N] or NULL.
+ *      (non-decreasing, offsets[0] = 0, offsets[M] = N); gate fp32 [N] or
+ *      NULL.  The device checks offsets and every perm entry it uses: a
+ *      violation skips the affected work and is reported by
+ *      moga_sync_status() as MOGA_ERR_DEVICE_CHECK.
  * Out: out bf16 [N, H, d_h].
  * Limits: d_h in {64, 128}; 1 <= H; N * H < 2^31; 1 <= M <= 1024.
  * Workspace: moga_group_attn_workspace_size(N, H, d_h, M) bytes.
