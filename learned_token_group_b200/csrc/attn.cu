@@ -10,17 +10,24 @@
 // seg_table_kernel  groups sorted by size (largest first) with the prefix of
 //                   their query-tile counts: the persistent attention grid walks
 //                   this longest-first order.
-// attn_kernel<DH>   persistent varlen flash attention on tcgen05.  Per CTA:
-//                   warp 0 issues TMA loads (Q tile, double-buffered K/V),
-//                   warp 1 issues tcgen05.mma (S = Q K^T into one of two TMEM
-//                   S buffers, O += P V into a TMEM O buffer), warps 2-5 run the
-//                   online softmax on one query row per thread (S read from
-//                   TMEM, P written as bf16 into a 128B-swizzled smem tile, O
-//                   rescaled in TMEM only when a row max grows by more than
-//                   2^8), and the epilogue scales by gate/l and scatters each
-//                   row to out[perm[j]] (or adds into it for the STGA branch).
+// attn_kernel<DH>   persistent varlen flash attention on tcgen05.  A CTA works
+//                   on two 128-row query tiles (A, B) of one (segment, head)
+//                   at a time, streaming the segment's K/V tiles once for both.
+//                   Warp 0 issues TMA loads (Q_A, Q_B, double-buffered K and V
+//                   rings); warp 1 issues tcgen05.mma in the order
+//                   PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so the tensor core
+//                   works on one tile while the other tile's softmax runs;
+//                   warps 2-5 and 6-9 are the two softmax warpgroups (one query
+//                   row per thread): S is read from TMEM, P is written back as
+//                   bf16 over S in TMEM and consumed from there by the P V
+//                   product, O is rescaled in TMEM only when a row max grows by
+//                   more than 2^8; the epilogue scales by gate/l and scatters
+//                   each row to out[perm[j]] (or adds into it for the STGA
+//                   branch).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+
+#include <type_traits>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -29,7 +36,7 @@ namespace moga {
 
 namespace {
 
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-5 / 6-9 softmax of tiles A / B
 constexpr int kStages = 2;
 
 __device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
@@ -100,8 +107,9 @@ __global__ void window_perm_kernel(WinGeom g, int N, int32_t* __restrict__ perm_
   perm_w[start + ((t - t0) * eh + (h - h0)) * ew + (w - w0)] = i;
 }
 
-// table = [tile_prefix (M+1) | seg_start (M) | seg_len (M)], groups in
-// descending size order (ties: lower group first).
+// table = [unit_prefix (M+1) | seg_start (M) | seg_len (M)], groups in
+// descending size order (ties: lower group first); a unit is a pair of
+// 128-row query tiles of one head.
 __global__ void __launch_bounds__(1024)
 seg_table_kernel(const int32_t* __restrict__ offsets, int M, int H, int64_t N, int32_t* __restrict__ table,
                  int* status) {
@@ -143,7 +151,7 @@ seg_table_kernel(const int32_t* __restrict__ offsets, int M, int H, int64_t N, i
       table[r] = run;
       table[M + 1 + r] = offsets[g];
       table[2 * M + 1 + r] = n;
-      run += ((n + kTile - 1) / kTile) * H;
+      run += (((n + kTile - 1) / kTile + 1) / 2) * H;  // pairs of query tiles per head
     }
     table[M] = run;
   }
@@ -152,50 +160,51 @@ seg_table_kernel(const int32_t* __restrict__ offsets, int M, int H, int64_t N, i
 template <int DH>
 struct Plan {
   static constexpr int kChunks = DH / 64;
-  static constexpr int kTileBytes = kTile * DH * 2;  // one 128-row bf16 operand
-  static constexpr int kQ = 0;
-  static constexpr int kK0 = kTileBytes;
-  static constexpr int kStageBytes = 2 * kTileBytes;  // K then V
-  static constexpr int kP = kK0 + kStages * kStageBytes;
-  static constexpr int kPBytes = kTile * kTile * 2;
-  static constexpr int kBar = kP + kPBytes;
+  static constexpr int kTileBytes = kTile * DH * 2;   // one 128-row bf16 operand tile
+  static constexpr int kQA = 0;                        // query tile A
+  static constexpr int kQB = kTileBytes;               // query tile B
+  static constexpr int kK0 = 2 * kTileBytes;           // K ring [kStages]
+  static constexpr int kV0 = kK0 + kStages * kTileBytes;  // V ring [kStages]
+  static constexpr int kBar = kV0 + kStages * kTileBytes;
   static constexpr int kTable = kBar + 256;
   static size_t bytes(int table_ints) { return (size_t)kTable + (size_t)table_ints * 4 + 1024; }
 };
 
-struct TileInfo {
-  int h, start, len, q0;
+// A work unit is a pair of consecutive 128-row query tiles (A, B) of one
+// (segment, head); both stream the same K/V tiles.
+struct Unit {
+  int h, start, len, q0;  // q0: first row of tile A inside the segment; tile B starts at q0 + 128
 };
 
 struct Decoder {
-  const AttnArgs* a;
-  const int* tab;  // shared copy of the segment table (groups)
+  int mode;
+  int nseg;
+  const int* tab;  // groups: shared copy of [unit_prefix (M+1) | seg_start (M) | seg_len (M)]
   WinGeom g;
-  int tpw;         // query tiles per window (windows)
-  __device__ __forceinline__ TileInfo operator()(int idx) const {
-    TileInfo t;
-    if (a->mode == 0) {
-      const int M = a->nseg;
-      int lo = 0, hi = M - 1;  // largest r with prefix[r] <= idx
+  int upw;         // windows: units per window
+  __device__ __forceinline__ Unit operator()(int idx) const {
+    Unit u;
+    if (mode == 0) {
+      int lo = 0, hi = nseg - 1;  // largest r with prefix[r] <= idx
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (tab[mid] <= idx) lo = mid; else hi = mid - 1;
       }
       const int local = idx - tab[lo];
-      t.start = tab[M + 1 + lo];
-      t.len = tab[2 * M + 1 + lo];
-      const int ntq = (t.len + kTile - 1) / kTile;
-      t.h = local / ntq;
-      t.q0 = (local - t.h * ntq) * kTile;
+      u.start = tab[nseg + 1 + lo];
+      u.len = tab[2 * nseg + 1 + lo];
+      const int npair = ((u.len + kTile - 1) / kTile + 1) / 2;
+      u.h = local / npair;
+      u.q0 = (local - u.h * npair) * 2 * kTile;
     } else {
-      const int qt = idx % tpw;
-      const int rest = idx / tpw;
-      const int seg = rest % a->nseg;
-      t.h = rest / a->nseg;
-      window_of(g, seg, t.start, t.len);
-      t.q0 = qt * kTile;
+      const int qp = idx % upw;
+      const int rest = idx / upw;
+      const int seg = rest % nseg;
+      u.h = rest / nseg;
+      window_of(g, seg, u.start, u.len);
+      u.q0 = qp * 2 * kTile;
     }
-    return t;
+    return u;
   }
 };
 
@@ -210,15 +219,16 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P::kBar);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* kv_full = bars + 2;    // [kStages]
-  uint64_t* kv_empty = bars + 4;   // [kStages]
-  uint64_t* s_full = bars + 6;     // [2]
-  uint64_t* s_empty = bars + 8;    // [2]
-  uint64_t* p_full = bars + 10;
-  uint64_t* o_ready = bars + 11;
-  uint64_t* done_bar = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 14);
+  uint64_t* k_full = bars + 2;    // [kStages]
+  uint64_t* k_empty = bars + 4;   // [kStages]
+  uint64_t* v_full = bars + 6;    // [kStages]
+  uint64_t* v_empty = bars + 8;   // [kStages]
+  uint64_t* s_full = bars + 10;   // [2]: S of tile A / B computed
+  uint64_t* p_full = bars + 12;   // [2]: P of tile A / B written (O rescaled)
+  uint64_t* o_full = bars + 14;   // [2]: last P V of tile A / B done
+  uint64_t* done_bar = bars + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 18);
   int* tab = reinterpret_cast<int*>(smem + P::kTable);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -227,29 +237,31 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&s_empty[b], 128);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_full[x], 128);
+      mbar_init(&o_full[x], 1);
     }
-    mbar_init(p_full, 128);
-    mbar_init(o_ready, 1);
     mbar_init(done_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  int total;
   Decoder dec;
-  dec.a = &a;
+  dec.mode = a.mode;
+  dec.nseg = a.nseg;
   dec.tab = tab;
+  dec.upw = 1;
   if (a.mode == 0) {
     const int n = 3 * a.nseg + 1;
     for (int i = threadIdx.x; i < n; i += blockDim.x) tab[i] = a.table[i];
   } else {
     dec.g = WinGeom{a.T, a.Hg, a.Wg, a.wt, a.wh, a.ww, (a.Hg + a.wh - 1) / a.wh, (a.Wg + a.ww - 1) / a.ww};
-    dec.tpw = (a.wt * a.wh * a.ww + kTile - 1) / kTile;
+    dec.upw = ((a.wt * a.wh * a.ww + kTile - 1) / kTile + 1) / 2;
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -258,10 +270,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  total = (a.mode == 0) ? tab[a.nseg] : a.nseg * dec.tpw * a.H;
+  const int total = (a.mode == 0) ? tab[a.nseg] : a.nseg * dec.upw * a.H;
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem;             // S buffers: columns [0,128) and [128,256)
-  const uint32_t tO = tmem + 256;       // O: columns [256, 256 + DH)
+  // TMEM columns: S/P of tile A [0,128), S/P of tile B [128,256), O of A [256,..), O of B [384,..).
+  // P (bf16, two per column) overwrites the first 64 columns of its tile's S.
+  auto tS = [tmem](int x) { return tmem + (uint32_t)(x * 128); };
+  auto tO = [tmem](int x) { return tmem + 256u + (uint32_t)(x * 128); };
   WaitCtx wc{abort_flag, status, wait_ns};
   const int64_t N = a.N;
 
@@ -271,38 +285,49 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       tma_prefetch_desc(&tq);
       tma_prefetch_desc(&tk);
       tma_prefetch_desc(&tv);
-      uint32_t it = 0, tcnt = 0;
+      uint32_t ucnt = 0, kc = 0, vc = 0;
       bool ok = true;
       for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
-        const TileInfo ti = dec(idx);
-        if (ti.q0 >= ti.len) continue;
-        const int nkv = (ti.len + kTile - 1) / kTile;
-        if (!mbar_wait(q_empty, (tcnt & 1) ^ 1, wc)) break;
-        const int rowq = (int)((int64_t)ti.h * N + ti.start + ti.q0);
-        mbar_expect_tx(q_full, P::kTileBytes);
+        const Unit u = dec(idx);
+        if (u.q0 >= u.len) continue;
+        const bool hb = u.q0 + kTile < u.len;
+        const int nkv = (u.len + kTile - 1) / kTile;
+        if (!mbar_wait(q_empty, (ucnt & 1) ^ 1, wc)) break;
+        const int rowq = (int)((int64_t)u.h * N + u.start + u.q0);
+        mbar_expect_tx(q_full, (hb ? 2 : 1) * P::kTileBytes);
 #pragma unroll
-        for (int c = 0; c < P::kChunks; ++c) tma_load_2d(&tq, q_full, smem + P::kQ + c * 16384, c * 64, rowq);
-        for (int kv = 0; kv < nkv; ++kv, ++it) {
-          const int st = it % kStages;
-          if (!mbar_wait(&kv_empty[st], ((it / kStages) & 1) ^ 1, wc)) { ok = false; break; }
-          const int rowk = (int)((int64_t)ti.h * N + ti.start + kv * kTile);
-          uint8_t* ks = smem + P::kK0 + st * P::kStageBytes;
-          mbar_expect_tx(&kv_full[st], 2 * P::kTileBytes);
+        for (int c = 0; c < P::kChunks; ++c) tma_load_2d(&tq, q_full, smem + P::kQA + c * 16384, c * 64, rowq);
+        if (hb) {
 #pragma unroll
-          for (int c = 0; c < P::kChunks; ++c) {
-            tma_load_2d(&tk, &kv_full[st], ks + c * 16384, c * 64, rowk);
-            tma_load_2d(&tv, &kv_full[st], ks + P::kTileBytes + c * 16384, c * 64, rowk);
-          }
+          for (int c = 0; c < P::kChunks; ++c)
+            tma_load_2d(&tq, q_full, smem + P::kQB + c * 16384, c * 64, rowq + kTile);
         }
-        ++tcnt;
+        ++ucnt;
+        for (int j = 0; j < nkv; ++j) {
+          const int rowk = (int)((int64_t)u.h * N + u.start + j * kTile);
+          const int ks = kc % kStages;
+          if (!mbar_wait(&k_empty[ks], ((kc / kStages) & 1) ^ 1, wc)) { ok = false; break; }
+          mbar_expect_tx(&k_full[ks], P::kTileBytes);
+#pragma unroll
+          for (int c = 0; c < P::kChunks; ++c)
+            tma_load_2d(&tk, &k_full[ks], smem + P::kK0 + ks * P::kTileBytes + c * 16384, c * 64, rowk);
+          ++kc;
+          const int vs = vc % kStages;
+          if (!mbar_wait(&v_empty[vs], ((vc / kStages) & 1) ^ 1, wc)) { ok = false; break; }
+          mbar_expect_tx(&v_full[vs], P::kTileBytes);
+#pragma unroll
+          for (int c = 0; c < P::kChunks; ++c)
+            tma_load_2d(&tv, &v_full[vs], smem + P::kV0 + vs * P::kTileBytes + c * 16384, c * 64, rowk);
+          ++vc;
+        }
       }
       // Drain every load this thread issued before the CTA exits.
       volatile int zero = 0;
       WaitCtx dc{&zero, nullptr, 100000000ull};
-      if (tcnt > 0) mbar_wait(q_full, (tcnt - 1) & 1, dc);
-      for (int s = 0; s < kStages && (uint32_t)s < it; ++s) {
-        const uint32_t last = it - 1 - ((it - 1 - s) % kStages);
-        mbar_wait(&kv_full[s], (last / kStages) & 1, dc);
+      if (ucnt > 0) mbar_wait(q_full, (ucnt - 1) & 1, dc);
+      for (int s = 0; s < kStages; ++s) {
+        if ((uint32_t)s < kc) mbar_wait(&k_full[s], ((kc - 1 - ((kc - 1 - s) % kStages)) / kStages) & 1, dc);
+        if ((uint32_t)s < vc) mbar_wait(&v_full[s], ((vc - 1 - ((vc - 1 - s) % kStages)) / kStages) & 1, dc);
       }
     }
   } else if (warp == 1) {
@@ -310,59 +335,83 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idO = idesc_bf16(128, DH, false, true);
-      const uint32_t q_addr = smem_u32(smem + P::kQ);
-      const uint32_t p_addr = smem_u32(smem + P::kP);
-      uint32_t it = 0, tcnt = 0, pcnt = 0;
+      uint32_t ucnt = 0, kc = 0, vc = 0, pc0 = 0, pc1 = 0;
       bool ok = true;
-      auto issue_pv = [&](int st, bool acc) {
-        const uint32_t v_addr = smem_u32(smem + P::kK0 + st * P::kStageBytes + P::kTileBytes);
+      // S_x = Q_x K^T (both K-major in smem, 128B swizzle)
+      auto issue_s = [&](int x, int ks) {
+        const uint32_t qa = smem_u32(smem + (x ? P::kQB : P::kQA));
+        const uint32_t ka = smem_u32(smem + P::kK0 + ks * P::kTileBytes);
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(p_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(v_addr + kk * 2048, 16384, 1024);
-          umma_bf16(tO, ad, bd, idO, (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_bf16(tS(x), sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idS,
+                    kk > 0 ? 1u : 0u);
         }
       };
-      for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
-        const TileInfo ti = dec(idx);
-        if (ti.q0 >= ti.len) continue;
-        const int nkv = (ti.len + kTile - 1) / kTile;
-        if (!mbar_wait(q_full, tcnt & 1, wc)) break;
-        tc_fence_after();
-        int prev_st = -1;
-        for (int kv = 0; kv < nkv; ++kv, ++it) {
-          const int st = it % kStages;
-          if (!mbar_wait(&kv_full[st], (it / kStages) & 1, wc)) { ok = false; break; }
-          const int sb = it & 1;
-          if (!mbar_wait(&s_empty[sb], ((it >> 1) & 1) ^ 1, wc)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(smem + P::kK0 + st * P::kStageBytes);
+      // O_x += P_x V (P in TMEM over S_x, V MN-major in smem)
+      auto issue_pv = [&](int x, int vs, bool acc) {
+        const uint32_t va = smem_u32(smem + P::kV0 + vs * P::kTileBytes);
 #pragma unroll
-          for (int kk = 0; kk < DH / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            umma_bf16(tS + sb * 128, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024), idS,
-                      kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&s_full[sb]);
-          if (kv == nkv - 1) umma_commit(q_empty);
-          if (prev_st >= 0) {
-            if (!mbar_wait(p_full, pcnt & 1, wc)) { ok = false; break; }
-            ++pcnt;
-            tc_fence_after();
-            issue_pv(prev_st, kv - 1 > 0);
-            umma_commit(&kv_empty[prev_st]);
-            umma_commit(o_ready);
-          }
-          prev_st = st;
-        }
-        if (!ok) break;
-        if (!mbar_wait(p_full, pcnt & 1, wc)) break;
-        ++pcnt;
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          umma_bf16_ts(tO(x), tS(x) + kk * 8, sdesc_sw128(va + kk * 2048, 16384, 1024), idO,
+                       (acc || kk > 0) ? 1u : 0u);
+      };
+      for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
+        const Unit u = dec(idx);
+        if (u.q0 >= u.len) continue;
+        const bool hb = u.q0 + kTile < u.len;
+        const int nkv = (u.len + kTile - 1) / kTile;
+        if (!mbar_wait(q_full, ucnt & 1, wc)) break;
+        ++ucnt;
+        int ks = kc % kStages;
+        if (!mbar_wait(&k_full[ks], (kc / kStages) & 1, wc)) break;
         tc_fence_after();
-        issue_pv(prev_st, nkv - 1 > 0);
-        umma_commit(&kv_empty[prev_st]);
-        umma_commit(o_ready);
-        ++tcnt;
+        issue_s(0, ks);
+        umma_commit(&s_full[0]);
+        if (hb) {
+          issue_s(1, ks);
+          umma_commit(&s_full[1]);
+        }
+        umma_commit(&k_empty[ks]);
+        ++kc;
+        if (nkv == 1) umma_commit(q_empty);
+        for (int j = 0; j < nkv; ++j) {
+          const int vs = vc % kStages;
+          const bool more = j + 1 < nkv;
+          if (!mbar_wait(&v_full[vs], (vc / kStages) & 1, wc)) { ok = false; break; }
+          if (!mbar_wait(&p_full[0], pc0 & 1, wc)) { ok = false; break; }
+          ++pc0;
+          tc_fence_after();
+          issue_pv(0, vs, j > 0);
+          ks = kc % kStages;
+          if (more) {
+            if (!mbar_wait(&k_full[ks], (kc / kStages) & 1, wc)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(0, ks);
+            umma_commit(&s_full[0]);
+          } else {
+            umma_commit(&o_full[0]);
+          }
+          if (hb) {
+            if (!mbar_wait(&p_full[1], pc1 & 1, wc)) { ok = false; break; }
+            ++pc1;
+            tc_fence_after();
+            issue_pv(1, vs, j > 0);
+            if (more) {
+              issue_s(1, ks);
+              umma_commit(&s_full[1]);
+            } else {
+              umma_commit(&o_full[1]);
+            }
+          }
+          umma_commit(&v_empty[vs]);
+          ++vc;
+          if (more) {
+            umma_commit(&k_empty[ks]);
+            ++kc;
+            if (j + 2 == nkv) umma_commit(q_empty);  // the unit's last S products are issued
+          }
+        }
       }
       umma_commit(done_bar);
       volatile int zero = 0;
@@ -371,90 +420,121 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     }
   } else {
     // ---------------------------------------------------------------- softmax + epilogue
-    const int sub = warp & 3;
+    const int x = (warp - 2) >> 2;  // warps 2-5: tile A, warps 6-9: tile B
+    const int sub = warp & 3;       // TMEM sub-partition this warp may access
     const int row = sub * 32 + lane;
     const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
+    const uint32_t tSx = tS(x) + lane_base, tOx = tO(x) + lane_base;
     const float scale_log2 = 1.4426950408889634f * rsqrtf((float)DH);
-    uint8_t* p_row = smem + P::kP + row * 128;
-    uint32_t it = 0, ocnt = 0;
+    uint32_t sc = 0, oc = 0;
     bool ok = true;
     for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
-      const TileInfo ti = dec(idx);
-      if (ti.q0 >= ti.len) continue;
-      const int nkv = (ti.len + kTile - 1) / kTile;
+      const Unit u = dec(idx);
+      if (u.q0 >= u.len) continue;
+      const bool hb = u.q0 + kTile < u.len;
+      if (x == 1 && !hb) continue;
+      const int nkv = (u.len + kTile - 1) / kTile;
       float m_run = -INFINITY, l = 0.f;
-      for (int kv = 0; kv < nkv; ++kv, ++it) {
-        const int sb = it & 1;
-        if (!mbar_wait(&s_full[sb], (it >> 1) & 1, wc)) { ok = false; break; }
+      for (int j = 0; j < nkv; ++j) {
+        if (!mbar_wait(&s_full[x], sc & 1, wc)) { ok = false; break; }
+        ++sc;
         tc_fence_after();
-        float s[kTile];
+        // pass 1: row max of S (raw scores), 32 columns at a time; the next
+        // chunk's TMEM load is in flight while the current one is reduced.
+        const int valid = u.len - j * kTile;  // keys of this tile inside the segment
+        float mx = -INFINITY;
+        // Only the segment's last KV tile has keys to mask (warp-uniform branch).
+        auto row_max = [&](auto masked) {
+          float cur[32], nxt[32];
+          tmem_ld32(tSx, cur);
 #pragma unroll
-        for (int c = 0; c < kTile / 32; ++c) tmem_ld32(tS + lane_base + sb * 128 + c * 32, s + c * 32);
-        tmem_ld_wait();
-        tc_fence_before();
-        mbar_arrive(&s_empty[sb]);
-        const int valid = min(kTile, ti.len - kv * kTile);
-        float rmax = -INFINITY;
+          for (int c = 0; c < kTile / 32; ++c) {
+            tmem_ld_wait();
+            if (c + 1 < kTile / 32) tmem_ld32(tSx + (c + 1) * 32, nxt);
 #pragma unroll
-        for (int j = 0; j < kTile; ++j) {
-          s[j] = (j < valid) ? s[j] * scale_log2 : -INFINITY;
-          rmax = fmaxf(rmax, s[j]);
-        }
-        if (kv > 0) {
-          // O and the P buffer are busy until the previous P V product lands.
-          if (!mbar_wait(o_ready, ocnt & 1, wc)) { ok = false; break; }
-          ++ocnt;
-          tc_fence_after();
-          const bool need = rmax > m_run + 8.0f;
-          if (__any_sync(0xffffffffu, need)) {
-            const float alpha = need ? fast_exp2(m_run - rmax) : 1.0f;
-            if (need) {
-              l *= alpha;
-              m_run = rmax;
+            for (int e = 0; e < 32; ++e) {
+              if constexpr (decltype(masked)::value)
+                mx = fmaxf(mx, (c * 32 + e < valid) ? cur[e] : -INFINITY);
+              else
+                mx = fmaxf(mx, cur[e]);
             }
 #pragma unroll
-            for (int c = 0; c < DH / 32; ++c) {
-              float o[32];
-              tmem_ld32(tO + lane_base + c * 32, o);
-              tmem_ld_wait();
-#pragma unroll
-              for (int j = 0; j < 32; ++j) o[j] *= alpha;
-              tmem_st32(tO + lane_base + c * 32, o);
-            }
-            tmem_st_wait();
+            for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
           }
+        };
+        if (valid >= kTile) row_max(std::false_type{}); else row_max(std::true_type{});
+        const float m_new = fmaxf(m_run, mx * scale_log2);
+        // O_x was last written by the previous P V product, which completed
+        // before this S (the MMA thread issued it first).  The running max is
+        // moved (and O rescaled) only when it grows by more than 2^8; P and l
+        // use the same stale max otherwise, so the result is unchanged.
+        float alpha = 1.0f;
+        bool rescale = false;
+        if (j == 0) {
+          m_run = m_new;
         } else {
-          m_run = rmax;
-        }
-#pragma unroll
-        for (int u = 0; u < kTile / 8; ++u) {
-          float p[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            p[e] = fast_exp2(s[u * 8 + e] - m_run);
-            l += p[e];
+          const bool need = m_new > m_run + 8.0f;
+          rescale = __any_sync(0xffffffffu, need);
+          if (need) {
+            alpha = fast_exp2(m_run - m_new);
+            l *= alpha;
+            m_run = m_new;
           }
-          uint4 pk;
-          pk.x = pack_bf16x2(p[0], p[1]);
-          pk.y = pack_bf16x2(p[2], p[3]);
-          pk.z = pack_bf16x2(p[4], p[5]);
-          pk.w = pack_bf16x2(p[6], p[7]);
-          *reinterpret_cast<uint4*>(p_row + (u >> 3) * 16384 + (((u & 7) ^ (row & 7)) << 4)) = pk;
         }
-        fence_proxy_async_smem();
+        // pass 2: P = 2^(S*scale - m), summed into l and written back over S
+        // as packed bf16 (two keys per TMEM column).
+        const float nm = -m_run;
+        auto write_p = [&](auto masked) {
+          float cur[32], nxt[32];
+          tmem_ld32(tSx, cur);
+#pragma unroll
+          for (int c = 0; c < kTile / 32; ++c) {
+            tmem_ld_wait();
+            if (c + 1 < kTile / 32) tmem_ld32(tSx + (c + 1) * 32, nxt);
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              float p0 = fast_exp2(fmaf(cur[2 * e], scale_log2, nm));
+              float p1 = fast_exp2(fmaf(cur[2 * e + 1], scale_log2, nm));
+              if constexpr (decltype(masked)::value) {
+                if (c * 32 + 2 * e >= valid) p0 = 0.0f;
+                if (c * 32 + 2 * e + 1 >= valid) p1 = 0.0f;
+              }
+              l += p0 + p1;
+              pk[e] = pack_bf16x2(p0, p1);
+            }
+            // columns [16c, 16c+16) hold S of keys already read into registers
+            tmem_st16u(tSx + c * 16, pk);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
+          }
+        };
+        if (valid >= kTile) write_p(std::false_type{}); else write_p(std::true_type{});
+        if (rescale) {
+#pragma unroll
+          for (int c = 0; c < DH / 32; ++c) {
+            float o[32];
+            tmem_ld32(tOx + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            tmem_st32(tOx + c * 32, o);
+          }
+        }
+        tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(p_full);
+        mbar_arrive(&p_full[x]);
       }
       if (!ok) break;
       // epilogue: wait for the last P V product, normalise, gate, scatter
-      if (!mbar_wait(o_ready, ocnt & 1, wc)) break;
-      ++ocnt;
+      if (!mbar_wait(&o_full[x], oc & 1, wc)) break;
+      ++oc;
       tc_fence_after();
-      const int r = ti.q0 + row;
-      bool live = r < ti.len;
+      const int r = u.q0 + x * kTile + row;
+      bool live = r < u.len;
       int64_t src = 0;
       if (live) {
-        src = a.perm[ti.start + r];
+        src = a.perm[u.start + r];
         if (src < 0 || src >= N) {
           live = false;
           if (status) atomicOr(status, DEV_RANGE);
@@ -462,21 +542,21 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       }
       const float gt = (live && a.gate) ? a.gate[src] : 1.0f;
       const float inv = a.out_scale * gt / l;
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) + (src * a.H + ti.h) * (int64_t)DH;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) + (src * a.H + u.h) * (int64_t)DH;
 #pragma unroll
       for (int c = 0; c < DH / 32; ++c) {
         float o[32];
-        tmem_ld32(tO + lane_base + c * 32, o);
+        tmem_ld32(tOx + c * 32, o);
         tmem_ld_wait();
         if (live) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int q4 = 0; q4 < 4; ++q4) {
             float w[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) w[e] = o[u * 8 + e] * inv;
+            for (int e = 0; e < 8; ++e) w[e] = o[q4 * 8 + e] * inv;
             if (a.accumulate) {
-              const uint4 old = dst[u];
+              const uint4 old = dst[q4];
               const __nv_bfloat162* ob = reinterpret_cast<const __nv_bfloat162*>(&old);
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
@@ -490,7 +570,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             pk.y = pack_bf16x2(w[2], w[3]);
             pk.z = pack_bf16x2(w[4], w[5]);
             pk.w = pack_bf16x2(w[6], w[7]);
-            dst[u] = pk;
+            dst[q4] = pk;
           }
         }
       }
@@ -520,7 +600,7 @@ cudaError_t launch_attention_dh(const DevCtx& c, const AttnArgs& a) {
   int grid = c.num_sms;
   if (a.mode == 1) {
     const int64_t tpw = ceil_div((int64_t)a.wt * a.wh * a.ww, kTile);
-    const int64_t total = (int64_t)a.nseg * tpw * a.H;
+    const int64_t total = (int64_t)a.nseg * ((tpw + 1) / 2) * a.H;
     if (total < grid) grid = (int)total;
   }
   if (grid < 1) return cudaSuccess;
