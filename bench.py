@@ -57,7 +57,8 @@ def _peaks():
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "enforced.power.limit")
 
     def __init__(self, device_index: int):
         self.proc = None
@@ -100,7 +101,8 @@ class ClockSampler:
                 if len(parts) < 9:
                     continue
                 try:
-                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+                    lim = float(parts[9]) if len(parts) > 9 else float("nan")
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9], lim))
                 except ValueError:
                     continue
         if not rows:
@@ -110,7 +112,7 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in load for i, v in enumerate(r[3]) if v.lower() == "active"})
         return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": max(r[1] for r in rows),
-                "power_w_max": pmax, "samples": len(load), "reasons": reasons}
+                "power_w_max": pmax, "power_limit_w": rows[-1][4], "samples": len(load), "reasons": reasons}
 
 
 # ----------------------------------------------------------------------------- helpers

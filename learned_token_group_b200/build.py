@@ -46,8 +46,9 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
     tmp = LIB + ".tmp"
+    extra = os.environ.get("MOGA_NVCC_FLAGS", "").split()  # e.g. tuning -D overrides
     cmd = [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
-           "-Xptxas", "-v" if verbose else "-O3", "-I", os.path.join(ROOT, "include"),
+           "-Xptxas", "-v" if verbose else "-O3", "-I", os.path.join(ROOT, "include"), *extra,
            "-o", tmp] + [os.path.join(CSRC, f) for f in SOURCES]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:

@@ -36,7 +36,21 @@ namespace moga {
 
 namespace {
 
-constexpr int kAttnThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-5 / 6-9 softmax of tiles A / B
+// One key pair in every kExp2PolyEvery goes through the FMA-pipe polynomial
+// instead of MUFU ex2 (0 disables), balancing the two units in the softmax.
+#ifndef MOGA_EXP2_POLY_EVERY
+#define MOGA_EXP2_POLY_EVERY 8
+#endif
+constexpr int kExp2PolyEvery = MOGA_EXP2_POLY_EVERY;
+// Warpgroup 0: warp 0 TMA, warp 1 MMA (+ TMEM allocation), warps 2-3 idle;
+// warpgroups 1 and 2: softmax + epilogue of query tiles A and B.
+constexpr int kAttnThreads = 384;
+// Register split after launch (384 threads x 168): warpgroup 0 drops to 104,
+// the softmax warpgroups rise to 192: 128*104 + 256*192 = 62464 <= 64512
+// (multiples of 8; this split compiles without spills).
+constexpr int kRegsCtl = 104;
+constexpr int kRegsSoftmax = 192;
+static_assert(128 * kRegsCtl + 256 * kRegsSoftmax <= kAttnThreads * 168, "register split exceeds the launch");
 constexpr int kStages = 2;
 
 __device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
@@ -279,6 +293,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
   WaitCtx wc{abort_flag, status, wait_ns};
   const int64_t N = a.N;
 
+  if (warp < 4) {
+  regs_dec<kRegsCtl>();
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
@@ -418,9 +434,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       WaitCtx dc{&zero, nullptr, 100000000ull};
       mbar_wait(done_bar, 0, dc);
     }
+  }
   } else {
+    regs_inc<kRegsSoftmax>();
     // ---------------------------------------------------------------- softmax + epilogue
-    const int x = (warp - 2) >> 2;  // warps 2-5: tile A, warps 6-9: tile B
+    const int x = (warp - 4) >> 2;  // warps 4-7: tile A, warps 8-11: tile B
     const int sub = warp & 3;       // TMEM sub-partition this warp may access
     const int row = sub * 32 + lane;
     const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
@@ -434,35 +452,27 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       const bool hb = u.q0 + kTile < u.len;
       if (x == 1 && !hb) continue;
       const int nkv = (u.len + kTile - 1) / kTile;
-      float m_run = -INFINITY, l = 0.f;
+      float m_run = -INFINITY;
+      uint64_t l2 = f2_pack(0.f, 0.f);  // row sum of P, kept as two partial sums
       for (int j = 0; j < nkv; ++j) {
         if (!mbar_wait(&s_full[x], sc & 1, wc)) { ok = false; break; }
         ++sc;
         tc_fence_after();
-        // pass 1: row max of S (raw scores), 32 columns at a time; the next
-        // chunk's TMEM load is in flight while the current one is reduced.
+        // The whole S row (128 fp32) is read from TMEM once.
         const int valid = u.len - j * kTile;  // keys of this tile inside the segment
-        float mx = -INFINITY;
-        // Only the segment's last KV tile has keys to mask (warp-uniform branch).
-        auto row_max = [&](auto masked) {
-          float cur[32], nxt[32];
-          tmem_ld32(tSx, cur);
+        float sr[kTile];
 #pragma unroll
-          for (int c = 0; c < kTile / 32; ++c) {
-            tmem_ld_wait();
-            if (c + 1 < kTile / 32) tmem_ld32(tSx + (c + 1) * 32, nxt);
+        for (int c = 0; c < kTile / 32; ++c) tmem_ld32(tSx + c * 32, sr + c * 32);
+        tmem_ld_wait();
+        if (valid < kTile) {  // only the segment's last KV tile has keys to mask
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              if constexpr (decltype(masked)::value)
-                mx = fmaxf(mx, (c * 32 + e < valid) ? cur[e] : -INFINITY);
-              else
-                mx = fmaxf(mx, cur[e]);
-            }
+          for (int c = 0; c < kTile; ++c)
+            if (c >= valid) sr[c] = -INFINITY;
+        }
+        float mx = fmax3(sr[0], sr[1], sr[2]);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
-          }
-        };
-        if (valid >= kTile) row_max(std::false_type{}); else row_max(std::true_type{});
+        for (int c = 3; c + 1 < kTile; c += 2) mx = fmax3(mx, sr[c], sr[c + 1]);
+        mx = fmaxf(mx, sr[kTile - 1]);
         const float m_new = fmaxf(m_run, mx * scale_log2);
         // O_x was last written by the previous P V product, which completed
         // before this S (the MMA thread issued it first).  The running max is
@@ -477,39 +487,35 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
           rescale = __any_sync(0xffffffffu, need);
           if (need) {
             alpha = fast_exp2(m_run - m_new);
-            l *= alpha;
+            l2 = f2_mul(l2, f2_pack(alpha, alpha));
             m_run = m_new;
           }
         }
-        // pass 2: P = 2^(S*scale - m), summed into l and written back over S
-        // as packed bf16 (two keys per TMEM column).
-        const float nm = -m_run;
-        auto write_p = [&](auto masked) {
-          float cur[32], nxt[32];
-          tmem_ld32(tSx, cur);
+        // P = 2^(S*scale - m), summed into l and written back over S as packed
+        // bf16 (two keys per TMEM column); pairs of keys go through the packed
+        // fp32x2 FMA/ADD units.  Masked keys are -inf, so their P is 0.
+        const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
+        const uint64_t nm2 = f2_pack(-m_run, -m_run);
 #pragma unroll
-          for (int c = 0; c < kTile / 32; ++c) {
-            tmem_ld_wait();
-            if (c + 1 < kTile / 32) tmem_ld32(tSx + (c + 1) * 32, nxt);
-            uint32_t pk[16];
+        for (int c = 0; c < kTile / 32; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float p0 = fast_exp2(fmaf(cur[2 * e], scale_log2, nm));
-              float p1 = fast_exp2(fmaf(cur[2 * e + 1], scale_log2, nm));
-              if constexpr (decltype(masked)::value) {
-                if (c * 32 + 2 * e >= valid) p0 = 0.0f;
-                if (c * 32 + 2 * e + 1 >= valid) p1 = 0.0f;
-              }
-              l += p0 + p1;
-              pk[e] = pack_bf16x2(p0, p1);
+          for (int e = 0; e < 16; ++e) {
+            const uint64_t t2 = f2_fma(f2_pack(sr[c * 32 + 2 * e], sr[c * 32 + 2 * e + 1]), sc2, nm2);
+            float p0, p1;
+            if (kExp2PolyEvery > 0 && e % (kExp2PolyEvery > 0 ? kExp2PolyEvery : 1) == kExp2PolyEvery - 1) {
+              f2_unpack(exp2_poly_x2(t2), p0, p1);
+            } else {
+              float t0, t1;
+              f2_unpack(t2, t0, t1);
+              p0 = fast_exp2(t0);
+              p1 = fast_exp2(t1);
             }
-            // columns [16c, 16c+16) hold S of keys already read into registers
-            tmem_st16u(tSx + c * 16, pk);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
+            l2 = f2_add(l2, f2_pack(p0, p1));
+            pk[e] = pack_bf16x2(p0, p1);
           }
-        };
-        if (valid >= kTile) write_p(std::false_type{}); else write_p(std::true_type{});
+          tmem_st16u(tSx + c * 16, pk);
+        }
         if (rescale) {
 #pragma unroll
           for (int c = 0; c < DH / 32; ++c) {
@@ -540,8 +546,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
           if (status) atomicOr(status, DEV_RANGE);
         }
       }
+      float l_lo, l_hi;
+      f2_unpack(l2, l_lo, l_hi);
       const float gt = (live && a.gate) ? a.gate[src] : 1.0f;
-      const float inv = a.out_scale * gt / l;
+      const float inv = a.out_scale * gt / (l_lo + l_hi);
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) + (src * a.H + u.h) * (int64_t)DH;
 #pragma unroll
       for (int c = 0; c < DH / 32; ++c) {

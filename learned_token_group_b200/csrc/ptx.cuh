@@ -238,9 +238,77 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Packed fp32 pairs (sm_100 f32x2 instructions): one issue slot for two lanes of work.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// Three-input maximum (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^t for a pair of arguments on the FMA pipe (no MUFU): t = n + f with
+// n = round(t) (magic-number rounding) and f in [-1/2, 1/2]; 2^f from a
+// degree-3 polynomial fitted for minimax relative error by Lawson's iteration
+// (coefficients from csrc/exp2_poly.py; relative error <= 7.5e-5); 2^n is
+// applied by adding n to the exponent field.  Arguments below -126 are
+// clamped to -126 so that the exponent field cannot wrap (the result is then
+// below 2^-126, i.e. 0 for bf16 P); -inf (a masked key) gives a tiny positive
+// value, not NaN.
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t t2) {
+  constexpr float kC0 = 0.999928073f, kC1 = 0.693260987f, kC2 = 0.242611135f, kC3 = 0.0551716668f;
+  float t0, t1;
+  f2_unpack(t2, t0, t1);
+  const uint64_t tc = f2_pack(fmaxf(t0, -126.0f), fmaxf(t1, -126.0f));
+  const uint64_t r = f2_add(tc, f2_pack(12582912.0f, 12582912.0f));   // 1.5 * 2^23: round to integer
+  const uint64_t n = f2_add(r, f2_pack(-12582912.0f, -12582912.0f));
+  const uint64_t f = f2_fma(n, f2_pack(-1.0f, -1.0f), tc);
+  uint64_t p = f2_fma(f, f2_pack(kC3, kC3), f2_pack(kC2, kC2));
+  p = f2_fma(p, f, f2_pack(kC1, kC1));
+  p = f2_fma(p, f, f2_pack(kC0, kC0));
+  float p0, p1, r0, r1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(r, r0, r1);
+  const float e0 = __int_as_float(__float_as_int(p0) + (__float_as_int(r0) << 23));
+  const float e1 = __int_as_float(__float_as_int(p1) + (__float_as_int(r1) << 23));
+  return f2_pack(e0, e1);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Warpgroup-wide register reallocation (all 128 threads of the warpgroup).
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
