@@ -66,6 +66,7 @@ def get_lib():
         "moga_kernel_launches": (ctypes.c_uint64, []),
         "moga_route_noalloc": (_I, [_P, _P, _P, _I, _I64, _I, _I, _P, _P, _P, _P, _P, _P]),
         "moga_set_timing_events": (_I, [_I, _P, _P]),
+        "moga_debug_inject": (_I, [_I]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

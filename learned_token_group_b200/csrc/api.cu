@@ -16,6 +16,7 @@ namespace {
 
 std::atomic<uint64_t> g_wait_ns{4000000000ull};
 std::atomic<uint64_t> g_launches{0};
+std::atomic<int> g_debug_inject{0};
 constexpr int kNumStages = 6;
 std::atomic<void*> g_ev_begin[kNumStages];
 std::atomic<void*> g_ev_end[kNumStages];
@@ -208,6 +209,7 @@ moga_status group_attn_body(const DevCtx& c, const void* q, const void* k, const
   a.mode = 0;
   a.table = table;
   a.nseg = M;
+  a.debug_withhold_first_k = g_debug_inject.load(std::memory_order_relaxed) == 1;
   mark(MOGA_STAGE_GROUP_ATTN, true, c.stream);
   const cudaError_t e = launch_attention(c, a);
   mark(MOGA_STAGE_GROUP_ATTN, false, c.stream);
@@ -317,6 +319,12 @@ int moga_version(void) { return (1 << 16) | 0; }
 uint64_t moga_set_wait_limit_ns(uint64_t ns) { return g_wait_ns.exchange(ns ? ns : 1); }
 
 uint64_t moga_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+moga_status moga_debug_inject(int mode) {
+  if (mode < 0 || mode > 1) return MOGA_ERR_INVALID_ARG;
+  g_debug_inject.store(mode, std::memory_order_relaxed);
+  return MOGA_OK;
+}
 
 moga_status moga_set_timing_events(int stage, void* begin, void* end) {
   if (stage < 0 || stage >= kNumStages) return MOGA_ERR_INVALID_ARG;

@@ -323,6 +323,13 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
           const int rowk = (int)((int64_t)u.h * N + u.start + j * kTile);
           const int ks = kc % kStages;
           if (!mbar_wait(&k_empty[ks], ((kc / kStages) & 1) ^ 1, wc)) { ok = false; break; }
+          if (a.debug_withhold_first_k && kc == 0) {
+            // Test hook: this K tile never arrives, so the MMA warp's bounded
+            // wait runs out and the kernel reports a timeout.  No load is in
+            // flight for it, so the slot is not counted for the drain below.
+            ok = false;
+            break;
+          }
           mbar_expect_tx(&k_full[ks], P::kTileBytes);
 #pragma unroll
           for (int c = 0; c < P::kChunks; ++c)

@@ -65,6 +65,7 @@ struct AttnArgs {
   const int32_t* table;   // groups: [3*(M+1)] = tile_prefix | seg_start | seg_len (sorted)
   int nseg;               // groups: M ; windows: number of windows
   int T, Hg, Wg, wt, wh, ww;
+  int debug_withhold_first_k;  // test hook: the producer skips each CTA's first K tile
 };
 cudaError_t launch_attention(const DevCtx& c, const AttnArgs& a);
 

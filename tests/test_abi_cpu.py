@@ -106,6 +106,12 @@ def test_layer_validation(lib):
     assert lib.moga_sync_status(None, None) == INVALID
 
 
+def test_debug_inject_modes(lib):
+    assert lib.moga_debug_inject(2) == INVALID
+    assert lib.moga_debug_inject(-1) == INVALID
+    assert lib.moga_debug_inject(0) == OK
+
+
 def test_wait_limit_roundtrip(lib):
     old = lib.moga_set_wait_limit_ns(123456)
     assert lib.moga_set_wait_limit_ns(old) == 123456
