@@ -308,7 +308,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         if (u.q0 >= u.len) continue;
         const bool hb = u.q0 + kTile < u.len;
         const int nkv = (u.len + kTile - 1) / kTile;
-        if (!mbar_wait(q_empty, (ucnt & 1) ^ 1, wc)) break;
+        if (!mbar_wait(q_empty, (ucnt & 1) ^ 1, wc, 1, ucnt)) break;
         const int rowq = (int)((int64_t)u.h * N + u.start + u.q0);
         mbar_expect_tx(q_full, (hb ? 2 : 1) * P::kTileBytes);
 #pragma unroll
@@ -322,7 +322,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         for (int j = 0; j < nkv; ++j) {
           const int rowk = (int)((int64_t)u.h * N + u.start + j * kTile);
           const int ks = kc % kStages;
-          if (!mbar_wait(&k_empty[ks], ((kc / kStages) & 1) ^ 1, wc)) { ok = false; break; }
+          if (!mbar_wait(&k_empty[ks], ((kc / kStages) & 1) ^ 1, wc, 2, kc)) { ok = false; break; }
           if (a.debug_withhold_first_k && kc == 0) {
             // Test hook: this K tile never arrives, so the MMA warp's bounded
             // wait runs out and the kernel reports a timeout.  No load is in
@@ -336,7 +336,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             tma_load_2d(&tk, &k_full[ks], smem + P::kK0 + ks * P::kTileBytes + c * 16384, c * 64, rowk);
           ++kc;
           const int vs = vc % kStages;
-          if (!mbar_wait(&v_empty[vs], ((vc / kStages) & 1) ^ 1, wc)) { ok = false; break; }
+          if (!mbar_wait(&v_empty[vs], ((vc / kStages) & 1) ^ 1, wc, 3, vc)) { ok = false; break; }
           mbar_expect_tx(&v_full[vs], P::kTileBytes);
 #pragma unroll
           for (int c = 0; c < P::kChunks; ++c)
@@ -384,10 +384,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         if (u.q0 >= u.len) continue;
         const bool hb = u.q0 + kTile < u.len;
         const int nkv = (u.len + kTile - 1) / kTile;
-        if (!mbar_wait(q_full, ucnt & 1, wc)) break;
+        if (!mbar_wait(q_full, ucnt & 1, wc, 4, ucnt)) break;
         ++ucnt;
         int ks = kc % kStages;
-        if (!mbar_wait(&k_full[ks], (kc / kStages) & 1, wc)) break;
+        if (!mbar_wait(&k_full[ks], (kc / kStages) & 1, wc, 5, kc)) break;
         tc_fence_after();
         issue_s(0, ks);
         umma_commit(&s_full[0]);
@@ -401,14 +401,14 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         for (int j = 0; j < nkv; ++j) {
           const int vs = vc % kStages;
           const bool more = j + 1 < nkv;
-          if (!mbar_wait(&v_full[vs], (vc / kStages) & 1, wc)) { ok = false; break; }
-          if (!mbar_wait(&p_full[0], pc0 & 1, wc)) { ok = false; break; }
+          if (!mbar_wait(&v_full[vs], (vc / kStages) & 1, wc, 7, vc)) { ok = false; break; }
+          if (!mbar_wait(&p_full[0], pc0 & 1, wc, 13, pc0)) { ok = false; break; }
           ++pc0;
           tc_fence_after();
           issue_pv(0, vs, j > 0);
           ks = kc % kStages;
           if (more) {
-            if (!mbar_wait(&k_full[ks], (kc / kStages) & 1, wc)) { ok = false; break; }
+            if (!mbar_wait(&k_full[ks], (kc / kStages) & 1, wc, 8, kc)) { ok = false; break; }
             tc_fence_after();
             issue_s(0, ks);
             umma_commit(&s_full[0]);
@@ -416,7 +416,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             umma_commit(&o_full[0]);
           }
           if (hb) {
-            if (!mbar_wait(&p_full[1], pc1 & 1, wc)) { ok = false; break; }
+            if (!mbar_wait(&p_full[1], pc1 & 1, wc, 29, pc1)) { ok = false; break; }
             ++pc1;
             tc_fence_after();
             issue_pv(1, vs, j > 0);
@@ -460,9 +460,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       if (x == 1 && !hb) continue;
       const int nkv = (u.len + kTile - 1) / kTile;
       float m_run = -INFINITY;
-      uint64_t l2 = f2_pack(0.f, 0.f);  // row sum of P, kept as two partial sums
+      uint64_t la = f2_pack(0.f, 0.f), lb = la, lc = la, ld = la;  // row sum of P, 8 partial sums
       for (int j = 0; j < nkv; ++j) {
-        if (!mbar_wait(&s_full[x], sc & 1, wc)) { ok = false; break; }
+        if (!mbar_wait(&s_full[x], sc & 1, wc, 6 + 16 * x, sc)) { ok = false; break; }
         ++sc;
         tc_fence_after();
         // The whole S row (128 fp32) is read from TMEM once.
@@ -476,10 +476,16 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
           for (int c = 0; c < kTile; ++c)
             if (c >= valid) sr[c] = -INFINITY;
         }
-        float mx = fmax3(sr[0], sr[1], sr[2]);
+        // row max as a tree: 8 independent chains of 3-input maxima
+        float m8[8];
 #pragma unroll
-        for (int c = 3; c + 1 < kTile; c += 2) mx = fmax3(mx, sr[c], sr[c + 1]);
-        mx = fmaxf(mx, sr[kTile - 1]);
+        for (int i = 0; i < 8; ++i) {
+          float m = fmax3(sr[16 * i], sr[16 * i + 1], sr[16 * i + 2]);
+#pragma unroll
+          for (int k = 3; k + 1 < 16; k += 2) m = fmax3(m, sr[16 * i + k], sr[16 * i + k + 1]);
+          m8[i] = fmaxf(m, sr[16 * i + 15]);
+        }
+        const float mx = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
         const float m_new = fmaxf(m_run, mx * scale_log2);
         // O_x was last written by the previous P V product, which completed
         // before this S (the MMA thread issued it first).  The running max is
@@ -494,7 +500,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
           rescale = __any_sync(0xffffffffu, need);
           if (need) {
             alpha = fast_exp2(m_run - m_new);
-            l2 = f2_mul(l2, f2_pack(alpha, alpha));
+            const uint64_t a2 = f2_pack(alpha, alpha);
+            la = f2_mul(la, a2);
+            lb = f2_mul(lb, a2);
+            lc = f2_mul(lc, a2);
+            ld = f2_mul(ld, a2);
             m_run = m_new;
           }
         }
@@ -518,7 +528,13 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
               p0 = fast_exp2(t0);
               p1 = fast_exp2(t1);
             }
-            l2 = f2_add(l2, f2_pack(p0, p1));
+            const uint64_t pp = f2_pack(p0, p1);
+            switch (e & 3) {
+              case 0: la = f2_add(la, pp); break;
+              case 1: lb = f2_add(lb, pp); break;
+              case 2: lc = f2_add(lc, pp); break;
+              default: ld = f2_add(ld, pp); break;
+            }
             pk[e] = pack_bf16x2(p0, p1);
           }
           tmem_st16u(tSx + c * 16, pk);
@@ -540,7 +556,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       }
       if (!ok) break;
       // epilogue: wait for the last P V product, normalise, gate, scatter
-      if (!mbar_wait(&o_full[x], oc & 1, wc)) break;
+      if (!mbar_wait(&o_full[x], oc & 1, wc, 9 + 16 * x, oc)) break;
       ++oc;
       tc_fence_after();
       const int r = u.q0 + x * kTile + row;
@@ -554,7 +570,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         }
       }
       float l_lo, l_hi;
-      f2_unpack(l2, l_lo, l_hi);
+      f2_unpack(f2_add(f2_add(la, lb), f2_add(lc, ld)), l_lo, l_hi);
       const float gt = (live && a.gate) ? a.gate[src] : 1.0f;
       const float inv = a.out_scale * gt / (l_lo + l_hi);
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) + (src * a.H + u.h) * (int64_t)DH;

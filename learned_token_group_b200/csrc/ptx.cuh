@@ -59,18 +59,31 @@ struct WaitCtx {
 
 // Wait until the phase with `parity` of `bar` completes. Returns false (and
 // raises the abort flag) if the wait exceeds ctx.limit_ns or another role of
-// this CTA already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& ctx) {
+// this CTA already aborted.  The first wait to time out also records where it
+// gave up in status[1] (site | block << 8) and status[2] (parity | count << 1,
+// count = the caller's progress counter), for diagnosis.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& ctx, int site = 0,
+                                          uint32_t count = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   uint32_t spins = 0;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((++spins & 255u) == 0) {
-      if (*ctx.abort_flag) return false;
+      if (*ctx.abort_flag) {
+        // Where this role stood when the CTA gave up: status[8 + site] keeps
+        // the progress count + 1 of the first block to report that site.
+        if (ctx.status && site > 0 && site < 56) atomicCAS(&ctx.status[8 + site], 0, (int)(count + 1));
+        return false;
+      }
       if (global_timer_ns() - t0 > ctx.limit_ns) {
         *ctx.abort_flag = 1;
-        if (ctx.status) atomicOr(ctx.status, DEV_TIMEOUT);
+        if (ctx.status) {
+          if (atomicOr(ctx.status, DEV_TIMEOUT) == 0) {
+            ctx.status[1] = site | ((int)blockIdx.x << 8);
+            ctx.status[2] = (int)(parity | (count << 1));
+          }
+        }
         return false;
       }
     }
@@ -299,6 +312,13 @@ __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t t2) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Shared-memory atomic add with acquire-release ordering at CTA scope.
+__device__ __forceinline__ int atom_add_acq_rel_cta(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(smem_u32(p)), "r"(v) : "memory");
+  return old;
 }
 
 // Warpgroup-wide register reallocation (all 128 threads of the warpgroup).
