@@ -88,6 +88,20 @@ moga_status moga_route(const void* x, const void* W_r, const float* b_r, moga_dt
                        int M, int32_t* group_id, float* gate, int32_t* perm, int32_t* offsets,
                        int32_t* max_seqlen, void* ws, size_t ws_bytes, void* stream);
 
+/* moga_route_ex: moga_route plus the group-balancing statistics of the pages'
+ * "Group Balancing Loss" section (Eq. 6), in the reading
+ *   F_i = fraction of tokens routed to group i   (= (offsets[i+1]-offsets[i])/N)
+ *   P_i = (1/N) * sum over all tokens x of p(i|x)
+ *   balance = M * sum_i F_i P_i               (1 when balanced and confident)
+ * prob_mean (fp32 [M], device) receives P, balance (fp32 [1], device) the
+ * metric; either may be NULL (both NULL = plain moga_route).  The sums are
+ * taken in a fixed order, so the results are deterministic.
+ * Workspace: moga_route_ex_workspace_size(N, M) bytes. */
+size_t moga_route_ex_workspace_size(int64_t N, int M);
+moga_status moga_route_ex(const void* x, const void* W_r, const float* b_r, moga_dtype dt, int64_t N, int d, int M,
+                          int32_t* group_id, float* gate, int32_t* perm, int32_t* offsets, int32_t* max_seqlen,
+                          float* prob_mean, float* balance, void* ws, size_t ws_bytes, void* stream);
+
 /* moga_route_noalloc: the same routing as moga_route, for callers that cannot
  * allocate device memory themselves (for example code running inside a
  * framework whose allocator owns the GPU, or a pre-recorded launch sequence
@@ -166,6 +180,23 @@ moga_status moga_layer(const void* x, const void* W_r, const float* b_r, moga_dt
                        const void* k, const void* v, int64_t N, int d, int H, int d_h, int M, int T, int Hg,
                        int Wg, const int* window, void* out, int32_t* group_id, float* gate, int32_t* perm,
                        int32_t* offsets, void* ws, size_t ws_bytes, void* stream);
+
+/* moga_layer_ex: the visual block with a choice of branches, as in the pages'
+ * "Spatial-Temporal Group Attention (STGA)" section (each token's output is
+ * the mean of its MoGA group, its STGA window and its per-frame group):
+ *   branches bit 0: the STGA window branch (window required),
+ *   branches bit 1: the per-frame branch, attention among all tokens of each
+ *                   latent frame (window 1 x Hg x Wg),
+ *   out = arithmetic mean of MoGA(x) and the branches that are on.
+ * branches = 1 is moga_layer with a window, branches = 0 is MoGA alone.
+ * Other arguments, outputs and limits as moga_layer; T, Hg, Wg are required
+ * whenever branches != 0.
+ * Workspace: moga_layer_ex_workspace_size(N, H, d_h, M, branches) bytes. */
+size_t moga_layer_ex_workspace_size(int64_t N, int H, int d_h, int M, int branches);
+moga_status moga_layer_ex(const void* x, const void* W_r, const float* b_r, moga_dtype x_dt, const void* q,
+                          const void* k, const void* v, int64_t N, int d, int H, int d_h, int M, int T, int Hg,
+                          int Wg, const int* window, int branches, void* out, int32_t* group_id, float* gate,
+                          int32_t* perm, int32_t* offsets, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------- device status
  * moga_sync_status: synchronises `stream`, reads the device status word kept

@@ -63,6 +63,11 @@ def get_lib():
         "moga_layer": (_I, [_P, _P, _P, _I, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _I, _P,
                             _P, _P, _P, _P, _P, _P, _SZ, _P]),
         "moga_sync_status": (_I, [_P, _P]),
+        "moga_layer_ex_workspace_size": (_SZ, [_I64, _I, _I, _I, _I]),
+        "moga_route_ex_workspace_size": (_SZ, [_I64, _I]),
+        "moga_route_ex": (_I, [_P, _P, _P, _I, _I64, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+        "moga_layer_ex": (_I, [_P, _P, _P, _I, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _I, _P, _I,
+                               _P, _P, _P, _P, _P, _P, _SZ, _P]),
         "moga_kernel_launches": (ctypes.c_uint64, []),
         "moga_route_noalloc": (_I, [_P, _P, _P, _I, _I64, _I, _I, _P, _P, _P, _P, _P, _P]),
         "moga_set_timing_events": (_I, [_I, _P, _P]),
@@ -164,6 +169,32 @@ def route(x: torch.Tensor, W_r: torch.Tensor, b_r: Optional[torch.Tensor], M: in
     return out
 
 
+def route_stats(x: torch.Tensor, W_r: torch.Tensor, b_r: Optional[torch.Tensor], M: int):
+    """moga_route_ex: routing plus balancing statistics.
+
+    Returns dict(group_id, gate, perm, offsets, max_seqlen, prob_mean [M], balance [1]).
+    """
+    lib = get_lib()
+    _dev_tensor(x, "x")
+    _dev_tensor(W_r, "W_r", x.dtype)
+    dt = {torch.float32: MOGA_F32, torch.bfloat16: MOGA_BF16}[x.dtype]
+    N, d = x.shape
+    dev = x.device
+    out = {"group_id": torch.empty(N, dtype=torch.int32, device=dev),
+           "gate": torch.empty(N, dtype=torch.float32, device=dev),
+           "perm": torch.empty(N, dtype=torch.int32, device=dev),
+           "offsets": torch.empty(M + 1, dtype=torch.int32, device=dev),
+           "max_seqlen": torch.empty(1, dtype=torch.int32, device=dev),
+           "prob_mean": torch.empty(M, dtype=torch.float32, device=dev),
+           "balance": torch.empty(1, dtype=torch.float32, device=dev)}
+    ws = workspace(lib.moga_route_ex_workspace_size(N, M), dev)
+    st = lib.moga_route_ex(_ptr(x), _ptr(W_r), _ptr(b_r), dt, N, d, M, _ptr(out["group_id"]), _ptr(out["gate"]),
+                           _ptr(out["perm"]), _ptr(out["offsets"]), _ptr(out["max_seqlen"]), _ptr(out["prob_mean"]),
+                           _ptr(out["balance"]), _ptr(ws), ws.numel(), _stream(dev))
+    _check(st, "moga_route_ex")
+    return out
+
+
 def group_attn(q, k, v, perm, offsets, gate, M: int, out_scale: float = 1.0, out=None, ws=None):
     """moga_group_attn: out[perm[j]] = out_scale * gate * SA within each segment."""
     lib = get_lib()
@@ -208,17 +239,23 @@ def stga_window_attn(q, k, v, grid: Sequence[int], window: Sequence[int], accumu
 
 
 class MogaLayer:
-    """Preallocated outputs + workspace for repeated moga_layer calls."""
+    """Preallocated outputs + workspace for repeated calls of one visual block.
 
-    def __init__(self, N, d, H, d_h, M, grid=None, window=None, x_dtype=torch.bfloat16, device="cuda"):
+    window: STGA window (or None); per_frame: add the per-frame branch (the
+    block output is then the mean of all branches that are on).
+    """
+
+    def __init__(self, N, d, H, d_h, M, grid=None, window=None, x_dtype=torch.bfloat16, device="cuda",
+                 per_frame: bool = False):
         lib = get_lib()
         self.N, self.d, self.H, self.d_h, self.M = N, d, H, d_h, M
         self.grid = tuple(grid) if grid is not None else (0, 0, 0)
         self.window = tuple(window) if window is not None else None
+        self.branches = (1 if self.window else 0) | (2 if per_frame else 0)
         self.x_dt = {torch.float32: MOGA_F32, torch.bfloat16: MOGA_BF16}[x_dtype]
         self.device = torch.device(device)
         self._w3 = _int3(self.window) if self.window else None
-        need = lib.moga_layer_workspace_size(N, H, d_h, M, *self.grid, self._w3)
+        need = lib.moga_layer_ex_workspace_size(N, H, d_h, M, self.branches)
         self.ws = workspace(need, self.device)
         self.out = torch.empty((N, H, d_h), dtype=torch.bfloat16, device=self.device)
         self.group_id = torch.empty(N, dtype=torch.int32, device=self.device)
@@ -228,21 +265,28 @@ class MogaLayer:
 
     def __call__(self, x, W_r, b_r, q, k, v):
         lib = get_lib()
-        st = lib.moga_layer(_ptr(x), _ptr(W_r), _ptr(b_r), self.x_dt, _ptr(q), _ptr(k), _ptr(v), self.N, self.d,
-                            self.H, self.d_h, self.M, *self.grid, self._w3, _ptr(self.out), _ptr(self.group_id),
-                            _ptr(self.gate), _ptr(self.perm), _ptr(self.offsets), _ptr(self.ws), self.ws.numel(),
-                            _stream(self.device))
-        _check(st, "moga_layer")
+        if self.branches & 2:
+            st = lib.moga_layer_ex(_ptr(x), _ptr(W_r), _ptr(b_r), self.x_dt, _ptr(q), _ptr(k), _ptr(v), self.N,
+                                   self.d, self.H, self.d_h, self.M, *self.grid, self._w3, self.branches,
+                                   _ptr(self.out), _ptr(self.group_id), _ptr(self.gate), _ptr(self.perm),
+                                   _ptr(self.offsets), _ptr(self.ws), self.ws.numel(), _stream(self.device))
+            _check(st, "moga_layer_ex")
+        else:
+            st = lib.moga_layer(_ptr(x), _ptr(W_r), _ptr(b_r), self.x_dt, _ptr(q), _ptr(k), _ptr(v), self.N,
+                                self.d, self.H, self.d_h, self.M, *self.grid, self._w3, _ptr(self.out),
+                                _ptr(self.group_id), _ptr(self.gate), _ptr(self.perm), _ptr(self.offsets),
+                                _ptr(self.ws), self.ws.numel(), _stream(self.device))
+            _check(st, "moga_layer")
         return self.out
 
 
-def moga_layer(x, W_r, b_r, q, k, v, M: int, grid=None, window=None):
-    """One MoGA block: returns dict(out, group_id, gate, perm, offsets)."""
+def moga_layer(x, W_r, b_r, q, k, v, M: int, grid=None, window=None, per_frame: bool = False):
+    """One MoGA block: returns dict(out, group_id, gate, perm, offsets, ws)."""
     N, d = x.shape
     _, H, d_h = q.shape
     for n, t in (("x", x), ("q", q), ("k", k), ("v", v)):
         _dev_tensor(t, n)
-    layer = MogaLayer(N, d, H, d_h, M, grid, window, x.dtype, x.device)
+    layer = MogaLayer(N, d, H, d_h, M, grid, window, x.dtype, x.device, per_frame=per_frame)
     layer(x, W_r, b_r, q, k, v)
     return {"out": layer.out, "group_id": layer.group_id, "gate": layer.gate, "perm": layer.perm,
             "offsets": layer.offsets, "ws": layer.ws}

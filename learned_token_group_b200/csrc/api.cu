@@ -96,14 +96,16 @@ struct Carve {
 };
 
 struct RouteWs {
-  size_t hist, base, total;
+  size_t hist, base, pstat, total;
 };
-RouteWs route_ws(int64_t N, int M) {
+// with_stats adds the per-(tile, warp) sums of routing probabilities.
+RouteWs route_ws(int64_t N, int M, bool with_stats = false) {
   Carve c;
   RouteWs w;
   const size_t cells = (size_t)ceil_div(N, kTile) * (size_t)M;
   w.hist = c.take(cells * 4);
   w.base = c.take(cells * 4);
+  w.pstat = with_stats ? c.take(cells * 4 * 4) : 0;
   w.total = c.off;
   return w;
 }
@@ -156,25 +158,30 @@ moga_status check_window(int T, int Hg, int Wg, const int* window, int64_t* N) {
 // ------------------------------------------------------------------ bodies (args already validated)
 moga_status route_body(const DevCtx& c, const void* x, const void* W, const float* b, moga_dtype dt, int64_t N,
                        int d, int M, int32_t* gid, float* gate, int32_t* perm, int32_t* offsets,
-                       int32_t* max_seqlen, uint8_t* ws) {
+                       int32_t* max_seqlen, uint8_t* ws, float* prob_mean = nullptr, float* balance = nullptr) {
+  const bool stats = prob_mean || balance;
   if (N == 0) {
     cudaError_t e = cudaMemsetAsync(offsets, 0, (size_t)(M + 1) * 4, c.stream);
     if (e == cudaSuccess) e = cudaMemsetAsync(max_seqlen, 0, 4, c.stream);
+    if (e == cudaSuccess && prob_mean) e = cudaMemsetAsync(prob_mean, 0, (size_t)M * 4, c.stream);
+    if (e == cudaSuccess && balance) e = cudaMemsetAsync(balance, 0, 4, c.stream);
     return from_cuda(e);
   }
-  const RouteWs w = route_ws(N, M);
+  const RouteWs w = route_ws(N, M, stats);
   int32_t* hist = reinterpret_cast<int32_t*>(ws + w.hist);
   int32_t* base = reinterpret_cast<int32_t*>(ws + w.base);
+  float* pstat = stats ? reinterpret_cast<float*>(ws + w.pstat) : nullptr;
   cudaError_t e;
   mark(MOGA_STAGE_ROUTER, true, c.stream);
   if (dt == MOGA_BF16 && M <= 256 && d >= 64)
-    e = launch_route_tc(c, x, W, b, N, d, M, gid, gate, hist);
+    e = launch_route_tc(c, x, W, b, N, d, M, gid, gate, hist, pstat);
   else
-    e = launch_route_simt(c, x, W, b, dt == MOGA_BF16, N, d, M, gid, gate, hist);
+    e = launch_route_simt(c, x, W, b, dt == MOGA_BF16, N, d, M, gid, gate, hist, pstat);
   mark(MOGA_STAGE_ROUTER, false, c.stream);
   if (e != cudaSuccess) return MOGA_ERR_CUDA;
   mark(MOGA_STAGE_SORT, true, c.stream);
-  if ((e = launch_scan(c, hist, ceil_div(N, kTile), M, base, offsets, max_seqlen)) != cudaSuccess)
+  if ((e = launch_scan(c, hist, ceil_div(N, kTile), M, base, offsets, max_seqlen, pstat, N, prob_mean,
+                       balance)) != cudaSuccess)
     return MOGA_ERR_CUDA;
   if ((e = launch_scatter(c, gid, base, N, M, perm)) != cudaSuccess) return MOGA_ERR_CUDA;
   mark(MOGA_STAGE_SORT, false, c.stream);
@@ -217,8 +224,10 @@ moga_status group_attn_body(const DevCtx& c, const void* q, const void* k, const
   return from_cuda(e);
 }
 
+// accumulate == 0: out = STGA; otherwise out += add_scale * STGA.
 moga_status stga_body(const DevCtx& c, const void* q, const void* k, const void* v, int T, int Hg, int Wg,
-                      const int* window, int H, int d_h, int accumulate, void* out, uint8_t* ws) {
+                      const int* window, int H, int d_h, int accumulate, void* out, uint8_t* ws,
+                      float add_scale = 0.5f) {
   const int64_t N = (int64_t)T * Hg * Wg;
   const AttnWs w = attn_ws(N, H, d_h, 0, true);
   int32_t* permw = reinterpret_cast<int32_t*>(ws + w.permw);
@@ -238,7 +247,7 @@ moga_status stga_body(const DevCtx& c, const void* q, const void* k, const void*
   a.N = N;
   a.H = H;
   a.d_h = d_h;
-  a.out_scale = accumulate ? 0.5f : 1.0f;
+  a.out_scale = accumulate ? add_scale : 1.0f;
   a.accumulate = accumulate ? 1 : 0;
   a.mode = 1;
   a.table = nullptr;
@@ -351,6 +360,26 @@ moga_status moga_route(const void* x, const void* W_r, const float* b_r, moga_dt
   return route_body(c, x, W_r, b_r, dt, N, d, M, group_id, gate, perm, offsets, max_seqlen, (uint8_t*)ws);
 }
 
+size_t moga_route_ex_workspace_size(int64_t N, int M) {
+  if (N < 0 || M < 1) return 0;
+  return route_ws(N, M, true).total;
+}
+
+moga_status moga_route_ex(const void* x, const void* W_r, const float* b_r, moga_dtype dt, int64_t N, int d, int M,
+                          int32_t* group_id, float* gate, int32_t* perm, int32_t* offsets, int32_t* max_seqlen,
+                          float* prob_mean, float* balance, void* ws, size_t ws_bytes, void* stream) {
+  moga_status st = check_route_args(x, W_r, b_r, dt, N, d, M, group_id, gate, perm, offsets, max_seqlen);
+  if (st != MOGA_OK) return st;
+  if ((prob_mean && !aligned4(prob_mean)) || (balance && !aligned4(balance))) return MOGA_ERR_INVALID_ARG;
+  if (!ws || !aligned16(ws)) return MOGA_ERR_INVALID_ARG;
+  const bool stats = prob_mean || balance;
+  if (ws_bytes < route_ws(N, M, stats).total) return MOGA_ERR_WORKSPACE;
+  DevCtx c;
+  if (!make_ctx(&c, ws, stream)) return MOGA_ERR_CUDA;
+  return route_body(c, x, W_r, b_r, dt, N, d, M, group_id, gate, perm, offsets, max_seqlen, (uint8_t*)ws,
+                    prob_mean, balance);
+}
+
 moga_status moga_route_noalloc(const void* x, const void* W_r, const float* b_r, moga_dtype dt, int64_t N, int d,
                                int M, int32_t* group_id, float* gate, int32_t* perm, int32_t* offsets,
                                int32_t* max_seqlen, void* stream) {
@@ -448,6 +477,58 @@ moga_status moga_layer(const void* x, const void* W_r, const float* b_r, moga_dt
   const float scale = window ? 0.5f : 1.0f;
   if ((st = group_attn_body(c, q, k, v, perm, offsets, gate, N, H, d_h, M, scale, out, w)) != MOGA_OK) return st;
   if (window) return stga_body(c, q, k, v, T, Hg, Wg, window, H, d_h, 1, out, w);
+  return MOGA_OK;
+}
+
+size_t moga_layer_ex_workspace_size(int64_t N, int H, int d_h, int M, int branches) {
+  if (N < 0 || H < 1 || M < 1 || branches < 0 || branches > 3) return 0;
+  size_t need = route_ws(N, M).total;
+  const size_t ga = attn_ws(N, H, d_h, M, false).total;
+  if (ga > need) need = ga;
+  if (branches) {
+    const size_t sw = attn_ws(N, H, d_h, 0, true).total;
+    if (sw > need) need = sw;
+  }
+  return need;
+}
+
+moga_status moga_layer_ex(const void* x, const void* W_r, const float* b_r, moga_dtype x_dt, const void* q,
+                          const void* k, const void* v, int64_t N, int d, int H, int d_h, int M, int T, int Hg,
+                          int Wg, const int* window, int branches, void* out, int32_t* group_id, float* gate,
+                          int32_t* perm, int32_t* offsets, void* ws, size_t ws_bytes, void* stream) {
+  if (branches < 0 || branches > 3) return MOGA_ERR_INVALID_ARG;
+  moga_status st = check_route_args(x, W_r, b_r, x_dt, N, d, M, group_id, gate, perm, offsets, offsets);
+  if (st != MOGA_OK) return st;
+  if ((st = check_qkv(q, k, v, out)) != MOGA_OK) return st;
+  if ((st = check_attn_shape(N, H, d_h)) != MOGA_OK) return st;
+  const int frame_window[3] = {1, Hg, Wg};
+  if (branches & 1) {
+    int64_t n = 0;
+    if ((st = check_window(T, Hg, Wg, window, &n)) != MOGA_OK) return st;
+    if (n != N) return MOGA_ERR_INVALID_ARG;
+  }
+  if (branches & 2) {
+    int64_t n = 0;
+    if ((st = check_window(T, Hg, Wg, frame_window, &n)) != MOGA_OK) return st;
+    if (n != N) return MOGA_ERR_INVALID_ARG;
+  }
+  if (!ws || !aligned16(ws)) return MOGA_ERR_INVALID_ARG;
+  if (ws_bytes < moga_layer_ex_workspace_size(N, H, d_h, M, branches)) return MOGA_ERR_WORKSPACE;
+  DevCtx c;
+  if (!make_ctx(&c, ws, stream)) return MOGA_ERR_CUDA;
+  uint8_t* w = (uint8_t*)ws;
+  int32_t* max_seqlen = reinterpret_cast<int32_t*>(w + 16);
+  if ((st = route_body(c, x, W_r, b_r, x_dt, N, d, M, group_id, gate, perm, offsets, max_seqlen, w)) != MOGA_OK)
+    return st;
+  if (N == 0) return MOGA_OK;
+  // out = mean of the branches that are on: each adds 1/nb of its output.
+  const int nb = 1 + (branches & 1) + ((branches >> 1) & 1);
+  const float scale = 1.0f / (float)nb;
+  if ((st = group_attn_body(c, q, k, v, perm, offsets, gate, N, H, d_h, M, scale, out, w)) != MOGA_OK) return st;
+  if ((branches & 1) && (st = stga_body(c, q, k, v, T, Hg, Wg, window, H, d_h, 1, out, w, scale)) != MOGA_OK)
+    return st;
+  if ((branches & 2) && (st = stga_body(c, q, k, v, T, Hg, Wg, frame_window, H, d_h, 1, out, w, scale)) != MOGA_OK)
+    return st;
   return MOGA_OK;
 }
 

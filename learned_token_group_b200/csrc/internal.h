@@ -28,13 +28,16 @@ struct DevCtx {
 
 // ------------------------------------------------------------------ routing
 // Router logits + softmax gate + argmax + per-tile group histogram.
+// pstat (nullable): per (tile, warp) sums of p(i|x) over the warp's tokens, [tiles][4][M].
 cudaError_t launch_route_tc(const DevCtx& c, const void* x, const void* W, const float* b, int64_t N, int d,
-                            int M, int32_t* group_id, float* gate, int32_t* hist);
+                            int M, int32_t* group_id, float* gate, int32_t* hist, float* pstat);
 cudaError_t launch_route_simt(const DevCtx& c, const void* x, const void* W, const float* b, bool bf16,
-                              int64_t N, int d, int M, int32_t* group_id, float* gate, int32_t* hist);
-// Exclusive scan of the per-tile histograms -> offsets, max_seqlen, per-tile bases.
+                              int64_t N, int d, int M, int32_t* group_id, float* gate, int32_t* hist, float* pstat);
+// Exclusive scan of the per-tile histograms -> offsets, max_seqlen, per-tile
+// bases; with pstat also the mean routing probabilities and the balance metric.
 cudaError_t launch_scan(const DevCtx& c, const int32_t* hist, int64_t ntiles, int M, int32_t* base,
-                        int32_t* offsets, int32_t* max_seqlen);
+                        int32_t* offsets, int32_t* max_seqlen, const float* pstat, int64_t N, float* prob_mean,
+                        float* balance);
 // Stable scatter of token indices into perm.
 cudaError_t launch_scatter(const DevCtx& c, const int32_t* group_id, const int32_t* base, int64_t N, int M,
                            int32_t* perm);

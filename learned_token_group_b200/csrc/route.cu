@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
 route_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                 const float* __restrict__ bias, int N, int d, int M, int mpad, int stages, int stage_bytes,
                 int32_t* __restrict__ group_id, float* __restrict__ gate, int32_t* __restrict__ hist,
-                int* status, unsigned long long wait_ns) {
+                float* __restrict__ pstat, int* status, unsigned long long wait_ns) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -188,9 +188,27 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
           if (col < M) online_softmax_step(v[j] + (bias ? __ldg(bias + col) : 0.f), col, mx, arg, sum);
         }
       }
+      const int64_t tok = (int64_t)t * kTile + row;
+      if (pstat) {
+        // Balancing statistics: this warp's sum over its 32 tokens of
+        // p(i|x) for every group i (butterfly reduction, fixed order).
+        const float inv = 1.0f / sum;
+        for (int c0 = 0; c0 < mpad; c0 += 16) {
+          float v[16];
+          tmem_ld16(base + c0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int col = c0 + j;
+            float pj = (col < M && tok < N) ? expf(v[j] + (bias ? __ldg(bias + col) : 0.f) - mx) * inv : 0.f;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) pj += __shfl_xor_sync(0xffffffffu, pj, o);
+            if (lane == 0 && col < M) pstat[((int64_t)t * 4 + sub) * M + col] = pj;
+          }
+        }
+      }
       tc_fence_before();
       mbar_arrive(&acc_empty[ab]);
-      const int64_t tok = (int64_t)t * kTile + row;
       if (tok < N) {
         group_id[tok] = arg;
         gate[tok] = 1.0f / sum;
@@ -218,12 +236,15 @@ __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return _
 template <typename T>
 __global__ void __launch_bounds__(128)
 route_simt_kernel(const T* __restrict__ x, const T* __restrict__ W, const float* __restrict__ bias, int N, int d,
-                  int M, int32_t* __restrict__ group_id, float* __restrict__ gate, int32_t* __restrict__ hist) {
+                  int M, int32_t* __restrict__ group_id, float* __restrict__ gate, int32_t* __restrict__ hist,
+                  float* __restrict__ pstat) {
   extern __shared__ float logit_s[];          // [4][M]
   int* hist_s = reinterpret_cast<int*>(logit_s + 4 * M);  // [M]
+  float* ps = logit_s + 5 * M;                           // [4][M] per-warp sums of p(i|x)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x;
   for (int m = threadIdx.x; m < M; m += blockDim.x) hist_s[m] = 0;
+  for (int m = threadIdx.x; m < 4 * M; m += blockDim.x) ps[m] = 0.f;
   __syncthreads();
   float* lg = logit_s + warp * M;
   for (int r = warp; r < kTile; r += 4) {
@@ -246,19 +267,26 @@ route_simt_kernel(const T* __restrict__ x, const T* __restrict__ W, const float*
       group_id[tok] = arg;
       gate[tok] = 1.0f / sum;
       atomicAdd(&hist_s[arg], 1);
+      if (pstat)
+        for (int m = 0; m < M; ++m) ps[warp * M + m] += expf(lg[m] - mx) / sum;
     }
     __syncwarp();
   }
   __syncthreads();
   for (int m = threadIdx.x; m < M; m += blockDim.x) hist[(int64_t)t * M + m] = hist_s[m];
+  if (pstat)
+    for (int m = threadIdx.x; m < 4 * M; m += blockDim.x) pstat[(int64_t)t * 4 * M + m] = ps[m];
 }
 
 // One CTA: column sums of hist per group in C chunks, exclusive scans, bases.
 __global__ void __launch_bounds__(1024)
 scan_kernel(const int32_t* __restrict__ hist, int ntiles, int M, int32_t* __restrict__ base,
-            int32_t* __restrict__ offsets, int32_t* __restrict__ max_seqlen) {
+            int32_t* __restrict__ offsets, int32_t* __restrict__ max_seqlen, const float* __restrict__ pstat,
+            int N, float* __restrict__ prob_mean, float* __restrict__ balance) {
   __shared__ int part[1024];
   __shared__ int offs_s[1025];
+  __shared__ float fpart[1024];
+  __shared__ float pm_s[1024];
   const int C = max(1, 1024 / M);
   const int tid = threadIdx.x;
   const int per = (ntiles + C - 1) / C;
@@ -269,8 +297,22 @@ scan_kernel(const int32_t* __restrict__ hist, int ntiles, int M, int32_t* __rest
     int s = 0;
     for (int t = t0; t < t1; ++t) s += hist[(int64_t)t * M + g];
     part[c * M + g] = s;
+    if (pstat) {
+      // mean routing probability: per-tile, per-warp partials summed in a
+      // fixed order (tile, then warp), so the result is deterministic
+      float f = 0.f;
+      for (int t = t0; t < t1; ++t)
+        for (int w = 0; w < 4; ++w) f += pstat[((int64_t)t * 4 + w) * M + g];
+      fpart[c * M + g] = f;
+    }
   }
   __syncthreads();
+  if (pstat && tid < M) {
+    float f = 0.f;
+    for (int cc = 0; cc < C; ++cc) f += fpart[cc * M + tid];
+    pm_s[tid] = f / (float)N;
+    if (prob_mean) prob_mean[tid] = pm_s[tid];
+  }
   if (tid < M) {
     int run = 0;
     for (int cc = 0; cc < C; ++cc) {
@@ -293,6 +335,12 @@ scan_kernel(const int32_t* __restrict__ hist, int ntiles, int M, int32_t* __rest
     offs_s[M] = run;
     offsets[M] = run;
     *max_seqlen = mx;
+    if (pstat && balance) {
+      // M * sum_i F_i P_i with F_i the fraction of tokens routed to group i
+      float b = 0.f;
+      for (int m = 0; m < M; ++m) b += ((float)(offs_s[m + 1] - offs_s[m]) / (float)N) * pm_s[m];
+      *balance = (float)M * b;
+    }
   }
   __syncthreads();
   if (active) {
@@ -331,7 +379,7 @@ scatter_kernel(const int32_t* __restrict__ group_id, const int32_t* __restrict__
 }  // namespace
 
 cudaError_t launch_route_tc(const DevCtx& c, const void* x, const void* W, const float* b, int64_t N, int d,
-                            int M, int32_t* group_id, float* gate, int32_t* hist) {
+                            int M, int32_t* group_id, float* gate, int32_t* hist, float* pstat) {
   const RouteSmemPlan p = route_plan(M);
   if (p.mpad > kRouteMaxMPad) return cudaErrorInvalidValue;
   CUtensorMap mx, mw;
@@ -345,34 +393,36 @@ cudaError_t launch_route_tc(const DevCtx& c, const void* x, const void* W, const
   if (e != cudaSuccess) return e;
   const int grid = (int)(ntiles < c.num_sms ? ntiles : c.num_sms);
   route_tc_kernel<<<grid, kRouteThreads, p.total, c.stream>>>(mx, mw, b, (int)N, d, M, p.mpad, p.stages,
-                                                               p.stage_bytes, group_id, gate, hist, c.status,
+                                                               p.stage_bytes, group_id, gate, hist, pstat, c.status,
                                                                (unsigned long long)c.wait_ns);
   return cudaGetLastError();
 }
 
 cudaError_t launch_route_simt(const DevCtx& c, const void* x, const void* W, const float* b, bool bf16,
-                              int64_t N, int d, int M, int32_t* group_id, float* gate, int32_t* hist) {
+                              int64_t N, int d, int M, int32_t* group_id, float* gate, int32_t* hist, float* pstat) {
   const int64_t ntiles = ceil_div(N, kTile);
-  const size_t smem = (size_t)5 * M * sizeof(float);
+  const size_t smem = (size_t)9 * M * sizeof(float);
   if (bf16) {
     auto k = route_simt_kernel<__nv_bfloat16>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<(unsigned)ntiles, 128, smem, c.stream>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)W, b, (int)N, d,
-                                                  M, group_id, gate, hist);
+                                                  M, group_id, gate, hist, pstat);
   } else {
     auto k = route_simt_kernel<float>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<(unsigned)ntiles, 128, smem, c.stream>>>((const float*)x, (const float*)W, b, (int)N, d, M, group_id,
-                                                  gate, hist);
+                                                  gate, hist, pstat);
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_scan(const DevCtx& c, const int32_t* hist, int64_t ntiles, int M, int32_t* base,
-                        int32_t* offsets, int32_t* max_seqlen) {
-  scan_kernel<<<1, 1024, 0, c.stream>>>(hist, (int)ntiles, M, base, offsets, max_seqlen);
+                        int32_t* offsets, int32_t* max_seqlen, const float* pstat, int64_t N, float* prob_mean,
+                        float* balance) {
+  scan_kernel<<<1, 1024, 0, c.stream>>>(hist, (int)ntiles, M, base, offsets, max_seqlen, pstat, (int)N, prob_mean,
+                                        balance);
   return cudaGetLastError();
 }
 

@@ -32,7 +32,9 @@ Readings where the pages leave a step open (each one is pinned by a test):
   sorted position j (the inverse of the pages' original-to-permuted index).
 * STGA windows: non-overlapping boxes of (wt, wh, ww) tokens anchored at the
   grid origin, clipped at the grid edges; token index (t*Hg + h)*Wg + w.
-* combine: out = (MoGA + STGA) / 2 when STGA is on, MoGA alone otherwise.
+* combine: out = (MoGA + STGA) / 2 when STGA is on, MoGA alone otherwise; with
+  the per-frame branch (attention inside each latent frame) the block output
+  is the plain mean of all branches that are on.
 
 Every function here is pinned by ``tests/test_oracle_pins.py`` to something
 other than itself (closed forms, a library attention routine, numpy's stable
@@ -46,8 +48,8 @@ from typing import Iterable, List, Optional, Sequence, Tuple
 import numpy as np
 
 __all__ = [
-    "route", "counting_sort", "attention_rows", "group_attention",
-    "stga_windows", "stga_attention", "moga_layer",
+    "route", "balance_stats", "counting_sort", "attention_rows", "group_attention",
+    "stga_windows", "stga_attention", "frame_attention", "moga_layer",
 ]
 
 _ROW_BLOCK = 16384
@@ -93,6 +95,31 @@ def route(x, W_r, b_r=None) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
             top2 = np.sort(r, axis=1)[:, -2:]
             margin[r0:r1] = top2[:, 1] - top2[:, 0]
     return gid, gate, margin
+
+
+def balance_stats(x, W_r, b_r=None):
+    """Group-balancing statistics ("Group Balancing Loss", Eq. 6).
+
+    Reading taken (the pages' P_i definition and their limiting values
+    disagree): F_i = fraction of tokens whose argmax group is i, P_i = mean of
+    p(i|x) over ALL tokens, metric = M * sum_i F_i * P_i (1 when balanced and
+    confident, M when collapsed onto one group).  Returns (F, P, metric).
+    """
+    W = _f64(W_r)
+    M = W.shape[0]
+    b = np.zeros(M) if b_r is None else _f64(b_r)
+    N = x.shape[0]
+    counts = np.zeros(M)
+    psum = np.zeros(M)
+    for r0 in range(0, N, _ROW_BLOCK):
+        r = _f64(x[r0:r0 + _ROW_BLOCK]) @ W.T + b
+        e = np.exp(r - r.max(axis=1, keepdims=True))
+        p = e / e.sum(axis=1, keepdims=True)
+        psum += p.sum(axis=0)
+        counts += np.bincount(np.argmax(r, axis=1), minlength=M)
+    F = counts / N
+    P = psum / N
+    return F, P, float(M * np.sum(F * P))
 
 
 def counting_sort(group_id, M: int) -> Tuple[np.ndarray, np.ndarray, int]:
@@ -218,22 +245,34 @@ def stga_attention(q, k, v, T: int, Hg: int, Wg: int, window,
     return _attend_sets(q, k, v, stga_windows(T, Hg, Wg, window), row_pos, hs, None, out)
 
 
+def frame_attention(q, k, v, T: int, Hg: int, Wg: int, rows=None, heads=None) -> np.ndarray:
+    """Per-frame branch: full attention among the tokens of each latent frame
+    (the STGA definition with a window of one whole frame)."""
+    return stga_attention(q, k, v, T, Hg, Wg, (1, Hg, Wg), rows=rows, heads=heads)
+
+
 def moga_layer(x, W_r, b_r, q, k, v, M: int, grid=None, window=None,
-               rows=None, heads=None):
-    """One visual attention block: route, group attention, optional STGA, mean.
+               rows=None, heads=None, per_frame: bool = False):
+    """One visual attention block: route, group attention, optional STGA and
+    per-frame branches, and the arithmetic mean of the branches that are on.
 
     Returns a dict with group_id, gate, margin, perm, offsets, max_seqlen,
-    moga (Eq. 5 output), stga (or None) and out (the block output).
+    moga (Eq. 5 output), stga / frame (or None) and out (the block output).
     """
     gid, gate, margin = route(x, W_r, b_r)
     perm, offsets, max_seqlen = counting_sort(gid, M)
     moga = group_attention(q, k, v, gid, gate, M, rows=rows, heads=heads)
-    stga = None
-    out = moga
+    branches = [moga]
+    stga = frame = None
     if window is not None:
         T, Hg, Wg = grid
         stga = stga_attention(q, k, v, T, Hg, Wg, window, rows=rows, heads=heads)
-        out = 0.5 * (moga + stga)
+        branches.append(stga)
+    if per_frame:
+        T, Hg, Wg = grid
+        frame = frame_attention(q, k, v, T, Hg, Wg, rows=rows, heads=heads)
+        branches.append(frame)
+    out = branches[0] if len(branches) == 1 else sum(branches) / len(branches)
     return {"group_id": gid, "gate": gate, "margin": margin, "perm": perm,
             "offsets": offsets, "max_seqlen": max_seqlen, "moga": moga,
-            "stga": stga, "out": out}
+            "stga": stga, "frame": frame, "out": out}

@@ -112,6 +112,33 @@ def test_debug_inject_modes(lib):
     assert lib.moga_debug_inject(0) == OK
 
 
+def test_layer_ex_validation(lib):
+    w = (ctypes.c_int * 3)(3, 8, 8)
+    f = lib.moga_layer_ex
+    args = [P, P, None, 1, P, P, P, 384, 256, 2, 128, 4, 3, 8, 16, w, 3, P, P, P, P, P, P, BIG, None]
+    bad = list(args)
+    bad[16] = 4                                       # unknown branch bit
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[15] = None                                    # STGA branch without a window
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[13], bad[16] = 9, 2                           # per-frame branch: grid must cover N
+    assert f(*bad) == INVALID
+    small = list(args)
+    small[23] = 4096
+    assert f(*small) == WORKSPACE
+    assert lib.moga_layer_ex_workspace_size(384, 2, 128, 4, 2) >= lib.moga_layer_ex_workspace_size(384, 2, 128, 4, 0)
+    assert lib.moga_layer_ex_workspace_size(384, 2, 128, 4, 5) == 0
+
+
+def test_route_ex_validation(lib):
+    f = lib.moga_route_ex
+    assert f(P, P, None, 1, 1000, 64, 4, P, P, P, P, P, P + 2, None, P, BIG, None) == INVALID  # misaligned
+    assert f(P, P, None, 1, 1000, 64, 4, P, P, P, P, P, P, P, P, 256, None) == WORKSPACE
+    assert lib.moga_route_ex_workspace_size(1000, 4) > lib.moga_route_workspace_size(1000, 4)
+
+
 def test_wait_limit_roundtrip(lib):
     old = lib.moga_set_wait_limit_ns(123456)
     assert lib.moga_set_wait_limit_ns(old) == 123456

@@ -103,3 +103,43 @@ def test_layer_bitwise_deterministic(name):
         outs.append((layer.out.clone(), layer.perm.clone(), layer.gate.clone()))
     for a, b in zip(*outs):
         assert torch.equal(a, b)
+
+
+THREE = [
+    custom(384, H=2, d_h=128, d=256, M=4, x_kind="clustered", grid=(3, 8, 16), window=(3, 8, 8), name="small3"),
+    custom(2 * 30 * 52, H=1, d_h=64, d=128, M=6, x_kind="clustered", grid=(2, 30, 52), window=(3, 8, 8),
+           name="frame_grid3"),
+]
+
+
+@pytest.mark.parametrize("wl", THREE, ids=[w.name for w in THREE])
+def test_layer_three_branches(wl):
+    """MoGA + STGA + per-frame attention, averaged (moga_layer_ex, branches = 3)."""
+    inp = make_inputs(wl, seed=2, device="cuda")
+    res = moga.moga_layer(inp["x"], inp["W_r"], inp["b_r"], inp["q"], inp["k"], inp["v"], wl.M, wl.grid,
+                          wl.window, per_frame=True)
+    moga.sync_status(res["ws"])
+    gid, _ = check_route(res, inp["x"], inp["W_r"], inp["b_r"], wl.M, GATE_TOL_BF16)
+    gate = np_cpu(res["gate"]).astype(np.float64)
+    q, k, v = (np_cpu(inp[n]) for n in "qkv")
+    ref = (oracle.group_attention(q, k, v, gid, gate, wl.M) + oracle.stga_attention(q, k, v, *wl.grid, wl.window)
+           + oracle.frame_attention(q, k, v, *wl.grid)) / 3
+    compare_out(res["out"], ref, groups=gid)
+
+
+def test_layer_three_branches_wan_sampled():
+    wl = WORKLOADS["wan_32k"]
+    inp = make_inputs(wl, seed=3, device="cuda")
+    res = moga.moga_layer(inp["x"], inp["W_r"], inp["b_r"], inp["q"], inp["k"], inp["v"], wl.M, wl.grid,
+                          wl.window, per_frame=True)
+    moga.sync_status(res["ws"])
+    gid, _ = check_route(res, inp["x"], inp["W_r"], inp["b_r"], wl.M, GATE_TOL_BF16)
+    rows = _sample_rows(gid, wl.M, wl.grid, wl.window, np.random.default_rng(5), per_group=24)
+    heads = [0, wl.H - 1]
+    gate = np_cpu(res["gate"]).astype(np.float64)
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    ref = (oracle.group_attention(q, k, v, gid, gate, wl.M, rows=rows, heads=heads)
+           + oracle.stga_attention(q, k, v, *wl.grid, wl.window, rows=rows, heads=heads)
+           + oracle.frame_attention(q, k, v, *wl.grid, rows=rows, heads=heads)) / 3
+    out = res["out"][torch.from_numpy(rows).cuda()][:, heads]
+    compare_out(out, ref, groups=gid[rows])

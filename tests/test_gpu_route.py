@@ -69,3 +69,26 @@ def test_route_workload(name):
     if name == "skew_187k":
         assert (counts[56:] == 0).all()
         assert sorted(counts[48:56].tolist()) == [1, 2, 3, 5, 8, 13, 21, 34]
+
+
+@pytest.mark.parametrize("name", ["tiny", "wan_32k", "skew_187k"])
+def test_route_balance_stats(name):
+    """moga_route_ex: routing identical to moga_route, plus P_i and the balance
+    metric against the oracle, bitwise repeatable."""
+    import oracle
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl, seed=0, device="cuda", with_qkv=False)
+    res = moga.route_stats(inp["x"], inp["W_r"], inp["b_r"], wl.M)
+    ref = moga.route(inp["x"], inp["W_r"], inp["b_r"], wl.M)
+    again = moga.route_stats(inp["x"], inp["W_r"], inp["b_r"], wl.M)
+    torch.cuda.synchronize()
+    for key in ("group_id", "perm", "offsets", "gate"):
+        assert np.array_equal(np_cpu(res[key]), np_cpu(ref[key]))
+    F, P, b = oracle.balance_stats(np_cpu(inp["x"]), np_cpu(inp["W_r"]),
+                                   None if inp["b_r"] is None else np_cpu(inp["b_r"]))
+    pm = np_cpu(res["prob_mean"]).astype(np.float64)
+    assert np.abs(pm - P).max() <= 1e-5, np.abs(pm - P).max()
+    assert abs(float(np_cpu(res["balance"])[0]) - b) <= 1e-4 * max(1.0, b)
+    assert np.array_equal(np_cpu(again["prob_mean"]), np_cpu(res["prob_mean"]))
+    assert np.array_equal(np_cpu(again["balance"]), np_cpu(res["balance"]))
+    print(f"{name}: balance metric {b:.4f} (GPU {float(np_cpu(res['balance'])[0]):.4f})")

@@ -294,10 +294,60 @@ def check_golden(o):
     assert np.allclose(out[:, 0, 0], s["expect"]["stga"], rtol=0, atol=1e-14)
 
 
+def check_three_branch_mean(o):
+    rng = np.random.default_rng(11)
+    # brute force: frames are windows (1, Hg, Wg); the block output is the mean of three branches
+    grid, N = (3, 3, 4), 36
+    x = rng.normal(size=(N, 5))
+    W = rng.normal(size=(3, 5))
+    q, k, v = (rng.normal(size=(N, 2, 4)) for _ in range(3))
+    res = o.moga_layer(x, W, None, q, k, v, 3, grid=grid, window=(2, 2, 2), per_frame=True)
+    g0, p0 = _brute_route(x.tolist(), W.tolist(), None)
+    ref = (_brute_masked_dense(q, k, v, g0, p0) + _brute_stga(q, k, v, grid, (2, 2, 2))
+           + _brute_stga(q, k, v, grid, (1, 3, 4))) / 3
+    assert np.allclose(res["out"], ref, rtol=0, atol=1e-12)
+    # one frame, M = 1, whole-grid window: every branch is full attention
+    grid1 = (1, 4, 5)
+    q1, k1, v1 = (rng.normal(size=(20, 2, 8)) for _ in range(3))
+    res = o.moga_layer(rng.normal(size=(20, 3)), rng.normal(size=(1, 3)), None, q1, k1, v1, 1,
+                       grid=grid1, window=grid1, per_frame=True)
+    assert np.allclose(res["out"], _sdpa(q1, k1, v1), rtol=0, atol=1e-12)
+
+
+def check_balance_stats(o):
+    M = 4
+    # W = 0: every p(i|x) = 1/M, all tokens tie into group 0 -> F = e_0, P = 1/M, metric 1
+    F, P, b = o.balance_stats(np.ones((10, 3)), np.zeros((M, 3)))
+    assert np.allclose(F, [1, 0, 0, 0]) and np.allclose(P, 0.25) and abs(b - 1.0) < 1e-15
+    # confident and balanced: x = 60 e_{i mod M}, W = I -> F = P = 1/M, metric -> 1
+    x = np.zeros((8 * M, M))
+    x[np.arange(8 * M), np.arange(8 * M) % M] = 60.0
+    F, P, b = o.balance_stats(x, np.eye(M))
+    assert np.allclose(F, 1 / M) and np.allclose(P, 1 / M, atol=1e-20) and abs(b - 1.0) < 1e-12
+    # collapsed and confident: everything in group 2 -> metric -> M
+    x = np.zeros((12, M))
+    x[:, 2] = 60.0
+    F, P, b = o.balance_stats(x, np.eye(M))
+    assert abs(b - M) < 1e-12
+    # brute force on a random case
+    rng = np.random.default_rng(12)
+    x, W, bias = rng.normal(size=(15, 6)), rng.normal(size=(3, 6)), rng.normal(size=3)
+    g0, _ = _brute_route(x.tolist(), W.tolist(), bias.tolist())
+    p_all = []
+    for i in range(15):
+        r = [sum(x[i, c] * W[m, c] for c in range(6)) + bias[m] for m in range(3)]
+        z = sum(math.exp(v - max(r)) for v in r)
+        p_all.append([math.exp(v - max(r)) / z for v in r])
+    Fb = np.bincount(g0, minlength=3) / 15
+    Pb = np.mean(p_all, axis=0)
+    F, P, b = o.balance_stats(x, W, bias)
+    assert np.allclose(F, Fb) and np.allclose(P, Pb, atol=1e-14) and abs(b - 3 * np.sum(Fb * Pb)) < 1e-13
+
+
 CHECKS = [check_route_closed_form, check_route_ties_and_M1, check_route_brute, check_counting_sort,
           check_full_attention_when_M1, check_group_equals_subset_attention, check_special_cases,
           check_brute_force_tiny, check_permutation_equivariance, check_stga, check_layer_combine,
-          check_golden]
+          check_golden, check_three_branch_mean, check_balance_stats]
 
 
 @pytest.mark.parametrize("check", CHECKS, ids=[c.__name__ for c in CHECKS])
