@@ -237,6 +237,15 @@ def run_reference(args, wl, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(value: float, dist, device=None) -> float:
+    """The slowest rank's time (every rank must call this, in the same order)."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_ours(args, wl, rank, world, dist):
     import learned_token_group_b200 as moga
 
@@ -272,11 +281,7 @@ def run_ours(args, wl, rank, world, dist):
         barrier()
         launches = moga.kernel_launches() - l0
     moga.sync_status(layer.ws)
-    ms = ev0.elapsed_time(ev1) / args.steps
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dist, dev)
     clocks = clk.summary()
     if args.lean:
         if rank == 0:
@@ -328,13 +333,39 @@ def run_ours(args, wl, rank, world, dist):
     ev1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = ev0.elapsed_time(ev1) / n_e2e
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / n_e2e, dist, dev)
     moga.sync_status(layer.ws)
 
+    # ---- the widened rows: three-branch block (adds the per-frame branch) and
+    # routing with balancing statistics, each timed over K steps
+    widened = {}
+    if wl.window is not None and not args.no_extras:
+        layer3 = moga.MogaLayer(wl.N, wl.d, wl.H, wl.d_h, wl.M, wl.grid, wl.window,
+                                torch.float32 if wl.x_dtype == "f32" else torch.bfloat16, dev, per_frame=True)
+        step3 = lambda: layer3(inp["x"], inp["W_r"], inp["b_r"], inp["q"], inp["k"], inp["v"])
+        step3()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step3()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        moga.sync_status(layer3.ws)
+        widened["three_branch_layer_ms"] = ev0.elapsed_time(ev1) / args.steps
+        del layer3
+        rt = lambda: moga.route(inp["x"], inp["W_r"], inp["b_r"], wl.M, out=r_out, ws=r_ws)
+        rs = lambda: moga.route_stats(inp["x"], inp["W_r"], inp["b_r"], wl.M)
+        r_out = moga.route(inp["x"], inp["W_r"], inp["b_r"], wl.M)
+        r_ws = moga.workspace(moga.get_lib().moga_route_workspace_size(wl.N, wl.M), dev)
+        for name, fn in (("route_ms", rt), ("route_with_balance_stats_ms", rs)):
+            fn()
+            torch.cuda.synchronize()
+            ev0.record(stream)
+            for _ in range(args.steps):
+                fn()
+            ev1.record(stream)
+            torch.cuda.synchronize()
+            widened[name] = ev0.elapsed_time(ev1) / args.steps
     if rank != 0:
         return
     peaks = _peaks()
@@ -377,6 +408,7 @@ def run_ours(args, wl, rank, world, dist):
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": int(launches),
         "clocks": clocks,
+        "widened": widened,
     }
     print(json.dumps(line), flush=True)
 
@@ -390,6 +422,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the widened-row timings")
     ap.add_argument("--lean", action="store_true",
                     help="warm-up and timed steps only (for hardware-counter captures)")
     args = ap.parse_args()
