@@ -128,9 +128,9 @@ moga_status moga_route_noalloc(const void* x, const void* W_r, const float* b_r,
                                int32_t* max_seqlen, void* stream);
 
 /* ---------------------------------------------------------------- grouped attention
- * moga_group_attn: Algorithm 1 steps 2 (gather), 3 (attention inside each
- * group segment) and 4 (un-permute), with the gate of Eq. 5 fused into the
- * store:   out[perm[j], h, :] = out_scale * gate[perm[j]] *
+ * moga_group_attn: Algorithm 1 steps 2 (gather Q/K/V into group order), 3
+ * (attention inside each group segment) and 4 (un-permute), with the gate of
+ * Eq. 5 fused into the store:   out[perm[j], h, :] = out_scale * gate[perm[j]] *
  *              SA(q[perm[j],h], K_seg(j),h, V_seg(j),h)
  * where seg(j) is the segment of offsets that contains j.  gate may be NULL
  * (gate = 1).  Tokens of empty groups do not exist, so every token's row of
@@ -227,7 +227,7 @@ typedef enum {
   MOGA_STAGE_SORT = 1,        /* scan + stable scatter -> offsets, perm */
   MOGA_STAGE_GATHER = 2,      /* segment table + gather of Q/K/V into group order */
   MOGA_STAGE_GROUP_ATTN = 3,  /* grouped attention kernel (incl. gate + un-permute) */
-  MOGA_STAGE_STGA_PREP = 4,   /* window permutation + gather into window order */
+  MOGA_STAGE_STGA_PREP = 4,   /* window-order permutation (+ gather for windows over 256 tokens) */
   MOGA_STAGE_STGA_ATTN = 5    /* STGA window attention kernel (incl. the mean) */
 } moga_stage;
 uint64_t moga_kernel_launches(void);

@@ -110,21 +110,31 @@ RouteWs route_ws(int64_t N, int M, bool with_stats = false) {
   return w;
 }
 
+// Grouped attention (and windows larger than two query tiles) streams each
+// segment's K/V many times, so it reads a gathered head-major copy of Q/K/V
+// with tiled loads; small STGA windows read q, k, v in place by token index.
+constexpr int64_t kDirectWindowMax = 2 * kTile;
+
 struct AttnWs {
   size_t table, permw, qh, kh, vh, total;
 };
-AttnWs attn_ws(int64_t N, int H, int d_h, int nseg_table, bool window_perm) {
+AttnWs attn_ws(int64_t N, int H, int d_h, int nseg_table, bool window_perm, bool copy = true) {
   Carve c;
   AttnWs w;
   w.table = c.take((size_t)(3 * nseg_table + 1) * 4);
   w.permw = window_perm ? c.take((size_t)N * 4) : 0;
-  const size_t mat = (size_t)N * H * d_h * 2;
-  w.qh = c.take(mat);
-  w.kh = c.take(mat);
-  w.vh = c.take(mat);
+  w.qh = w.kh = w.vh = 0;
+  if (copy) {
+    const size_t mat = (size_t)N * H * d_h * 2;
+    w.qh = c.take(mat);
+    w.kh = c.take(mat);
+    w.vh = c.take(mat);
+  }
   w.total = c.off;
   return w;
 }
+
+bool stga_direct(const int* window) { return (int64_t)window[0] * window[1] * window[2] <= kDirectWindowMax; }
 
 moga_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MOGA_OK : MOGA_ERR_CUDA; }
 
@@ -202,9 +212,10 @@ moga_status group_attn_body(const DevCtx& c, const void* q, const void* k, const
   mark(MOGA_STAGE_GATHER, false, c.stream);
   count(2);
   AttnArgs a{};
-  a.qh = ws + w.qh;
-  a.kh = ws + w.kh;
-  a.vh = ws + w.vh;
+  a.direct = 0;
+  a.q = ws + w.qh;
+  a.k = ws + w.kh;
+  a.v = ws + w.vh;
   a.perm = perm;
   a.gate = gate;
   a.out = out;
@@ -229,18 +240,27 @@ moga_status stga_body(const DevCtx& c, const void* q, const void* k, const void*
                       const int* window, int H, int d_h, int accumulate, void* out, uint8_t* ws,
                       float add_scale = 0.5f) {
   const int64_t N = (int64_t)T * Hg * Wg;
-  const AttnWs w = attn_ws(N, H, d_h, 0, true);
+  const bool direct = stga_direct(window);
+  const AttnWs w = attn_ws(N, H, d_h, 0, true, !direct);
   int32_t* permw = reinterpret_cast<int32_t*>(ws + w.permw);
   mark(MOGA_STAGE_STGA_PREP, true, c.stream);
   if (launch_window_perm(c, T, Hg, Wg, window, permw) != cudaSuccess) return MOGA_ERR_CUDA;
-  if (launch_gather(c, q, k, v, permw, N, H, d_h, ws + w.qh, ws + w.kh, ws + w.vh) != cudaSuccess)
-    return MOGA_ERR_CUDA;
-  mark(MOGA_STAGE_STGA_PREP, false, c.stream);
-  count(2);
+  count(1);
   AttnArgs a{};
-  a.qh = ws + w.qh;
-  a.kh = ws + w.kh;
-  a.vh = ws + w.vh;
+  a.direct = direct ? 1 : 0;
+  if (direct) {
+    a.q = q;
+    a.k = k;
+    a.v = v;
+  } else {
+    if (launch_gather(c, q, k, v, permw, N, H, d_h, ws + w.qh, ws + w.kh, ws + w.vh) != cudaSuccess)
+      return MOGA_ERR_CUDA;
+    count(1);
+    a.q = ws + w.qh;
+    a.k = ws + w.kh;
+    a.v = ws + w.vh;
+  }
+  mark(MOGA_STAGE_STGA_PREP, false, c.stream);
   a.perm = permw;
   a.gate = nullptr;
   a.out = out;
@@ -420,7 +440,7 @@ moga_status moga_group_attn(const void* q, const void* k, const void* v, const i
 size_t stga_window_attn_workspace_size(int T, int Hg, int Wg, const int* window, int H, int d_h) {
   int64_t N = 0;
   if (check_window(T, Hg, Wg, window, &N) != MOGA_OK || H < 1) return 0;
-  return attn_ws(N, H, d_h, 0, true).total;
+  return attn_ws(N, H, d_h, 0, true, !stga_direct(window)).total;
 }
 
 moga_status stga_window_attn(const void* q, const void* k, const void* v, int T, int Hg, int Wg,
@@ -433,7 +453,7 @@ moga_status stga_window_attn(const void* q, const void* k, const void* v, int T,
   if ((st = check_attn_shape(N, H, d_h)) != MOGA_OK) return st;
   if (accumulate != 0 && accumulate != 1) return MOGA_ERR_INVALID_ARG;
   if (!ws || !aligned16(ws)) return MOGA_ERR_INVALID_ARG;
-  if (ws_bytes < attn_ws(N, H, d_h, 0, true).total) return MOGA_ERR_WORKSPACE;
+  if (ws_bytes < attn_ws(N, H, d_h, 0, true, !stga_direct(window)).total) return MOGA_ERR_WORKSPACE;
   DevCtx c;
   if (!make_ctx(&c, ws, stream)) return MOGA_ERR_CUDA;
   return stga_body(c, q, k, v, T, Hg, Wg, window, H, d_h, accumulate, out, (uint8_t*)ws);
@@ -445,7 +465,7 @@ size_t moga_layer_workspace_size(int64_t N, int H, int d_h, int M, int T, int Hg
   const size_t ga = attn_ws(N, H, d_h, M, false).total;
   if (ga > need) need = ga;
   if (window) {
-    const size_t sw = attn_ws(N, H, d_h, 0, true).total;
+    const size_t sw = attn_ws(N, H, d_h, 0, true, !stga_direct(window)).total;
     if (sw > need) need = sw;
   }
   return need;

@@ -3,9 +3,6 @@
 // Attention" / "MoGA Pseudocode and Kernel Integration") and STGA window
 // attention (same page, "Spatial-Temporal Group Attention").
 //
-// gather_kernel     Q^,K^,V^[h][j] = q,k,v[perm[j]][h]: 16-byte vector copies,
-//                   one warp per token row, head-major destination so that each
-//                   (segment, head) is a dense [rows x d_h] matrix for TMA.
 // window_perm_kernel  position of every grid token in window order (STGA).
 // seg_table_kernel  groups sorted by size (largest first) with the prefix of
 //                   their query-tile counts: the persistent attention grid walks
@@ -13,8 +10,9 @@
 // attn_kernel<DH>   persistent varlen flash attention on tcgen05.  A CTA works
 //                   on two 128-row query tiles (A, B) of one (segment, head)
 //                   at a time, streaming the segment's K/V tiles once for both.
-//                   Warp 0 issues TMA loads (Q_A, Q_B, double-buffered K and V
-//                   rings); warp 1 issues tcgen05.mma in the order
+//                   Warp 0 loads Q_A, Q_B and double-buffered K and V tiles
+//                   straight from q, k, v by token index (TMA tile::gather4,
+//                   four rows per load, 32 lanes per tile); warp 1 issues tcgen05.mma in the order
 //                   PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so the tensor core
 //                   works on one tile while the other tile's softmax runs;
 //                   warps 2-5 and 6-9 are the two softmax warpgroups (one query
@@ -222,7 +220,9 @@ struct Decoder {
   }
 };
 
-template <int DH>
+// kDirect: load Q/K/V rows straight from q, k, v by token index (tile::gather4);
+// otherwise 128-row tiles of a gathered head-major copy (2-D tiled TMA).
+template <int DH, bool kDirect>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
             const __grid_constant__ CUtensorMap tv, const AttnArgs a, int* status, unsigned long long wait_ns) {
@@ -296,7 +296,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
   if (warp < 4) {
   regs_dec<kRegsCtl>();
   if (warp == 0) {
-    // ---------------------------------------------------------------- TMA producer
+    if constexpr (!kDirect) {
+    // ---------------------------------------------------------------- TMA producer (tiled)
+    // 128-row tiles of the gathered head-major copy [H][N][d_h] (row h*N + j).
     if (lane == 0) {
       tma_prefetch_desc(&tq);
       tma_prefetch_desc(&tk);
@@ -352,6 +354,91 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         if ((uint32_t)s < kc) mbar_wait(&k_full[s], ((kc - 1 - ((kc - 1 - s) % kStages)) / kStages) & 1, dc);
         if ((uint32_t)s < vc) mbar_wait(&v_full[s], ((vc - 1 - ((vc - 1 - s) % kStages)) / kStages) & 1, dc);
       }
+    }
+    } else {
+    // ---------------------------------------------------------------- TMA producer (whole warp)
+    // Q/K/V rows are fetched straight from q, k, v [N, H, d_h] by token index
+    // (perm: segment position -> token), four rows per tile::gather4 load and
+    // lane, so no gathered copy of Q/K/V is ever written.  Positions past the
+    // segment end repeat its last token (those keys and queries are masked).
+    if (lane == 0) {
+      tma_prefetch_desc(&tq);
+      tma_prefetch_desc(&tk);
+      tma_prefetch_desc(&tv);
+    }
+    const int H = a.H;
+    auto rows4 = [&](int pos0, int pos_end, int h, int* r) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int pp = min(pos0 + 4 * lane + i, pos_end - 1);
+        const int tok = a.perm[pp];
+        r[i] = (tok >= 0 && (int64_t)tok < N) ? tok * H + h : -1;  // out of range: zero fill
+      }
+    };
+    auto gather_tile = [&](const CUtensorMap* map, uint64_t* bar, uint8_t* dst, const int* r) {
+#pragma unroll
+      for (int c = 0; c < P::kChunks; ++c)
+        tma_gather4(map, bar, dst + c * 16384 + lane * 512, c * 64, r[0], r[1], r[2], r[3]);
+    };
+    uint32_t ucnt = 0, kc = 0, vc = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
+      const Unit u = dec(idx);
+      if (u.q0 >= u.len) continue;
+      const bool hb = u.q0 + kTile < u.len;
+      const int nkv = (u.len + kTile - 1) / kTile;
+      const int seg_end = u.start + u.len;
+      // Token indices are read one tile ahead, so that their global-memory
+      // latency overlaps the waits for free buffers.
+      int rqa[4], rqb[4], rk[4];
+      rows4(u.start + u.q0, seg_end, u.h, rqa);
+      if (hb) rows4(u.start + u.q0 + kTile, seg_end, u.h, rqb);
+      rows4(u.start, seg_end, u.h, rk);
+      int w = 1;
+      if (lane == 0) w = mbar_wait(q_empty, (ucnt & 1) ^ 1, wc, 1, ucnt);
+      if (!__shfl_sync(0xffffffffu, w, 0)) break;
+      if (lane == 0) mbar_expect_tx(q_full, (hb ? 2 : 1) * P::kTileBytes);
+      __syncwarp();
+      gather_tile(&tq, q_full, smem + P::kQA, rqa);
+      if (hb) gather_tile(&tq, q_full, smem + P::kQB, rqb);
+      ++ucnt;
+      for (int j = 0; j < nkv; ++j) {
+        const int ks = kc % kStages;
+        if (lane == 0) {
+          w = mbar_wait(&k_empty[ks], ((kc / kStages) & 1) ^ 1, wc, 2, kc);
+          // Test hook: this K tile never arrives, so the MMA warp's bounded
+          // wait runs out and the kernel reports a timeout.  No load is in
+          // flight for it, so the slot is not counted for the drain below.
+          if (w && a.debug_withhold_first_k && kc == 0) w = 0;
+          if (w) mbar_expect_tx(&k_full[ks], P::kTileBytes);
+        }
+        if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+        __syncwarp();
+        gather_tile(&tk, &k_full[ks], smem + P::kK0 + ks * P::kTileBytes, rk);  // K and V share rows
+        ++kc;
+        const int vs = vc % kStages;
+        if (lane == 0) {
+          w = mbar_wait(&v_empty[vs], ((vc / kStages) & 1) ^ 1, wc, 3, vc);
+          if (w) mbar_expect_tx(&v_full[vs], P::kTileBytes);
+        }
+        if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+        __syncwarp();
+        gather_tile(&tv, &v_full[vs], smem + P::kV0 + vs * P::kTileBytes, rk);
+        ++vc;
+        if (j + 1 < nkv) rows4(u.start + (j + 1) * kTile, seg_end, u.h, rk);
+      }
+    }
+    // Drain every load this warp issued before the CTA exits.
+    __syncwarp();
+    if (lane == 0) {
+      volatile int zero = 0;
+      WaitCtx dc{&zero, nullptr, 100000000ull};
+      if (ucnt > 0) mbar_wait(q_full, (ucnt - 1) & 1, dc);
+      for (int s = 0; s < kStages; ++s) {
+        if ((uint32_t)s < kc) mbar_wait(&k_full[s], ((kc - 1 - ((kc - 1 - s) % kStages)) / kStages) & 1, dc);
+        if ((uint32_t)s < vc) mbar_wait(&v_full[s], ((vc - 1 - ((vc - 1 - s) % kStages)) / kStages) & 1, dc);
+      }
+    }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -621,12 +708,16 @@ cudaError_t launch_attention_dh(const DevCtx& c, const AttnArgs& a) {
   using P = Plan<DH>;
   CUtensorMap mq, mk, mv;
   const uint64_t rows = (uint64_t)a.N * (uint64_t)a.H;
-  if (!make_tmap_2d(&mq, a.qh, DH, rows, DH * 2, kTile)) return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&mk, a.kh, DH, rows, DH * 2, kTile)) return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&mv, a.vh, DH, rows, DH * 2, kTile)) return cudaErrorInvalidValue;
+  // direct: q, k, v [N, H, d_h] viewed as [N*H rows, d_h] with one-row boxes
+  // (gather4); tiled: the gathered copy [H*N rows, d_h] with 128-row boxes.
+  const uint32_t box_rows = a.direct ? 1u : (uint32_t)kTile;
+  if (!make_tmap_2d(&mq, a.q, DH, rows, DH * 2, box_rows)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&mk, a.k, DH, rows, DH * 2, box_rows)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&mv, a.v, DH, rows, DH * 2, box_rows)) return cudaErrorInvalidValue;
   const int table_ints = a.mode == 0 ? 3 * a.nseg + 1 : 0;
   const size_t smem = P::bytes(table_ints);
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = a.direct ? attn_kernel<DH, true> : attn_kernel<DH, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int grid = c.num_sms;
   if (a.mode == 1) {
@@ -635,7 +726,7 @@ cudaError_t launch_attention_dh(const DevCtx& c, const AttnArgs& a) {
     if (total < grid) grid = (int)total;
   }
   if (grid < 1) return cudaSuccess;
-  attn_kernel<DH><<<grid, kAttnThreads, smem, c.stream>>>(mq, mk, mv, a, c.status, (unsigned long long)c.wait_ns);
+  kern<<<grid, kAttnThreads, smem, c.stream>>>(mq, mk, mv, a, c.status, (unsigned long long)c.wait_ns);
   return cudaGetLastError();
 }
 

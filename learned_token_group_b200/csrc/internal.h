@@ -43,19 +43,23 @@ cudaError_t launch_scatter(const DevCtx& c, const int32_t* group_id, const int32
                            int32_t* perm);
 
 // ------------------------------------------------------------------ attention
-// Q/K/V rows gathered by perm into head-major [H][N][d_h] buffers.
-cudaError_t launch_gather(const DevCtx& c, const void* q, const void* k, const void* v, const int32_t* perm,
-                          int64_t N, int H, int d_h, void* qh, void* kh, void* vh);
 // Window-order permutation of the STGA grid.
 cudaError_t launch_window_perm(const DevCtx& c, int T, int Hg, int Wg, const int* window, int32_t* perm_w);
 // Sorted segment table (largest group first) for the grouped attention.
 cudaError_t launch_seg_table(const DevCtx& c, const int32_t* offsets, int M, int H, int64_t N, int32_t* table);
 
+// Q/K/V rows gathered by perm into head-major [H][N][d_h] buffers.
+cudaError_t launch_gather(const DevCtx& c, const void* q, const void* k, const void* v, const int32_t* perm,
+                          int64_t N, int H, int d_h, void* qh, void* kh, void* vh);
+
 struct AttnArgs {
-  const void* qh;
-  const void* kh;
-  const void* vh;
-  const int32_t* perm;    // sorted position -> original token
+  // direct = 1: q, k, v are the caller's [N, H, d_h] tensors, read by token
+  // index (perm); direct = 0: they are gathered head-major copies [H][N][d_h].
+  int direct;
+  const void* q;
+  const void* k;
+  const void* v;
+  const int32_t* perm;    // segment position -> original token
   const float* gate;      // per original token, or null (gate = 1)
   void* out;              // bf16 [N, H, d_h]
   int64_t N;
