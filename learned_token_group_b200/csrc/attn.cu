@@ -10,18 +10,20 @@
 // attn_kernel<DH>   persistent varlen flash attention on tcgen05.  A CTA works
 //                   on two 128-row query tiles (A, B) of one (segment, head)
 //                   at a time, streaming the segment's K/V tiles once for both.
-//                   Warp 0 loads Q_A, Q_B and double-buffered K and V tiles
-//                   straight from q, k, v by token index (TMA tile::gather4,
-//                   four rows per load, 32 lanes per tile); warp 1 issues tcgen05.mma in the order
+//                   Loads: grouped attention (and large windows) read 128-row
+//                   tiles of a gathered head-major copy with 2-D TMA (warp 0);
+//                   windows of up to 256 tokens are copied straight from
+//                   q, k, v by token index with cp.async by warps 0, 2 and 3.
+//                   Warp 1 issues tcgen05.mma in the order
 //                   PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so the tensor core
 //                   works on one tile while the other tile's softmax runs;
-//                   warps 2-5 and 6-9 are the two softmax warpgroups (one query
+//                   warps 4-7 and 8-11 are the two softmax warpgroups (one query
 //                   row per thread): S is read from TMEM, P is written back as
 //                   bf16 over S in TMEM and consumed from there by the P V
 //                   product, O is rescaled in TMEM only when a row max grows by
 //                   more than 2^8; the epilogue scales by gate/l and scatters
-//                   each row to out[perm[j]] (or adds into it for the STGA
-//                   branch).
+//                   each row to out[perm[j]] (or, for a later branch of the
+//                   block, adds into it with vector reductions).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -194,6 +196,7 @@ struct Decoder {
   const int* tab;  // groups: shared copy of [unit_prefix (M+1) | seg_start (M) | seg_len (M)]
   WinGeom g;
   int upw;         // windows: units per window
+  int H;           // windows read in place: heads vary fastest
   __device__ __forceinline__ Unit operator()(int idx) const {
     Unit u;
     if (mode == 0) {
@@ -209,10 +212,20 @@ struct Decoder {
       u.h = local / npair;
       u.q0 = (local - u.h * npair) * 2 * kTile;
     } else {
+      // Units in place go window by window with the heads innermost, so the
+      // CTAs running at once read whole token rows of q, k, v (all heads)
+      // close together in time.  With a gathered head-major copy each head's
+      // window is contiguous already, and heads go outermost.
       const int qp = idx % upw;
       const int rest = idx / upw;
-      const int seg = rest % nseg;
-      u.h = rest / nseg;
+      int seg;
+      if (H > 0) {
+        u.h = rest % H;
+        seg = rest / H;
+      } else {
+        seg = rest % nseg;
+        u.h = rest / nseg;
+      }
       window_of(g, seg, u.start, u.len);
       u.q0 = qp * 2 * kTile;
     }
@@ -220,7 +233,7 @@ struct Decoder {
   }
 };
 
-// kDirect: load Q/K/V rows straight from q, k, v by token index (tile::gather4);
+// kDirect: copy Q/K/V rows straight from q, k, v by token index (cp.async);
 // otherwise 128-row tiles of a gathered head-major copy (2-D tiled TMA).
 template <int DH, bool kDirect>
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -270,6 +283,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
   dec.nseg = a.nseg;
   dec.tab = tab;
   dec.upw = 1;
+  dec.H = kDirect ? a.H : 0;
   if (a.mode == 0) {
     const int n = 3 * a.nseg + 1;
     for (int i = threadIdx.x; i < n; i += blockDim.x) tab[i] = a.table[i];
@@ -295,8 +309,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
 
   if (warp < 4) {
   regs_dec<kRegsCtl>();
-  if (warp == 0) {
-    if constexpr (!kDirect) {
+  if (!kDirect && warp == 0) {
     // ---------------------------------------------------------------- TMA producer (tiled)
     // 128-row tiles of the gathered head-major copy [H][N][d_h] (row h*N + j).
     if (lane == 0) {
@@ -355,92 +368,120 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         if ((uint32_t)s < vc) mbar_wait(&v_full[s], ((vc - 1 - ((vc - 1 - s) % kStages)) / kStages) & 1, dc);
       }
     }
-    } else {
-    // ---------------------------------------------------------------- TMA producer (whole warp)
-    // Q/K/V rows are fetched straight from q, k, v [N, H, d_h] by token index
-    // (perm: segment position -> token), four rows per tile::gather4 load and
-    // lane, so no gathered copy of Q/K/V is ever written.  Positions past the
-    // segment end repeat its last token (those keys and queries are masked).
-    if (lane == 0) {
-      tma_prefetch_desc(&tq);
-      tma_prefetch_desc(&tk);
-      tma_prefetch_desc(&tv);
-    }
+  }
+  if (kDirect && warp != 1) {
+    // ---------------------------------------------------------------- cp.async loaders (warps 0, 2, 3)
+    // Q/K/V rows are copied straight from q, k, v [N, H, d_h] by token index
+    // (perm: segment position -> token), so no gathered copy is ever written.
+    // Warp 0 copies Q_A and Q_B, warp 2 the K tiles and warp 3 the V tiles:
+    // each lane moves 16-byte pieces with cp.async into the 128-byte swizzled
+    // layout the MMA descriptors expect, waits for its pieces, fences them for
+    // the async proxy, and lane 0 then arrives on the tile's barrier.  Each
+    // empty barrier thus has one waiter that follows its phases in order.
+    // Three warps keep up to 128 KB in flight, which single-row TMA gathers
+    // could not (their per-instruction cost capped an SM near 8 B/cycle).
+    // Positions past the segment end repeat its last token (masked later).
+    const int li = warp == 0 ? 0 : warp - 1;  // 0: Q, 1: K, 2: V
+    constexpr int kPieces = DH * 2 / 16;       // 16-byte pieces per row
+    constexpr int kRowsPerOp = 32 / kPieces;   // rows one warp-wide copy covers
+    const int piece = lane % kPieces, sub = lane / kPieces;
+    const uint32_t piece_off = (uint32_t)((piece >> 3) * (kTile * 128));  // 64-column chunk
+    const int pj = piece & 7;
+    int* toks = tab + li * 2 * kTile;  // this loader's token rows (two tiles for Q)
     const int H = a.H;
-    auto rows4 = [&](int pos0, int pos_end, int h, int* r) {
+    uint32_t ucnt = 0, t = 0;
+    bool ok = true;
+    // Row indices of tile rows [pos0, pos0 + 128), four per lane: token * H + h,
+    // or -1 (zero-filled) for a token out of range or a row past the segment
+    // end.  Read before the slot is free so that their latency overlaps the
+    // wait.
+    auto fetch_rows = [&](int pos0, int seg_end, int h, int (&tr)[4]) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int pp = min(pos0 + 4 * lane + i, pos_end - 1);
-        const int tok = a.perm[pp];
-        r[i] = (tok >= 0 && (int64_t)tok < N) ? tok * H + h : -1;  // out of range: zero fill
+        const int pp = pos0 + 4 * lane + i;
+        const int tok = a.perm[min(pp, seg_end - 1)];
+        tr[i] = (pp < seg_end && tok >= 0 && (int64_t)tok < N) ? tok * H + h : -1;
       }
     };
-    auto gather_tile = [&](const CUtensorMap* map, uint64_t* bar, uint8_t* dst, const int* r) {
+    // Issues the copies of one tile whose row indices are in tr (staged in
+    // tk, 128 ints); the caller waits for them.  Only the copies covering the
+    // tile's first nrows rows are issued (a warp-uniform count): rows past the
+    // segment end keep what the slot held, which is finite (earlier tiles or
+    // the initial zeros), and belong to masked keys or dropped queries.
+    auto copy_tile = [&](const void* g, uint8_t* dst, const int (&tr)[4], int* tk, int nrows) {
 #pragma unroll
-      for (int c = 0; c < P::kChunks; ++c)
-        tma_gather4(map, bar, dst + c * 16384 + lane * 512, c * 64, r[0], r[1], r[2], r[3]);
+      for (int i = 0; i < 4; ++i) tk[4 * lane + i] = tr[i];
+      __syncwarp();
+      const char* gb = static_cast<const char*>(g) + piece * 16;
+      const uint32_t db = smem_u32(dst) + piece_off;
+      const int nops = (min(nrows, kTile) + kRowsPerOp - 1) / kRowsPerOp;  // warp-uniform
+#pragma unroll 8
+      for (int i = 0; i < nops; ++i) {
+        const int r = i * kRowsPerOp + sub;
+        const int row = tk[r];
+        const char* src = row >= 0 ? gb + (int64_t)row * (DH * 2) : gb;
+        cp_async16(db + r * 128 + ((pj ^ (r & 7)) << 4), src, row >= 0 ? 16 : 0);
+      }
     };
-    uint32_t ucnt = 0, kc = 0, vc = 0;
-    bool ok = true;
+    auto finish = [&]() {
+      cp_async_commit_wait_all();
+      fence_proxy_async_smem();
+      __syncwarp();
+    };
+    // Lane 0 waits; the whole warp learns the outcome.
+    auto warp_wait = [&](uint64_t* bar, uint32_t parity, int site, uint32_t count) {
+      int w = 1;
+      if (lane == 0) w = mbar_wait(bar, parity, wc, site, count);
+      return __shfl_sync(0xffffffffu, w, 0) != 0;
+    };
+    if (li > 0) {
+      // Rows past a segment's end are never copied, so the K and V rings
+      // start as zeros: every row the tensor core reads is then finite (a
+      // masked key's P is 0, and 0 times a finite V row adds nothing).
+      uint4* ring = reinterpret_cast<uint4*>(smem + (li == 1 ? P::kK0 : P::kV0));
+      for (int i = lane; i < kStages * P::kTileBytes / 16; i += 32) ring[i] = make_uint4(0, 0, 0, 0);
+      fence_proxy_async_smem();
+      __syncwarp();
+    }
     for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
       const Unit u = dec(idx);
       if (u.q0 >= u.len) continue;
       const bool hb = u.q0 + kTile < u.len;
       const int nkv = (u.len + kTile - 1) / kTile;
       const int seg_end = u.start + u.len;
-      // Token indices are read one tile ahead, so that their global-memory
-      // latency overlaps the waits for free buffers.
-      int rqa[4], rqb[4], rk[4];
-      rows4(u.start + u.q0, seg_end, u.h, rqa);
-      if (hb) rows4(u.start + u.q0 + kTile, seg_end, u.h, rqb);
-      rows4(u.start, seg_end, u.h, rk);
-      int w = 1;
-      if (lane == 0) w = mbar_wait(q_empty, (ucnt & 1) ^ 1, wc, 1, ucnt);
-      if (!__shfl_sync(0xffffffffu, w, 0)) break;
-      if (lane == 0) mbar_expect_tx(q_full, (hb ? 2 : 1) * P::kTileBytes);
-      __syncwarp();
-      gather_tile(&tq, q_full, smem + P::kQA, rqa);
-      if (hb) gather_tile(&tq, q_full, smem + P::kQB, rqb);
-      ++ucnt;
-      for (int j = 0; j < nkv; ++j) {
-        const int ks = kc % kStages;
-        if (lane == 0) {
-          w = mbar_wait(&k_empty[ks], ((kc / kStages) & 1) ^ 1, wc, 2, kc);
-          // Test hook: this K tile never arrives, so the MMA warp's bounded
-          // wait runs out and the kernel reports a timeout.  No load is in
-          // flight for it, so the slot is not counted for the drain below.
-          if (w && a.debug_withhold_first_k && kc == 0) w = 0;
-          if (w) mbar_expect_tx(&k_full[ks], P::kTileBytes);
+      if (li == 0) {
+        int ra[4], rb[4];
+        fetch_rows(u.start + u.q0, seg_end, u.h, ra);
+        if (hb) fetch_rows(u.start + u.q0 + kTile, seg_end, u.h, rb);
+        if (!warp_wait(q_empty, (ucnt & 1) ^ 1, 1, ucnt)) { ok = false; break; }
+        copy_tile(a.q, smem + P::kQA, ra, toks, u.len - u.q0);
+        if (hb) copy_tile(a.q, smem + P::kQB, rb, toks + kTile, u.len - u.q0 - kTile);
+        finish();
+        if (lane == 0) mbar_arrive(q_full);
+        ++ucnt;
+        continue;
+      }
+      const bool is_v = li == 2;
+      for (int j = 0; j < nkv; ++j, ++t) {
+        int tr[4];
+        const int s = t % kStages;
+        fetch_rows(u.start + j * kTile, seg_end, u.h, tr);
+        if (!warp_wait(is_v ? &v_empty[s] : &k_empty[s], ((t / kStages) & 1) ^ 1, is_v ? 3 : 2, t)) {
+          ok = false;
+          break;
         }
-        if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
-        __syncwarp();
-        gather_tile(&tk, &k_full[ks], smem + P::kK0 + ks * P::kTileBytes, rk);  // K and V share rows
-        ++kc;
-        const int vs = vc % kStages;
-        if (lane == 0) {
-          w = mbar_wait(&v_empty[vs], ((vc / kStages) & 1) ^ 1, wc, 3, vc);
-          if (w) mbar_expect_tx(&v_full[vs], P::kTileBytes);
-        }
-        if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
-        __syncwarp();
-        gather_tile(&tv, &v_full[vs], smem + P::kV0 + vs * P::kTileBytes, rk);
-        ++vc;
-        if (j + 1 < nkv) rows4(u.start + (j + 1) * kTile, seg_end, u.h, rk);
+        // Test hook: the first K tile never arrives, so the MMA warp's
+        // bounded wait runs out and the kernel reports a timeout.
+        if (!is_v && t == 0 && a.debug_withhold_first_k) { ok = false; break; }
+        copy_tile(is_v ? a.v : a.k, smem + (is_v ? P::kV0 : P::kK0) + s * P::kTileBytes, tr, toks,
+                  u.len - j * kTile);
+        finish();
+        if (lane == 0) mbar_arrive(is_v ? &v_full[s] : &k_full[s]);
       }
     }
-    // Drain every load this warp issued before the CTA exits.
-    __syncwarp();
-    if (lane == 0) {
-      volatile int zero = 0;
-      WaitCtx dc{&zero, nullptr, 100000000ull};
-      if (ucnt > 0) mbar_wait(q_full, (ucnt - 1) & 1, dc);
-      for (int s = 0; s < kStages; ++s) {
-        if ((uint32_t)s < kc) mbar_wait(&k_full[s], ((kc - 1 - ((kc - 1 - s) % kStages)) / kStages) & 1, dc);
-        if ((uint32_t)s < vc) mbar_wait(&v_full[s], ((vc - 1 - ((vc - 1 - s) % kStages)) / kStages) & 1, dc);
-      }
-    }
-    }
-  } else if (warp == 1) {
+    // Every copy was waited for before its arrive, so nothing is in flight.
+  }
+  if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
@@ -546,6 +587,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       const bool hb = u.q0 + kTile < u.len;
       if (x == 1 && !hb) continue;
       const int nkv = (u.len + kTile - 1) / kTile;
+      // The output row of this thread's query is fetched now, so its latency
+      // hides behind the key loop.
+      const int r = u.q0 + x * kTile + row;
+      bool live = r < u.len;
+      const int src = live ? a.perm[u.start + r] : 0;
       float m_run = -INFINITY;
       uint64_t la = f2_pack(0.f, 0.f), lb = la, lc = la, ld = la;  // row sum of P, 8 partial sums
       for (int j = 0; j < nkv; ++j) {
@@ -646,21 +692,15 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       if (!mbar_wait(&o_full[x], oc & 1, wc, 9 + 16 * x, oc)) break;
       ++oc;
       tc_fence_after();
-      const int r = u.q0 + x * kTile + row;
-      bool live = r < u.len;
-      int64_t src = 0;
-      if (live) {
-        src = a.perm[u.start + r];
-        if (src < 0 || src >= N) {
-          live = false;
-          if (status) atomicOr(status, DEV_RANGE);
-        }
+      if (live && (src < 0 || src >= N)) {
+        live = false;
+        if (status) atomicOr(status, DEV_RANGE);
       }
       float l_lo, l_hi;
       f2_unpack(f2_add(f2_add(la, lb), f2_add(lc, ld)), l_lo, l_hi);
       const float gt = (live && a.gate) ? a.gate[src] : 1.0f;
       const float inv = a.out_scale * gt / (l_lo + l_hi);
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) + (src * a.H + u.h) * (int64_t)DH;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) + ((int64_t)src * a.H + u.h) * (int64_t)DH;
 #pragma unroll
       for (int c = 0; c < DH / 32; ++c) {
         float o[32];
@@ -673,22 +713,17 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             float w[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) w[e] = o[q4 * 8 + e] * inv;
-            if (a.accumulate) {
-              const uint4 old = dst[q4];
-              const __nv_bfloat162* ob = reinterpret_cast<const __nv_bfloat162*>(&old);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(ob[e]);
-                w[2 * e] += f.x;
-                w[2 * e + 1] += f.y;
-              }
-            }
             uint4 pk;
             pk.x = pack_bf16x2(w[0], w[1]);
             pk.y = pack_bf16x2(w[2], w[3]);
             pk.z = pack_bf16x2(w[4], w[5]);
             pk.w = pack_bf16x2(w[6], w[7]);
-            dst[q4] = pk;
+            // accumulate (a later branch of the block): out += this branch,
+            // added by the memory system; otherwise a plain store.
+            if (a.accumulate)
+              red_add_bf16x8(dst + q4, pk);
+            else
+              dst[q4] = pk;
           }
         }
       }
@@ -708,13 +743,14 @@ cudaError_t launch_attention_dh(const DevCtx& c, const AttnArgs& a) {
   using P = Plan<DH>;
   CUtensorMap mq, mk, mv;
   const uint64_t rows = (uint64_t)a.N * (uint64_t)a.H;
-  // direct: q, k, v [N, H, d_h] viewed as [N*H rows, d_h] with one-row boxes
-  // (gather4); tiled: the gathered copy [H*N rows, d_h] with 128-row boxes.
-  const uint32_t box_rows = a.direct ? 1u : (uint32_t)kTile;
+  // tiled: the gathered copy [H*N rows, d_h] with 128-row boxes.  The
+  // in-place kernel copies rows itself and does not read the maps.
+  const uint32_t box_rows = (uint32_t)kTile;
   if (!make_tmap_2d(&mq, a.q, DH, rows, DH * 2, box_rows)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&mk, a.k, DH, rows, DH * 2, box_rows)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&mv, a.v, DH, rows, DH * 2, box_rows)) return cudaErrorInvalidValue;
-  const int table_ints = a.mode == 0 ? 3 * a.nseg + 1 : 0;
+  // groups: the segment table; in place: the loaders' token rows (2 tiles each)
+  const int table_ints = a.mode == 0 ? 3 * a.nseg + 1 : (a.direct ? 6 * kTile : 0);
   const size_t smem = P::bytes(table_ints);
   auto kern = a.direct ? attn_kernel<DH, true> : attn_kernel<DH, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -102,18 +102,6 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* ba
       : "memory");
 }
 
-// Four rows of a 2-D tensor (box one row high, 64 bf16 columns) gathered by
-// row index into four consecutive 128-byte shared-memory rows (sm_100 TMA
-// tile::gather4); the tensor map's swizzle applies as for tiled loads.
-__device__ __forceinline__ void tma_gather4(const CUtensorMap* map, uint64_t* bar, void* dst, int col, int r0, int r1,
-                                            int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(smem_u32(bar)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-      : "memory");
-}
-
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (tensor core operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -324,6 +312,23 @@ __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t t2) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// 16-byte asynchronous global -> shared copy through L2 only (cp.async.cg);
+// src_bytes = 0 fills the 16 bytes with zeros and reads nothing.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+// out[0..8) += v (eight bf16 values) as one fire-and-forget vector reduction:
+// the add is done by the memory system, so the thread does not wait for the
+// old values to arrive.  Each sum is rounded to bf16 once.
+__device__ __forceinline__ void red_add_bf16x8(void* gptr, const uint4& v) {
+  asm volatile("red.global.add.noftz.v4.bf16x2 [%0], {%1, %2, %3, %4};" ::"l"(gptr), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
 }
 
 // Shared-memory atomic add with acquire-release ordering at CTA scope.
