@@ -198,6 +198,49 @@ moga_status moga_layer_ex(const void* x, const void* W_r, const float* b_r, moga
                           int Wg, const int* window, int branches, void* out, int32_t* group_id, float* gate,
                           int32_t* perm, int32_t* offsets, void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- host pipeline
+ * A pipeline runs the visual block of moga_layer_ex (same arithmetic, same
+ * branches) on inputs that live in HOST memory and returns the output to host
+ * memory, step after step, with the copies of one step overlapping the
+ * compute of its neighbours: step i+1's inputs travel host -> device while
+ * step i computes and step i-1's output travels back.  It owns two device
+ * slots of inputs and outputs, one workspace and three streams (copy in,
+ * compute, copy out), all on the device that is current at creation.
+ * Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister): the
+ * copies are then asynchronous DMA; pageable memory still works but the copies
+ * stop overlapping.  The pipeline is not thread-safe: one host thread at a time.
+ *
+ * moga_pipe_create: shapes and branches as moga_layer_ex (window required when
+ * branches & 1; T, Hg, Wg required when branches != 0).  Allocates about
+ * 2 x (inputs + outputs) + the layer workspace of device memory.
+ * On success *pipe receives the handle.  Invalid shapes return
+ * MOGA_ERR_INVALID_ARG / MOGA_ERR_UNSUPPORTED before any CUDA call.
+ */
+typedef struct moga_pipe moga_pipe;
+moga_status moga_pipe_create(int64_t N, int d, int H, int d_h, int M, moga_dtype x_dt, int T, int Hg, int Wg,
+                             const int* window, int branches, moga_pipe** pipe);
+
+/* moga_pipe_submit: enqueues one step and returns without waiting.
+ * In (host): x [N, d] (x_dt), W_r [M, d] (x_dt), b_r fp32 [M] or NULL,
+ *            q, k, v bf16 [N, H, d_h].
+ * Out (host): out bf16 [N, H, d_h]; group_id int32 [N] and gate fp32 [N]
+ *            optional (NULL = not returned).
+ * Every host buffer must stay valid, and the inputs unchanged, until
+ * moga_pipe_sync() returns; the outputs hold the step's result from then on.
+ * Returns MOGA_ERR_INVALID_ARG for a NULL required pointer or a NULL pipe, and
+ * MOGA_ERR_CUDA if enqueueing failed. */
+moga_status moga_pipe_submit(moga_pipe* pipe, const void* x, const void* W_r, const float* b_r, const void* q,
+                             const void* k, const void* v, void* out, int32_t* group_id, float* gate);
+
+/* moga_pipe_sync: waits for every submitted step, then reads and clears the
+ * device status word; returns MOGA_OK, MOGA_ERR_TIMEOUT, MOGA_ERR_DEVICE_CHECK
+ * or MOGA_ERR_CUDA (the first error of any step since the last sync). */
+moga_status moga_pipe_sync(moga_pipe* pipe);
+
+/* moga_pipe_destroy: waits for outstanding steps and frees everything.
+ * NULL is a no-op. */
+moga_status moga_pipe_destroy(moga_pipe* pipe);
+
 /* ---------------------------------------------------------------- device status
  * moga_sync_status: synchronises `stream`, reads the device status word kept
  * at the start of a workspace `ws` used by the calls above, clears it, and

@@ -20,7 +20,7 @@ import torch
 
 __all__ = ["MogaError", "get_lib", "LIB_PATH", "HEADER_PATH", "route", "group_attn", "stga_window_attn",
            "moga_layer", "sync_status", "workspace", "MogaLayer", "exported_names", "kernel_launches",
-           "set_timing_events", "STAGES"]
+           "set_timing_events", "STAGES", "Pipeline"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoga.so")
@@ -72,6 +72,10 @@ def get_lib():
         "moga_route_noalloc": (_I, [_P, _P, _P, _I, _I64, _I, _I, _P, _P, _P, _P, _P, _P]),
         "moga_set_timing_events": (_I, [_I, _P, _P]),
         "moga_debug_inject": (_I, [_I]),
+        "moga_pipe_create": (_I, [_I64, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I, ctypes.POINTER(_P)]),
+        "moga_pipe_submit": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+        "moga_pipe_sync": (_I, [_P]),
+        "moga_pipe_destroy": (_I, [_P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -290,3 +294,76 @@ def moga_layer(x, W_r, b_r, q, k, v, M: int, grid=None, window=None, per_frame: 
     layer(x, W_r, b_r, q, k, v)
     return {"out": layer.out, "group_id": layer.group_id, "gate": layer.gate, "perm": layer.perm,
             "offsets": layer.offsets, "ws": layer.ws}
+
+
+def _host_tensor(t: torch.Tensor, name: str, dtype, shape):
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+class Pipeline:
+    """Host-to-host pipeline of one visual block (moga_pipe_* in moga.h).
+
+    ``submit`` enqueues one step on host tensors (page-locked ones make the
+    copies asynchronous) and returns at once; consecutive steps overlap their
+    copies with their neighbours' compute.  ``sync`` waits for every submitted
+    step; the host tensors handed to ``submit`` are kept alive until then.
+    """
+
+    def __init__(self, N, d, H, d_h, M, grid=None, window=None, x_dtype=torch.bfloat16, device="cuda",
+                 per_frame: bool = False):
+        lib = get_lib()
+        self.N, self.d, self.H, self.d_h, self.M = N, d, H, d_h, M
+        self.x_dtype = x_dtype
+        grid = tuple(grid) if grid is not None else (0, 0, 0)
+        self.window = tuple(window) if window is not None else None
+        self.branches = (1 if self.window else 0) | (2 if per_frame else 0)
+        x_dt = {torch.float32: MOGA_F32, torch.bfloat16: MOGA_BF16}[x_dtype]
+        handle = ctypes.c_void_p()
+        with torch.cuda.device(torch.device(device)):
+            st = lib.moga_pipe_create(N, d, H, d_h, M, x_dt, *grid, _int3(self.window) if self.window else None,
+                                      self.branches, ctypes.byref(handle))
+        _check(st, "moga_pipe_create")
+        self._h = handle
+        self._keep = []
+
+    def submit(self, x, W_r, b_r, q, k, v, out, group_id=None, gate=None):
+        N, d, H, d_h, M = self.N, self.d, self.H, self.d_h, self.M
+        _host_tensor(x, "x", self.x_dtype, (N, d))
+        _host_tensor(W_r, "W_r", self.x_dtype, (M, d))
+        if b_r is not None:
+            _host_tensor(b_r, "b_r", torch.float32, (M,))
+        for n, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+            _host_tensor(t, n, torch.bfloat16, (N, H, d_h))
+        if group_id is not None:
+            _host_tensor(group_id, "group_id", torch.int32, (N,))
+        if gate is not None:
+            _host_tensor(gate, "gate", torch.float32, (N,))
+        st = get_lib().moga_pipe_submit(self._h, _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(q), _ptr(k), _ptr(v),
+                                        _ptr(out), _ptr(group_id), _ptr(gate))
+        self._keep.append((x, W_r, b_r, q, k, v, out, group_id, gate))
+        _check(st, "moga_pipe_submit")
+
+    def sync(self):
+        st = get_lib().moga_pipe_sync(self._h)
+        self._keep.clear()
+        _check(st, "moga_pipe_sync")
+
+    def close(self):
+        if self._h:
+            get_lib().moga_pipe_destroy(self._h)
+            self._h = None
+            self._keep.clear()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

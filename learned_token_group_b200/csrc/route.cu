@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(128)
 scatter_kernel(const int32_t* __restrict__ group_id, const int32_t* __restrict__ base, int N, int M,
                int32_t* __restrict__ perm) {
   extern __shared__ int cnt[];  // [4][M]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < 4 * M; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
   const int t = blockIdx.x;

@@ -147,3 +147,22 @@ def test_route_ex_validation(lib):
 def test_wait_limit_roundtrip(lib):
     old = lib.moga_set_wait_limit_ns(123456)
     assert lib.moga_set_wait_limit_ns(old) == 123456
+
+
+def test_pipe_validation(lib):
+    """The host pipeline rejects bad shapes before any CUDA call, and a NULL
+    handle everywhere."""
+    h = ctypes.c_void_p()
+    w = (ctypes.c_int * 3)(3, 8, 8)
+    create = lib.moga_pipe_create
+    assert create(384, 256, 2, 128, 4, 1, 3, 8, 16, w, 1, None) == INVALID          # no handle slot
+    assert create(-1, 256, 2, 128, 4, 1, 0, 0, 0, None, 0, ctypes.byref(h)) == INVALID
+    assert create(384, 256, 2, 96, 4, 1, 0, 0, 0, None, 0, ctypes.byref(h)) == UNSUPPORTED
+    assert create(384, 256, 2, 128, 4, 7, 0, 0, 0, None, 0, ctypes.byref(h)) == INVALID  # dtype
+    assert create(384, 256, 2, 128, 4, 1, 3, 8, 16, None, 1, ctypes.byref(h)) == INVALID  # window missing
+    assert create(384, 256, 2, 128, 4, 1, 3, 8, 15, w, 1, ctypes.byref(h)) == INVALID     # grid != N
+    assert create(384, 256, 2, 128, 4, 1, 3, 8, 16, w, 4, ctypes.byref(h)) == INVALID     # branch bits
+    assert h.value is None
+    assert lib.moga_pipe_submit(None, P, P, None, P, P, P, P, None, None) == INVALID
+    assert lib.moga_pipe_sync(None) == INVALID
+    assert lib.moga_pipe_destroy(None) == OK
