@@ -32,6 +32,14 @@ Readings where the pages leave a step open (each one is pinned by a test):
   sorted position j (the inverse of the pages' original-to-permuted index).
 * STGA windows: non-overlapping boxes of (wt, wh, ww) tokens anchored at the
   grid origin, clipped at the grid edges; token index (t*Hg + h)*Wg + w.
+* shot-aware STGA: temporal groups never cross a shot boundary.  Within each
+  shot, temporal windows of wt frames tile the shot from its first frame and
+  are clipped at its last (wt = 0: one window per shot).  Keys and values, not
+  queries, of a shot's first temporal window are augmented with the last
+  aug_prev frames of the previous shot, and those of its last temporal window
+  with the first aug_next frames of the next shot, in the window's spatial tile
+  (the pages say "two latent frames from adjacent shots": aug_prev = aug_next
+  = 2 by default, each clipped to the neighbouring shot's length).
 * combine: out = (MoGA + STGA) / 2 when STGA is on, MoGA alone otherwise; with
   the per-frame branch (attention inside each latent frame) the block output
   is the plain mean of all branches that are on.
@@ -50,6 +58,7 @@ import numpy as np
 __all__ = [
     "route", "balance_stats", "counting_sort", "attention_rows", "group_attention",
     "stga_windows", "stga_attention", "frame_attention", "moga_layer",
+    "shot_windows", "stga_shot_attention",
 ]
 
 _ROW_BLOCK = 16384
@@ -249,6 +258,71 @@ def frame_attention(q, k, v, T: int, Hg: int, Wg: int, rows=None, heads=None) ->
     """Per-frame branch: full attention among the tokens of each latent frame
     (the STGA definition with a window of one whole frame)."""
     return stga_attention(q, k, v, T, Hg, Wg, (1, Hg, Wg), rows=rows, heads=heads)
+
+
+def _tile_tokens(frames: np.ndarray, hs: np.ndarray, ws: np.ndarray, Hg: int, Wg: int) -> np.ndarray:
+    """Token indices (t*Hg + h)*Wg + w of a box of frames x rows x columns, sorted."""
+    idx = ((frames[:, None, None] * Hg + hs[None, :, None]) * Wg + ws[None, None, :]).reshape(-1)
+    return np.sort(idx)
+
+
+def shot_windows(T: int, Hg: int, Wg: int, window, shot_start: Sequence[int],
+                 aug_prev: int = 2, aug_next: int = 2) -> List[Tuple[np.ndarray, np.ndarray]]:
+    """(query tokens, key/value tokens) of every shot-aware STGA window
+    ("Spatial-Temporal Group Attention": frames of different shots are in
+    distinct temporal groups; keys and values, not queries, see two latent
+    frames of the adjacent shots).
+
+    shot_start: 0 = s_0 < s_1 < ... < s_S = T; shot j holds frames
+    [s_j, s_{j+1}).  Windows go shot by shot, then temporal window, then
+    spatial rows, then columns; the query sets cover every token once.
+    """
+    wt, wh, ww = (int(w) for w in window)
+    s = [int(v) for v in shot_start]
+    assert s[0] == 0 and s[-1] == T and all(a < b for a, b in zip(s, s[1:]))
+    S = len(s) - 1
+    pairs = []
+    for j in range(S):
+        a, b = s[j], s[j + 1]
+        step = wt if wt > 0 else b - a
+        for t0 in range(a, b, step):
+            t1 = min(b, t0 + step)
+            extra = []
+            if t0 == a and j > 0:                     # first window of the shot
+                extra.append(np.arange(max(s[j - 1], a - aug_prev), a))
+            if t1 == b and j < S - 1:                 # last window of the shot
+                extra.append(np.arange(b, min(s[j + 2], b + aug_next)))
+            own = np.arange(t0, t1)
+            kv_frames = np.concatenate([own] + extra) if extra else own
+            for h0 in range(0, Hg, wh):
+                for w0 in range(0, Wg, ww):
+                    hs = np.arange(h0, min(Hg, h0 + wh))
+                    ws = np.arange(w0, min(Wg, w0 + ww))
+                    pairs.append((_tile_tokens(own, hs, ws, Hg, Wg),
+                                  _tile_tokens(kv_frames, hs, ws, Hg, Wg)))
+    return pairs
+
+
+def stga_shot_attention(q, k, v, T: int, Hg: int, Wg: int, window, shot_start,
+                        aug_prev: int = 2, aug_next: int = 2,
+                        rows: Optional[Sequence[int]] = None,
+                        heads: Optional[Sequence[int]] = None) -> np.ndarray:
+    """Shot-aware STGA: each query attends to its window's tokens plus the
+    window's boundary frames of the adjacent shots (see ``shot_windows``).
+
+    Output layout as for ``group_attention``.
+    """
+    N, H, d_h = q.shape
+    assert T * Hg * Wg == N
+    out, row_pos, hs = _row_layout(N, H, d_h, rows, heads)
+    for qidx, kidx in shot_windows(T, Hg, Wg, window, shot_start, aug_prev, aug_next):
+        qi = qidx[row_pos[qidx] >= 0]
+        if qi.size == 0:
+            continue
+        for hp, h in enumerate(hs):
+            o = attention_rows(_f64(q[qi, h]), _f64(k[kidx, h]), _f64(v[kidx, h]))
+            out[row_pos[qi], hp] = o
+    return out
 
 
 def moga_layer(x, W_r, b_r, q, k, v, M: int, grid=None, window=None,

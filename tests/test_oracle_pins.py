@@ -94,6 +94,52 @@ def _brute_stga(q, k, v, grid, window):
     return out
 
 
+def _brute_shot_stga(q, k, v, grid, window, shot_start, aug_prev, aug_next):
+    """Pure-Python shot-aware window attention from coordinates: key j is
+    visible to query i iff both lie in the same spatial tile and j's frame is
+    in i's temporal window, or in the previous shot's last aug_prev frames
+    when i's window starts its shot, or in the next shot's first aug_next
+    frames when i's window ends its shot."""
+    T, Hg, Wg = grid
+    wt, wh, ww = window
+    s = list(shot_start)
+    N, H, E = q.shape
+
+    def coords(i):
+        t, rem = divmod(i, Hg * Wg)
+        hh, w = divmod(rem, Wg)
+        return t, hh, w
+
+    def visible(i, jj):
+        t, hh, w = coords(i)
+        t2, h2, w2 = coords(jj)
+        if h2 // wh != hh // wh or w2 // ww != w // ww:
+            return False
+        sh = max(n for n in range(len(s) - 1) if s[n] <= t)
+        step = wt if wt > 0 else s[sh + 1] - s[sh]
+        a = s[sh] + ((t - s[sh]) // step) * step
+        b = min(s[sh + 1], a + step)
+        if a <= t2 < b:
+            return True
+        if a == s[sh] and sh > 0 and max(s[sh - 1], s[sh] - aug_prev) <= t2 < s[sh]:
+            return True
+        if b == s[sh + 1] and sh + 1 < len(s) - 1 and s[sh + 1] <= t2 < min(s[sh + 2], s[sh + 1] + aug_next):
+            return True
+        return False
+
+    out = np.zeros((N, H, E))
+    for i in range(N):
+        keys = [jj for jj in range(N) if visible(i, jj)]
+        for h in range(H):
+            sc = [sum(float(q[i, h, c]) * float(k[jj, h, c]) for c in range(E)) / math.sqrt(E) for jj in keys]
+            mx = max(sc)
+            w = [math.exp(a - mx) for a in sc]
+            z = sum(w)
+            for c in range(E):
+                out[i, h, c] = sum(wj * float(v[jj, h, c]) for jj, wj in zip(keys, w)) / z
+    return out
+
+
 def _read_golden(name):
     sections, cur = {}, None
     env = {"e": math.e, "log": math.log, "__builtins__": {}}
@@ -344,10 +390,50 @@ def check_balance_stats(o):
     assert np.allclose(F, Fb) and np.allclose(P, Pb, atol=1e-14) and abs(b - 3 * np.sum(Fb * Pb)) < 1e-13
 
 
+def check_shot_stga(o):
+    rng = np.random.default_rng(21)
+    # brute force: temporal windows inside shots, augmented keys at the cuts
+    for grid, window, shots, aug in (((5, 3, 4), (2, 2, 3), [0, 2, 5], (1, 2)),
+                                     ((6, 2, 3), (0, 2, 2), [0, 1, 3, 6], (2, 2)),
+                                     ((7, 2, 2), (2, 1, 2), [0, 3, 4, 7], (2, 1))):
+        N = grid[0] * grid[1] * grid[2]
+        q, k, v = (rng.normal(size=(N, 2, 3)) for _ in range(3))
+        out = o.stga_shot_attention(q, k, v, *grid, window, shots, *aug)
+        assert np.allclose(out, _brute_shot_stga(q, k, v, grid, window, shots, *aug), rtol=0, atol=1e-12)
+    # one shot: plain STGA, whatever the augmentation
+    q, k, v = (rng.normal(size=(6 * 4 * 4, 2, 4)) for _ in range(3))
+    plain = o.stga_attention(q, k, v, 6, 4, 4, (3, 2, 2))
+    assert np.allclose(o.stga_shot_attention(q, k, v, 6, 4, 4, (3, 2, 2), [0, 6], 2, 2), plain, rtol=0, atol=1e-13)
+    # cuts on window boundaries and no augmentation: plain STGA again
+    assert np.allclose(o.stga_shot_attention(q, k, v, 6, 4, 4, (3, 2, 2), [0, 3, 6], 0, 0), plain, rtol=0,
+                       atol=1e-13)
+    # queries are not augmented: every token appears in exactly one query set,
+    # and key sets are query sets plus boundary frames only
+    pairs = o.shot_windows(9, 2, 2, (2, 2, 2), [0, 4, 9], 2, 2)
+    allq = np.sort(np.concatenate([a for a, _ in pairs]))
+    assert np.array_equal(allq, np.arange(36))
+    assert all(np.isin(a, b).all() for a, b in pairs)
+    # perturbations: the frame before the previous shot's last two is invisible
+    # to the next shot's first window; the last frame before the cut is visible
+    grid, shots = (8, 2, 2), [0, 4, 8]
+    q, k, v = (rng.normal(size=(32, 1, 4)) for _ in range(3))
+    base = o.stga_shot_attention(q, k, v, *grid, (0, 2, 2), shots, 2, 2)
+    first_win = np.arange(16, 32)                          # shot 1, frames 4..7, the only tile
+    k2, v2 = k.copy(), v.copy()
+    k2[4:8] += 3.0                                         # frame 1 (4 tokens) of shot 0
+    v2[4:8] -= 2.0
+    assert np.allclose(o.stga_shot_attention(q, k2, v2, *grid, (0, 2, 2), shots, 2, 2)[first_win],
+                       base[first_win], rtol=0, atol=0)
+    k3 = k.copy()
+    k3[12:16] += 3.0                                       # frame 3: shot 0's last frame
+    assert not np.allclose(o.stga_shot_attention(q, k3, v, *grid, (0, 2, 2), shots, 2, 2)[first_win],
+                           base[first_win])
+
+
 CHECKS = [check_route_closed_form, check_route_ties_and_M1, check_route_brute, check_counting_sort,
           check_full_attention_when_M1, check_group_equals_subset_attention, check_special_cases,
           check_brute_force_tiny, check_permutation_equivariance, check_stga, check_layer_combine,
-          check_golden, check_three_branch_mean, check_balance_stats]
+          check_golden, check_three_branch_mean, check_balance_stats, check_shot_stga]
 
 
 @pytest.mark.parametrize("check", CHECKS, ids=[c.__name__ for c in CHECKS])
@@ -402,6 +488,19 @@ def _windows_off_by_one(T, Hg, Wg, window):
     return _ORIG_WIN(T, Hg, Wg, (window[0], window[1], window[2] + 1))
 
 
+def _shot_aug_on_queries(T, Hg, Wg, window, shot_start, aug_prev=2, aug_next=2):
+    return [(b, b) for _, b in _ORIG_SHOT(T, Hg, Wg, window, shot_start, aug_prev, aug_next)]
+
+
+def _shot_aug_short(T, Hg, Wg, window, shot_start, aug_prev=2, aug_next=2):
+    return _ORIG_SHOT(T, Hg, Wg, window, shot_start, max(aug_prev - 1, 0), aug_next)
+
+
+def _shot_ignores_cuts(T, Hg, Wg, window, shot_start, aug_prev=2, aug_next=2):
+    return _ORIG_SHOT(T, Hg, Wg, window, [0, T], aug_prev, aug_next)
+
+
+_ORIG_SHOT = oracle.shot_windows
 _ORIG_GA = oracle.group_attention
 _ORIG_WIN = oracle.stga_windows
 _ORIG_ROUTE = oracle.route
@@ -415,6 +514,9 @@ MUTANTS = {
     "unstable_group_order": ("counting_sort", _unstable_sort),
     "gate_dropped": ("group_attention", _no_gate),
     "window_width_off_by_one": ("stga_windows", _windows_off_by_one),
+    "shot_augments_queries": ("shot_windows", _shot_aug_on_queries),
+    "shot_augmentation_short": ("shot_windows", _shot_aug_short),
+    "shot_cuts_ignored": ("shot_windows", _shot_ignores_cuts),
 }
 
 
