@@ -166,6 +166,34 @@ moga_status stga_window_attn(const void* q, const void* k, const void* v, int T,
                              const int* window, int H, int d_h, int accumulate, void* out, void* ws,
                              size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- shot-aware STGA
+ * stga_shot_attn: the STGA branch with shots ("Spatial-Temporal Group
+ * Attention (STGA)" section: frames of different shots are in distinct
+ * temporal groups; keys and values, not queries, are augmented with latent
+ * frames of the adjacent shots).  Reading taken:
+ *   - shot_start (DEVICE int32 [nshots + 1]): 0 = s_0 < s_1 < ... < s_nshots
+ *     = T; shot j holds latent frames [s_j, s_{j+1}).  Checked on the device:
+ *     a violation skips all work and moga_sync_status() reports
+ *     MOGA_ERR_DEVICE_CHECK.
+ *   - window (host int[3]) = (wt, wh, ww): temporal windows of wt frames tile
+ *     each shot from its first frame and are clipped at its last; wt = 0 makes
+ *     one temporal window per shot (the pages' Wan setting is (0, Hg/2, Wg/2),
+ *     a 2x2 spatial partition).  Spatial tiles as in stga_window_attn.
+ *   - the keys/values of a shot's first temporal window add the previous
+ *     shot's last aug_prev frames, those of its last temporal window the next
+ *     shot's first aug_next frames (each clipped to that shot), in the same
+ *     spatial tile; the pages' choice is aug_prev = aug_next = 2.
+ * accumulate = 0: out = out_scale * SA; accumulate = 1: out += out_scale * SA
+ * (the block's mean of branches).  q, k, v, out: bf16 [T*Hg*Wg, H, d_h].
+ * Workspace: stga_shot_attn_workspace_size(...) bytes (an upper bound that
+ * holds for every split of T frames into nshots shots).
+ */
+size_t stga_shot_attn_workspace_size(int T, int Hg, int Wg, const int* window, int nshots, int aug_prev,
+                                     int aug_next, int H, int d_h);
+moga_status stga_shot_attn(const void* q, const void* k, const void* v, int T, int Hg, int Wg, const int* window,
+                           const int32_t* shot_start, int nshots, int aug_prev, int aug_next, int H, int d_h,
+                           float out_scale, int accumulate, void* out, void* ws, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------- full layer
  * moga_layer: one visual attention block = moga_route, then moga_group_attn,
  * then (when window != NULL) stga_window_attn, combined as

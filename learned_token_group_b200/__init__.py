@@ -20,7 +20,7 @@ import torch
 
 __all__ = ["MogaError", "get_lib", "LIB_PATH", "HEADER_PATH", "route", "group_attn", "stga_window_attn",
            "moga_layer", "sync_status", "workspace", "MogaLayer", "exported_names", "kernel_launches",
-           "set_timing_events", "STAGES", "Pipeline"]
+           "set_timing_events", "STAGES", "Pipeline", "stga_shot_attn"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoga.so")
@@ -72,6 +72,8 @@ def get_lib():
         "moga_route_noalloc": (_I, [_P, _P, _P, _I, _I64, _I, _I, _P, _P, _P, _P, _P, _P]),
         "moga_set_timing_events": (_I, [_I, _P, _P]),
         "moga_debug_inject": (_I, [_I]),
+        "stga_shot_attn_workspace_size": (_SZ, [_I, _I, _I, _P, _I, _I, _I, _I, _I]),
+        "stga_shot_attn": (_I, [_P, _P, _P, _I, _I, _I, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _P, _SZ, _P]),
         "moga_pipe_create": (_I, [_I64, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I, ctypes.POINTER(_P)]),
         "moga_pipe_submit": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
         "moga_pipe_sync": (_I, [_P]),
@@ -240,6 +242,36 @@ def stga_window_attn(q, k, v, grid: Sequence[int], window: Sequence[int], accumu
                               _ptr(out), _ptr(ws), ws.numel(), _stream(q.device))
     _check(st, "stga_window_attn")
     return out
+
+
+def stga_shot_attn(q, k, v, grid: Sequence[int], window: Sequence[int], shot_start: torch.Tensor,
+                   aug_prev: int = 2, aug_next: int = 2, out_scale: float = 1.0, accumulate: bool = False,
+                   out=None, ws=None):
+    """Shot-aware STGA over a (T, Hg, Wg) grid (stga_shot_attn in moga.h).
+
+    shot_start: device int32 [nshots + 1] frame boundaries (0 ... T); window
+    (wt, wh, ww) with wt = 0 for one temporal window per shot.
+    """
+    lib = get_lib()
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _dev_tensor(t, n, torch.bfloat16)
+    _dev_tensor(shot_start, "shot_start", torch.int32)
+    N, H, d_h = q.shape
+    T, Hg, Wg = (int(g) for g in grid)
+    w3 = _int3(window)
+    nshots = shot_start.numel() - 1
+    if out is None:
+        if accumulate:
+            raise ValueError("accumulate=True needs an existing out tensor")
+        out = torch.empty_like(q)
+    if ws is None:
+        ws = workspace(lib.stga_shot_attn_workspace_size(T, Hg, Wg, w3, nshots, aug_prev, aug_next, H, d_h),
+                       q.device)
+    st = lib.stga_shot_attn(_ptr(q), _ptr(k), _ptr(v), T, Hg, Wg, w3, _ptr(shot_start), nshots, int(aug_prev),
+                            int(aug_next), H, d_h, float(out_scale), int(bool(accumulate)), _ptr(out), _ptr(ws),
+                            ws.numel(), _stream(q.device))
+    _check(st, "stga_shot_attn")
+    return out, ws
 
 
 class MogaLayer:

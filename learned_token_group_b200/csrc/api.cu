@@ -308,6 +308,36 @@ moga_status check_qkv(const void* q, const void* k, const void* v, const void* o
   return MOGA_OK;
 }
 
+// Shot windows: window table, query index list, key/value index list.
+struct ShotWs {
+  size_t wtab, qperm, kvperm, total;
+  int64_t cap;
+};
+ShotWs shot_ws(int T, int Hg, int Wg, const int* window, int nshots, int aug_prev, int aug_next) {
+  Carve c;
+  ShotWs w;
+  w.cap = shot_window_cap(T, Hg, Wg, window, nshots);
+  w.wtab = c.take(shot_table_ints(w.cap) * 4);
+  w.qperm = c.take((size_t)T * Hg * Wg * 4);
+  w.kvperm = c.take((size_t)shot_kv_cap(T, Hg, Wg, nshots, aug_prev, aug_next) * 4);
+  w.total = c.off;
+  return w;
+}
+
+moga_status check_shots(int T, int Hg, int Wg, const int* window, int nshots, int aug_prev, int aug_next,
+                        int64_t* N) {
+  if (!window || T < 1 || Hg < 1 || Wg < 1) return MOGA_ERR_INVALID_ARG;
+  if (window[0] < 0 || window[1] < 1 || window[2] < 1) return MOGA_ERR_INVALID_ARG;
+  if (nshots < 1 || nshots > T || aug_prev < 0 || aug_next < 0 || aug_prev > T || aug_next > T)
+    return MOGA_ERR_INVALID_ARG;
+  const int64_t n = (int64_t)T * Hg * Wg;
+  if (n >= (int64_t)1 << 31 || shot_kv_cap(T, Hg, Wg, nshots, aug_prev, aug_next) >= (int64_t)1 << 31 ||
+      (int64_t)shot_table_ints(shot_window_cap(T, Hg, Wg, window, nshots)) >= (int64_t)1 << 31)
+    return MOGA_ERR_UNSUPPORTED;
+  *N = n;
+  return MOGA_OK;
+}
+
 }  // namespace
 
 bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
@@ -457,6 +487,71 @@ moga_status stga_window_attn(const void* q, const void* k, const void* v, int T,
   DevCtx c;
   if (!make_ctx(&c, ws, stream)) return MOGA_ERR_CUDA;
   return stga_body(c, q, k, v, T, Hg, Wg, window, H, d_h, accumulate, out, (uint8_t*)ws);
+}
+
+size_t stga_shot_attn_workspace_size(int T, int Hg, int Wg, const int* window, int nshots, int aug_prev,
+                                     int aug_next, int H, int d_h) {
+  int64_t N = 0;
+  if (check_shots(T, Hg, Wg, window, nshots, aug_prev, aug_next, &N) != MOGA_OK) return 0;
+  if (check_attn_shape(N, H, d_h) != MOGA_OK) return 0;
+  return shot_ws(T, Hg, Wg, window, nshots, aug_prev, aug_next).total;
+}
+
+moga_status stga_shot_attn(const void* q, const void* k, const void* v, int T, int Hg, int Wg, const int* window,
+                           const int32_t* shot_start, int nshots, int aug_prev, int aug_next, int H, int d_h,
+                           float out_scale, int accumulate, void* out, void* ws, size_t ws_bytes, void* stream) {
+  moga_status st = check_qkv(q, k, v, out);
+  if (st != MOGA_OK) return st;
+  int64_t N = 0;
+  if ((st = check_shots(T, Hg, Wg, window, nshots, aug_prev, aug_next, &N)) != MOGA_OK) return st;
+  if ((st = check_attn_shape(N, H, d_h)) != MOGA_OK) return st;
+  if (!shot_start || !aligned4(shot_start) || (accumulate != 0 && accumulate != 1)) return MOGA_ERR_INVALID_ARG;
+  if (!(out_scale == out_scale)) return MOGA_ERR_INVALID_ARG;  // NaN
+  if (!ws || !aligned16(ws)) return MOGA_ERR_INVALID_ARG;
+  const ShotWs w = shot_ws(T, Hg, Wg, window, nshots, aug_prev, aug_next);
+  if (ws_bytes < w.total) return MOGA_ERR_WORKSPACE;
+  DevCtx c;
+  if (!make_ctx(&c, ws, stream)) return MOGA_ERR_CUDA;
+  uint8_t* wb = (uint8_t*)ws;
+  int32_t* wtab = reinterpret_cast<int32_t*>(wb + w.wtab);
+  int32_t* qperm = reinterpret_cast<int32_t*>(wb + w.qperm);
+  int32_t* kvperm = reinterpret_cast<int32_t*>(wb + w.kvperm);
+  mark(MOGA_STAGE_STGA_PREP, true, c.stream);
+  if (launch_shot_table(c, shot_start, nshots, T, Hg, Wg, window, aug_prev, aug_next, H, w.cap, wtab) !=
+      cudaSuccess)
+    return MOGA_ERR_CUDA;
+  if (launch_shot_perm(c, wtab, w.cap, Hg, Wg, window, qperm, kvperm) != cudaSuccess) return MOGA_ERR_CUDA;
+  count(2);
+  mark(MOGA_STAGE_STGA_PREP, false, c.stream);
+  AttnArgs a{};
+  a.direct = 1;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.perm = qperm;
+  a.kvperm = kvperm;
+  a.gate = nullptr;
+  a.out = out;
+  a.N = N;
+  a.H = H;
+  a.d_h = d_h;
+  a.out_scale = out_scale;
+  a.accumulate = accumulate;
+  a.mode = 2;
+  a.table = wtab;
+  a.nseg = (int)w.cap;
+  a.T = T;
+  a.Hg = Hg;
+  a.Wg = Wg;
+  a.wt = window[0];
+  a.wh = window[1];
+  a.ww = window[2];
+  a.debug_withhold_first_k = 0;
+  mark(MOGA_STAGE_STGA_ATTN, true, c.stream);
+  const cudaError_t e = launch_attention(c, a);
+  mark(MOGA_STAGE_STGA_ATTN, false, c.stream);
+  count(1);
+  return from_cuda(e);
 }
 
 size_t moga_layer_workspace_size(int64_t N, int H, int d_h, int M, int T, int Hg, int Wg, const int* window) {

@@ -187,9 +187,13 @@ struct Plan {
 // A work unit is a pair of consecutive 128-row query tiles (A, B) of one
 // (segment, head); both stream the same K/V tiles.
 struct Unit {
-  int h, start, len, q0;  // q0: first row of tile A inside the segment; tile B starts at q0 + 128
+  int h, start, len, q0;  // query segment; q0: first row of tile A in it (tile B starts at q0 + 128)
+  int kvs, kvl;           // key/value segment (the query segment except for shot windows)
 };
 
+// kShots: the decoder of the in-place kernel, which also serves shot windows
+// (mode 2); the tiled kernel never sees them and keeps the smaller decoder.
+template <bool kShots>
 struct Decoder {
   int mode;
   int nseg;
@@ -197,6 +201,8 @@ struct Decoder {
   WinGeom g;
   int upw;         // windows: units per window
   int H;           // windows read in place: heads vary fastest
+  const int* gtab; // shot windows: window table in device memory
+  int cap;         // shot windows: table capacity
   __device__ __forceinline__ Unit operator()(int idx) const {
     Unit u;
     if (mode == 0) {
@@ -211,7 +217,9 @@ struct Decoder {
       const int npair = ((u.len + kTile - 1) / kTile + 1) / 2;
       u.h = local / npair;
       u.q0 = (local - u.h * npair) * 2 * kTile;
-    } else {
+      u.kvs = u.start;
+      u.kvl = u.len;
+    } else if (!kShots || mode == 1) {
       // Units in place go window by window with the heads innermost, so the
       // CTAs running at once read whole token rows of q, k, v (all heads)
       // close together in time.  With a gathered head-major copy each head's
@@ -228,6 +236,25 @@ struct Decoder {
       }
       window_of(g, seg, u.start, u.len);
       u.q0 = qp * 2 * kTile;
+      u.kvs = u.start;
+      u.kvl = u.len;
+    } else {
+      // shot windows: binary search of the unit prefix in the global table
+      const int nwin = gtab[0];
+      const int* pre = gtab + kShotHdr;
+      int lo = 0, hi = nwin - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pre[mid] <= idx) lo = mid; else hi = mid - 1;
+      }
+      const int* e = gtab + kShotHdr + cap + 1 + (size_t)lo * kShotEnt;
+      const int local = idx - pre[lo];
+      u.start = e[0];
+      u.len = e[1];
+      u.kvs = e[2];
+      u.kvl = e[3];
+      u.h = local % H;
+      u.q0 = (local / H) * 2 * kTile;
     }
     return u;
   }
@@ -278,16 +305,18 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     *abort_flag = 0;
     fence_mbar_init();
   }
-  Decoder dec;
+  Decoder<kDirect> dec;
   dec.mode = a.mode;
   dec.nseg = a.nseg;
   dec.tab = tab;
   dec.upw = 1;
   dec.H = kDirect ? a.H : 0;
+  dec.gtab = a.table;
+  dec.cap = a.nseg;
   if (a.mode == 0) {
     const int n = 3 * a.nseg + 1;
     for (int i = threadIdx.x; i < n; i += blockDim.x) tab[i] = a.table[i];
-  } else {
+  } else if (a.mode == 1) {
     dec.g = WinGeom{a.T, a.Hg, a.Wg, a.wt, a.wh, a.ww, (a.Hg + a.wh - 1) / a.wh, (a.Wg + a.ww - 1) / a.ww};
     dec.upw = ((a.wt * a.wh * a.ww + kTile - 1) / kTile + 1) / 2;
   }
@@ -298,7 +327,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const int total = (a.mode == 0) ? tab[a.nseg] : a.nseg * dec.upw * a.H;
+  const int total = a.mode == 0 ? tab[a.nseg] : a.mode == 1 ? a.nseg * dec.upw * a.H : a.table[1];
   const uint32_t tmem = *tmem_slot;
   // TMEM columns: S/P of tile A [0,128), S/P of tile B [128,256), O of A [256,..), O of B [384,..).
   // P (bf16, two per column) overwrites the first 64 columns of its tile's S.
@@ -322,7 +351,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         const Unit u = dec(idx);
         if (u.q0 >= u.len) continue;
         const bool hb = u.q0 + kTile < u.len;
-        const int nkv = (u.len + kTile - 1) / kTile;
+        const int nkv = (u.kvl + kTile - 1) / kTile;
         if (!mbar_wait(q_empty, (ucnt & 1) ^ 1, wc, 1, ucnt)) break;
         const int rowq = (int)((int64_t)u.h * N + u.start + u.q0);
         mbar_expect_tx(q_full, (hb ? 2 : 1) * P::kTileBytes);
@@ -335,7 +364,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         }
         ++ucnt;
         for (int j = 0; j < nkv; ++j) {
-          const int rowk = (int)((int64_t)u.h * N + u.start + j * kTile);
+          const int rowk = (int)((int64_t)u.h * N + u.kvs + j * kTile);
           const int ks = kc % kStages;
           if (!mbar_wait(&k_empty[ks], ((kc / kStages) & 1) ^ 1, wc, 2, kc)) { ok = false; break; }
           if (a.debug_withhold_first_k && kc == 0) {
@@ -372,7 +401,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
   if (kDirect && warp != 1) {
     // ---------------------------------------------------------------- cp.async loaders (warps 0, 2, 3)
     // Q/K/V rows are copied straight from q, k, v [N, H, d_h] by token index
-    // (perm: segment position -> token), so no gathered copy is ever written.
+    // (perm / kvperm: segment position -> token), so no gathered copy is ever
+    // written.
     // Warp 0 copies Q_A and Q_B, warp 2 the K tiles and warp 3 the V tiles:
     // each lane moves 16-byte pieces with cp.async into the 128-byte swizzled
     // layout the MMA descriptors expect, waits for its pieces, fences them for
@@ -380,8 +410,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     // empty barrier thus has one waiter that follows its phases in order.
     // Three warps keep up to 128 KB in flight, which single-row TMA gathers
     // could not (their per-instruction cost capped an SM near 8 B/cycle).
-    // Positions past the segment end repeat its last token (masked later).
     const int li = warp == 0 ? 0 : warp - 1;  // 0: Q, 1: K, 2: V
+    const int32_t* kvperm = a.kvperm ? a.kvperm : a.perm;
     constexpr int kPieces = DH * 2 / 16;       // 16-byte pieces per row
     constexpr int kRowsPerOp = 32 / kPieces;   // rows one warp-wide copy covers
     const int piece = lane % kPieces, sub = lane / kPieces;
@@ -395,11 +425,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     // or -1 (zero-filled) for a token out of range or a row past the segment
     // end.  Read before the slot is free so that their latency overlaps the
     // wait.
-    auto fetch_rows = [&](int pos0, int seg_end, int h, int (&tr)[4]) {
+    auto fetch_rows = [&](const int32_t* idx, int pos0, int seg_end, int h, int (&tr)[4]) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int pp = pos0 + 4 * lane + i;
-        const int tok = a.perm[min(pp, seg_end - 1)];
+        const int tok = idx[min(pp, seg_end - 1)];
         tr[i] = (pp < seg_end && tok >= 0 && (int64_t)tok < N) ? tok * H + h : -1;
       }
     };
@@ -447,12 +477,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       const Unit u = dec(idx);
       if (u.q0 >= u.len) continue;
       const bool hb = u.q0 + kTile < u.len;
-      const int nkv = (u.len + kTile - 1) / kTile;
-      const int seg_end = u.start + u.len;
+      const int nkv = (u.kvl + kTile - 1) / kTile;
+      const int seg_end = u.start + u.len, kv_end = u.kvs + u.kvl;
       if (li == 0) {
         int ra[4], rb[4];
-        fetch_rows(u.start + u.q0, seg_end, u.h, ra);
-        if (hb) fetch_rows(u.start + u.q0 + kTile, seg_end, u.h, rb);
+        fetch_rows(a.perm, u.start + u.q0, seg_end, u.h, ra);
+        if (hb) fetch_rows(a.perm, u.start + u.q0 + kTile, seg_end, u.h, rb);
         if (!warp_wait(q_empty, (ucnt & 1) ^ 1, 1, ucnt)) { ok = false; break; }
         copy_tile(a.q, smem + P::kQA, ra, toks, u.len - u.q0);
         if (hb) copy_tile(a.q, smem + P::kQB, rb, toks + kTile, u.len - u.q0 - kTile);
@@ -465,7 +495,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       for (int j = 0; j < nkv; ++j, ++t) {
         int tr[4];
         const int s = t % kStages;
-        fetch_rows(u.start + j * kTile, seg_end, u.h, tr);
+        fetch_rows(kvperm, u.kvs + j * kTile, kv_end, u.h, tr);
         if (!warp_wait(is_v ? &v_empty[s] : &k_empty[s], ((t / kStages) & 1) ^ 1, is_v ? 3 : 2, t)) {
           ok = false;
           break;
@@ -474,7 +504,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         // bounded wait runs out and the kernel reports a timeout.
         if (!is_v && t == 0 && a.debug_withhold_first_k) { ok = false; break; }
         copy_tile(is_v ? a.v : a.k, smem + (is_v ? P::kV0 : P::kK0) + s * P::kTileBytes, tr, toks,
-                  u.len - j * kTile);
+                  u.kvl - j * kTile);
         finish();
         if (lane == 0) mbar_arrive(is_v ? &v_full[s] : &k_full[s]);
       }
@@ -511,7 +541,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         const Unit u = dec(idx);
         if (u.q0 >= u.len) continue;
         const bool hb = u.q0 + kTile < u.len;
-        const int nkv = (u.len + kTile - 1) / kTile;
+        const int nkv = (u.kvl + kTile - 1) / kTile;
         if (!mbar_wait(q_full, ucnt & 1, wc, 4, ucnt)) break;
         ++ucnt;
         int ks = kc % kStages;
@@ -586,7 +616,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       if (u.q0 >= u.len) continue;
       const bool hb = u.q0 + kTile < u.len;
       if (x == 1 && !hb) continue;
-      const int nkv = (u.len + kTile - 1) / kTile;
+      const int nkv = (u.kvl + kTile - 1) / kTile;
       // The output row of this thread's query is fetched now, so its latency
       // hides behind the key loop.
       const int r = u.q0 + x * kTile + row;
@@ -599,7 +629,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         ++sc;
         tc_fence_after();
         // The whole S row (128 fp32) is read from TMEM once.
-        const int valid = u.len - j * kTile;  // keys of this tile inside the segment
+        const int valid = u.kvl - j * kTile;  // keys of this tile inside the key/value segment
         float sr[kTile];
 #pragma unroll
         for (int c = 0; c < kTile / 32; ++c) tmem_ld32(tSx + c * 32, sr + c * 32);

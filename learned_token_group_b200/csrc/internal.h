@@ -59,7 +59,8 @@ struct AttnArgs {
   const void* q;
   const void* k;
   const void* v;
-  const int32_t* perm;    // segment position -> original token
+  const int32_t* perm;    // segment position -> original token (queries; also keys/values unless kvperm)
+  const int32_t* kvperm;  // mode 2: key/value position -> original token
   const float* gate;      // per original token, or null (gate = 1)
   void* out;              // bf16 [N, H, d_h]
   int64_t N;
@@ -67,14 +68,43 @@ struct AttnArgs {
   int d_h;
   float out_scale;
   int accumulate;         // 0: out = scale*gate*O ; 1: out += scale*O
-  // segment source: groups (sorted table in device memory) or STGA windows
-  int mode;               // 0 groups, 1 windows
-  const int32_t* table;   // groups: [3*(M+1)] = tile_prefix | seg_start | seg_len (sorted)
-  int nseg;               // groups: M ; windows: number of windows
+  // segment source: groups (sorted table in device memory), STGA windows
+  // (decoded from the grid), or shot windows (mode 2: a window table in
+  // device memory whose key/value segments differ from the query segments;
+  // read in place only)
+  int mode;               // 0 groups, 1 windows, 2 shot windows
+  const int32_t* table;   // groups: [3*(M+1)] = tile_prefix | seg_start | seg_len (sorted); mode 2: window table
+  int nseg;               // groups: M ; windows: number of windows ; mode 2: table capacity (windows)
   int T, Hg, Wg, wt, wh, ww;
   int debug_withhold_first_k;  // test hook: the producer skips each CTA's first K tile
 };
 cudaError_t launch_attention(const DevCtx& c, const AttnArgs& a);
+
+// ------------------------------------------------------------------ shot windows
+// Window table of shot-aware STGA (int32, device):
+//   [0] windows, [1] work units (query-tile pairs x heads), [2] key/value rows, [3] spare,
+//   [4, 4 + cap + 1)   unit prefix per window,
+//   then cap entries of kShotEnt ints: q_start, q_len, kv_start, kv_len,
+//   t0, t1 (own frames), pf0, pf1 (previous shot's frames), nf0, nf1 (next
+//   shot's frames), tile row, tile column.
+constexpr int kShotHdr = 4;
+constexpr int kShotEnt = 12;
+inline size_t shot_table_ints(int64_t cap) { return (size_t)(kShotHdr + cap + 1 + kShotEnt * cap); }
+// Upper bound on the number of windows of any shot split of T frames into nshots shots.
+inline int64_t shot_window_cap(int T, int Hg, int Wg, const int* w, int nshots) {
+  const int64_t tw = w[0] > 0 ? ((int64_t)T + (int64_t)nshots * (w[0] - 1)) / w[0] : nshots;
+  return tw * ceil_div(Hg, w[1]) * ceil_div(Wg, w[2]);
+}
+// Upper bound on key/value rows: every token once plus the boundary frames of each cut.
+inline int64_t shot_kv_cap(int T, int Hg, int Wg, int nshots, int aug_prev, int aug_next) {
+  return (int64_t)T * Hg * Wg + (int64_t)(nshots - 1) * (aug_prev + aug_next) * Hg * Wg;
+}
+// Builds the window table from the device shot boundaries (checked on the device).
+cudaError_t launch_shot_table(const DevCtx& c, const int32_t* shot_start, int nshots, int T, int Hg, int Wg,
+                              const int* window, int aug_prev, int aug_next, int H, int64_t cap, int32_t* wtab);
+// Query and key/value index lists of every window of the table.
+cudaError_t launch_shot_perm(const DevCtx& c, const int32_t* wtab, int64_t cap, int Hg, int Wg, const int* window,
+                             int32_t* qperm, int32_t* kvperm);
 
 // Number of STGA windows for a grid.
 inline int64_t stga_num_windows(int T, int Hg, int Wg, const int* w) {

@@ -166,3 +166,38 @@ def test_pipe_validation(lib):
     assert lib.moga_pipe_submit(None, P, P, None, P, P, P, P, None, None) == INVALID
     assert lib.moga_pipe_sync(None) == INVALID
     assert lib.moga_pipe_destroy(None) == OK
+
+
+def test_shot_attn_validation(lib):
+    w = (ctypes.c_int * 3)(0, 15, 26)
+    f = lib.stga_shot_attn
+    args = [P, P, P, 20, 30, 52, w, P, 4, 2, 2, 2, 128, 1.0, 0, P, P, BIG, None]
+    bad = list(args)
+    bad[8] = 0                                        # no shots
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[8] = 21                                       # more shots than frames
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[9] = -1                                       # negative augmentation
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[7] = None                                     # shot boundaries missing
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[14] = 2                                       # accumulate must be 0 or 1
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[12] = 96
+    assert f(*bad) == UNSUPPORTED
+    w_bad = (ctypes.c_int * 3)(1, 0, 26)
+    bad = list(args)
+    bad[6] = w_bad
+    assert f(*bad) == INVALID
+    small = list(args)
+    small[17] = 4096
+    assert f(*small) == WORKSPACE
+    n1 = lib.stga_shot_attn_workspace_size(20, 30, 52, w, 4, 2, 2, 2, 128)
+    n2 = lib.stga_shot_attn_workspace_size(20, 30, 52, w, 8, 2, 2, 2, 128)
+    assert 0 < n1 < n2
+    assert lib.stga_shot_attn_workspace_size(20, 30, 52, w, 0, 2, 2, 2, 128) == 0
