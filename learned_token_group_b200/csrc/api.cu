@@ -308,18 +308,38 @@ moga_status check_qkv(const void* q, const void* k, const void* v, const void* o
   return MOGA_OK;
 }
 
-// Shot windows: window table, query index list, key/value index list.
+// Shot windows whose key/value segments span at most four tiles are read in
+// place; longer ones (the pages' whole-shot windows) stream each K/V tile for
+// many query tiles and read gathered head-major copies with tiled loads.
+bool shot_direct(int T, int Hg, int Wg, const int* w, int nshots, int aug_prev, int aug_next) {
+  const int64_t frames = (int64_t)(w[0] > 0 ? w[0] : T - nshots + 1) + aug_prev + aug_next;
+  const int64_t area = (int64_t)(w[1] < Hg ? w[1] : Hg) * (w[2] < Wg ? w[2] : Wg);
+  return frames * area <= 4 * kTile;
+}
+
+// Shot windows: window table, query index list, key/value index list, and
+// (tiled) the gathered copies of Q (N rows per head) and K/V (kv_cap rows).
 struct ShotWs {
-  size_t wtab, qperm, kvperm, total;
-  int64_t cap;
+  size_t wtab, qperm, kvperm, qh, kh, vh, total;
+  int64_t cap, kv_cap;
+  bool direct;
 };
-ShotWs shot_ws(int T, int Hg, int Wg, const int* window, int nshots, int aug_prev, int aug_next) {
+ShotWs shot_ws(int T, int Hg, int Wg, const int* window, int nshots, int aug_prev, int aug_next, int H, int d_h) {
   Carve c;
   ShotWs w;
+  const int64_t N = (int64_t)T * Hg * Wg;
   w.cap = shot_window_cap(T, Hg, Wg, window, nshots);
+  w.kv_cap = shot_kv_cap(T, Hg, Wg, nshots, aug_prev, aug_next);
+  w.direct = shot_direct(T, Hg, Wg, window, nshots, aug_prev, aug_next);
   w.wtab = c.take(shot_table_ints(w.cap) * 4);
-  w.qperm = c.take((size_t)T * Hg * Wg * 4);
-  w.kvperm = c.take((size_t)shot_kv_cap(T, Hg, Wg, nshots, aug_prev, aug_next) * 4);
+  w.qperm = c.take((size_t)N * 4);
+  w.kvperm = c.take((size_t)w.kv_cap * 4);
+  w.qh = w.kh = w.vh = 0;
+  if (!w.direct) {
+    w.qh = c.take((size_t)N * H * d_h * 2);
+    w.kh = c.take((size_t)w.kv_cap * H * d_h * 2);
+    w.vh = c.take((size_t)w.kv_cap * H * d_h * 2);
+  }
   w.total = c.off;
   return w;
 }
@@ -331,7 +351,7 @@ moga_status check_shots(int T, int Hg, int Wg, const int* window, int nshots, in
   if (nshots < 1 || nshots > T || aug_prev < 0 || aug_next < 0 || aug_prev > T || aug_next > T)
     return MOGA_ERR_INVALID_ARG;
   const int64_t n = (int64_t)T * Hg * Wg;
-  if (n >= (int64_t)1 << 31 || shot_kv_cap(T, Hg, Wg, nshots, aug_prev, aug_next) >= (int64_t)1 << 31 ||
+  if (n >= (int64_t)1 << 31 || shot_kv_cap(T, Hg, Wg, nshots, aug_prev, aug_next) >= (int64_t)1 << 30 ||
       (int64_t)shot_table_ints(shot_window_cap(T, Hg, Wg, window, nshots)) >= (int64_t)1 << 31)
     return MOGA_ERR_UNSUPPORTED;
   *N = n;
@@ -494,7 +514,7 @@ size_t stga_shot_attn_workspace_size(int T, int Hg, int Wg, const int* window, i
   int64_t N = 0;
   if (check_shots(T, Hg, Wg, window, nshots, aug_prev, aug_next, &N) != MOGA_OK) return 0;
   if (check_attn_shape(N, H, d_h) != MOGA_OK) return 0;
-  return shot_ws(T, Hg, Wg, window, nshots, aug_prev, aug_next).total;
+  return shot_ws(T, Hg, Wg, window, nshots, aug_prev, aug_next, H, d_h).total;
 }
 
 moga_status stga_shot_attn(const void* q, const void* k, const void* v, int T, int Hg, int Wg, const int* window,
@@ -508,7 +528,9 @@ moga_status stga_shot_attn(const void* q, const void* k, const void* v, int T, i
   if (!shot_start || !aligned4(shot_start) || (accumulate != 0 && accumulate != 1)) return MOGA_ERR_INVALID_ARG;
   if (!(out_scale == out_scale)) return MOGA_ERR_INVALID_ARG;  // NaN
   if (!ws || !aligned16(ws)) return MOGA_ERR_INVALID_ARG;
-  const ShotWs w = shot_ws(T, Hg, Wg, window, nshots, aug_prev, aug_next);
+  if ((int64_t)shot_kv_cap(T, Hg, Wg, nshots, aug_prev, aug_next) * H >= (int64_t)1 << 31)
+    return MOGA_ERR_UNSUPPORTED;
+  const ShotWs w = shot_ws(T, Hg, Wg, window, nshots, aug_prev, aug_next, H, d_h);
   if (ws_bytes < w.total) return MOGA_ERR_WORKSPACE;
   DevCtx c;
   if (!make_ctx(&c, ws, stream)) return MOGA_ERR_CUDA;
@@ -522,12 +544,24 @@ moga_status stga_shot_attn(const void* q, const void* k, const void* v, int T, i
     return MOGA_ERR_CUDA;
   if (launch_shot_perm(c, wtab, w.cap, Hg, Wg, window, qperm, kvperm) != cudaSuccess) return MOGA_ERR_CUDA;
   count(2);
-  mark(MOGA_STAGE_STGA_PREP, false, c.stream);
   AttnArgs a{};
-  a.direct = 1;
+  a.direct = w.direct ? 1 : 0;
   a.q = q;
   a.k = k;
   a.v = v;
+  if (!w.direct) {
+    // queries: every token once; keys/values: the device-computed count of rows
+    if (launch_gather_rows(c, q, nullptr, qperm, nullptr, N, N, H, d_h, N, wb + w.qh, nullptr) != cudaSuccess ||
+        launch_gather_rows(c, k, v, kvperm, wtab + 2, w.kv_cap, N, H, d_h, w.kv_cap, wb + w.kh, wb + w.vh) !=
+            cudaSuccess)
+      return MOGA_ERR_CUDA;
+    count(2);
+    a.q = wb + w.qh;
+    a.k = wb + w.kh;
+    a.v = wb + w.vh;
+    a.kv_rows = w.kv_cap;
+  }
+  mark(MOGA_STAGE_STGA_PREP, false, c.stream);
   a.perm = qperm;
   a.kvperm = kvperm;
   a.gate = nullptr;

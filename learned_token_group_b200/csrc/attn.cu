@@ -92,6 +92,46 @@ gather_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k, const ui
   }
 }
 
+// da[h][j] = a[idx[j]][h] (and db from b when given) for j < rows, where rows
+// is *rows_dev when given (a count the device computed) else rows_max; the
+// destinations are head-major with a per-head row stride.  Used for the
+// query and key/value lists of shot windows, whose lengths differ.
+__global__ void __launch_bounds__(256)
+gather_rows_kernel(const uint4* __restrict__ a, const uint4* __restrict__ b, const int32_t* __restrict__ idx,
+                   const int32_t* __restrict__ rows_dev, int64_t rows_max, int64_t N, int H, int vph,
+                   int64_t stride, uint4* __restrict__ da, uint4* __restrict__ db, int* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t w0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t rows = rows_dev ? min((int64_t)*rows_dev, rows_max) : rows_max;
+  const int vpr = H * vph;
+  for (int64_t j = w0; j < rows; j += nw) {
+    const int64_t src = idx[j];
+    if (src < 0 || src >= N) {
+      if (lane == 0 && status) atomicOr(status, DEV_RANGE);
+      continue;
+    }
+#pragma unroll 2
+    for (int u = lane; u < vpr; u += 32) {
+      const int h = u / vph, c = u - h * vph;
+      const int64_t dst = ((int64_t)h * stride + j) * vph + c;
+      da[dst] = ldg_stream(a + src * vpr + u);
+      if (b) db[dst] = ldg_stream(b + src * vpr + u);
+    }
+  }
+  // The last tile of the last segment may read up to a tile past `rows`:
+  // those rows are zeroed so that every value the tensor core reads is finite.
+  const int64_t tail = min(rows + kTile, rows_max);
+  for (int64_t j = rows + w0; j < tail; j += nw) {
+    for (int u = lane; u < vpr; u += 32) {
+      const int h = u / vph, c = u - h * vph;
+      const int64_t dst = ((int64_t)h * stride + j) * vph + c;
+      da[dst] = make_uint4(0, 0, 0, 0);
+      if (b) db[dst] = make_uint4(0, 0, 0, 0);
+    }
+  }
+}
+
 struct WinGeom {
   int T, Hg, Wg, wt, wh, ww, nbh, nbw;
 };
@@ -200,7 +240,8 @@ struct Decoder {
   const int* tab;  // groups: shared copy of [unit_prefix (M+1) | seg_start (M) | seg_len (M)]
   WinGeom g;
   int upw;         // windows: units per window
-  int H;           // windows read in place: heads vary fastest
+  int H;           // windows read in place: heads vary fastest (0: heads outermost)
+  int heads;       // shot windows: number of heads (heads vary fastest)
   const int* gtab; // shot windows: window table in device memory
   int cap;         // shot windows: table capacity
   __device__ __forceinline__ Unit operator()(int idx) const {
@@ -253,8 +294,8 @@ struct Decoder {
       u.len = e[1];
       u.kvs = e[2];
       u.kvl = e[3];
-      u.h = local % H;
-      u.q0 = (local / H) * 2 * kTile;
+      u.h = local % heads;
+      u.q0 = (local / heads) * 2 * kTile;
     }
     return u;
   }
@@ -262,7 +303,9 @@ struct Decoder {
 
 // kDirect: copy Q/K/V rows straight from q, k, v by token index (cp.async);
 // otherwise 128-row tiles of a gathered head-major copy (2-D tiled TMA).
-template <int DH, bool kDirect>
+// kShots: the unit decoder also reads shot-window tables (mode 2); the
+// grouped-attention instantiation leaves it out.
+template <int DH, bool kDirect, bool kShots>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
             const __grid_constant__ CUtensorMap tv, const AttnArgs a, int* status, unsigned long long wait_ns) {
@@ -305,12 +348,13 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     *abort_flag = 0;
     fence_mbar_init();
   }
-  Decoder<kDirect> dec;
+  Decoder<kShots> dec;
   dec.mode = a.mode;
   dec.nseg = a.nseg;
   dec.tab = tab;
   dec.upw = 1;
   dec.H = kDirect ? a.H : 0;
+  dec.heads = a.H;
   dec.gtab = a.table;
   dec.cap = a.nseg;
   if (a.mode == 0) {
@@ -335,6 +379,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
   auto tO = [tmem](int x) { return tmem + 256u + (uint32_t)(x * 128); };
   WaitCtx wc{abort_flag, status, wait_ns};
   const int64_t N = a.N;
+  const int64_t kv_rows = a.kv_rows > 0 ? a.kv_rows : N;  // per-head rows of the K/V copies
 
   if (warp < 4) {
   regs_dec<kRegsCtl>();
@@ -364,7 +409,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         }
         ++ucnt;
         for (int j = 0; j < nkv; ++j) {
-          const int rowk = (int)((int64_t)u.h * N + u.kvs + j * kTile);
+          const int rowk = (int)((int64_t)u.h * kv_rows + u.kvs + j * kTile);
           const int ks = kc % kStages;
           if (!mbar_wait(&k_empty[ks], ((kc / kStages) & 1) ^ 1, wc, 2, kc)) { ok = false; break; }
           if (a.debug_withhold_first_k && kc == 0) {
@@ -621,6 +666,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       // hides behind the key loop.
       const int r = u.q0 + x * kTile + row;
       bool live = r < u.len;
+      if (live && (u.h < 0 || u.h >= a.H || u.start < 0 || (int64_t)u.start + r >= N)) {  // outside the tensors
+        live = false;
+        if (status) atomicOr(status, DEV_RANGE);
+      }
       const int src = live ? a.perm[u.start + r] : 0;
       float m_run = -INFINITY;
       uint64_t la = f2_pack(0.f, 0.f), lb = la, lc = la, ld = la;  // row sum of P, 8 partial sums
@@ -773,16 +822,19 @@ cudaError_t launch_attention_dh(const DevCtx& c, const AttnArgs& a) {
   using P = Plan<DH>;
   CUtensorMap mq, mk, mv;
   const uint64_t rows = (uint64_t)a.N * (uint64_t)a.H;
-  // tiled: the gathered copy [H*N rows, d_h] with 128-row boxes.  The
-  // in-place kernel copies rows itself and does not read the maps.
+  const uint64_t kv_rows = (uint64_t)(a.kv_rows > 0 ? a.kv_rows : a.N) * (uint64_t)a.H;
+  // tiled: the gathered copies, Q [H*N rows, d_h] and K/V [H*kv_rows, d_h],
+  // with 128-row boxes.  The in-place kernel copies rows itself and does not
+  // read the maps.
   const uint32_t box_rows = (uint32_t)kTile;
   if (!make_tmap_2d(&mq, a.q, DH, rows, DH * 2, box_rows)) return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&mk, a.k, DH, rows, DH * 2, box_rows)) return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&mv, a.v, DH, rows, DH * 2, box_rows)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&mk, a.k, DH, kv_rows, DH * 2, box_rows)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&mv, a.v, DH, kv_rows, DH * 2, box_rows)) return cudaErrorInvalidValue;
   // groups: the segment table; in place: the loaders' token rows (2 tiles each)
   const int table_ints = a.mode == 0 ? 3 * a.nseg + 1 : (a.direct ? 6 * kTile : 0);
   const size_t smem = P::bytes(table_ints);
-  auto kern = a.direct ? attn_kernel<DH, true> : attn_kernel<DH, false>;
+  auto kern = a.direct ? attn_kernel<DH, true, true>
+                       : (a.mode == 2 ? attn_kernel<DH, false, true> : attn_kernel<DH, false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int grid = c.num_sms;
@@ -807,6 +859,19 @@ cudaError_t launch_gather(const DevCtx& c, const void* q, const void* k, const v
   if (blocks > cap) blocks = cap;
   gather_kernel<<<(unsigned)blocks, 256, 0, c.stream>>>((const uint4*)q, (const uint4*)k, (const uint4*)v, perm, N,
                                                          H, vph, (uint4*)qh, (uint4*)kh, (uint4*)vh, c.status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const DevCtx& c, const void* a, const void* b, const int32_t* idx,
+                               const int32_t* rows_dev, int64_t rows_max, int64_t N, int H, int d_h, int64_t stride,
+                               void* da, void* db) {
+  if (rows_max == 0) return cudaSuccess;
+  int64_t blocks = ceil_div(rows_max, 8);
+  const int64_t cap = (int64_t)c.num_sms * 8;
+  if (blocks > cap) blocks = cap;
+  gather_rows_kernel<<<(unsigned)blocks, 256, 0, c.stream>>>((const uint4*)a, (const uint4*)b, idx, rows_dev,
+                                                             rows_max, N, H, d_h / 8, stride, (uint4*)da,
+                                                             (uint4*)db, c.status);
   return cudaGetLastError();
 }
 

@@ -52,6 +52,12 @@ cudaError_t launch_seg_table(const DevCtx& c, const int32_t* offsets, int M, int
 cudaError_t launch_gather(const DevCtx& c, const void* q, const void* k, const void* v, const int32_t* perm,
                           int64_t N, int H, int d_h, void* qh, void* kh, void* vh);
 
+// Rows idx[0..rows) of a (and b) gathered head-major into da (db) with a
+// per-head row stride; rows = *rows_dev when given, else rows_max.
+cudaError_t launch_gather_rows(const DevCtx& c, const void* a, const void* b, const int32_t* idx,
+                               const int32_t* rows_dev, int64_t rows_max, int64_t N, int H, int d_h, int64_t stride,
+                               void* da, void* db);
+
 struct AttnArgs {
   // direct = 1: q, k, v are the caller's [N, H, d_h] tensors, read by token
   // index (perm); direct = 0: they are gathered head-major copies [H][N][d_h].
@@ -64,6 +70,7 @@ struct AttnArgs {
   const float* gate;      // per original token, or null (gate = 1)
   void* out;              // bf16 [N, H, d_h]
   int64_t N;
+  int64_t kv_rows;        // tiled mode 2: per-head rows of the K/V copies (0: N)
   int H;
   int d_h;
   float out_scale;

@@ -67,15 +67,17 @@ def test_shot_stga_accumulate_and_scale():
     compare_out(out, ref)
 
 
-def test_one_shot_equals_plain_stga():
+@pytest.mark.parametrize("window,plain", [((3, 8, 8), (3, 8, 8)),       # read in place on both sides
+                                          ((0, 30, 52), (6, 30, 52))])   # gathered copies, tiled loads
+def test_one_shot_equals_plain_stga(window, plain):
     """With a single shot there is nothing to augment: the result is the
     plain STGA branch (same window order, same tiles)."""
-    grid, window = (6, 30, 52), (3, 8, 8)
+    grid = (6, 30, 52)
     q, k, v = _qkv(9360, 2, 128, seed=9)
     ss = torch.tensor([0, 6], dtype=torch.int32, device="cuda")
     a, ws = moga.stga_shot_attn(q, k, v, grid, window, ss, 2, 2)
     moga.sync_status(ws)
-    b = moga.stga_window_attn(q, k, v, grid, window)
+    b = moga.stga_window_attn(q, k, v, grid, plain)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
 
