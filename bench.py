@@ -204,6 +204,36 @@ def _recorded_traffic(name):
     return None
 
 
+def _shot_split(T: int):
+    """A fixed, uneven split of T latent frames into shots (fractions of a
+    120-frame video cut at frames 24, 40, 60, 88 and 100)."""
+    cuts = sorted({int(round(T * f)) for f in (0.2, 1 / 3, 0.5, 11 / 15, 5 / 6)} - {0, T})
+    return [0] + cuts + [T]
+
+
+def _shot_flops(wl, window, shots, aug_prev, aug_next):
+    """Useful FLOPs 4 * sum over windows of q_len * kv_len * d_h * H
+    (window geometry only: frames x tile area, per shot)."""
+    T, Hg, Wg = wl.grid
+    wt, wh, ww = window
+    total = 0
+    for j in range(len(shots) - 1):
+        a, b = shots[j], shots[j + 1]
+        step = wt if wt > 0 else b - a
+        for t0 in range(a, b, step):
+            t1 = min(b, t0 + step)
+            extra = 0
+            if t0 == a and j > 0:
+                extra += a - max(shots[j - 1], a - aug_prev)
+            if t1 == b and j + 1 < len(shots) - 1:
+                extra += min(shots[j + 2], b + aug_next) - b
+            for h0 in range(0, Hg, wh):
+                for w0 in range(0, Wg, ww):
+                    area = (min(Hg, h0 + wh) - h0) * (min(Wg, w0 + ww) - w0)
+                    total += (t1 - t0) * area * (t1 - t0 + extra) * area
+    return 4.0 * total * wl.d_h * wl.H
+
+
 def _blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -392,6 +422,26 @@ def run_ours(args, wl, rank, world, dist):
             ev1.record(stream)
             torch.cuda.synchronize()
             widened[name] = ev0.elapsed_time(ev1) / args.steps
+        # shot-aware STGA over a fixed split of the latent frames into shots:
+        # the pages' 2x2 spatial partition with whole-shot temporal groups, and
+        # the workload's window inside shots; two boundary frames each way
+        shots = _shot_split(wl.grid[0])
+        ss = torch.tensor(shots, dtype=torch.int32, device=dev)
+        half = (0, (wl.grid[1] + 1) // 2, (wl.grid[2] + 1) // 2)
+        for tag, win in (("shot_stga_2x2_whole_shot", half), ("shot_stga_window", tuple(wl.window))):
+            out_s, ws_s = moga.stga_shot_attn(inp["q"], inp["k"], inp["v"], wl.grid, win, ss, 2, 2)
+            torch.cuda.synchronize()
+            ev0.record(stream)
+            for _ in range(args.steps):
+                moga.stga_shot_attn(inp["q"], inp["k"], inp["v"], wl.grid, win, ss, 2, 2, out=out_s, ws=ws_s)
+            ev1.record(stream)
+            torch.cuda.synchronize()
+            moga.sync_status(ws_s)
+            ms_s = ev0.elapsed_time(ev1) / args.steps
+            widened[tag + "_ms"] = ms_s
+            widened[tag + "_tflops"] = _shot_flops(wl, win, shots, 2, 2) / (ms_s * 1e-3) / 1e12
+            del out_s, ws_s
+        widened["shot_split"] = shots
     if rank != 0:
         return
     peaks = _peaks()
