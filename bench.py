@@ -278,6 +278,55 @@ def max_over_ranks(value: float, dist, device=None) -> float:
     return float(t.item())
 
 
+def measure_context(moga, wl, steps, seed, dev, dist):
+    """One more workload of the metric: layer time over `steps` steps (device
+    events, max over ranks), then one pass with per-stage events, reduced to
+    grouped-attention TFLOP/s and router / gather bandwidth."""
+    inp = make_inputs(wl, seed=seed, device=dev)
+    xdt = torch.float32 if wl.x_dtype == "f32" else torch.bfloat16
+    layer = moga.MogaLayer(wl.N, wl.d, wl.H, wl.d_h, wl.M, wl.grid, wl.window, xdt, dev)
+    step = lambda: layer(inp["x"], inp["W_r"], inp["b_r"], inp["q"], inp["k"], inp["v"])
+    step()
+    moga.sync_status(layer.ws)
+    stream = torch.cuda.current_stream(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / steps, dist, dev)
+    stages = list(moga.STAGES)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in stages]
+    for b_ev, e_ev in evs:
+        b_ev.record(stream)
+        e_ev.record(stream)
+    torch.cuda.synchronize()
+    for s_i, name in enumerate(stages):
+        moga.set_timing_events(name, *evs[s_i])
+    step()
+    for name in stages:
+        moga.set_timing_events(name, None, None)
+    torch.cuda.synchronize()
+    moga.sync_status(layer.ws)
+    st = {name: evs[s_i][0].elapsed_time(evs[s_i][1]) for s_i, name in enumerate(stages)}
+    counts = np.diff(layer.offsets.cpu().numpy().astype(np.int64))
+    flops = 4.0 * float((counts.astype(np.float64) ** 2).sum()) * wl.d_h * wl.H
+    peaks = _peaks()
+    tf = flops / (st["group_attn"] * 1e-3) / 1e12
+    xb = wl.N * wl.d * (2 if wl.x_dtype == "bf16" else 4) + 8 * wl.N
+    gb = 6 * wl.N * wl.H * wl.d_h * 2 + 4 * wl.N
+    out = {"workload": wl.describe(), "steps": steps, "ms_per_step": ms, "tokens_per_s": wl.N / (ms * 1e-3),
+           "stage_ms": st, "group_attn_tflops": tf, "group_attn_frac_of_peak": tf / peaks["bf16_tflops"],
+           "router_GBs": xb / (st["router"] * 1e-3) / 1e9, "gather_GBs": gb / (st["gather"] * 1e-3) / 1e9,
+           "largest_group": int(counts.max()), "nonempty_groups": int((counts > 0).sum())}
+    out["router_frac_of_hbm"] = out["router_GBs"] / peaks["hbm_gbs"]
+    out["gather_frac_of_hbm"] = out["gather_GBs"] / peaks["hbm_gbs"]
+    del layer, inp
+    return out
+
+
 def run_ours(args, wl, rank, world, dist):
     import learned_token_group_b200 as moga
 
@@ -442,6 +491,13 @@ def run_ours(args, wl, rank, world, dist):
             widened[tag + "_tflops"] = _shot_flops(wl, win, shots, 2, 2) / (ms_s * 1e-3) / 1e12
             del out_s, ws_s
         widened["shot_split"] = shots
+    # ---- the other contexts the metric names: the same block at 580k tokens
+    # (40 heads, M = 32) and the skewed-routing stress case
+    contexts = {}
+    if wl.name == DEFAULT_CONFIG and not args.no_extras:
+        for name, steps in (("minute_580k", 2), ("skew_187k", 5)):
+            contexts[name] = measure_context(moga, WORKLOADS[name], steps, args.seed + rank, dev, dist)
+            torch.cuda.empty_cache()
     if rank != 0:
         return
     peaks = _peaks()
@@ -491,6 +547,7 @@ def run_ours(args, wl, rank, world, dist):
         "gpu_launches": int(launches),
         "clocks": clocks,
         "widened": widened,
+        "contexts": contexts,
     }
     print(json.dumps(line), flush=True)
 

@@ -26,6 +26,15 @@ namespace {
 constexpr int kRouteThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int kRouteMaxMPad = 256;
 
+// 64-column chunks of x per ring stage: a stage loads kRouteChunks adjacent
+// 128-byte pieces of each of its 128 rows back to back, so DRAM sees
+// kRouteChunks * 128 contiguous bytes per row (long rows of large d models
+// otherwise arrive as scattered 128-byte pieces).
+#ifndef MOGA_ROUTE_CHUNKS
+#define MOGA_ROUTE_CHUNKS 2
+#endif
+constexpr int kRouteChunks = MOGA_ROUTE_CHUNKS;
+
 struct RouteSmemPlan {
   int mpad, stages, stage_bytes, x_bytes, w_bytes;
   size_t total;
@@ -35,8 +44,8 @@ inline RouteSmemPlan route_plan(int M) {
   RouteSmemPlan p;
   p.mpad = (int)align_up((size_t)M, 16);
   if (p.mpad < 16) p.mpad = 16;
-  p.x_bytes = kTile * 128;
-  p.w_bytes = p.mpad * 128;
+  p.x_bytes = kTile * 128 * kRouteChunks;
+  p.w_bytes = p.mpad * 128 * kRouteChunks;
   p.stage_bytes = p.x_bytes + p.w_bytes;
   p.stages = (int)((200 * 1024) / p.stage_bytes);
   if (p.stages > 8) p.stages = 8;
@@ -78,8 +87,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = (N + kTile - 1) / kTile;
-  const int nk = (d + 63) / 64;
-  const uint32_t x_bytes = kTile * 128, w_bytes = (uint32_t)mpad * 128;
+  const int nk = (d + 64 * kRouteChunks - 1) / (64 * kRouteChunks);  // ring stages per tile
+  const uint32_t x_bytes = kTile * 128 * kRouteChunks, w_bytes = (uint32_t)mpad * 128 * kRouteChunks;
   uint32_t ncols = 32;
   while (ncols < (uint32_t)(2 * mpad)) ncols <<= 1;
 
@@ -117,9 +126,13 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
           const int s = it % stages;
           if (!mbar_wait(&empty[s], ((it / stages) & 1) ^ 1, wc)) { ok = false; break; }
           uint8_t* xs = ring + (size_t)s * stage_bytes;
-          mbar_expect_tx(&full[s], x_bytes + w_bytes);
-          tma_load_2d(&tmap_x, &full[s], xs, kc * 64, t * kTile);
-          tma_load_2d(&tmap_w, &full[s], xs + x_bytes, kc * 64, 0);
+          mbar_expect_tx(&full[s], x_bytes + w_bytes);  // boxes past d are zero-filled, still full size
+#pragma unroll
+          for (int c = 0; c < kRouteChunks; ++c)
+            tma_load_2d(&tmap_x, &full[s], xs + c * (kTile * 128), (kc * kRouteChunks + c) * 64, t * kTile);
+#pragma unroll
+          for (int c = 0; c < kRouteChunks; ++c)
+            tma_load_2d(&tmap_w, &full[s], xs + x_bytes + c * (mpad * 128), (kc * kRouteChunks + c) * 64, 0);
         }
       }
       // Drain: every issued load must land before the CTA may exit.
@@ -149,10 +162,13 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
           const uint32_t xa = smem_u32(ring + (size_t)s * stage_bytes);
           const uint32_t wa = xa + x_bytes;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = sdesc_sw128(xa + kk * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(wa + kk * 32, 16, 1024);
-            umma_bf16(dt, ad, bd, idesc, (kc | kk) != 0);
+          for (int c = 0; c < kRouteChunks; ++c) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = sdesc_sw128(xa + c * (kTile * 128) + kk * 32, 16, 1024);
+              const uint64_t bd = sdesc_sw128(wa + c * (mpad * 128) + kk * 32, 16, 1024);
+              umma_bf16(dt, ad, bd, idesc, (kc | c | kk) != 0);
+            }
           }
           umma_commit(&empty[s]);
         }
