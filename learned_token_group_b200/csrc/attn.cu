@@ -36,6 +36,13 @@ namespace moga {
 
 namespace {
 
+// Windows of at most 192 tokens use the small-window plan (double-buffered
+// query tiles, compact half tiles); 0 sends them through the general plan.
+#ifndef MOGA_STGA_SMALL
+#define MOGA_STGA_SMALL 1
+#endif
+constexpr bool kSmallWindows = MOGA_STGA_SMALL != 0;
+
 // One key pair in every kExp2PolyEvery goes through the FMA-pipe polynomial
 // instead of MUFU ex2 (0 disables), balancing the two units in the softmax.
 #ifndef MOGA_EXP2_POLY_EVERY
@@ -222,6 +229,22 @@ struct Plan {
   static constexpr int kBar = kV0 + kStages * kTileBytes;
   static constexpr int kTable = kBar + 256;
   static size_t bytes(int table_ints) { return (size_t)kTable + (size_t)table_ints * 4 + 1024; }
+  // Small windows (at most 192 tokens, read in place): query tile B and the
+  // second K and V tiles hold at most 64 rows and are stored compactly (64
+  // rows per 64-column chunk), which frees room for a second pair of query
+  // tiles.  Compact query tiles come first and full ones follow, so a
+  // 128-row operand read of a compact tile stays in shared memory; its rows
+  // past 64 only reach query rows that are dropped or keys that are masked.
+  static constexpr int kChunkFull = kTile * 128;               // bytes of one 64-column chunk, 128 rows
+  static constexpr int kChunkHalf = 64 * 128;                  // the same for 64 rows
+  static constexpr int kHalfBytes = kChunks * kChunkHalf;
+  static constexpr int kSQB = 0;                                // [2] compact query tiles B
+  static constexpr int kSQA = 2 * kHalfBytes;                   // [2] query tiles A
+  static constexpr int kSK0 = kSQA + 2 * kTileBytes;            // K tile 0, then compact K tile 1
+  static constexpr int kSK1 = kSK0 + kTileBytes;
+  static constexpr int kSV0 = kSK1 + kHalfBytes;                // V tile 0, then compact V tile 1
+  static constexpr int kSV1 = kSV0 + kTileBytes;
+  static_assert(kSV1 + kHalfBytes <= kBar, "small-window plan must fit the standard one");
 };
 
 // A work unit is a pair of consecutive 128-row query tiles (A, B) of one
@@ -305,7 +328,10 @@ struct Decoder {
 // otherwise 128-row tiles of a gathered head-major copy (2-D tiled TMA).
 // kShots: the unit decoder also reads shot-window tables (mode 2); the
 // grouped-attention instantiation leaves it out.
-template <int DH, bool kDirect, bool kShots>
+// kSmall: in place, windows of at most 192 tokens (see Plan): compact tiles,
+// K/V tile j always in slot j, and two query buffers used in turn, so the
+// next window's queries load while this one computes.
+template <int DH, bool kDirect, bool kShots, bool kSmall>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
             const __grid_constant__ CUtensorMap tv, const AttnArgs a, int* status, unsigned long long wait_ns) {
@@ -314,25 +340,27 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P::kBar);
-  uint64_t* q_full = bars + 0;
-  uint64_t* q_empty = bars + 1;
-  uint64_t* k_full = bars + 2;    // [kStages]
-  uint64_t* k_empty = bars + 4;   // [kStages]
-  uint64_t* v_full = bars + 6;    // [kStages]
-  uint64_t* v_empty = bars + 8;   // [kStages]
-  uint64_t* s_full = bars + 10;   // [2]: S of tile A / B computed
-  uint64_t* p_full = bars + 12;   // [2]: P of tile A / B written (O rescaled)
-  uint64_t* o_full = bars + 14;   // [2]: last P V of tile A / B done
-  uint64_t* done_bar = bars + 16;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 18);
+  uint64_t* q_full = bars + 0;    // [2] (the second pair only for small windows)
+  uint64_t* q_empty = bars + 2;   // [2]
+  uint64_t* k_full = bars + 4;    // [kStages]
+  uint64_t* k_empty = bars + 6;   // [kStages]
+  uint64_t* v_full = bars + 8;    // [kStages]
+  uint64_t* v_empty = bars + 10;  // [kStages]
+  uint64_t* s_full = bars + 12;   // [2]: S of tile A / B computed
+  uint64_t* p_full = bars + 14;   // [2]: P of tile A / B written (O rescaled)
+  uint64_t* o_full = bars + 16;   // [2]: last P V of tile A / B done
+  uint64_t* done_bar = bars + 18;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 20);
   int* tab = reinterpret_cast<int*>(smem + P::kTable);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&q_full[b], 1);
+      mbar_init(&q_empty[b], 1);
+    }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
@@ -460,11 +488,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     constexpr int kPieces = DH * 2 / 16;       // 16-byte pieces per row
     constexpr int kRowsPerOp = 32 / kPieces;   // rows one warp-wide copy covers
     const int piece = lane % kPieces, sub = lane / kPieces;
-    const uint32_t piece_off = (uint32_t)((piece >> 3) * (kTile * 128));  // 64-column chunk
+    const int pchunk = piece >> 3;  // 64-column chunk of this lane's piece
     const int pj = piece & 7;
     int* toks = tab + li * 2 * kTile;  // this loader's token rows (two tiles for Q)
     const int H = a.H;
     uint32_t ucnt = 0, t = 0;
+    uint32_t sc0 = 0, sc1 = 0;  // small windows: uses of K/V slot 0 and 1 by this loader
     bool ok = true;
     // Row indices of tile rows [pos0, pos0 + 128), four per lane: token * H + h,
     // or -1 (zero-filled) for a token out of range or a row past the segment
@@ -483,12 +512,13 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     // tile's first nrows rows are issued (a warp-uniform count): rows past the
     // segment end keep what the slot held, which is finite (earlier tiles or
     // the initial zeros), and belong to masked keys or dropped queries.
-    auto copy_tile = [&](const void* g, uint8_t* dst, const int (&tr)[4], int* tk, int nrows) {
+    // chunk: byte stride between 64-column chunks (full or compact tile).
+    auto copy_tile = [&](const void* g, uint8_t* dst, const int (&tr)[4], int* tk, int nrows, int chunk) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) tk[4 * lane + i] = tr[i];
       __syncwarp();
       const char* gb = static_cast<const char*>(g) + piece * 16;
-      const uint32_t db = smem_u32(dst) + piece_off;
+      const uint32_t db = smem_u32(dst) + (uint32_t)(pchunk * chunk);
       const int nops = (min(nrows, kTile) + kRowsPerOp - 1) / kRowsPerOp;  // warp-uniform
 #pragma unroll 8
       for (int i = 0; i < nops; ++i) {
@@ -509,12 +539,21 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       if (lane == 0) w = mbar_wait(bar, parity, wc, site, count);
       return __shfl_sync(0xffffffffu, w, 0) != 0;
     };
-    if (li > 0) {
+    {
       // Rows past a segment's end are never copied, so the K and V rings
-      // start as zeros: every row the tensor core reads is then finite (a
-      // masked key's P is 0, and 0 times a finite V row adds nothing).
-      uint4* ring = reinterpret_cast<uint4*>(smem + (li == 1 ? P::kK0 : P::kV0));
-      for (int i = lane; i < kStages * P::kTileBytes / 16; i += 32) ring[i] = make_uint4(0, 0, 0, 0);
+      // (and, for small windows, the query buffers) start as zeros: every
+      // row the tensor core reads is then finite (a masked key's P is 0, and
+      // 0 times a finite V row adds nothing).
+      int off, bytes;
+      if constexpr (kSmall) {
+        off = li == 0 ? P::kSQB : li == 1 ? P::kSK0 : P::kSV0;
+        bytes = li == 0 ? P::kSK0 : P::kTileBytes + P::kHalfBytes;
+      } else {
+        off = li == 1 ? P::kK0 : P::kV0;
+        bytes = li == 0 ? 0 : kStages * P::kTileBytes;
+      }
+      uint4* ring = reinterpret_cast<uint4*>(smem + off);
+      for (int i = lane; i < bytes / 16; i += 32) ring[i] = make_uint4(0, 0, 0, 0);
       fence_proxy_async_smem();
       __syncwarp();
     }
@@ -528,28 +567,51 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         int ra[4], rb[4];
         fetch_rows(a.perm, u.start + u.q0, seg_end, u.h, ra);
         if (hb) fetch_rows(a.perm, u.start + u.q0 + kTile, seg_end, u.h, rb);
-        if (!warp_wait(q_empty, (ucnt & 1) ^ 1, 1, ucnt)) { ok = false; break; }
-        copy_tile(a.q, smem + P::kQA, ra, toks, u.len - u.q0);
-        if (hb) copy_tile(a.q, smem + P::kQB, rb, toks + kTile, u.len - u.q0 - kTile);
+        // small windows: query buffers alternate by unit, each with its own barriers
+        const int qb = kSmall ? (int)(ucnt & 1) : 0;
+        const uint32_t qph = kSmall ? (ucnt >> 1) : ucnt;
+        if (!warp_wait(&q_empty[qb], (qph & 1) ^ 1, 1, ucnt)) { ok = false; break; }
+        if constexpr (kSmall) {
+          copy_tile(a.q, smem + P::kSQA + qb * P::kTileBytes, ra, toks, u.len - u.q0, P::kChunkFull);
+          if (hb) copy_tile(a.q, smem + P::kSQB + qb * P::kHalfBytes, rb, toks + kTile, u.len - u.q0 - kTile,
+                            P::kChunkHalf);
+        } else {
+          copy_tile(a.q, smem + P::kQA, ra, toks, u.len - u.q0, P::kChunkFull);
+          if (hb) copy_tile(a.q, smem + P::kQB, rb, toks + kTile, u.len - u.q0 - kTile, P::kChunkFull);
+        }
         finish();
-        if (lane == 0) mbar_arrive(q_full);
+        if (lane == 0) mbar_arrive(&q_full[qb]);
         ++ucnt;
         continue;
       }
       const bool is_v = li == 2;
       for (int j = 0; j < nkv; ++j, ++t) {
         int tr[4];
-        const int s = t % kStages;
+        // slot and phase: a ring of kStages tiles, or (small windows) tile j in slot j
+        const int s = kSmall ? j : (int)(t % kStages);
+        const uint32_t ph = kSmall ? (j ? sc1 : sc0) : t / kStages;
         fetch_rows(kvperm, u.kvs + j * kTile, kv_end, u.h, tr);
-        if (!warp_wait(is_v ? &v_empty[s] : &k_empty[s], ((t / kStages) & 1) ^ 1, is_v ? 3 : 2, t)) {
+        if (!warp_wait(is_v ? &v_empty[s] : &k_empty[s], (ph & 1) ^ 1, is_v ? 3 : 2, t)) {
           ok = false;
           break;
         }
         // Test hook: the first K tile never arrives, so the MMA warp's
         // bounded wait runs out and the kernel reports a timeout.
         if (!is_v && t == 0 && a.debug_withhold_first_k) { ok = false; break; }
-        copy_tile(is_v ? a.v : a.k, smem + (is_v ? P::kV0 : P::kK0) + s * P::kTileBytes, tr, toks,
-                  u.kvl - j * kTile);
+        uint8_t* dst;
+        int chunk = P::kChunkFull;
+        if constexpr (kSmall) {
+          dst = smem + (is_v ? (j ? P::kSV1 : P::kSV0) : (j ? P::kSK1 : P::kSK0));
+          if (j) {
+            chunk = P::kChunkHalf;
+            ++sc1;
+          } else {
+            ++sc0;
+          }
+        } else {
+          dst = smem + (is_v ? P::kV0 : P::kK0) + s * P::kTileBytes;
+        }
+        copy_tile(is_v ? a.v : a.k, dst, tr, toks, u.kvl - j * kTile, chunk);
         finish();
         if (lane == 0) mbar_arrive(is_v ? &v_full[s] : &k_full[s]);
       }
@@ -562,58 +624,77 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idO = idesc_bf16(128, DH, false, true);
       uint32_t ucnt = 0, kc = 0, vc = 0, pc0 = 0, pc1 = 0;
+      uint32_t kc0 = 0, kc1 = 0, vc0 = 0, vc1 = 0;  // small windows: uses of K/V slot 0 and 1
       bool ok = true;
-      // S_x = Q_x K^T (both K-major in smem, 128B swizzle)
-      auto issue_s = [&](int x, int ks) {
-        const uint32_t qa = smem_u32(smem + (x ? P::kQB : P::kQA));
-        const uint32_t ka = smem_u32(smem + P::kK0 + ks * P::kTileBytes);
+      // S_x = Q_x K^T (both K-major in smem, 128B swizzle); qc / kch: byte
+      // stride between the 64-column chunks of the query / key tile.
+      auto issue_s = [&](int x, uint32_t qa, int qc, uint32_t ka, int kch) {
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_bf16(tS(x), sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idS,
-                    kk > 0 ? 1u : 0u);
+          const uint32_t qo = (kk >> 2) * qc + (kk & 3) * 32, ko = (kk >> 2) * kch + (kk & 3) * 32;
+          umma_bf16(tS(x), sdesc_sw128(qa + qo, 16, 1024), sdesc_sw128(ka + ko, 16, 1024), idS, kk > 0 ? 1u : 0u);
         }
       };
-      // O_x += P_x V (P in TMEM over S_x, V MN-major in smem)
-      auto issue_pv = [&](int x, int vs, bool acc) {
-        const uint32_t va = smem_u32(smem + P::kV0 + vs * P::kTileBytes);
+      // O_x += P_x V over the first nk 16-key steps (P in TMEM over S_x, V
+      // MN-major in smem, vch between its 64-column chunks); later steps hold
+      // only masked keys (P = 0) and are skipped.
+      auto issue_pv = [&](int x, uint32_t va, int vch, int nk, bool acc) {
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          umma_bf16_ts(tO(x), tS(x) + kk * 8, sdesc_sw128(va + kk * 2048, 16384, 1024), idO,
-                       (acc || kk > 0) ? 1u : 0u);
+          if (kk < nk)
+            umma_bf16_ts(tO(x), tS(x) + kk * 8, sdesc_sw128(va + kk * 2048, vch, 1024), idO,
+                         (acc || kk > 0) ? 1u : 0u);
       };
+      // K/V tile j of a unit: a ring of kStages slots, or (small windows) slot j.
+      auto kslot = [&](int j) { return kSmall ? j : (int)(kc % kStages); };
+      auto vslot = [&](int j) { return kSmall ? j : (int)(vc % kStages); };
+      auto kphase = [&](int j) { return kSmall ? (j ? kc1 : kc0) : kc / kStages; };
+      auto vphase = [&](int j) { return kSmall ? (j ? vc1 : vc0) : vc / kStages; };
+      auto kaddr = [&](int sl) {
+        return smem_u32(smem + (kSmall ? (sl ? P::kSK1 : P::kSK0) : P::kK0 + sl * P::kTileBytes));
+      };
+      auto vaddr = [&](int sl) {
+        return smem_u32(smem + (kSmall ? (sl ? P::kSV1 : P::kSV0) : P::kV0 + sl * P::kTileBytes));
+      };
+      auto chunk_of = [&](int sl) { return (kSmall && sl) ? P::kChunkHalf : P::kChunkFull; };
       for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
         const Unit u = dec(idx);
         if (u.q0 >= u.len) continue;
         const bool hb = u.q0 + kTile < u.len;
         const int nkv = (u.kvl + kTile - 1) / kTile;
-        if (!mbar_wait(q_full, ucnt & 1, wc, 4, ucnt)) break;
+        const int qb = kSmall ? (int)(ucnt & 1) : 0;
+        const uint32_t qph = kSmall ? (ucnt >> 1) : ucnt;
+        if (!mbar_wait(&q_full[qb], qph & 1, wc, 4, ucnt)) break;
         ++ucnt;
-        int ks = kc % kStages;
-        if (!mbar_wait(&k_full[ks], (kc / kStages) & 1, wc, 5, kc)) break;
+        const uint32_t qa_addr = smem_u32(smem + (kSmall ? P::kSQA + qb * P::kTileBytes : P::kQA));
+        const uint32_t qb_addr = smem_u32(smem + (kSmall ? P::kSQB + qb * P::kHalfBytes : P::kQB));
+        const int qb_chunk = kSmall ? P::kChunkHalf : P::kChunkFull;
+        int ks = kslot(0);
+        if (!mbar_wait(&k_full[ks], kphase(0) & 1, wc, 5, kc)) break;
         tc_fence_after();
-        issue_s(0, ks);
+        issue_s(0, qa_addr, P::kChunkFull, kaddr(ks), chunk_of(ks));
         umma_commit(&s_full[0]);
         if (hb) {
-          issue_s(1, ks);
+          issue_s(1, qb_addr, qb_chunk, kaddr(ks), chunk_of(ks));
           umma_commit(&s_full[1]);
         }
         umma_commit(&k_empty[ks]);
-        ++kc;
-        if (nkv == 1) umma_commit(q_empty);
+        if (kSmall) ++kc0; else ++kc;
+        if (nkv == 1) umma_commit(&q_empty[qb]);
         for (int j = 0; j < nkv; ++j) {
-          const int vs = vc % kStages;
+          const int vs = vslot(j);
           const bool more = j + 1 < nkv;
-          if (!mbar_wait(&v_full[vs], (vc / kStages) & 1, wc, 7, vc)) { ok = false; break; }
+          const int nk = (min(kTile, u.kvl - j * kTile) + 15) / 16;
+          if (!mbar_wait(&v_full[vs], vphase(j) & 1, wc, 7, vc)) { ok = false; break; }
           if (!mbar_wait(&p_full[0], pc0 & 1, wc, 13, pc0)) { ok = false; break; }
           ++pc0;
           tc_fence_after();
-          issue_pv(0, vs, j > 0);
-          ks = kc % kStages;
+          issue_pv(0, vaddr(vs), chunk_of(vs), nk, j > 0);
+          ks = kslot(j + 1);
           if (more) {
-            if (!mbar_wait(&k_full[ks], (kc / kStages) & 1, wc, 8, kc)) { ok = false; break; }
+            if (!mbar_wait(&k_full[ks], kphase(j + 1) & 1, wc, 8, kc)) { ok = false; break; }
             tc_fence_after();
-            issue_s(0, ks);
+            issue_s(0, qa_addr, P::kChunkFull, kaddr(ks), chunk_of(ks));
             umma_commit(&s_full[0]);
           } else {
             umma_commit(&o_full[0]);
@@ -622,20 +703,20 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             if (!mbar_wait(&p_full[1], pc1 & 1, wc, 29, pc1)) { ok = false; break; }
             ++pc1;
             tc_fence_after();
-            issue_pv(1, vs, j > 0);
+            issue_pv(1, vaddr(vs), chunk_of(vs), nk, j > 0);
             if (more) {
-              issue_s(1, ks);
+              issue_s(1, qb_addr, qb_chunk, kaddr(ks), chunk_of(ks));
               umma_commit(&s_full[1]);
             } else {
               umma_commit(&o_full[1]);
             }
           }
           umma_commit(&v_empty[vs]);
-          ++vc;
+          if (kSmall) { if (j) ++vc1; else ++vc0; } else { ++vc; }
           if (more) {
             umma_commit(&k_empty[ks]);
-            ++kc;
-            if (j + 2 == nkv) umma_commit(q_empty);  // the unit's last S products are issued
+            if (kSmall) ++kc1; else ++kc;  // tile j + 1 of a small window is tile 1
+            if (j + 2 == nkv) umma_commit(&q_empty[qb]);  // the unit's last S products are issued
           }
         }
       }
@@ -833,8 +914,11 @@ cudaError_t launch_attention_dh(const DevCtx& c, const AttnArgs& a) {
   // groups: the segment table; in place: the loaders' token rows (2 tiles each)
   const int table_ints = a.mode == 0 ? 3 * a.nseg + 1 : (a.direct ? 6 * kTile : 0);
   const size_t smem = P::bytes(table_ints);
-  auto kern = a.direct ? attn_kernel<DH, true, true>
-                       : (a.mode == 2 ? attn_kernel<DH, false, true> : attn_kernel<DH, false, false>);
+  // windows of at most 192 tokens fit the small-window plan (query tile B and
+  // the second K/V tiles of at most 64 rows)
+  const bool small = a.direct && a.mode == 1 && (int64_t)a.wt * a.wh * a.ww <= kTile + 64 && kSmallWindows;
+  auto kern = a.direct ? (small ? attn_kernel<DH, true, true, true> : attn_kernel<DH, true, true, false>)
+                       : (a.mode == 2 ? attn_kernel<DH, false, true, false> : attn_kernel<DH, false, false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int grid = c.num_sms;
