@@ -635,13 +635,14 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
           umma_bf16(tS(x), sdesc_sw128(qa + qo, 16, 1024), sdesc_sw128(ka + ko, 16, 1024), idS, kk > 0 ? 1u : 0u);
         }
       };
-      // O_x += P_x V over the first nk 16-key steps (P in TMEM over S_x, V
-      // MN-major in smem, vch between its 64-column chunks); later steps hold
-      // only masked keys (P = 0) and are skipped.
+      // O_x += P_x V (P in TMEM over S_x, V MN-major in smem, vch between its
+      // 64-column chunks).  Small windows issue only the first nk 16-key steps:
+      // the rest hold masked keys (P = 0) and, in a compact tile, no rows at
+      // all.  Full tiles issue all eight without a test on the issue path.
       auto issue_pv = [&](int x, uint32_t va, int vch, int nk, bool acc) {
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          if (kk < nk)
+          if (!kSmall || kk < nk)
             umma_bf16_ts(tO(x), tS(x) + kk * 8, sdesc_sw128(va + kk * 2048, vch, 1024), idO,
                          (acc || kk > 0) ? 1u : 0u);
       };
