@@ -491,6 +491,21 @@ def run_ours(args, wl, rank, world, dist):
             widened[tag + "_tflops"] = _shot_flops(wl, win, shots, 2, 2) / (ms_s * 1e-3) / 1e12
             del out_s, ws_s
         widened["shot_split"] = shots
+        # the pages' whole block in one call: MoGA, whole-shot 2x2 STGA and
+        # per-frame attention, averaged (moga_layer_shots)
+        blk = moga.moga_layer_shots(inp["x"], inp["W_r"], inp["b_r"], inp["q"], inp["k"], inp["v"], wl.M,
+                                    wl.grid, half, ss, 2, 2, per_frame=True)
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            moga.moga_layer_shots(inp["x"], inp["W_r"], inp["b_r"], inp["q"], inp["k"], inp["v"], wl.M, wl.grid,
+                                  half, ss, 2, 2, per_frame=True, res=blk)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        moga.sync_status(blk["ws"])
+        widened["pages_block_ms"] = ev0.elapsed_time(ev1) / args.steps
+        widened["pages_block"] = "MoGA + shot-aware STGA (whole shots, 2x2 tiles, 2+2 boundary frames) + per-frame"
+        del blk
     # ---- the other contexts the metric names: the same block at 580k tokens
     # (40 heads, M = 32) and the skewed-routing stress case
     contexts = {}

@@ -194,6 +194,21 @@ moga_status stga_shot_attn(const void* q, const void* k, const void* v, int T, i
                            const int32_t* shot_start, int nshots, int aug_prev, int aug_next, int H, int d_h,
                            float out_scale, int accumulate, void* out, void* ws, size_t ws_bytes, void* stream);
 
+/* moga_layer_shots: the visual block of the pages' Wan setting, one call:
+ * moga_route, grouped attention, shot-aware STGA (stga_shot_attn with the
+ * given window, shots and augmentation) and, when per_frame = 1, the
+ * per-frame branch; out = arithmetic mean of the branches (2 or 3 of them).
+ * Arguments and outputs as moga_layer_ex and stga_shot_attn (shot_start is
+ * device int32 [nshots + 1]; T * Hg * Wg must equal N).
+ * Workspace: moga_layer_shots_workspace_size(...) bytes. */
+size_t moga_layer_shots_workspace_size(int64_t N, int H, int d_h, int M, int T, int Hg, int Wg, const int* window,
+                                       int nshots, int aug_prev, int aug_next, int per_frame);
+moga_status moga_layer_shots(const void* x, const void* W_r, const float* b_r, moga_dtype x_dt, const void* q,
+                             const void* k, const void* v, int64_t N, int d, int H, int d_h, int M, int T, int Hg,
+                             int Wg, const int* window, const int32_t* shot_start, int nshots, int aug_prev,
+                             int aug_next, int per_frame, void* out, int32_t* group_id, float* gate, int32_t* perm,
+                             int32_t* offsets, void* ws, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------- full layer
  * moga_layer: one visual attention block = moga_route, then moga_group_attn,
  * then (when window != NULL) stga_window_attn, combined as

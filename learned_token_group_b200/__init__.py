@@ -20,7 +20,7 @@ import torch
 
 __all__ = ["MogaError", "get_lib", "LIB_PATH", "HEADER_PATH", "route", "group_attn", "stga_window_attn",
            "moga_layer", "sync_status", "workspace", "MogaLayer", "exported_names", "kernel_launches",
-           "set_timing_events", "STAGES", "Pipeline", "stga_shot_attn"]
+           "set_timing_events", "STAGES", "Pipeline", "stga_shot_attn", "moga_layer_shots"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoga.so")
@@ -74,6 +74,9 @@ def get_lib():
         "moga_debug_inject": (_I, [_I]),
         "stga_shot_attn_workspace_size": (_SZ, [_I, _I, _I, _P, _I, _I, _I, _I, _I]),
         "stga_shot_attn": (_I, [_P, _P, _P, _I, _I, _I, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _P, _SZ, _P]),
+        "moga_layer_shots_workspace_size": (_SZ, [_I64, _I, _I, _I, _I, _I, _I, _P, _I, _I, _I, _I]),
+        "moga_layer_shots": (_I, [_P, _P, _P, _I, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I,
+                                  _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
         "moga_pipe_create": (_I, [_I64, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I, ctypes.POINTER(_P)]),
         "moga_pipe_submit": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
         "moga_pipe_sync": (_I, [_P]),
@@ -272,6 +275,39 @@ def stga_shot_attn(q, k, v, grid: Sequence[int], window: Sequence[int], shot_sta
                             ws.numel(), _stream(q.device))
     _check(st, "stga_shot_attn")
     return out, ws
+
+
+def moga_layer_shots(x, W_r, b_r, q, k, v, M: int, grid, window, shot_start: torch.Tensor, aug_prev: int = 2,
+                     aug_next: int = 2, per_frame: bool = True, res=None):
+    """The pages' visual block in one call: MoGA, shot-aware STGA and (per_frame)
+    the per-frame branch, averaged.  Returns dict(out, group_id, gate, perm,
+    offsets, ws); pass that dict back as ``res`` to reuse its buffers."""
+    lib = get_lib()
+    N, d = x.shape
+    _, H, d_h = q.shape
+    for n, t in (("x", x), ("q", q), ("k", k), ("v", v)):
+        _dev_tensor(t, n)
+    _dev_tensor(shot_start, "shot_start", torch.int32)
+    T, Hg, Wg = (int(g) for g in grid)
+    w3 = _int3(window)
+    nshots = shot_start.numel() - 1
+    dev = x.device
+    x_dt = {torch.float32: MOGA_F32, torch.bfloat16: MOGA_BF16}[x.dtype]
+    need = lib.moga_layer_shots_workspace_size(N, H, d_h, M, T, Hg, Wg, w3, nshots, aug_prev, aug_next,
+                                               int(bool(per_frame)))
+    if res is None or res["ws"].numel() < need:
+        res = {"out": torch.empty((N, H, d_h), dtype=torch.bfloat16, device=dev),
+               "group_id": torch.empty(N, dtype=torch.int32, device=dev),
+               "gate": torch.empty(N, dtype=torch.float32, device=dev),
+               "perm": torch.empty(N, dtype=torch.int32, device=dev),
+               "offsets": torch.empty(M + 1, dtype=torch.int32, device=dev), "ws": workspace(need, dev)}
+    ws = res["ws"]
+    st = lib.moga_layer_shots(_ptr(x), _ptr(W_r), _ptr(b_r), x_dt, _ptr(q), _ptr(k), _ptr(v), N, d, H, d_h, M, T,
+                              Hg, Wg, w3, _ptr(shot_start), nshots, int(aug_prev), int(aug_next),
+                              int(bool(per_frame)), _ptr(res["out"]), _ptr(res["group_id"]), _ptr(res["gate"]),
+                              _ptr(res["perm"]), _ptr(res["offsets"]), _ptr(ws), ws.numel(), _stream(dev))
+    _check(st, "moga_layer_shots")
+    return res
 
 
 class MogaLayer:

@@ -358,6 +358,77 @@ moga_status check_shots(int T, int Hg, int Wg, const int* window, int nshots, in
   return MOGA_OK;
 }
 
+moga_status check_shot_args(int T, int Hg, int Wg, const int* window, const int32_t* shot_start, int nshots,
+                            int aug_prev, int aug_next, int H, int d_h, int64_t* N) {
+  moga_status st = check_shots(T, Hg, Wg, window, nshots, aug_prev, aug_next, N);
+  if (st != MOGA_OK) return st;
+  if ((st = check_attn_shape(*N, H, d_h)) != MOGA_OK) return st;
+  if (!shot_start || !aligned4(shot_start)) return MOGA_ERR_INVALID_ARG;
+  if ((int64_t)shot_kv_cap(T, Hg, Wg, nshots, aug_prev, aug_next) * H >= (int64_t)1 << 31)
+    return MOGA_ERR_UNSUPPORTED;
+  return MOGA_OK;
+}
+
+// Shot-aware STGA into out (accumulate: out += out_scale * SA), arguments
+// already validated, workspace large enough for shot_ws.
+moga_status shot_body(const DevCtx& c, const void* q, const void* k, const void* v, int T, int Hg, int Wg,
+                      const int* window, const int32_t* shot_start, int nshots, int aug_prev, int aug_next, int H,
+                      int d_h, float out_scale, int accumulate, void* out, uint8_t* wb) {
+  const int64_t N = (int64_t)T * Hg * Wg;
+  const ShotWs w = shot_ws(T, Hg, Wg, window, nshots, aug_prev, aug_next, H, d_h);
+  int32_t* wtab = reinterpret_cast<int32_t*>(wb + w.wtab);
+  int32_t* qperm = reinterpret_cast<int32_t*>(wb + w.qperm);
+  int32_t* kvperm = reinterpret_cast<int32_t*>(wb + w.kvperm);
+  mark(MOGA_STAGE_STGA_PREP, true, c.stream);
+  if (launch_shot_table(c, shot_start, nshots, T, Hg, Wg, window, aug_prev, aug_next, H, w.cap, wtab) !=
+      cudaSuccess)
+    return MOGA_ERR_CUDA;
+  if (launch_shot_perm(c, wtab, w.cap, Hg, Wg, window, qperm, kvperm) != cudaSuccess) return MOGA_ERR_CUDA;
+  count(2);
+  AttnArgs a{};
+  a.direct = w.direct ? 1 : 0;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  if (!w.direct) {
+    // queries: every token once; keys/values: the device-computed count of rows
+    if (launch_gather_rows(c, q, nullptr, qperm, nullptr, N, N, H, d_h, N, wb + w.qh, nullptr) != cudaSuccess ||
+        launch_gather_rows(c, k, v, kvperm, wtab + 2, w.kv_cap, N, H, d_h, w.kv_cap, wb + w.kh, wb + w.vh) !=
+            cudaSuccess)
+      return MOGA_ERR_CUDA;
+    count(2);
+    a.q = wb + w.qh;
+    a.k = wb + w.kh;
+    a.v = wb + w.vh;
+    a.kv_rows = w.kv_cap;
+  }
+  mark(MOGA_STAGE_STGA_PREP, false, c.stream);
+  a.perm = qperm;
+  a.kvperm = kvperm;
+  a.gate = nullptr;
+  a.out = out;
+  a.N = N;
+  a.H = H;
+  a.d_h = d_h;
+  a.out_scale = out_scale;
+  a.accumulate = accumulate;
+  a.mode = 2;
+  a.table = wtab;
+  a.nseg = (int)w.cap;
+  a.T = T;
+  a.Hg = Hg;
+  a.Wg = Wg;
+  a.wt = window[0];
+  a.wh = window[1];
+  a.ww = window[2];
+  a.debug_withhold_first_k = 0;
+  mark(MOGA_STAGE_STGA_ATTN, true, c.stream);
+  const cudaError_t e = launch_attention(c, a);
+  mark(MOGA_STAGE_STGA_ATTN, false, c.stream);
+  count(1);
+  return from_cuda(e);
+}
+
 }  // namespace
 
 bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
@@ -523,69 +594,61 @@ moga_status stga_shot_attn(const void* q, const void* k, const void* v, int T, i
   moga_status st = check_qkv(q, k, v, out);
   if (st != MOGA_OK) return st;
   int64_t N = 0;
-  if ((st = check_shots(T, Hg, Wg, window, nshots, aug_prev, aug_next, &N)) != MOGA_OK) return st;
-  if ((st = check_attn_shape(N, H, d_h)) != MOGA_OK) return st;
-  if (!shot_start || !aligned4(shot_start) || (accumulate != 0 && accumulate != 1)) return MOGA_ERR_INVALID_ARG;
-  if (!(out_scale == out_scale)) return MOGA_ERR_INVALID_ARG;  // NaN
+  if ((st = check_shot_args(T, Hg, Wg, window, shot_start, nshots, aug_prev, aug_next, H, d_h, &N)) != MOGA_OK)
+    return st;
+  if ((accumulate != 0 && accumulate != 1) || !(out_scale == out_scale)) return MOGA_ERR_INVALID_ARG;  // NaN
   if (!ws || !aligned16(ws)) return MOGA_ERR_INVALID_ARG;
-  if ((int64_t)shot_kv_cap(T, Hg, Wg, nshots, aug_prev, aug_next) * H >= (int64_t)1 << 31)
-    return MOGA_ERR_UNSUPPORTED;
-  const ShotWs w = shot_ws(T, Hg, Wg, window, nshots, aug_prev, aug_next, H, d_h);
-  if (ws_bytes < w.total) return MOGA_ERR_WORKSPACE;
+  if (ws_bytes < shot_ws(T, Hg, Wg, window, nshots, aug_prev, aug_next, H, d_h).total) return MOGA_ERR_WORKSPACE;
   DevCtx c;
   if (!make_ctx(&c, ws, stream)) return MOGA_ERR_CUDA;
-  uint8_t* wb = (uint8_t*)ws;
-  int32_t* wtab = reinterpret_cast<int32_t*>(wb + w.wtab);
-  int32_t* qperm = reinterpret_cast<int32_t*>(wb + w.qperm);
-  int32_t* kvperm = reinterpret_cast<int32_t*>(wb + w.kvperm);
-  mark(MOGA_STAGE_STGA_PREP, true, c.stream);
-  if (launch_shot_table(c, shot_start, nshots, T, Hg, Wg, window, aug_prev, aug_next, H, w.cap, wtab) !=
-      cudaSuccess)
-    return MOGA_ERR_CUDA;
-  if (launch_shot_perm(c, wtab, w.cap, Hg, Wg, window, qperm, kvperm) != cudaSuccess) return MOGA_ERR_CUDA;
-  count(2);
-  AttnArgs a{};
-  a.direct = w.direct ? 1 : 0;
-  a.q = q;
-  a.k = k;
-  a.v = v;
-  if (!w.direct) {
-    // queries: every token once; keys/values: the device-computed count of rows
-    if (launch_gather_rows(c, q, nullptr, qperm, nullptr, N, N, H, d_h, N, wb + w.qh, nullptr) != cudaSuccess ||
-        launch_gather_rows(c, k, v, kvperm, wtab + 2, w.kv_cap, N, H, d_h, w.kv_cap, wb + w.kh, wb + w.vh) !=
-            cudaSuccess)
-      return MOGA_ERR_CUDA;
-    count(2);
-    a.q = wb + w.qh;
-    a.k = wb + w.kh;
-    a.v = wb + w.vh;
-    a.kv_rows = w.kv_cap;
-  }
-  mark(MOGA_STAGE_STGA_PREP, false, c.stream);
-  a.perm = qperm;
-  a.kvperm = kvperm;
-  a.gate = nullptr;
-  a.out = out;
-  a.N = N;
-  a.H = H;
-  a.d_h = d_h;
-  a.out_scale = out_scale;
-  a.accumulate = accumulate;
-  a.mode = 2;
-  a.table = wtab;
-  a.nseg = (int)w.cap;
-  a.T = T;
-  a.Hg = Hg;
-  a.Wg = Wg;
-  a.wt = window[0];
-  a.wh = window[1];
-  a.ww = window[2];
-  a.debug_withhold_first_k = 0;
-  mark(MOGA_STAGE_STGA_ATTN, true, c.stream);
-  const cudaError_t e = launch_attention(c, a);
-  mark(MOGA_STAGE_STGA_ATTN, false, c.stream);
-  count(1);
-  return from_cuda(e);
+  return shot_body(c, q, k, v, T, Hg, Wg, window, shot_start, nshots, aug_prev, aug_next, H, d_h, out_scale,
+                   accumulate, out, (uint8_t*)ws);
+}
+
+size_t moga_layer_shots_workspace_size(int64_t N, int H, int d_h, int M, int T, int Hg, int Wg, const int* window,
+                                       int nshots, int aug_prev, int aug_next, int per_frame) {
+  if (N < 0 || H < 1 || M < 1 || (per_frame != 0 && per_frame != 1)) return 0;
+  if (stga_shot_attn_workspace_size(T, Hg, Wg, window, nshots, aug_prev, aug_next, H, d_h) == 0) return 0;
+  size_t need = moga_layer_ex_workspace_size(N, H, d_h, M, per_frame ? 2 : 0);
+  const size_t sw = shot_ws(T, Hg, Wg, window, nshots, aug_prev, aug_next, H, d_h).total;
+  return need > sw ? need : sw;
+}
+
+moga_status moga_layer_shots(const void* x, const void* W_r, const float* b_r, moga_dtype x_dt, const void* q,
+                             const void* k, const void* v, int64_t N, int d, int H, int d_h, int M, int T, int Hg,
+                             int Wg, const int* window, const int32_t* shot_start, int nshots, int aug_prev,
+                             int aug_next, int per_frame, void* out, int32_t* group_id, float* gate, int32_t* perm,
+                             int32_t* offsets, void* ws, size_t ws_bytes, void* stream) {
+  if (per_frame != 0 && per_frame != 1) return MOGA_ERR_INVALID_ARG;
+  moga_status st = check_route_args(x, W_r, b_r, x_dt, N, d, M, group_id, gate, perm, offsets, offsets);
+  if (st != MOGA_OK) return st;
+  if ((st = check_qkv(q, k, v, out)) != MOGA_OK) return st;
+  if ((st = check_attn_shape(N, H, d_h)) != MOGA_OK) return st;
+  int64_t n = 0;
+  if ((st = check_shot_args(T, Hg, Wg, window, shot_start, nshots, aug_prev, aug_next, H, d_h, &n)) != MOGA_OK)
+    return st;
+  if (n != N) return MOGA_ERR_INVALID_ARG;
+  if (!ws || !aligned16(ws)) return MOGA_ERR_INVALID_ARG;
+  if (ws_bytes < moga_layer_shots_workspace_size(N, H, d_h, M, T, Hg, Wg, window, nshots, aug_prev, aug_next,
+                                                 per_frame))
+    return MOGA_ERR_WORKSPACE;
+  DevCtx c;
+  if (!make_ctx(&c, ws, stream)) return MOGA_ERR_CUDA;
+  uint8_t* w = (uint8_t*)ws;
+  int32_t* max_seqlen = reinterpret_cast<int32_t*>(w + 16);
+  if ((st = route_body(c, x, W_r, b_r, x_dt, N, d, M, group_id, gate, perm, offsets, max_seqlen, w)) != MOGA_OK)
+    return st;
+  if (N == 0) return MOGA_OK;
+  // out = mean of MoGA, shot-aware STGA and (when on) the per-frame branch
+  const float scale = 1.0f / (float)(2 + per_frame);
+  const int frame_window[3] = {1, Hg, Wg};
+  if ((st = group_attn_body(c, q, k, v, perm, offsets, gate, N, H, d_h, M, scale, out, w)) != MOGA_OK) return st;
+  if ((st = shot_body(c, q, k, v, T, Hg, Wg, window, shot_start, nshots, aug_prev, aug_next, H, d_h, scale, 1, out,
+                      w)) != MOGA_OK)
+    return st;
+  if (per_frame && (st = stga_body(c, q, k, v, T, Hg, Wg, frame_window, H, d_h, 1, out, w, scale)) != MOGA_OK)
+    return st;
+  return MOGA_OK;
 }
 
 size_t moga_layer_workspace_size(int64_t N, int H, int d_h, int M, int T, int Hg, int Wg, const int* window) {

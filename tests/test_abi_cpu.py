@@ -201,3 +201,23 @@ def test_shot_attn_validation(lib):
     n2 = lib.stga_shot_attn_workspace_size(20, 30, 52, w, 8, 2, 2, 2, 128)
     assert 0 < n1 < n2
     assert lib.stga_shot_attn_workspace_size(20, 30, 52, w, 0, 2, 2, 2, 128) == 0
+
+
+def test_layer_shots_validation(lib):
+    w = (ctypes.c_int * 3)(0, 15, 26)
+    f = lib.moga_layer_shots
+    args = [P, P, None, 1, P, P, P, 9360, 256, 2, 128, 4, 6, 30, 52, w, P, 2, 2, 2, 1, P, P, P, P, P, P, BIG, None]
+    bad = list(args)
+    bad[20] = 2                                       # per_frame must be 0 or 1
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[12] = 5                                       # grid must cover N
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[16] = None                                    # shot boundaries missing
+    assert f(*bad) == INVALID
+    small = list(args)
+    small[27] = 4096
+    assert f(*small) == WORKSPACE
+    assert lib.moga_layer_shots_workspace_size(9360, 2, 128, 4, 6, 30, 52, w, 2, 2, 2, 1) >= \
+        lib.moga_layer_shots_workspace_size(9360, 2, 128, 4, 6, 30, 52, w, 2, 2, 2, 0) > 0

@@ -122,3 +122,25 @@ def test_shot_stga_video_sampled(window):
                                      rows=rows, heads=heads)
     got = out[torch.from_numpy(rows).cuda()][:, heads]
     compare_out(got, ref, groups=_window_ids(wl.grid, window, VIDEO_SHOTS, 2, 2)[rows])
+
+
+@pytest.mark.parametrize("per_frame", [True, False])
+def test_layer_shots_block(per_frame):
+    """moga_layer_shots: the mean of MoGA, shot-aware STGA and (optionally)
+    per-frame attention, against the oracle's branches combined the same way."""
+    grid, window, shots = (6, 8, 16), (0, 4, 8), [0, 2, 6]
+    wl = custom(768, H=2, d_h=128, d=128, M=4, x_kind="clustered", grid=grid, name="shots_block")
+    inp = make_inputs(wl, seed=17, device="cuda")
+    ss = torch.tensor(shots, dtype=torch.int32, device="cuda")
+    res = moga.moga_layer_shots(inp["x"], inp["W_r"], inp["b_r"], inp["q"], inp["k"], inp["v"], wl.M, grid, window,
+                                ss, 2, 2, per_frame=per_frame)
+    moga.sync_status(res["ws"])
+    gid = np_cpu(res["group_id"]).astype(np.int64)
+    gate = np_cpu(res["gate"]).astype(np.float64)
+    q, k, v = (np_cpu(inp[n]) for n in ("q", "k", "v"))
+    ref = oracle.group_attention(q, k, v, gid, gate, wl.M) + oracle.stga_shot_attention(q, k, v, *grid, window,
+                                                                                       shots, 2, 2)
+    if per_frame:
+        ref = ref + oracle.frame_attention(q, k, v, *grid)
+    ref = ref / (3 if per_frame else 2)
+    compare_out(res["out"], ref, groups=gid)
