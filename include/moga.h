@@ -321,10 +321,11 @@ moga_status moga_set_timing_events(int stage, void* begin, void* end);
 
 /* moga_debug_inject: failure-detection test hook, process-wide.
  *   0: off (default).
- *   1: in later moga_group_attn / moga_layer calls, the grouped-attention
- *      kernel's loader withholds each CTA's first K tile, so the MMA warp's
- *      bounded wait runs out: the kernel drains, frees its tensor memory and
- *      exits, and moga_sync_status() reports MOGA_ERR_TIMEOUT.  Nothing faults
+ *   1: in later attention calls (grouped, STGA, shot-aware, and the layers
+ *      built on them), the attention kernel's loader withholds each CTA's
+ *      first K tile, so the MMA warp's bounded wait runs out: the kernel
+ *      drains, frees its tensor memory and exits, and moga_sync_status()
+ *      reports MOGA_ERR_TIMEOUT.  Nothing faults
  *      or hangs; the CUDA context stays usable.  Pair with a short
  *      moga_set_wait_limit_ns().
  * Returns MOGA_ERR_INVALID_ARG for other modes. */

@@ -278,6 +278,7 @@ moga_status stga_body(const DevCtx& c, const void* q, const void* k, const void*
   a.wt = window[0];
   a.wh = window[1];
   a.ww = window[2];
+  a.debug_withhold_first_k = g_debug_inject.load(std::memory_order_relaxed) == 1;
   mark(MOGA_STAGE_STGA_ATTN, true, c.stream);
   const cudaError_t e = launch_attention(c, a);
   mark(MOGA_STAGE_STGA_ATTN, false, c.stream);
@@ -421,7 +422,7 @@ moga_status shot_body(const DevCtx& c, const void* q, const void* k, const void*
   a.wt = window[0];
   a.wh = window[1];
   a.ww = window[2];
-  a.debug_withhold_first_k = 0;
+  a.debug_withhold_first_k = g_debug_inject.load(std::memory_order_relaxed) == 1;
   mark(MOGA_STAGE_STGA_ATTN, true, c.stream);
   const cudaError_t e = launch_attention(c, a);
   mark(MOGA_STAGE_STGA_ATTN, false, c.stream);

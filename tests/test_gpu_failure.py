@@ -81,3 +81,28 @@ def test_bad_perm_reported():
     moga.group_attn(inp["q"], inp["k"], inp["v"], bad, offsets, gate_t, M, ws=ws)
     assert _status(ws) == DEVICE_CHECK
     assert _status(ws) == 0
+
+
+@pytest.mark.parametrize("window", [(3, 8, 8), (2, 10, 12), (2, 30, 52)])
+def test_window_kernels_time_out_cleanly(window):
+    """The same hook on the STGA kernels: small-window plan (3x8x8), general
+    in-place plan (240-token windows) and the tiled copy (whole frames).  Each
+    loader gives up, the bounded waits run out, the status says so, and the
+    next call matches the oracle."""
+    lib = moga.get_lib()
+    grid = (4, 30, 52)
+    N = 4 * 30 * 52
+    inp = make_inputs(custom(N, H=2, d_h=128, d=64, M=2), seed=8, device="cuda")
+    ws = moga.workspace(lib.stga_window_attn_workspace_size(*grid, (ctypes.c_int * 3)(*window), 2, 128), "cuda")
+    old = lib.moga_set_wait_limit_ns(50_000_000)
+    try:
+        assert lib.moga_debug_inject(1) == 0
+        moga.stga_window_attn(inp["q"], inp["k"], inp["v"], grid, window, ws=ws)
+        assert _status(ws) == TIMEOUT
+    finally:
+        lib.moga_debug_inject(0)
+        lib.moga_set_wait_limit_ns(old)
+    out = moga.stga_window_attn(inp["q"], inp["k"], inp["v"], grid, window, ws=ws)
+    moga.sync_status(ws)
+    ref = oracle.stga_attention(np_cpu(inp["q"]), np_cpu(inp["k"]), np_cpu(inp["v"]), *grid, window)
+    compare_out(out, ref)

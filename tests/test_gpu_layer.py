@@ -143,3 +143,35 @@ def test_layer_three_branches_wan_sampled():
            + oracle.frame_attention(q, k, v, *wl.grid, rows=rows, heads=heads)) / 3
     out = res["out"][torch.from_numpy(rows).cuda()][:, heads]
     compare_out(out, ref, groups=gid[rows])
+
+
+def test_layer_replays_in_a_cuda_graph():
+    """A whole layer (router, sort, gathers, both attention kernels) captured
+    into a CUDA graph replays to the same bits as eager calls, also after the
+    inputs are overwritten in place."""
+    wl = WORKLOADS["wan_32k"]
+    inp = make_inputs(wl, seed=5, device="cuda")
+    layer = moga.MogaLayer(wl.N, wl.d, wl.H, wl.d_h, wl.M, wl.grid, wl.window, torch.bfloat16, "cuda")
+    args = lambda: (inp["x"], inp["W_r"], inp["b_r"], inp["q"], inp["k"], inp["v"])
+    layer(*args())
+    moga.sync_status(layer.ws)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        layer(*args())
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        layer(*args())
+    for seed in (5, 6):
+        new = make_inputs(wl, seed=seed, device="cuda")
+        for key in ("x", "q", "k", "v"):
+            inp[key].copy_(new[key])
+        layer.out.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        moga.sync_status(layer.ws)
+        got = layer.out.clone()
+        layer(*args())
+        moga.sync_status(layer.ws)
+        assert torch.equal(got, layer.out)
