@@ -88,6 +88,19 @@ moga_status moga_route(const void* x, const void* W_r, const float* b_r, moga_dt
                        int M, int32_t* group_id, float* gate, int32_t* perm, int32_t* offsets,
                        int32_t* max_seqlen, void* ws, size_t ws_bytes, void* stream);
 
+/* moga_sort: the index half of Algorithm 1 step 2 for caller-given group ids
+ * ("MoGA Pseudocode and Kernel Integration"): from group_id int32 [N] in
+ * [0, M) it writes perm int32 [N] (stable: tokens by group, then by index),
+ * offsets int32 [M+1] and max_seqlen int32 [1], exactly as moga_route does for
+ * its own ids.  Ids outside [0, M) are skipped on the device (offsets[M] then
+ * counts only valid tokens) and moga_sync_status() reports
+ * MOGA_ERR_DEVICE_CHECK.  Used when routing happened elsewhere (e.g. on other
+ * ranks of a sequence-parallel group).
+ * Workspace: moga_sort_workspace_size(N, M) bytes. */
+size_t moga_sort_workspace_size(int64_t N, int M);
+moga_status moga_sort(const int32_t* group_id, int64_t N, int M, int32_t* perm, int32_t* offsets,
+                      int32_t* max_seqlen, void* ws, size_t ws_bytes, void* stream);
+
 /* moga_route_ex: moga_route plus the group-balancing statistics of the pages'
  * "Group Balancing Loss" section (Eq. 6), in the reading
  *   F_i = fraction of tokens routed to group i   (= (offsets[i+1]-offsets[i])/N)

@@ -20,7 +20,7 @@ import torch
 
 __all__ = ["MogaError", "get_lib", "LIB_PATH", "HEADER_PATH", "route", "group_attn", "stga_window_attn",
            "moga_layer", "sync_status", "workspace", "MogaLayer", "exported_names", "kernel_launches",
-           "set_timing_events", "STAGES", "Pipeline", "stga_shot_attn", "moga_layer_shots"]
+           "set_timing_events", "STAGES", "Pipeline", "stga_shot_attn", "moga_layer_shots", "sort"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoga.so")
@@ -77,6 +77,8 @@ def get_lib():
         "moga_layer_shots_workspace_size": (_SZ, [_I64, _I, _I, _I, _I, _I, _I, _P, _I, _I, _I, _I]),
         "moga_layer_shots": (_I, [_P, _P, _P, _I, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I,
                                   _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+        "moga_sort_workspace_size": (_SZ, [_I64, _I]),
+        "moga_sort": (_I, [_P, _I64, _I, _P, _P, _P, _P, _SZ, _P]),
         "moga_pipe_create": (_I, [_I64, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I, ctypes.POINTER(_P)]),
         "moga_pipe_submit": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
         "moga_pipe_sync": (_I, [_P]),
@@ -176,6 +178,23 @@ def route(x: torch.Tensor, W_r: torch.Tensor, b_r: Optional[torch.Tensor], M: in
                         _stream(dev))
     _check(st, "moga_route")
     return out
+
+
+def sort(group_id: torch.Tensor, M: int, ws=None):
+    """Counting sort of caller-given group ids (moga_sort): dict(perm, offsets, max_seqlen, ws)."""
+    lib = get_lib()
+    _dev_tensor(group_id, "group_id", torch.int32)
+    N = group_id.numel()
+    dev = group_id.device
+    if ws is None:
+        ws = workspace(lib.moga_sort_workspace_size(N, M), dev)
+    res = {"perm": torch.empty(N, dtype=torch.int32, device=dev),
+           "offsets": torch.empty(M + 1, dtype=torch.int32, device=dev),
+           "max_seqlen": torch.empty(1, dtype=torch.int32, device=dev), "ws": ws}
+    st = lib.moga_sort(_ptr(group_id), N, M, _ptr(res["perm"]), _ptr(res["offsets"]), _ptr(res["max_seqlen"]),
+                       _ptr(ws), ws.numel(), _stream(dev))
+    _check(st, "moga_sort")
+    return res
 
 
 def route_stats(x: torch.Tensor, W_r: torch.Tensor, b_r: Optional[torch.Tensor], M: int):

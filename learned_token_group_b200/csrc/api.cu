@@ -502,6 +502,39 @@ moga_status moga_route(const void* x, const void* W_r, const float* b_r, moga_dt
   return route_body(c, x, W_r, b_r, dt, N, d, M, group_id, gate, perm, offsets, max_seqlen, (uint8_t*)ws);
 }
 
+size_t moga_sort_workspace_size(int64_t N, int M) {
+  if (N < 0 || M < 1) return 0;
+  return route_ws(N, M).total;
+}
+
+moga_status moga_sort(const int32_t* group_id, int64_t N, int M, int32_t* perm, int32_t* offsets,
+                      int32_t* max_seqlen, void* ws, size_t ws_bytes, void* stream) {
+  if (N < 0 || N >= ((int64_t)1 << 31) || M < 1 || M > 65536) return MOGA_ERR_INVALID_ARG;
+  if (!offsets || !max_seqlen || !aligned4(offsets) || !aligned4(max_seqlen)) return MOGA_ERR_INVALID_ARG;
+  if (N > 0 && (!group_id || !perm || !aligned4(group_id) || !aligned4(perm))) return MOGA_ERR_INVALID_ARG;
+  if (!ws || !aligned16(ws)) return MOGA_ERR_INVALID_ARG;
+  if (ws_bytes < moga_sort_workspace_size(N, M)) return MOGA_ERR_WORKSPACE;
+  DevCtx c;
+  if (!make_ctx(&c, ws, stream)) return MOGA_ERR_CUDA;
+  if (N == 0) {
+    cudaError_t e = cudaMemsetAsync(offsets, 0, (size_t)(M + 1) * 4, c.stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(max_seqlen, 0, 4, c.stream);
+    return from_cuda(e);
+  }
+  const RouteWs w = route_ws(N, M);
+  int32_t* hist = reinterpret_cast<int32_t*>((uint8_t*)ws + w.hist);
+  int32_t* base = reinterpret_cast<int32_t*>((uint8_t*)ws + w.base);
+  mark(MOGA_STAGE_SORT, true, c.stream);
+  if (launch_hist(c, group_id, N, M, hist) != cudaSuccess ||
+      launch_scan(c, hist, ceil_div(N, kTile), M, base, offsets, max_seqlen, nullptr, N, nullptr, nullptr) !=
+          cudaSuccess ||
+      launch_scatter(c, group_id, base, N, M, perm) != cudaSuccess)
+    return MOGA_ERR_CUDA;
+  mark(MOGA_STAGE_SORT, false, c.stream);
+  count(3);
+  return MOGA_OK;
+}
+
 size_t moga_route_ex_workspace_size(int64_t N, int M) {
   if (N < 0 || M < 1) return 0;
   return route_ws(N, M, true).total;

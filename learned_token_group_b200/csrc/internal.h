@@ -38,7 +38,10 @@ cudaError_t launch_route_simt(const DevCtx& c, const void* x, const void* W, con
 cudaError_t launch_scan(const DevCtx& c, const int32_t* hist, int64_t ntiles, int M, int32_t* base,
                         int32_t* offsets, int32_t* max_seqlen, const float* pstat, int64_t N, float* prob_mean,
                         float* balance);
-// Stable scatter of token indices into perm.
+// Per-tile group histograms of caller-given group ids (ids outside [0, M)
+// are skipped and reported as DEV_RANGE).
+cudaError_t launch_hist(const DevCtx& c, const int32_t* group_id, int64_t N, int M, int32_t* hist);
+// Stable scatter of token indices into perm (ids outside [0, M) are skipped).
 cudaError_t launch_scatter(const DevCtx& c, const int32_t* group_id, const int32_t* base, int64_t N, int M,
                            int32_t* perm);
 

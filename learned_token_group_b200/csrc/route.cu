@@ -377,8 +377,9 @@ scatter_kernel(const int32_t* __restrict__ group_id, const int32_t* __restrict__
   __syncthreads();
   const int t = blockIdx.x;
   const int64_t tok = (int64_t)t * kTile + threadIdx.x;
-  const bool valid = tok < N;
-  const int g = valid ? group_id[tok] : -1;
+  const int g0 = tok < N ? group_id[tok] : -1;
+  const bool valid = g0 >= 0 && g0 < M;  // ids out of range were reported by the histogram and are skipped
+  const int g = valid ? g0 : -1;
   const unsigned peers = __match_any_sync(0xffffffffu, g);
   unsigned lt;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt));
@@ -439,6 +440,31 @@ cudaError_t launch_scan(const DevCtx& c, const int32_t* hist, int64_t ntiles, in
                         float* balance) {
   scan_kernel<<<1, 1024, 0, c.stream>>>(hist, (int)ntiles, M, base, offsets, max_seqlen, pstat, (int)N, prob_mean,
                                         balance);
+  return cudaGetLastError();
+}
+
+// Per-tile histograms of given group ids (moga_sort); ids outside [0, M) are
+// skipped and reported.
+__global__ void __launch_bounds__(128)
+hist_kernel(const int32_t* __restrict__ group_id, int N, int M, int32_t* __restrict__ hist, int* status) {
+  extern __shared__ int h[];  // [M]
+  for (int i = threadIdx.x; i < M; i += blockDim.x) h[i] = 0;
+  __syncthreads();
+  const int64_t tok = (int64_t)blockIdx.x * kTile + threadIdx.x;
+  if (tok < N) {
+    const int g = group_id[tok];
+    if (g >= 0 && g < M)
+      atomicAdd(&h[g], 1);
+    else if (status)
+      atomicOr(status, DEV_RANGE);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < M; i += blockDim.x) hist[(int64_t)blockIdx.x * M + i] = h[i];
+}
+
+cudaError_t launch_hist(const DevCtx& c, const int32_t* group_id, int64_t N, int M, int32_t* hist) {
+  const int64_t ntiles = ceil_div(N, kTile);
+  hist_kernel<<<(unsigned)ntiles, 128, (size_t)M * sizeof(int), c.stream>>>(group_id, (int)N, M, hist, c.status);
   return cudaGetLastError();
 }
 
