@@ -458,6 +458,25 @@ def run_ours(args, wl, rank, world, dist):
         moga.sync_status(layer3.ws)
         widened["three_branch_layer_ms"] = ev0.elapsed_time(ev1) / args.steps
         del layer3
+        # the per-frame branch alone (whole-frame windows, read in place),
+        # added into an output as the block does
+        frame = (1, wl.grid[1], wl.grid[2])
+        ws_f = moga.workspace(moga.get_lib().stga_window_attn_workspace_size(
+            wl.grid[0], wl.grid[1], wl.grid[2], moga._int3(frame), wl.H, wl.d_h), dev)
+        out_f = moga.stga_window_attn(inp["q"], inp["k"], inp["v"], wl.grid, frame, ws=ws_f)
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            moga.stga_window_attn(inp["q"], inp["k"], inp["v"], wl.grid, frame, accumulate=True, out=out_f,
+                                  ws=ws_f)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        ms_f = ev0.elapsed_time(ev1) / args.steps
+        L = wl.grid[1] * wl.grid[2]
+        widened["per_frame_branch_ms"] = ms_f
+        widened["per_frame_branch_tflops"] = 4.0 * wl.grid[0] * L * L * wl.H * wl.d_h / (ms_f * 1e-3) / 1e12
+        moga.sync_status(ws_f)
+        del out_f, ws_f
         rt = lambda: moga.route(inp["x"], inp["W_r"], inp["b_r"], wl.M, out=r_out, ws=r_ws)
         rs = lambda: moga.route_stats(inp["x"], inp["W_r"], inp["b_r"], wl.M)
         r_out = moga.route(inp["x"], inp["W_r"], inp["b_r"], wl.M)

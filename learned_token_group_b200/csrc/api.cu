@@ -241,14 +241,20 @@ moga_status stga_body(const DevCtx& c, const void* q, const void* k, const void*
                       float add_scale = 0.5f) {
   const int64_t N = (int64_t)T * Hg * Wg;
   const bool direct = stga_direct(window);
+  // Windows of whole frames are runs of consecutive tokens: no permutation,
+  // no gathered copy, the tiled kernel reads q, k, v in place.
+  const bool contiguous = !direct && window[1] >= Hg && window[2] >= Wg;
   const AttnWs w = attn_ws(N, H, d_h, 0, true, !direct);
   int32_t* permw = reinterpret_cast<int32_t*>(ws + w.permw);
   mark(MOGA_STAGE_STGA_PREP, true, c.stream);
-  if (launch_window_perm(c, T, Hg, Wg, window, permw) != cudaSuccess) return MOGA_ERR_CUDA;
-  count(1);
+  if (!contiguous) {
+    if (launch_window_perm(c, T, Hg, Wg, window, permw) != cudaSuccess) return MOGA_ERR_CUDA;
+    count(1);
+  }
   AttnArgs a{};
   a.direct = direct ? 1 : 0;
-  if (direct) {
+  a.contiguous = contiguous ? 1 : 0;
+  if (direct || contiguous) {
     a.q = q;
     a.k = k;
     a.v = v;
@@ -261,7 +267,7 @@ moga_status stga_body(const DevCtx& c, const void* q, const void* k, const void*
     a.v = ws + w.vh;
   }
   mark(MOGA_STAGE_STGA_PREP, false, c.stream);
-  a.perm = permw;
+  a.perm = contiguous ? nullptr : permw;
   a.gate = nullptr;
   a.out = out;
   a.N = N;
@@ -441,6 +447,19 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t o
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_tokens(CUtensorMap* map, const void* base, uint64_t d_h, uint64_t H, uint64_t N) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d_h, H, N};
+  cuuint64_t strides[2] = {d_h * 2, H * d_h * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)kTile};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;

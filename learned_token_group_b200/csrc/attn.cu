@@ -381,7 +381,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
   dec.nseg = a.nseg;
   dec.tab = tab;
   dec.upw = 1;
-  dec.H = kDirect ? a.H : 0;
+  dec.H = (kDirect || a.contiguous) ? a.H : 0;
   dec.heads = a.H;
   dec.gtab = a.table;
   dec.cap = a.nseg;
@@ -420,24 +420,30 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       tma_prefetch_desc(&tv);
       uint32_t ucnt = 0, kc = 0, vc = 0;
       bool ok = true;
+      // One 128-row tile of head h starting at segment position pos: a row of
+      // the gathered head-major copy (rows = rows per head), or, for
+      // contiguous segments, 128 consecutive tokens read in place.
+      auto load_tile = [&](const CUtensorMap* map, uint64_t* bar, uint8_t* dst, int h, int64_t rows, int pos) {
+#pragma unroll
+        for (int c = 0; c < P::kChunks; ++c) {
+          if (a.contiguous)
+            tma_load_3d(map, bar, dst + c * 16384, c * 64, h, pos);
+          else
+            tma_load_2d(map, bar, dst + c * 16384, c * 64, (int)((int64_t)h * rows + pos));
+        }
+      };
       for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
         const Unit u = dec(idx);
         if (u.q0 >= u.len) continue;
         const bool hb = u.q0 + kTile < u.len;
         const int nkv = (u.kvl + kTile - 1) / kTile;
         if (!mbar_wait(q_empty, (ucnt & 1) ^ 1, wc, 1, ucnt)) break;
-        const int rowq = (int)((int64_t)u.h * N + u.start + u.q0);
         mbar_expect_tx(q_full, (hb ? 2 : 1) * P::kTileBytes);
-#pragma unroll
-        for (int c = 0; c < P::kChunks; ++c) tma_load_2d(&tq, q_full, smem + P::kQA + c * 16384, c * 64, rowq);
-        if (hb) {
-#pragma unroll
-          for (int c = 0; c < P::kChunks; ++c)
-            tma_load_2d(&tq, q_full, smem + P::kQB + c * 16384, c * 64, rowq + kTile);
-        }
+        load_tile(&tq, q_full, smem + P::kQA, u.h, N, u.start + u.q0);
+        if (hb) load_tile(&tq, q_full, smem + P::kQB, u.h, N, u.start + u.q0 + kTile);
         ++ucnt;
         for (int j = 0; j < nkv; ++j) {
-          const int rowk = (int)((int64_t)u.h * kv_rows + u.kvs + j * kTile);
+          const int posk = u.kvs + j * kTile;
           const int ks = kc % kStages;
           if (!mbar_wait(&k_empty[ks], ((kc / kStages) & 1) ^ 1, wc, 2, kc)) { ok = false; break; }
           if (a.debug_withhold_first_k && kc == 0) {
@@ -448,16 +454,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             break;
           }
           mbar_expect_tx(&k_full[ks], P::kTileBytes);
-#pragma unroll
-          for (int c = 0; c < P::kChunks; ++c)
-            tma_load_2d(&tk, &k_full[ks], smem + P::kK0 + ks * P::kTileBytes + c * 16384, c * 64, rowk);
+          load_tile(&tk, &k_full[ks], smem + P::kK0 + ks * P::kTileBytes, u.h, kv_rows, posk);
           ++kc;
           const int vs = vc % kStages;
           if (!mbar_wait(&v_empty[vs], ((vc / kStages) & 1) ^ 1, wc, 3, vc)) { ok = false; break; }
           mbar_expect_tx(&v_full[vs], P::kTileBytes);
-#pragma unroll
-          for (int c = 0; c < P::kChunks; ++c)
-            tma_load_2d(&tv, &v_full[vs], smem + P::kV0 + vs * P::kTileBytes + c * 16384, c * 64, rowk);
+          load_tile(&tv, &v_full[vs], smem + P::kV0 + vs * P::kTileBytes, u.h, kv_rows, posk);
           ++vc;
         }
       }
@@ -752,7 +754,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         live = false;
         if (status) atomicOr(status, DEV_RANGE);
       }
-      const int src = live ? a.perm[u.start + r] : 0;
+      const int src = live ? (a.perm ? a.perm[u.start + r] : u.start + r) : 0;
       float m_run = -INFINITY;
       uint64_t la = f2_pack(0.f, 0.f), lb = la, lc = la, ld = la;  // row sum of P, 8 partial sums
       for (int j = 0; j < nkv; ++j) {
@@ -909,9 +911,15 @@ cudaError_t launch_attention_dh(const DevCtx& c, const AttnArgs& a) {
   // with 128-row boxes.  The in-place kernel copies rows itself and does not
   // read the maps.
   const uint32_t box_rows = (uint32_t)kTile;
-  if (!make_tmap_2d(&mq, a.q, DH, rows, DH * 2, box_rows)) return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&mk, a.k, DH, kv_rows, DH * 2, box_rows)) return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&mv, a.v, DH, kv_rows, DH * 2, box_rows)) return cudaErrorInvalidValue;
+  if (a.contiguous) {  // the caller's [N, H, d_h] tensors, read in place
+    if (!make_tmap_tokens(&mq, a.q, DH, a.H, a.N) || !make_tmap_tokens(&mk, a.k, DH, a.H, a.N) ||
+        !make_tmap_tokens(&mv, a.v, DH, a.H, a.N))
+      return cudaErrorInvalidValue;
+  } else {
+    if (!make_tmap_2d(&mq, a.q, DH, rows, DH * 2, box_rows)) return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&mk, a.k, DH, kv_rows, DH * 2, box_rows)) return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&mv, a.v, DH, kv_rows, DH * 2, box_rows)) return cudaErrorInvalidValue;
+  }
   // groups: the segment table; in place: the loaders' token rows (2 tiles each)
   const int table_ints = a.mode == 0 ? 3 * a.nseg + 1 : (a.direct ? 6 * kTile : 0);
   const size_t smem = P::bytes(table_ints);

@@ -65,6 +65,10 @@ struct AttnArgs {
   // direct = 1: q, k, v are the caller's [N, H, d_h] tensors, read by token
   // index (perm); direct = 0: they are gathered head-major copies [H][N][d_h].
   int direct;
+  // contiguous = 1 (tiled kernel): segments are runs of consecutive tokens
+  // (windows of whole frames), so q, k, v are the caller's [N, H, d_h]
+  // tensors read in place with 3-D maps and perm is the identity (may be null).
+  int contiguous;
   const void* q;
   const void* k;
   const void* v;
@@ -126,5 +130,9 @@ inline int64_t stga_num_windows(int T, int Hg, int Wg, const int* w) {
 // unavailable or the encoding fails.
 bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
                   uint32_t box_rows);
+// Encodes a 3-D bf16 tensor map over [N tokens, H heads, d_h] (d_h innermost)
+// with a box of 64 columns x 1 head x 128 tokens and 128-byte swizzle: one
+// box is a 128-row operand tile of one head, read in place.
+bool make_tmap_tokens(CUtensorMap* map, const void* base, uint64_t d_h, uint64_t H, uint64_t N);
 
 }  // namespace moga

@@ -104,6 +104,10 @@ STGA_CASES = [
     ((1, 4, 6), (1, 4, 6), 2, 128),      # window = whole grid: full attention
     ((6, 30, 52), (3, 8, 8), 2, 128),    # the 480p latent grid, clipped edges
     ((2, 9, 7), (5, 16, 16), 1, 128),    # window larger than the grid
+    # whole-frame windows: runs of consecutive tokens, read in place
+    ((2, 30, 52), (1, 30, 52), 2, 128),  # per-frame attention, 1560 tokens (ragged tail)
+    ((5, 30, 52), (2, 30, 52), 1, 64),   # two frames per window, last window clipped
+    ((3, 7, 9), (2, 20, 20), 2, 64),     # wider than the frame, shorter than the clip
 ]
 
 
@@ -128,8 +132,9 @@ def test_stga_unit_window_is_v():
     assert (out.float() - v.float()).abs().max().item() == 0.0
 
 
-def test_stga_accumulate():
-    grid, window = (3, 10, 12), (3, 8, 8)
+@pytest.mark.parametrize("window", [(3, 8, 8), (1, 10, 12)])
+def test_stga_accumulate(window):
+    grid = (3, 10, 12)
     N = 360
     q, k, v = _qkv(N, 2, 128, seed=77)
     base = torch.randn((N, 2, 128), device="cuda").to(torch.bfloat16)
