@@ -43,6 +43,10 @@ Readings where the pages leave a step open (each one is pinned by a test):
 * combine: out = (MoGA + STGA) / 2 when STGA is on, MoGA alone otherwise; with
   the per-frame branch (attention inside each latent frame) the block output
   is the plain mean of all branches that are on.
+* gradients ("MoGA Router" and "Grouped Attention": the argmax is not
+  differentiable; gradients reach the router through the gate p(g(x)|x) of
+  Eq. 5 and reach q, k, v through the attention given the hard assignment).
+  The assignment g(x) is held fixed; no straight-through term is added.
 
 Every function here is pinned by ``tests/test_oracle_pins.py`` to something
 other than itself (closed forms, a library attention routine, numpy's stable
@@ -58,7 +62,8 @@ import numpy as np
 __all__ = [
     "route", "balance_stats", "counting_sort", "attention_rows", "group_attention",
     "stga_windows", "stga_attention", "frame_attention", "moga_layer",
-    "shot_windows", "stga_shot_attention",
+    "shot_windows", "stga_shot_attention", "attention_lse", "attention_rows_backward",
+    "moga_layer_backward",
 ]
 
 _ROW_BLOCK = 16384
@@ -350,3 +355,92 @@ def moga_layer(x, W_r, b_r, q, k, v, M: int, grid=None, window=None,
     return {"group_id": gid, "gate": gate, "margin": margin, "perm": perm,
             "offsets": offsets, "max_seqlen": max_seqlen, "moga": moga,
             "stga": stga, "frame": frame, "out": out}
+
+
+# ----------------------------------------------------------------------------- training
+def attention_lse(q_rows: np.ndarray, K: np.ndarray) -> np.ndarray:
+    """Natural-log log-sum-exp of each query row's scaled scores q K^T / sqrt(d_h)
+    (the normaliser of Eq. 1's softmax), written out as max + log(sum(exp))."""
+    s = (q_rows @ K.T) / math.sqrt(K.shape[1])
+    m = s.max(axis=1)
+    return m + np.log(np.exp(s - m[:, None]).sum(axis=1))
+
+
+def attention_rows_backward(Q: np.ndarray, K: np.ndarray, V: np.ndarray, dO: np.ndarray):
+    """Gradients of Eq. 1 over one token set of one head, given dO = dL/dO.
+
+    With S = Q K^T / sqrt(d_h), P = softmax_rows(S), O = P V:
+      dV = P^T dO;   dP = dO V^T;
+      dS = P * (dP - rowsum(P * dP))        (Jacobian of the row softmax);
+      dQ = dS K / sqrt(d_h);   dK = dS^T Q / sqrt(d_h).
+    Returns (dQ, dK, dV, O), float64.
+    """
+    c = 1.0 / math.sqrt(K.shape[1])
+    S = (Q @ K.T) * c
+    S = S - S.max(axis=1, keepdims=True)
+    P = np.exp(S)
+    P = P / P.sum(axis=1, keepdims=True)
+    O = P @ V
+    dV = P.T @ dO
+    dP = dO @ V.T
+    dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+    return (dS @ K) * c, (dS.T @ Q) * c, dV, O
+
+
+def moga_layer_backward(x, W_r, b_r, q, k, v, M: int, dout, grid=None, window=None,
+                        per_frame: bool = False):
+    """Gradients of L = sum(dout * out) for the block of ``moga_layer``.
+
+    out = mean over the branches that are on of: MoGA (Eq. 5: gate * SA within
+    the token's group), STGA (SA within each window), per-frame (SA within each
+    frame).  Each branch's share of dout is dout / (number of branches).  The
+    group assignment is held fixed (see the module notes); the gate
+    p = softmax(x W_r^T + b)_g carries the router's gradient:
+      dgate_i = sum_{h,c} w * dout[i,h,c] * SA_i[h,c];
+      dr_ij   = dgate_i * p_ig * ([j == g] - p_ij)      (softmax Jacobian);
+      dW_r = dr^T x;  db_r = sum_i dr_i;  dx = dr W_r   (the router's part of dx).
+    Returns a dict of float64 arrays dx [N, d], dW_r [M, d], db_r [M],
+    dq, dk, dv [N, H, d_h], plus dgate [N].
+    """
+    X = _f64(x)
+    W = _f64(W_r)
+    b = np.zeros(M) if b_r is None else _f64(b_r)
+    Q, Kt, Vt, dOut = _f64(q), _f64(k), _f64(v), _f64(dout)
+    N, H, d_h = Q.shape
+    r = X @ W.T + b                                         # Eq. 2
+    e = np.exp(r - r.max(axis=1, keepdims=True))
+    p = e / e.sum(axis=1, keepdims=True)                    # Eq. 3
+    g = np.argmax(r, axis=1)                                # Eq. 4
+    gate = p[np.arange(N), g]
+    nb = 1 + (window is not None) + bool(per_frame)
+    w = 1.0 / nb
+    dq = np.zeros_like(Q)
+    dk = np.zeros_like(Q)
+    dv = np.zeros_like(Q)
+    dgate = np.zeros(N)
+
+    def branch(sets, scale_rows):
+        for idx in sets:
+            if idx.size == 0:
+                continue
+            for h in range(H):
+                dO = w * dOut[idx, h]
+                if scale_rows is not None:
+                    dO = dO * scale_rows[idx][:, None]
+                gq, gk, gv, O = attention_rows_backward(Q[idx, h], Kt[idx, h], Vt[idx, h], dO)
+                dq[idx, h] += gq
+                dk[idx, h] += gk
+                dv[idx, h] += gv
+                if scale_rows is not None:                  # d/dgate of gate * SA
+                    dgate[idx] += w * (dOut[idx, h] * O).sum(axis=1)
+
+    branch([np.nonzero(g == m)[0] for m in range(M)], gate)
+    if window is not None:
+        branch(stga_windows(*grid, window), None)
+    if per_frame:
+        branch(stga_windows(*grid, (1, grid[1], grid[2])), None)
+    onehot = np.zeros((N, M))
+    onehot[np.arange(N), g] = 1.0
+    dr = (dgate * gate)[:, None] * (onehot - p)
+    return {"dx": dr @ W, "dW_r": dr.T @ X, "db_r": dr.sum(axis=0),
+            "dq": dq, "dk": dk, "dv": dv, "dgate": dgate}

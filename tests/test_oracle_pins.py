@@ -430,10 +430,119 @@ def check_shot_stga(o):
                            base[first_win])
 
 
+def _fd_problem(seed, M=3, window=(1, 2, 3), per_frame=True, bias=True):
+    rng = np.random.default_rng(seed)
+    grid, N, d, H, E = (2, 3, 4), 24, 5, 2, 4
+    x = rng.normal(size=(N, d))
+    W = rng.normal(size=(M, d))
+    b = rng.normal(size=M) if bias else None
+    q, k, v = (rng.normal(size=(N, H, E)) for _ in range(3))
+    dout = rng.normal(size=(N, H, E))
+    return dict(x=x, W_r=W, b_r=b, q=q, k=k, v=v, M=M, grid=grid, window=window, per_frame=per_frame, dout=dout)
+
+
+def check_backward_finite_differences(o):
+    """Every gradient of L = sum(dout * out) against central differences of
+    the (separately pinned) forward, on sampled coordinates of every input."""
+    for seed, kw in ((30, {}), (31, {"window": None, "per_frame": False}), (32, {"per_frame": False})):
+        pr = _fd_problem(seed, **kw)
+        fwd_args = {k_: pr[k_] for k_ in ("x", "W_r", "b_r", "q", "k", "v")}
+        M, grid, window, pf, dout = pr["M"], pr["grid"], pr["window"], pr["per_frame"], pr["dout"]
+
+        def loss(a):
+            res = o.moga_layer(a["x"], a["W_r"], a["b_r"], a["q"], a["k"], a["v"], M, grid=grid, window=window,
+                               per_frame=pf)
+            return float(np.sum(dout * res["out"]))
+
+        _, _, margin = o.route(pr["x"], pr["W_r"], pr["b_r"])
+        assert margin.min() > 1e-4          # a step of 1e-6 cannot move a token to another group
+        g = o.moga_layer_backward(pr["x"], pr["W_r"], pr["b_r"], pr["q"], pr["k"], pr["v"], M, dout, grid=grid,
+                                  window=window, per_frame=pf)
+        names = {"x": "dx", "W_r": "dW_r", "b_r": "db_r", "q": "dq", "k": "dk", "v": "dv"}
+        rng = np.random.default_rng(seed + 100)
+        eps = 1e-6
+        for name, gname in names.items():
+            base = fwd_args[name]
+            flat = base.reshape(-1)
+            for c in rng.choice(flat.size, size=min(flat.size, 12), replace=False):
+                a = dict(fwd_args)
+                plus = flat.copy()
+                plus[c] += eps
+                minus = flat.copy()
+                minus[c] -= eps
+                a[name] = plus.reshape(base.shape)
+                lp = loss(a)
+                a[name] = minus.reshape(base.shape)
+                lm = loss(a)
+                num = (lp - lm) / (2 * eps)
+                ana = g[gname].reshape(-1)[c]
+                assert abs(num - ana) <= 1e-6 * (1 + abs(num)), (seed, gname, int(c), num, ana)
+
+
+def check_backward_dense_autograd(o):
+    """The same gradients from torch autograd (float64) through a dense
+    formulation: every branch as N x N attention with a membership mask."""
+    pr = _fd_problem(40, M=4)
+    t = {k_: torch.tensor(pr[k_], dtype=torch.float64, requires_grad=True)
+         for k_ in ("x", "W_r", "b_r", "q", "k", "v")}
+    N, H, E = pr["q"].shape
+    T, Hg, Wg = pr["grid"]
+    r = t["x"] @ t["W_r"].T + t["b_r"]
+    p = torch.softmax(r, dim=1)
+    gid = torch.argmax(r.detach(), dim=1)
+    gate = p.gather(1, gid[:, None])[:, 0]
+    tok = torch.arange(N)
+    tt, hh, ww = tok // (Hg * Wg), (tok // Wg) % Hg, tok % Wg
+    wt, wh, wwid = pr["window"]
+    win = (tt // wt) * 1000 + (hh // wh) * 100 + ww // wwid
+    masks = [gid[:, None] == gid[None, :], win[:, None] == win[None, :], tt[:, None] == tt[None, :]]
+
+    def dense(mask):
+        s = torch.einsum("ihe,jhe->hij", t["q"], t["k"]) / math.sqrt(E)
+        s = s.masked_fill(~mask[None], float("-inf"))
+        return torch.einsum("hij,jhe->ihe", torch.softmax(s, dim=2), t["v"])
+
+    out = (gate[:, None, None] * dense(masks[0]) + dense(masks[1]) + dense(masks[2])) / 3
+    (out * torch.tensor(pr["dout"])).sum().backward()
+    g = o.moga_layer_backward(pr["x"], pr["W_r"], pr["b_r"], pr["q"], pr["k"], pr["v"], pr["M"], pr["dout"],
+                              grid=pr["grid"], window=pr["window"], per_frame=True)
+    for name, gname in (("x", "dx"), ("W_r", "dW_r"), ("b_r", "db_r"), ("q", "dq"), ("k", "dk"), ("v", "dv")):
+        assert np.allclose(g[gname], t[name].grad.numpy(), rtol=1e-9, atol=1e-11), gname
+
+
+def check_backward_special_cases(o):
+    pr = _fd_problem(50, M=1, window=None, per_frame=False)
+    g = o.moga_layer_backward(pr["x"], pr["W_r"], pr["b_r"], pr["q"], pr["k"], pr["v"], 1, pr["dout"])
+    # one group: the gate is identically 1, so the router gets no gradient
+    assert np.abs(g["dW_r"]).max() == 0 and np.abs(g["db_r"]).max() == 0 and np.abs(g["dx"]).max() == 0
+    # a token alone in its group: out = gate * v, so dv = gate * dout and dq = dk = 0
+    rng = np.random.default_rng(51)
+    N, d, H, E = 6, 3, 1, 4
+    x = np.eye(N, d) * 5.0
+    x[3:] = 0.0
+    x[3:, 0] = 5.0                     # tokens 0, 3, 4, 5 -> group 0; 1 -> group 1; 2 -> group 2
+    W = np.eye(3, d)
+    q, k, v, dout = (rng.normal(size=(N, H, E)) for _ in range(4))
+    g = o.moga_layer_backward(x, W, None, q, k, v, 3, dout)
+    _, gate, _ = o.route(x, W, None)
+    assert np.allclose(g["dv"][1], gate[1] * dout[1], rtol=0, atol=1e-14)
+    assert np.abs(g["dq"][1]).max() < 1e-15 and np.abs(g["dk"][1]).max() < 1e-15
+
+
+def check_attention_lse(o):
+    from scipy.special import logsumexp
+    rng = np.random.default_rng(60)
+    q, K = rng.normal(size=(7, 16)) * 3, rng.normal(size=(33, 16)) * 3
+    ref = logsumexp(q @ K.T / 4.0, axis=1)
+    assert np.allclose(o.attention_lse(q, K), ref, rtol=0, atol=1e-12)
+
+
 CHECKS = [check_route_closed_form, check_route_ties_and_M1, check_route_brute, check_counting_sort,
           check_full_attention_when_M1, check_group_equals_subset_attention, check_special_cases,
           check_brute_force_tiny, check_permutation_equivariance, check_stga, check_layer_combine,
-          check_golden, check_three_branch_mean, check_balance_stats, check_shot_stga]
+          check_golden, check_three_branch_mean, check_balance_stats, check_shot_stga,
+          check_backward_finite_differences, check_backward_dense_autograd, check_backward_special_cases,
+          check_attention_lse]
 
 
 @pytest.mark.parametrize("check", CHECKS, ids=[c.__name__ for c in CHECKS])
@@ -500,6 +609,41 @@ def _shot_ignores_cuts(T, Hg, Wg, window, shot_start, aug_prev=2, aug_next=2):
     return _ORIG_SHOT(T, Hg, Wg, window, [0, T], aug_prev, aug_next)
 
 
+def _bwd_no_jacobian_term(Q, K, V, dO):            # dS = P * dP, the row-sum term dropped
+    c = 1.0 / math.sqrt(K.shape[1])
+    S = (Q @ K.T) * c
+    P = np.exp(S - S.max(1, keepdims=True))
+    P = P / P.sum(1, keepdims=True)
+    dS = P * (dO @ V.T)
+    return (dS @ K) * c, (dS.T @ Q) * c, P.T @ dO, P @ V
+
+
+def _bwd_dk_untransposed(Q, K, V, dO):              # dK = dS Q instead of dS^T Q
+    dq, dk, dv, O = _ORIG_ABWD(Q, K, V, dO)
+    c = 1.0 / math.sqrt(K.shape[1])
+    S = (Q @ K.T) * c
+    P = np.exp(S - S.max(1, keepdims=True))
+    P = P / P.sum(1, keepdims=True)
+    dP = dO @ V.T
+    dS = P * (dP - (P * dP).sum(1, keepdims=True))
+    return dq, (dS @ Q) * c, dv, O
+
+
+def _bwd_router_sign(*a, **kw):                     # gradient ascent on the router
+    g = _ORIG_LBWD(*a, **kw)
+    for n in ("dx", "dW_r", "db_r"):
+        g[n] = -g[n]
+    return g
+
+
+def _lse_no_scale(q_rows, K):
+    s = q_rows @ K.T
+    m = s.max(axis=1)
+    return m + np.log(np.exp(s - m[:, None]).sum(axis=1))
+
+
+_ORIG_ABWD = oracle.attention_rows_backward
+_ORIG_LBWD = oracle.moga_layer_backward
 _ORIG_SHOT = oracle.shot_windows
 _ORIG_GA = oracle.group_attention
 _ORIG_WIN = oracle.stga_windows
@@ -517,6 +661,10 @@ MUTANTS = {
     "shot_augments_queries": ("shot_windows", _shot_aug_on_queries),
     "shot_augmentation_short": ("shot_windows", _shot_aug_short),
     "shot_cuts_ignored": ("shot_windows", _shot_ignores_cuts),
+    "bwd_softmax_jacobian_term_dropped": ("attention_rows_backward", _bwd_no_jacobian_term),
+    "bwd_dk_untransposed": ("attention_rows_backward", _bwd_dk_untransposed),
+    "bwd_router_sign_flipped": ("moga_layer_backward", _bwd_router_sign),
+    "lse_without_scale": ("attention_lse", _lse_no_scale),
 }
 
 
