@@ -237,6 +237,58 @@ moga_status moga_layer(const void* x, const void* W_r, const float* b_r, moga_dt
                        int Wg, const int* window, void* out, int32_t* group_id, float* gate, int32_t* perm,
                        int32_t* offsets, void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- training
+ * moga_layer_train: the forward of moga_layer that keeps what the backward
+ * pass needs.  Outputs as moga_layer plus
+ *   o_moga   bf16 [N, H, d_h]  MoGA branch alone, gate * SA (Eq. 5)
+ *   o_stga   bf16 [N, H, d_h]  STGA branch alone (window != NULL; else unused)
+ *   lse_moga fp32 [H, N]       natural-log log-sum-exp of each query's scaled
+ *                              scores q.k/sqrt(d_h) within its group, at the
+ *                              token's sorted position (perm order)
+ *   lse_stga fp32 [H, N]       the same within its STGA window, in window
+ *                              order (windows as in stga_window_attn, tokens
+ *                              of a window in index order)
+ *   out = 0.5 * (o_moga + o_stga), or o_moga when window == NULL (out may then
+ *   be o_moga itself; with a window the three outputs must be distinct).
+ * Workspace: moga_layer_train_workspace_size(...) bytes. */
+size_t moga_layer_train_workspace_size(int64_t N, int H, int d_h, int M, int T, int Hg, int Wg, const int* window);
+moga_status moga_layer_train(const void* x, const void* W_r, const float* b_r, moga_dtype x_dt, const void* q,
+                             const void* k, const void* v, int64_t N, int d, int H, int d_h, int M, int T, int Hg,
+                             int Wg, const int* window, void* out, void* o_moga, void* o_stga, float* lse_moga,
+                             float* lse_stga, int32_t* group_id, float* gate, int32_t* perm, int32_t* offsets,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* moga_layer_backward: gradients of a scalar loss L through the block, given
+ * dout = dL/dout (bf16 [N, H, d_h]) and what moga_layer_train returned
+ * ("MoGA Router" and "Grouped Attention" sections: the argmax assignment is
+ * not differentiable; the router learns through the gate p(g(x)|x) of Eq. 5,
+ * q, k, v through the attention of each branch with the assignment held
+ * fixed).  With w = 1/2 (window != NULL) or 1:
+ *   dq, dk, dv  bf16 [N, H, d_h]: w * gate * dout through MoGA's attention
+ *               plus w * dout through STGA's (overwritten, not accumulated);
+ *   dgate_i   = w * sum_{h,c} dout * o_moga / gate_i;
+ *   dr_ij     = dgate_i * p_ig * ([j == g_i] - p_ij) for the router's
+ *               softmax p = softmax(x W_r^T + b);
+ *   dx        = dr W_r   (x's dtype, [N, d]: the router's share of dL/dx;
+ *               q, k, v are inputs of the block, so the projections that
+ *               produce them are the caller's);
+ *   dW_r      = dr^T x   (fp32 [M, d], overwritten);
+ *   db_r      = sum_i dr_i (fp32 [M], overwritten; may be NULL).
+ * The inputs (x, W_r, b_r, q, k, v, group_id, gate, perm, offsets, o_moga,
+ * o_stga, lse_*) must be those of the forward call.  dW_r and db_r are
+ * summed in a fixed order (deterministic); bf16 outputs are rounded once per
+ * branch (the STGA share is added to the MoGA share in bf16).
+ * Workspace: moga_layer_backward_workspace_size(N, d, H, d_h, M) bytes
+ * (head-major copies of q, k, v and dO, plus per-token scratch). */
+size_t moga_layer_backward_workspace_size(int64_t N, int d, int H, int d_h, int M);
+moga_status moga_layer_backward(const void* dout, const void* x, const void* W_r, const float* b_r, moga_dtype x_dt,
+                                const void* q, const void* k, const void* v, int64_t N, int d, int H, int d_h, int M,
+                                int T, int Hg, int Wg, const int* window, const void* o_moga, const void* o_stga,
+                                const float* lse_moga, const float* lse_stga, const int32_t* group_id,
+                                const float* gate, const int32_t* perm, const int32_t* offsets, void* dx,
+                                float* dW_r, float* db_r, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                                void* stream);
+
 /* moga_layer_ex: the visual block with a choice of branches, as in the pages'
  * "Spatial-Temporal Group Attention (STGA)" section (each token's output is
  * the mean of its MoGA group, its STGA window and its per-frame group):

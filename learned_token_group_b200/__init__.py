@@ -20,7 +20,8 @@ import torch
 
 __all__ = ["MogaError", "get_lib", "LIB_PATH", "HEADER_PATH", "route", "group_attn", "stga_window_attn",
            "moga_layer", "sync_status", "workspace", "MogaLayer", "exported_names", "kernel_launches",
-           "set_timing_events", "STAGES", "Pipeline", "stga_shot_attn", "moga_layer_shots", "sort"]
+           "set_timing_events", "STAGES", "Pipeline", "stga_shot_attn", "moga_layer_shots", "sort",
+           "layer_train", "layer_backward", "MogaFunction"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoga.so")
@@ -83,6 +84,12 @@ def get_lib():
         "moga_pipe_submit": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
         "moga_pipe_sync": (_I, [_P]),
         "moga_pipe_destroy": (_I, [_P]),
+        "moga_layer_train_workspace_size": (_SZ, [_I64, _I, _I, _I, _I, _I, _I, _P]),
+        "moga_layer_train": (_I, [_P, _P, _P, _I, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _I, _P,
+                                  _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+        "moga_layer_backward_workspace_size": (_SZ, [_I64, _I, _I, _I, _I]),
+        "moga_layer_backward": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _I, _P,
+                                     _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -381,6 +388,95 @@ def moga_layer(x, W_r, b_r, q, k, v, M: int, grid=None, window=None, per_frame: 
     layer(x, W_r, b_r, q, k, v)
     return {"out": layer.out, "group_id": layer.group_id, "gate": layer.gate, "perm": layer.perm,
             "offsets": layer.offsets, "ws": layer.ws}
+
+
+def layer_train(x, W_r, b_r, q, k, v, M: int, grid=None, window=None, ws=None):
+    """Training forward of one block (moga_layer_train in moga.h): returns
+    dict(out, o_moga, o_stga, lse_moga, lse_stga, group_id, gate, perm,
+    offsets, ws); everything but out is what ``layer_backward`` needs."""
+    lib = get_lib()
+    N, d = x.shape
+    _, H, d_h = q.shape
+    for n, t in (("x", x), ("W_r", W_r), ("q", q), ("k", k), ("v", v)):
+        _dev_tensor(t, n)
+    dev = q.device
+    grid3 = tuple(int(g) for g in grid) if grid is not None else (0, 0, 0)
+    w3 = _int3(window) if window is not None else None
+    x_dt = {torch.float32: MOGA_F32, torch.bfloat16: MOGA_BF16}[x.dtype]
+    mat = lambda: torch.empty((N, H, d_h), dtype=torch.bfloat16, device=dev)
+    r = {"out": mat(), "o_moga": mat(), "o_stga": mat() if window is not None else None,
+         "lse_moga": torch.empty((H, N), dtype=torch.float32, device=dev),
+         "lse_stga": torch.empty((H, N), dtype=torch.float32, device=dev) if window is not None else None,
+         "group_id": torch.empty(N, dtype=torch.int32, device=dev),
+         "gate": torch.empty(N, dtype=torch.float32, device=dev),
+         "perm": torch.empty(N, dtype=torch.int32, device=dev),
+         "offsets": torch.empty(M + 1, dtype=torch.int32, device=dev)}
+    need = lib.moga_layer_train_workspace_size(N, H, d_h, M, *grid3, w3)
+    if ws is None or ws.numel() < need:
+        ws = workspace(need, dev)
+    st = lib.moga_layer_train(_ptr(x), _ptr(W_r), _ptr(b_r), x_dt, _ptr(q), _ptr(k), _ptr(v), N, d, H, d_h, M,
+                              *grid3, w3, _ptr(r["out"]), _ptr(r["o_moga"]), _ptr(r["o_stga"]),
+                              _ptr(r["lse_moga"]), _ptr(r["lse_stga"]), _ptr(r["group_id"]), _ptr(r["gate"]),
+                              _ptr(r["perm"]), _ptr(r["offsets"]), _ptr(ws), ws.numel(), _stream(dev))
+    _check(st, "moga_layer_train")
+    r["ws"] = ws
+    return r
+
+
+def layer_backward(dout, saved, x, W_r, b_r, q, k, v, M: int, grid=None, window=None, ws=None):
+    """Gradients of one block (moga_layer_backward in moga.h) from dout and
+    the dict ``layer_train`` returned: dict(dx, dW_r, db_r, dq, dk, dv, ws).
+    db_r is None when b_r is None."""
+    lib = get_lib()
+    N, d = x.shape
+    _, H, d_h = q.shape
+    _dev_tensor(dout, "dout", torch.bfloat16)
+    dev = q.device
+    grid3 = tuple(int(g) for g in grid) if grid is not None else (0, 0, 0)
+    w3 = _int3(window) if window is not None else None
+    x_dt = {torch.float32: MOGA_F32, torch.bfloat16: MOGA_BF16}[x.dtype]
+    g = {"dx": torch.empty_like(x), "dW_r": torch.empty((M, d), dtype=torch.float32, device=dev),
+         "db_r": torch.empty(M, dtype=torch.float32, device=dev) if b_r is not None else None,
+         "dq": torch.empty_like(q), "dk": torch.empty_like(q), "dv": torch.empty_like(q)}
+    need = lib.moga_layer_backward_workspace_size(N, d, H, d_h, M)
+    if ws is None or ws.numel() < need:
+        ws = workspace(need, dev)
+    s = saved
+    st = lib.moga_layer_backward(_ptr(dout), _ptr(x), _ptr(W_r), _ptr(b_r), x_dt, _ptr(q), _ptr(k), _ptr(v), N, d,
+                                 H, d_h, M, *grid3, w3, _ptr(s["o_moga"]), _ptr(s["o_stga"]), _ptr(s["lse_moga"]),
+                                 _ptr(s["lse_stga"]), _ptr(s["group_id"]), _ptr(s["gate"]), _ptr(s["perm"]),
+                                 _ptr(s["offsets"]), _ptr(g["dx"]), _ptr(g["dW_r"]), _ptr(g["db_r"]),
+                                 _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(ws), ws.numel(), _stream(dev))
+    _check(st, "moga_layer_backward")
+    g["ws"] = ws
+    return g
+
+
+class MogaFunction(torch.autograd.Function):
+    """The block as an autograd function: out = MogaFunction.apply(x, W_r,
+    b_r, q, k, v, M, grid, window).  Forward runs ``layer_train``, backward
+    ``layer_backward``; the group assignment is held fixed, so gradients
+    reach the router through the gate only."""
+
+    @staticmethod
+    def forward(ctx, x, W_r, b_r, q, k, v, M, grid=None, window=None):
+        r = layer_train(x.contiguous(), W_r.contiguous(), b_r, q.contiguous(), k.contiguous(), v.contiguous(), M,
+                        grid, window)
+        ctx.save_for_backward(x, W_r, q, k, v)
+        ctx.b_r = b_r
+        ctx.saved = {n: r[n] for n in ("o_moga", "o_stga", "lse_moga", "lse_stga", "group_id", "gate", "perm",
+                                       "offsets")}
+        ctx.args = (M, grid, window)
+        return r["out"]
+
+    @staticmethod
+    def backward(ctx, dout):
+        x, W_r, q, k, v = ctx.saved_tensors
+        M, grid, window = ctx.args
+        g = layer_backward(dout.contiguous().to(torch.bfloat16), ctx.saved, x, W_r, ctx.b_r, q, k, v, M, grid,
+                           window)
+        db = g["db_r"] if ctx.b_r is not None else None
+        return g["dx"], g["dW_r"].to(W_r.dtype), db, g["dq"], g["dk"], g["dv"], None, None, None
 
 
 def _host_tensor(t: torch.Tensor, name: str, dtype, shape):

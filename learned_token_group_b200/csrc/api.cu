@@ -201,7 +201,7 @@ moga_status route_body(const DevCtx& c, const void* x, const void* W, const floa
 
 moga_status group_attn_body(const DevCtx& c, const void* q, const void* k, const void* v, const int32_t* perm,
                             const int32_t* offsets, const float* gate, int64_t N, int H, int d_h, int M,
-                            float out_scale, void* out, uint8_t* ws) {
+                            float out_scale, void* out, uint8_t* ws, float* lse = nullptr) {
   if (N == 0) return MOGA_OK;
   const AttnWs w = attn_ws(N, H, d_h, M, false);
   int32_t* table = reinterpret_cast<int32_t*>(ws + w.table);
@@ -227,6 +227,7 @@ moga_status group_attn_body(const DevCtx& c, const void* q, const void* k, const
   a.mode = 0;
   a.table = table;
   a.nseg = M;
+  a.lse = lse;
   a.debug_withhold_first_k = g_debug_inject.load(std::memory_order_relaxed) == 1;
   mark(MOGA_STAGE_GROUP_ATTN, true, c.stream);
   const cudaError_t e = launch_attention(c, a);
@@ -238,7 +239,7 @@ moga_status group_attn_body(const DevCtx& c, const void* q, const void* k, const
 // accumulate == 0: out = STGA; otherwise out += add_scale * STGA.
 moga_status stga_body(const DevCtx& c, const void* q, const void* k, const void* v, int T, int Hg, int Wg,
                       const int* window, int H, int d_h, int accumulate, void* out, uint8_t* ws,
-                      float add_scale = 0.5f) {
+                      float add_scale = 0.5f, float* lse = nullptr) {
   const int64_t N = (int64_t)T * Hg * Wg;
   const bool direct = stga_direct(window);
   // Windows of whole frames are runs of consecutive tokens: no permutation,
@@ -284,12 +285,91 @@ moga_status stga_body(const DevCtx& c, const void* q, const void* k, const void*
   a.wt = window[0];
   a.wh = window[1];
   a.ww = window[2];
+  a.lse = lse;
   a.debug_withhold_first_k = g_debug_inject.load(std::memory_order_relaxed) == 1;
   mark(MOGA_STAGE_STGA_ATTN, true, c.stream);
   const cudaError_t e = launch_attention(c, a);
   mark(MOGA_STAGE_STGA_ATTN, false, c.stream);
   count(1);
   return from_cuda(e);
+}
+
+// ------------------------------------------------------------------ training
+struct BwdWs {
+  size_t table, permw, qh, kh, vh, doh, dsum, dgate, route, total;
+};
+BwdWs bwd_ws(int64_t N, int d, int H, int d_h, int M) {
+  Carve c;
+  BwdWs w;
+  const size_t mat = (size_t)N * H * d_h * 2;
+  w.table = c.take((size_t)(3 * M + 1) * 4);
+  w.permw = c.take((size_t)N * 4);
+  w.qh = c.take(mat);
+  w.kh = c.take(mat);
+  w.vh = c.take(mat);
+  w.doh = c.take(mat);
+  w.dsum = c.take((size_t)N * H * 4);
+  w.dgate = c.take((size_t)N * 4);
+  w.route = c.take(route_bwd_ws_bytes(N, d, M));
+  w.total = c.off;
+  return w;
+}
+
+// One branch of the attention backward: dO and D, then dK/dV, then dQ.
+// mode 0: groups (perm, offsets, gate); mode 1: STGA windows (window order).
+moga_status attn_bwd_branch(const DevCtx& c, const BwdWs& w, uint8_t* ws, int mode, const void* dout, const void* o,
+                            const float* lse, const void* q, const void* k, const void* v, const int32_t* perm,
+                            const int32_t* offsets, const float* gate, float wgt, int64_t N, int H, int d_h, int M,
+                            int T, int Hg, int Wg, const int* window, int accumulate, void* dq, void* dk, void* dv) {
+  int32_t* table = reinterpret_cast<int32_t*>(ws + w.table);
+  int32_t* permw = reinterpret_cast<int32_t*>(ws + w.permw);
+  float* dsum = reinterpret_cast<float*>(ws + w.dsum);
+  float* dgate = reinterpret_cast<float*>(ws + w.dgate);
+  const int32_t* sp = perm;
+  if (mode == 0) {
+    if (launch_seg_table(c, offsets, M, H, N, table, 1) != cudaSuccess) return MOGA_ERR_CUDA;
+  } else {
+    if (launch_window_perm(c, T, Hg, Wg, window, permw) != cudaSuccess) return MOGA_ERR_CUDA;
+    sp = permw;
+  }
+  if (launch_gather(c, q, k, v, sp, N, H, d_h, ws + w.qh, ws + w.kh, ws + w.vh) != cudaSuccess) return MOGA_ERR_CUDA;
+  if (launch_bwd_prep(c, dout, o, sp, mode == 0 ? gate : nullptr, wgt, N, H, d_h, ws + w.doh, dsum,
+                      mode == 0 ? dgate : nullptr) != cudaSuccess)
+    return MOGA_ERR_CUDA;
+  count(3);
+  BwdArgs a{};
+  a.q = ws + w.qh;
+  a.k = ws + w.kh;
+  a.v = ws + w.vh;
+  a.dout = ws + w.doh;
+  a.lse = lse;
+  a.dsum = dsum;
+  a.perm = sp;
+  a.N = N;
+  a.H = H;
+  a.d_h = d_h;
+  a.accumulate = accumulate;
+  a.mode = mode;
+  if (mode == 0) {
+    a.table = table;
+    a.nseg = M;
+  } else {
+    a.nseg = (int)stga_num_windows(T, Hg, Wg, window);
+    a.T = T;
+    a.Hg = Hg;
+    a.Wg = Wg;
+    a.wt = window[0];
+    a.wh = window[1];
+    a.ww = window[2];
+  }
+  a.out1 = dv;
+  a.out2 = dk;
+  if (launch_attn_bwd(c, a, false) != cudaSuccess) return MOGA_ERR_CUDA;
+  a.out1 = dq;
+  a.out2 = nullptr;
+  if (launch_attn_bwd(c, a, true) != cudaSuccess) return MOGA_ERR_CUDA;
+  count(2);
+  return MOGA_OK;
 }
 
 moga_status check_route_args(const void* x, const void* W_r, const float* b_r, moga_dtype dt, int64_t N, int d,
@@ -742,6 +822,101 @@ moga_status moga_layer(const void* x, const void* W_r, const float* b_r, moga_dt
   const float scale = window ? 0.5f : 1.0f;
   if ((st = group_attn_body(c, q, k, v, perm, offsets, gate, N, H, d_h, M, scale, out, w)) != MOGA_OK) return st;
   if (window) return stga_body(c, q, k, v, T, Hg, Wg, window, H, d_h, 1, out, w);
+  return MOGA_OK;
+}
+
+size_t moga_layer_train_workspace_size(int64_t N, int H, int d_h, int M, int T, int Hg, int Wg, const int* window) {
+  return moga_layer_workspace_size(N, H, d_h, M, T, Hg, Wg, window);
+}
+
+moga_status moga_layer_train(const void* x, const void* W_r, const float* b_r, moga_dtype x_dt, const void* q,
+                             const void* k, const void* v, int64_t N, int d, int H, int d_h, int M, int T, int Hg,
+                             int Wg, const int* window, void* out, void* o_moga, void* o_stga, float* lse_moga,
+                             float* lse_stga, int32_t* group_id, float* gate, int32_t* perm, int32_t* offsets,
+                             void* ws, size_t ws_bytes, void* stream) {
+  moga_status st = check_route_args(x, W_r, b_r, x_dt, N, d, M, group_id, gate, perm, offsets, offsets);
+  if (st != MOGA_OK) return st;
+  if ((st = check_qkv(q, k, v, out)) != MOGA_OK) return st;
+  if ((st = check_attn_shape(N, H, d_h)) != MOGA_OK) return st;
+  if (!o_moga || !aligned16(o_moga) || (N > 0 && (!lse_moga || !aligned4(lse_moga)))) return MOGA_ERR_INVALID_ARG;
+  if (window) {
+    int64_t n = 0;
+    if ((st = check_window(T, Hg, Wg, window, &n)) != MOGA_OK) return st;
+    if (n != N) return MOGA_ERR_INVALID_ARG;
+    if (!o_stga || !aligned16(o_stga) || (N > 0 && (!lse_stga || !aligned4(lse_stga)))) return MOGA_ERR_INVALID_ARG;
+    if (out == o_moga || out == o_stga || o_moga == o_stga) return MOGA_ERR_INVALID_ARG;
+  }
+  if (!ws || !aligned16(ws)) return MOGA_ERR_INVALID_ARG;
+  if (ws_bytes < moga_layer_train_workspace_size(N, H, d_h, M, T, Hg, Wg, window)) return MOGA_ERR_WORKSPACE;
+  DevCtx c;
+  if (!make_ctx(&c, ws, stream)) return MOGA_ERR_CUDA;
+  uint8_t* w = (uint8_t*)ws;
+  int32_t* max_seqlen = reinterpret_cast<int32_t*>(w + 16);
+  if ((st = route_body(c, x, W_r, b_r, x_dt, N, d, M, group_id, gate, perm, offsets, max_seqlen, w)) != MOGA_OK)
+    return st;
+  if (N == 0) return MOGA_OK;
+  if ((st = group_attn_body(c, q, k, v, perm, offsets, gate, N, H, d_h, M, 1.0f, o_moga, w, lse_moga)) != MOGA_OK)
+    return st;
+  const int64_t n = N * H * d_h;
+  if (window) {
+    if ((st = stga_body(c, q, k, v, T, Hg, Wg, window, H, d_h, 0, o_stga, w, 1.0f, lse_stga)) != MOGA_OK) return st;
+    if (launch_mean2(c, o_moga, o_stga, n, out) != cudaSuccess) return MOGA_ERR_CUDA;
+    count(1);
+  } else if (out != o_moga) {
+    if (cudaMemcpyAsync(out, o_moga, (size_t)n * 2, cudaMemcpyDeviceToDevice, c.stream) != cudaSuccess)
+      return MOGA_ERR_CUDA;
+  }
+  return MOGA_OK;
+}
+
+size_t moga_layer_backward_workspace_size(int64_t N, int d, int H, int d_h, int M) {
+  if (N < 0 || d < 1 || H < 1 || M < 1 || M > 1024 || (d_h != 64 && d_h != 128)) return 0;
+  return bwd_ws(N, d, H, d_h, M).total;
+}
+
+moga_status moga_layer_backward(const void* dout, const void* x, const void* W_r, const float* b_r, moga_dtype x_dt,
+                                const void* q, const void* k, const void* v, int64_t N, int d, int H, int d_h, int M,
+                                int T, int Hg, int Wg, const int* window, const void* o_moga, const void* o_stga,
+                                const float* lse_moga, const float* lse_stga, const int32_t* group_id,
+                                const float* gate, const int32_t* perm, const int32_t* offsets, void* dx,
+                                float* dW_r, float* db_r, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                                void* stream) {
+  // the routing results are inputs here; the forward's checks cover them
+  moga_status st = check_route_args(x, W_r, b_r, x_dt, N, d, M, group_id, gate, perm, offsets, offsets);
+  if (st != MOGA_OK) return st;
+  if ((st = check_qkv(q, k, v, dout)) != MOGA_OK) return st;
+  if ((st = check_attn_shape(N, H, d_h)) != MOGA_OK) return st;
+  if ((st = check_qkv(dq, dk, dv, o_moga)) != MOGA_OK) return st;
+  if (!dW_r || !aligned4(dW_r) || (db_r && !aligned4(db_r))) return MOGA_ERR_INVALID_ARG;
+  if (N > 0 && (!dx || !aligned16(dx) || !lse_moga || !aligned4(lse_moga))) return MOGA_ERR_INVALID_ARG;
+  if (window) {
+    int64_t n = 0;
+    if ((st = check_window(T, Hg, Wg, window, &n)) != MOGA_OK) return st;
+    if (n != N) return MOGA_ERR_INVALID_ARG;
+    if (!o_stga || !aligned16(o_stga) || (N > 0 && (!lse_stga || !aligned4(lse_stga)))) return MOGA_ERR_INVALID_ARG;
+  }
+  if (!ws || !aligned16(ws)) return MOGA_ERR_INVALID_ARG;
+  if (ws_bytes < moga_layer_backward_workspace_size(N, d, H, d_h, M)) return MOGA_ERR_WORKSPACE;
+  DevCtx c;
+  if (!make_ctx(&c, ws, stream)) return MOGA_ERR_CUDA;
+  uint8_t* w = (uint8_t*)ws;
+  const BwdWs bw = bwd_ws(N, d, H, d_h, M);
+  if (N == 0) {
+    cudaError_t e = cudaMemsetAsync(dW_r, 0, (size_t)M * d * 4, c.stream);
+    if (e == cudaSuccess && db_r) e = cudaMemsetAsync(db_r, 0, (size_t)M * 4, c.stream);
+    return from_cuda(e);
+  }
+  const float wgt = window ? 0.5f : 1.0f;
+  if ((st = attn_bwd_branch(c, bw, w, 0, dout, o_moga, lse_moga, q, k, v, perm, offsets, gate, wgt, N, H, d_h, M,
+                            T, Hg, Wg, window, 0, dq, dk, dv)) != MOGA_OK)
+    return st;
+  if (window && (st = attn_bwd_branch(c, bw, w, 1, dout, o_stga, lse_stga, q, k, v, nullptr, nullptr, nullptr, wgt,
+                                      N, H, d_h, M, T, Hg, Wg, window, 1, dq, dk, dv)) != MOGA_OK)
+    return st;
+  if (launch_route_bwd(c, x, W_r, b_r, x_dt == MOGA_BF16, N, d, M, group_id,
+                       reinterpret_cast<const float*>(w + bw.dgate), dx, dW_r, db_r, w + bw.route) != cudaSuccess)
+    return MOGA_ERR_CUDA;
+  count(3);
   return MOGA_OK;
 }
 

@@ -31,6 +31,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "windows.cuh"
 
 namespace moga {
 
@@ -139,20 +140,6 @@ gather_rows_kernel(const uint4* __restrict__ a, const uint4* __restrict__ b, con
   }
 }
 
-struct WinGeom {
-  int T, Hg, Wg, wt, wh, ww, nbh, nbw;
-};
-
-__device__ __forceinline__ void window_of(const WinGeom& g, int seg, int& start, int& len) {
-  const int tb = seg / (g.nbh * g.nbw);
-  const int hb = (seg / g.nbw) % g.nbh;
-  const int wb = seg % g.nbw;
-  const int t0 = tb * g.wt, h0 = hb * g.wh, w0 = wb * g.ww;
-  const int et = min(g.wt, g.T - t0), eh = min(g.wh, g.Hg - h0), ew = min(g.ww, g.Wg - w0);
-  start = t0 * g.Hg * g.Wg + et * (h0 * g.Wg + eh * w0);
-  len = et * eh * ew;
-}
-
 __global__ void window_perm_kernel(WinGeom g, int N, int32_t* __restrict__ perm_w) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= N) return;
@@ -172,8 +159,8 @@ __global__ void window_perm_kernel(WinGeom g, int N, int32_t* __restrict__ perm_
 // descending size order (ties: lower group first); a unit is a pair of
 // 128-row query tiles of one head.
 __global__ void __launch_bounds__(1024)
-seg_table_kernel(const int32_t* __restrict__ offsets, int M, int H, int64_t N, int32_t* __restrict__ table,
-                 int* status) {
+seg_table_kernel(const int32_t* __restrict__ offsets, int M, int H, int64_t N, int tiles_per_unit,
+                 int32_t* __restrict__ table, int* status) {
   __shared__ int n_s[1024];
   __shared__ int order[1024];
   __shared__ int bad;
@@ -212,7 +199,7 @@ seg_table_kernel(const int32_t* __restrict__ offsets, int M, int H, int64_t N, i
       table[r] = run;
       table[M + 1 + r] = offsets[g];
       table[2 * M + 1 + r] = n;
-      run += (((n + kTile - 1) / kTile + 1) / 2) * H;  // pairs of query tiles per head
+      run += (((n + kTile - 1) / kTile + tiles_per_unit - 1) / tiles_per_unit) * H;  // units per head
     }
     table[M] = run;
   }
@@ -861,6 +848,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       }
       float l_lo, l_hi;
       f2_unpack(f2_add(f2_add(la, lb), f2_add(lc, ld)), l_lo, l_hi);
+      // log-sum-exp of the scaled scores: S*scale = log2(e)^-1 (m + log2 l)
+      if (a.lse && live) a.lse[(int64_t)u.h * N + u.start + r] = (m_run + log2f(l_lo + l_hi)) * 0.6931471805599453f;
       const float gt = (live && a.gate) ? a.gate[src] : 1.0f;
       const float inv = a.out_scale * gt / (l_lo + l_hi);
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) + ((int64_t)src * a.H + u.h) * (int64_t)DH;
@@ -976,8 +965,9 @@ cudaError_t launch_window_perm(const DevCtx& c, int T, int Hg, int Wg, const int
   return cudaGetLastError();
 }
 
-cudaError_t launch_seg_table(const DevCtx& c, const int32_t* offsets, int M, int H, int64_t N, int32_t* table) {
-  seg_table_kernel<<<1, 1024, 0, c.stream>>>(offsets, M, H, N, table, c.status);
+cudaError_t launch_seg_table(const DevCtx& c, const int32_t* offsets, int M, int H, int64_t N, int32_t* table,
+                             int tiles_per_unit) {
+  seg_table_kernel<<<1, 1024, 0, c.stream>>>(offsets, M, H, N, tiles_per_unit, table, c.status);
   return cudaGetLastError();
 }
 

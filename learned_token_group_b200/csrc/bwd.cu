@@ -1,0 +1,807 @@
+// Gradients of the MoGA block (training): attention backward on tcgen05,
+// the per-token preparation of dO and D, and the router backward.
+//
+// "MoGA: Mixture-of-Groups Attention for End-to-End Long Video Generation"
+// (paper-graph-ui summary, section 3.4): the argmax assignment is not
+// differentiable, so the router learns through the gate p(g(x)|x) that scales
+// each token's group-attention output (Eq. 5, "Grouped Attention", "Gradient
+// flow"); q, k, v receive the gradient of each branch's attention with the
+// assignment held fixed.
+//
+// For one token set (a group or an STGA window) and one head, with
+// S = Q K^T / sqrt(d_h), P = softmax(S), O = P V and dO the branch's share of
+// the output gradient:
+//   D_i = sum_c dO_ic O_ic,   dP = dO V^T,   dS = P * (dP - D),
+//   dV = P^T dO,   dK = dS^T Q / sqrt(d_h),   dQ = dS K / sqrt(d_h).
+// P is rebuilt from the forward's log-sum-exp: P_ij = exp(S_ij - lse_i).
+//
+// attn_bwd_kernel<DH, kDQ> is one persistent kernel shape for both halves:
+// a CTA holds a 128-row "X" tile of one (segment, head) and streams the
+// segment's 64-row "Y" tiles past it.
+//   kDQ = false: X = (K, V) rows, Y = (Q, dO) rows:  S^T = K Q^T,
+//                dP^T = V dO^T, then dV += P^T dO and dK += dS^T Q;
+//   kDQ = true:  X = (Q, dO) rows, Y = (K, V) rows:  S = Q K^T, dP = dO V^T,
+//                then dQ += dS K.
+// Warp 0 loads tiles with TMA (and, for dK/dV, the per-column lse and D),
+// warp 1 issues tcgen05.mma, warps 4-11 (two warpgroups, each owning 32 of
+// the 64 Y columns of every TMEM lane) turn S and dP into bf16 P and dS in
+// TMEM, which the accumulating products read as their A operand.  Two S/dP
+// buffers alternate, so the tensor core computes tile i+1's S and tile i's
+// accumulations while the warpgroups work on tile i.  TMEM columns: buffer b
+// holds S at [128b, 128b+64) and dP at [128b+64, 128b+128); accumulators
+// start at 256 (dV then dK, or dQ).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+#include "windows.cuh"
+
+namespace moga {
+namespace {
+
+constexpr int kBwdThreads = 384;
+constexpr int kYRows = 64;
+constexpr int kYStages = 3;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int DH>
+struct BPlan {
+  static constexpr int kChunks = DH / 64;
+  static constexpr int kXBytes = kTile * DH * 2;    // 128-row bf16 tile
+  static constexpr int kYBytes = kYRows * DH * 2;   // 64-row bf16 tile
+  static constexpr int kXChunk = kTile * 128;       // bytes of one 64-column chunk of an X tile
+  static constexpr int kYChunk = kYRows * 128;      // the same for a Y tile
+  static constexpr int kX1 = 0;
+  static constexpr int kX2 = kXBytes;
+  static constexpr int kY0 = 2 * kXBytes;           // ring of kYStages x (Y1, Y2)
+  static constexpr int kYStage = 2 * kYBytes;
+  static constexpr int kVec = kY0 + kYStages * kYStage;  // ring of kYStages x (-lse*log2e [64], D [64]) fp32
+  static constexpr int kBar = kVec + kYStages * 2 * kYRows * 4;
+  static constexpr int kTable = kBar + 256;
+  static size_t bytes(int table_ints) { return (size_t)kTable + (size_t)table_ints * 4 + 1024; }
+};
+
+struct BUnit {
+  int h, start, len, x0;  // segment [start, start + len) of head h; X tile rows [x0, x0 + 128)
+};
+
+struct BDecoder {
+  int mode;        // 0 groups (table), 1 windows (geometry)
+  int nseg;
+  const int* tab;  // shared copy of [unit_prefix (M+1) | seg_start (M) | seg_len (M)]
+  WinGeom g;
+  int upw;         // windows: X tiles per window
+  __device__ __forceinline__ BUnit operator()(int idx) const {
+    BUnit u;
+    if (mode == 0) {
+      int lo = 0, hi = nseg - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (tab[mid] <= idx) lo = mid; else hi = mid - 1;
+      }
+      const int local = idx - tab[lo];
+      u.start = tab[nseg + 1 + lo];
+      u.len = tab[2 * nseg + 1 + lo];
+      const int nt = (u.len + kTile - 1) / kTile;
+      u.h = local / nt;
+      u.x0 = (local - u.h * nt) * kTile;
+    } else {
+      const int xt = idx % upw;
+      const int rest = idx / upw;
+      const int seg = rest % nseg;
+      u.h = rest / nseg;
+      window_of(g, seg, u.start, u.len);
+      u.x0 = xt * kTile;
+    }
+    return u;
+  }
+};
+
+template <int DH, bool kDQ>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__ CUtensorMap tx2,
+                const __grid_constant__ CUtensorMap ty1, const __grid_constant__ CUtensorMap ty2, const BwdArgs a,
+                int* status, unsigned long long wait_ns) {
+  using P = BPlan<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P::kBar);
+  uint64_t* x_full = bars + 0;
+  uint64_t* x_empty = bars + 1;
+  uint64_t* y_full = bars + 2;    // [kYStages]
+  uint64_t* y_empty = bars + 5;   // [kYStages]
+  uint64_t* s_full = bars + 8;    // [2]: S and dP of buffer b computed
+  uint64_t* p_full = bars + 10;   // [2]: P and dS of buffer b written
+  uint64_t* acc_full = bars + 12;
+  uint64_t* acc_empty = bars + 13;
+  uint64_t* done_bar = bars + 14;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 16);
+  int* tab = reinterpret_cast<int*>(smem + P::kTable);
+  float* vec = reinterpret_cast<float*>(smem + P::kVec);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(x_full, 1);
+    mbar_init(x_empty, 1);
+    for (int s = 0; s < kYStages; ++s) {
+      mbar_init(&y_full[s], kDQ ? 1 : 2);  // dK/dV: the TMA bytes and the lse/D vectors
+      mbar_init(&y_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 256);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 256);
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  BDecoder dec;
+  dec.mode = a.mode;
+  dec.nseg = a.nseg;
+  dec.tab = tab;
+  dec.upw = 1;
+  if (a.mode == 0) {
+    const int n = 3 * a.nseg + 1;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) tab[i] = a.table[i];
+  } else {
+    dec.g = WinGeom{a.T, a.Hg, a.Wg, a.wt, a.wh, a.ww, (a.Hg + a.wh - 1) / a.wh, (a.Wg + a.ww - 1) / a.ww};
+    dec.upw = (a.wt * a.wh * a.ww + kTile - 1) / kTile;
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const int total = a.mode == 0 ? tab[a.nseg] : a.nseg * dec.upw * a.H;
+  const uint32_t tmem = *tmem_slot;
+  auto tS = [tmem](int b) { return tmem + (uint32_t)(b * 128); };        // S (then P over its first columns)
+  auto tD = [tmem](int b) { return tmem + (uint32_t)(b * 128 + 64); };   // dP (then dS)
+  const uint32_t tAccA = tmem + 256u;                                      // dV, or dQ
+  const uint32_t tAccB = tmem + 256u + (uint32_t)DH;                       // dK
+  WaitCtx wc{abort_flag, status, wait_ns};
+  const int64_t N = a.N;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- loads
+    uint32_t uc = 0, yc = 0;
+    bool ok = true;
+    auto wwait = [&](uint64_t* bar, uint32_t parity, int site, uint32_t count) {
+      int w = 1;
+      if (lane == 0) w = mbar_wait(bar, parity, wc, site, count);
+      return __shfl_sync(0xffffffffu, w, 0) != 0;
+    };
+    if (lane == 0) {
+      tma_prefetch_desc(&tx1);
+      tma_prefetch_desc(&tx2);
+      tma_prefetch_desc(&ty1);
+      tma_prefetch_desc(&ty2);
+    }
+    for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
+      const BUnit u = dec(idx);
+      if (u.x0 >= u.len) continue;
+      const int ny = (u.len + kYRows - 1) / kYRows;
+      if (!wwait(x_empty, (uc & 1) ^ 1, 1, uc)) break;
+      if (lane == 0) {
+        const int row = (int)((int64_t)u.h * N + u.start + u.x0);
+        mbar_expect_tx(x_full, 2 * P::kXBytes);
+#pragma unroll
+        for (int c = 0; c < P::kChunks; ++c) {
+          tma_load_2d(&tx1, x_full, smem + P::kX1 + c * P::kXChunk, c * 64, row);
+          tma_load_2d(&tx2, x_full, smem + P::kX2 + c * P::kXChunk, c * 64, row);
+        }
+      }
+      ++uc;
+      for (int i = 0; i < ny; ++i) {
+        const int s = (int)(yc % kYStages);
+        if (!wwait(&y_empty[s], ((yc / kYStages) & 1) ^ 1, 2, yc)) { ok = false; break; }
+        if (lane == 0) {
+          const int row = (int)((int64_t)u.h * N + u.start + i * kYRows);
+          uint8_t* y1 = smem + P::kY0 + s * P::kYStage;
+          mbar_expect_tx(&y_full[s], 2 * P::kYBytes);
+#pragma unroll
+          for (int c = 0; c < P::kChunks; ++c) {
+            tma_load_2d(&ty1, &y_full[s], y1 + c * P::kYChunk, c * 64, row);
+            tma_load_2d(&ty2, &y_full[s], y1 + P::kYBytes + c * P::kYChunk, c * 64, row);
+          }
+        }
+        if (!kDQ) {
+          // per Y row (query): -lse * log2(e) and D; rows past the segment
+          // get -inf and 0, so their P and dS are exactly 0
+          float* v = vec + s * 2 * kYRows;
+          for (int c = lane; c < kYRows; c += 32) {
+            const int pos = i * kYRows + c;
+            const bool valid = pos < u.len;
+            const int64_t gi = (int64_t)u.h * N + u.start + pos;
+            v[c] = valid ? -a.lse[gi] * kLog2e : -INFINITY;
+            v[kYRows + c] = valid ? a.dsum[gi] : 0.0f;
+          }
+          __threadfence_block();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&y_full[s]);
+        }
+        ++yc;
+      }
+    }
+    // Drain every load this warp issued before the CTA exits.
+    if (lane == 0) {
+      volatile int zero = 0;
+      WaitCtx dc{&zero, nullptr, 100000000ull};
+      if (uc > 0) mbar_wait(x_full, (uc - 1) & 1, dc);
+      for (int s = 0; s < kYStages; ++s)
+        if ((uint32_t)s < yc) mbar_wait(&y_full[s], ((yc - 1 - ((yc - 1 - s) % kYStages)) / kYStages) & 1, dc);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(128, kYRows, false, false);
+      constexpr uint32_t idA = idesc_bf16(128, DH, false, true);
+      const uint32_t x1 = smem_u32(smem + P::kX1), x2 = smem_u32(smem + P::kX2);
+      uint32_t uc = 0, yc = 0;
+      bool ok = true;
+      // S (or S^T) = X1 Y1^T and dP (or dP^T) = X2 Y2^T, both operands K-major.
+      auto issue_s = [&](int b, int s) {
+        const uint32_t y1 = smem_u32(smem + P::kY0 + s * P::kYStage), y2 = y1 + P::kYBytes;
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint32_t xo = (kk >> 2) * P::kXChunk + (kk & 3) * 32, yo = (kk >> 2) * P::kYChunk + (kk & 3) * 32;
+          umma_bf16(tS(b), sdesc_sw128(x1 + xo, 16, 1024), sdesc_sw128(y1 + yo, 16, 1024), idS, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint32_t xo = (kk >> 2) * P::kXChunk + (kk & 3) * 32, yo = (kk >> 2) * P::kYChunk + (kk & 3) * 32;
+          umma_bf16(tD(b), sdesc_sw128(x2 + xo, 16, 1024), sdesc_sw128(y2 + yo, 16, 1024), idS, kk > 0 ? 1u : 0u);
+        }
+      };
+      // Accumulations over the 64 Y rows (four 16-row steps); P / dS of the
+      // step's rows sit in TMEM where the owning warpgroup wrote them
+      // (columns [32w, 32w + 16) of its S / dP region for Y rows [32w, 32w + 32)).
+      auto issue_acc = [&](int b, int s, bool acc) {
+        const uint32_t y1 = smem_u32(smem + P::kY0 + s * P::kYStage), y2 = y1 + P::kYBytes;
+#pragma unroll
+        for (int kk = 0; kk < kYRows / 16; ++kk) {
+          const uint32_t pc = 32u * (kk >> 1) + 8u * (kk & 1);
+          const uint32_t en = (acc || kk > 0) ? 1u : 0u;
+          if (kDQ) {
+            umma_bf16_ts(tAccA, tD(b) + pc, sdesc_sw128(y1 + kk * 2048, P::kYChunk, 1024), idA, en);  // dQ += dS K
+          } else {
+            umma_bf16_ts(tAccA, tS(b) + pc, sdesc_sw128(y2 + kk * 2048, P::kYChunk, 1024), idA, en);  // dV += P^T dO
+            umma_bf16_ts(tAccB, tD(b) + pc, sdesc_sw128(y1 + kk * 2048, P::kYChunk, 1024), idA, en);  // dK += dS^T Q
+          }
+        }
+      };
+      for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
+        const BUnit u = dec(idx);
+        if (u.x0 >= u.len) continue;
+        const int ny = (u.len + kYRows - 1) / kYRows;
+        if (!mbar_wait(x_full, uc & 1, wc, 3, uc)) break;
+        for (int i = 0; i <= ny && ok; ++i) {
+          if (i < ny) {
+            const int s = (int)(yc % kYStages), b = (int)(yc & 1);
+            if (!mbar_wait(&y_full[s], (yc / kYStages) & 1, wc, 4, yc)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(b, s);
+            umma_commit(&s_full[b]);
+            if (i + 1 == ny) umma_commit(x_empty);
+            ++yc;
+          }
+          if (i > 0) {
+            // tile yc - 1 - (i < ny): the previous Y tile of this unit
+            const uint32_t t = yc - 1 - (i < ny ? 1u : 0u);
+            const int s = (int)(t % kYStages), b = (int)(t & 1);
+            if (!mbar_wait(&p_full[b], (t >> 1) & 1, wc, 5, t)) { ok = false; break; }
+            if (i == 1 && uc > 0 && !mbar_wait(acc_empty, (uc - 1) & 1, wc, 6, uc)) { ok = false; break; }
+            tc_fence_after();
+            issue_acc(b, s, i > 1);
+            umma_commit(&y_empty[s]);
+            if (i == ny) umma_commit(acc_full);
+          }
+        }
+        ++uc;
+      }
+      umma_commit(done_bar);
+      volatile int zero = 0;
+      WaitCtx dc{&zero, nullptr, 100000000ull};
+      mbar_wait(done_bar, 0, dc);
+    }
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------------- P, dS and the epilogue
+    const int wg = (warp - 4) >> 2;   // Y columns [32 wg, 32 wg + 32) of every tile
+    const int sub = warp & 3;         // TMEM sub-partition of this warp
+    const int row = sub * 32 + lane;  // X row = TMEM lane
+    const uint32_t lb = (uint32_t)(sub * 32) << 16;
+    const float scale_log2 = kLog2e * rsqrtf((float)DH);
+    const float scale = rsqrtf((float)DH);
+    uint32_t uc = 0, yc = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
+      const BUnit u = dec(idx);
+      if (u.x0 >= u.len) continue;
+      const int ny = (u.len + kYRows - 1) / kYRows;
+      const int r = u.x0 + row;
+      bool live = r < u.len;
+      if (live && (u.h < 0 || u.h >= a.H || u.start < 0 || (int64_t)u.start + r >= N)) {
+        live = false;
+        if (status) atomicOr(status, DEV_RANGE);
+      }
+      float nl_row = -INFINITY, d_row = 0.0f;  // dQ: this query row's -lse*log2(e) and D
+      if (kDQ && live) {
+        const int64_t gi = (int64_t)u.h * N + u.start + r;
+        nl_row = -a.lse[gi] * kLog2e;
+        d_row = a.dsum[gi];
+      }
+      const int src = live ? (a.perm ? a.perm[u.start + r] : u.start + r) : 0;
+      for (int i = 0; i < ny; ++i, ++yc) {
+        const int b = (int)(yc & 1), s = (int)(yc % kYStages);
+        if (!mbar_wait(&s_full[b], (yc >> 1) & 1, wc, 7 + wg, yc)) { ok = false; break; }
+        tc_fence_after();
+        float sv[32], dv[32];
+        tmem_ld32(tS(b) + lb + 32 * wg, sv);
+        tmem_ld32(tD(b) + lb + 32 * wg, dv);
+        tmem_ld_wait();
+        uint32_t pk[16], dk[16];
+        if (kDQ) {
+          const int valid = u.len - i * kYRows - 32 * wg;  // keys of these columns inside the segment
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float p0 = fast_exp2(fmaf(sv[2 * e], scale_log2, nl_row));
+            float p1 = fast_exp2(fmaf(sv[2 * e + 1], scale_log2, nl_row));
+            p0 = 2 * e < valid ? p0 : 0.0f;
+            p1 = 2 * e + 1 < valid ? p1 : 0.0f;
+            pk[e] = pack_bf16x2(p0 * (dv[2 * e] - d_row), p1 * (dv[2 * e + 1] - d_row));
+          }
+        } else {
+          // the vectors are plain shared-memory stores of the load warp: wait
+          // on the stage's own barrier too (its phase is still this tile's,
+          // since the stage is refilled only after this tile's P and dS)
+          if (!mbar_wait(&y_full[s], (yc / kYStages) & 1, wc, 11 + wg, yc)) { ok = false; break; }
+          const float* nl = vec + s * 2 * kYRows + 32 * wg;
+          const float* dd = nl + kYRows;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = fast_exp2(fmaf(sv[2 * e], scale_log2, nl[2 * e]));
+            const float p1 = fast_exp2(fmaf(sv[2 * e + 1], scale_log2, nl[2 * e + 1]));
+            pk[e] = pack_bf16x2(p0, p1);
+            dk[e] = pack_bf16x2(p0 * (dv[2 * e] - dd[2 * e]), p1 * (dv[2 * e + 1] - dd[2 * e + 1]));
+          }
+        }
+        // dQ needs dS only (over dP); dK/dV need P (over S) and dS (over dP)
+        if (kDQ) {
+          tmem_st16u(tD(b) + lb + 32 * wg, pk);
+        } else {
+          tmem_st16u(tS(b) + lb + 32 * wg, pk);
+          tmem_st16u(tD(b) + lb + 32 * wg, dk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[b]);
+      }
+      if (!ok) break;
+      // ------------------------------------------------ epilogue
+      if (!mbar_wait(acc_full, uc & 1, wc, 9 + wg, uc)) break;
+      ++uc;
+      tc_fence_after();
+      if (live && (src < 0 || src >= N)) {
+        live = false;
+        if (status) atomicOr(status, DEV_RANGE);
+      }
+      // dK/dV: warpgroup 0 writes dV, warpgroup 1 dK (scaled); dQ: each
+      // warpgroup writes half of the columns (scaled).
+      uint32_t tacc;
+      void* outp;
+      int c0, nc;
+      float f;
+      if (kDQ) {
+        tacc = tAccA + (uint32_t)(wg * DH / 2);
+        outp = a.out1;
+        c0 = wg * DH / 2;
+        nc = DH / 2;
+        f = scale;
+      } else {
+        tacc = wg ? tAccB : tAccA;
+        outp = wg ? a.out2 : a.out1;
+        c0 = 0;
+        nc = DH;
+        f = wg ? scale : 1.0f;
+      }
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(outp) + ((int64_t)src * a.H + u.h) * (int64_t)DH + c0;
+      for (int c = 0; c < nc / 32; ++c) {
+        float o[32];
+        tmem_ld32(tacc + lb + c * 32, o);
+        tmem_ld_wait();
+        if (live) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 pk;
+            pk.x = pack_bf16x2(o[q4 * 8 + 0] * f, o[q4 * 8 + 1] * f);
+            pk.y = pack_bf16x2(o[q4 * 8 + 2] * f, o[q4 * 8 + 3] * f);
+            pk.z = pack_bf16x2(o[q4 * 8 + 4] * f, o[q4 * 8 + 5] * f);
+            pk.w = pack_bf16x2(o[q4 * 8 + 6] * f, o[q4 * 8 + 7] * f);
+            if (a.accumulate)
+              red_add_bf16x8(dst + q4, pk);
+            else
+              dst[q4] = pk;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(acc_empty);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int DH, bool kDQ>
+cudaError_t launch_bwd_dh(const DevCtx& c, const BwdArgs& a) {
+  using P = BPlan<DH>;
+  CUtensorMap m1, m2, m3, m4;
+  const uint64_t rows = (uint64_t)a.N * (uint64_t)a.H;
+  // X: 128-row boxes; Y: 64-row boxes (all [H][N][d_h] head-major copies)
+  const void* xs1 = kDQ ? a.q : a.k;
+  const void* xs2 = kDQ ? a.dout : a.v;
+  const void* ys1 = kDQ ? a.k : a.q;
+  const void* ys2 = kDQ ? a.v : a.dout;
+  if (!make_tmap_2d(&m1, xs1, DH, rows, DH * 2, kTile) || !make_tmap_2d(&m2, xs2, DH, rows, DH * 2, kTile) ||
+      !make_tmap_2d(&m3, ys1, DH, rows, DH * 2, kYRows) || !make_tmap_2d(&m4, ys2, DH, rows, DH * 2, kYRows))
+    return cudaErrorInvalidValue;
+  const int table_ints = a.mode == 0 ? 3 * a.nseg + 1 : 0;
+  const size_t smem = P::bytes(table_ints);
+  auto kern = attn_bwd_kernel<DH, kDQ>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int grid = c.num_sms;
+  if (a.mode == 1) {
+    const int64_t total = (int64_t)a.nseg * ceil_div((int64_t)a.wt * a.wh * a.ww, kTile) * a.H;
+    if (total < grid) grid = (int)total;
+  }
+  if (grid < 1) return cudaSuccess;
+  kern<<<grid, kBwdThreads, smem, c.stream>>>(m1, m2, m3, m4, a, c.status, (unsigned long long)c.wait_ns);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ dO, D and the gate gradient
+// One warp per segment position j (token src = perm[j]), all heads:
+//   dO_hat[h][j] = w * gate[src] * dout[src, h]          (bf16, head-major)
+//   D[h][j]      = w * sum_c dout[src, h, c] * o[src, h, c]
+//   dgate[src]   = sum_h D[h][j] / gate[src]              (when dgate is given)
+// where o is the branch's output as the forward stored it (for MoGA the
+// gated output gate * SA, so D equals sum_c dO_hat * SA).
+__global__ void __launch_bounds__(256)
+bwd_prep_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ o, const int32_t* __restrict__ perm,
+                const float* __restrict__ gate, float w, int64_t N, int H, int vph, uint4* __restrict__ dO_hat,
+                float* __restrict__ dsum, float* __restrict__ dgate, int* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t w0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int vpr = H * vph;
+  const int iters = (vpr + 31) / 32;
+  for (int64_t j = w0; j < N; j += nw) {
+    const int64_t src = perm ? perm[j] : j;
+    if (src < 0 || src >= N) {
+      if (lane == 0 && status) atomicOr(status, DEV_RANGE);
+      continue;
+    }
+    const float g = gate ? gate[src] : 1.0f;
+    const float sc = w * g;
+    float dg = 0.0f;
+    for (int it = 0; it < iters; ++it) {
+      const int u = it * 32 + lane;
+      const bool act = u < vpr;
+      const int h = u / vph, c = u - h * vph;
+      float part = 0.0f;
+      if (act) {
+        const uint4 dv = dout[src * vpr + u];
+        const uint4 ov = o[src * vpr + u];
+        const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+        const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 df = __bfloat1622float2(d2[e]);
+          const float2 of = __bfloat1622float2(o2[e]);
+          part = fmaf(df.x, of.x, part);
+          part = fmaf(df.y, of.y, part);
+          pk[e] = pack_bf16x2(df.x * sc, df.y * sc);
+        }
+        dO_hat[((int64_t)h * N + j) * vph + c] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      for (int off = vph >> 1; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+      if (act && c == 0) {
+        dsum[(int64_t)h * N + j] = w * part;
+        dg += w * part;
+      }
+    }
+    if (dgate) {
+      for (int off = 16; off > 0; off >>= 1) dg += __shfl_xor_sync(0xffffffffu, dg, off);
+      if (lane == 0) dgate[src] = dg / g;
+    }
+  }
+}
+
+// out = 0.5 * (a + b), bf16, n8 groups of 8 values
+__global__ void __launch_bounds__(256) mean2_kernel(const uint4* __restrict__ x, const uint4* __restrict__ y,
+                                                    int64_t n8, uint4* __restrict__ out) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 a = x[i], b = y[i];
+    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+    uint32_t pk[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 fa = __bfloat1622float2(a2[e]), fb = __bfloat1622float2(b2[e]);
+      pk[e] = pack_bf16x2(0.5f * (fa.x + fb.x), 0.5f * (fa.y + fb.y));
+    }
+    out[i] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  }
+}
+
+// ------------------------------------------------------------------ router backward
+// Eqs. 2-3 ("MoGA Router") differentiated through the gate:
+//   r = x W_r^T + b,  p = softmax(r),  gate = p_g (g = the forward's group id),
+//   dr_j = dgate * p_g * ([j == g] - p_j),
+//   dx = dr W_r,  dW_r = dr^T x,  db = sum over tokens of dr.
+template <typename T>
+struct Vec;
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int n = 8;
+  __device__ static void load(const __nv_bfloat16* p, float* v) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h[e]);
+      v[2 * e] = f.x;
+      v[2 * e + 1] = f.y;
+    }
+  }
+  __device__ static void store(__nv_bfloat16* p, const float* v) {
+    uint4 u;
+    u.x = pack_bf16x2(v[0], v[1]);
+    u.y = pack_bf16x2(v[2], v[3]);
+    u.z = pack_bf16x2(v[4], v[5]);
+    u.w = pack_bf16x2(v[6], v[7]);
+    *reinterpret_cast<uint4*>(p) = u;
+  }
+};
+template <>
+struct Vec<float> {
+  static constexpr int n = 4;
+  __device__ static void load(const float* p, float* v) {
+    const float4 f = *reinterpret_cast<const float4*>(p);
+    v[0] = f.x;
+    v[1] = f.y;
+    v[2] = f.z;
+    v[3] = f.w;
+  }
+  __device__ static void store(float* p, const float* v) { *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]); }
+};
+
+constexpr int kRbWarps = 8;
+constexpr int kRbGroups = 16;  // logits accumulated per pass over a row of x
+
+// One warp per token: logits, softmax, dr (kept in dr [N, M] for dW_r) and dx.
+template <typename T>
+__global__ void __launch_bounds__(kRbWarps * 32)
+route_bwd_kernel(const T* __restrict__ x, const T* __restrict__ W, const float* __restrict__ b,
+                 const int32_t* __restrict__ gid, const float* __restrict__ dgate, int64_t N, int d, int M,
+                 float* __restrict__ dr, T* __restrict__ dx, int* status) {
+  extern __shared__ float rb_smem[];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  float* lg = rb_smem + wid * M;  // this warp's logits, then dr
+  constexpr int V = Vec<T>::n;
+  const int nv = d / V;
+  for (int64_t i = (int64_t)blockIdx.x * kRbWarps + wid; i < N; i += (int64_t)gridDim.x * kRbWarps) {
+    const T* xr = x + i * d;
+    for (int j0 = 0; j0 < M; j0 += kRbGroups) {
+      float acc[kRbGroups];
+#pragma unroll
+      for (int jj = 0; jj < kRbGroups; ++jj) acc[jj] = 0.0f;
+      for (int cv = lane; cv < nv; cv += 32) {
+        float xv[V];
+        Vec<T>::load(xr + cv * V, xv);
+#pragma unroll
+        for (int jj = 0; jj < kRbGroups; ++jj) {
+          if (j0 + jj < M) {
+            float wv[V];
+            Vec<T>::load(W + (int64_t)(j0 + jj) * d + cv * V, wv);
+#pragma unroll
+            for (int e = 0; e < V; ++e) acc[jj] = fmaf(xv[e], wv[e], acc[jj]);
+          }
+        }
+      }
+#pragma unroll
+      for (int jj = 0; jj < kRbGroups; ++jj) {
+        float s = acc[jj];
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (lane == 0 && j0 + jj < M) lg[j0 + jj] = s + (b ? b[j0 + jj] : 0.0f);
+      }
+    }
+    __syncwarp();
+    const int g = gid[i];
+    if (g < 0 || g >= M) {
+      if (lane == 0 && status) atomicOr(status, DEV_RANGE);
+      for (int j = lane; j < M; j += 32) dr[i * M + j] = 0.0f;
+      for (int cv = lane; cv < nv; cv += 32) {
+        float z[V] = {};
+        Vec<T>::store(dx + i * d + cv * V, z);
+      }
+      __syncwarp();
+      continue;
+    }
+    float mx = -INFINITY;
+    for (int j = lane; j < M; j += 32) mx = fmaxf(mx, lg[j]);
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    float z = 0.0f;
+    for (int j = lane; j < M; j += 32) z += expf(lg[j] - mx);
+    for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+    const float pg = expf(lg[g] - mx) / z;
+    const float k = dgate[i] * pg;
+    __syncwarp();
+    for (int j = lane; j < M; j += 32) {
+      const float pj = expf(lg[j] - mx) / z;
+      const float v = k * ((j == g ? 1.0f : 0.0f) - pj);
+      lg[j] = v;
+      dr[i * M + j] = v;
+    }
+    __syncwarp();
+    for (int cv = lane; cv < nv; cv += 32) {
+      float o[V];
+#pragma unroll
+      for (int e = 0; e < V; ++e) o[e] = 0.0f;
+      for (int j = 0; j < M; ++j) {
+        const float rj = lg[j];
+        float wv[V];
+        Vec<T>::load(W + (int64_t)j * d + cv * V, wv);
+#pragma unroll
+        for (int e = 0; e < V; ++e) o[e] = fmaf(rj, wv[e], o[e]);
+      }
+      Vec<T>::store(dx + i * d + cv * V, o);
+    }
+    __syncwarp();
+  }
+}
+
+// Partial dW_r and db over one slice of the tokens: block (cx, s) covers
+// columns [64 cx, 64 cx + 64) and tokens of slice s; thread t owns column
+// 64 cx + t % 64 and groups t / 64 + 4 k.  Slices are reduced in a fixed
+// order afterwards, so the result does not depend on scheduling.
+template <typename T>
+__global__ void __launch_bounds__(256)
+route_dw_kernel(const T* __restrict__ x, const float* __restrict__ dr, int64_t N, int d, int M, int64_t per_slice,
+                float* __restrict__ pw, float* __restrict__ pb) {
+  const int t = threadIdx.x;
+  const int col = blockIdx.x * 64 + (t & 63);
+  const int s = blockIdx.y;
+  const int64_t i0 = (int64_t)s * per_slice, i1 = min(N, i0 + per_slice);
+  for (int j0 = 0; j0 < M; j0 += 64) {
+    float acc[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) acc[k] = 0.0f;
+    float bacc = 0.0f;
+    for (int64_t i = i0; i < i1; ++i) {
+      const float xv = col < d ? (float)x[i * d + col] : 0.0f;
+      const float* di = dr + i * M + j0;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const int j = (t >> 6) + 4 * k;
+        if (j0 + j < M) acc[k] = fmaf(di[j], xv, acc[k]);
+      }
+      if (blockIdx.x == 0 && t < 64 && j0 + t < M) bacc += di[t];
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int j = j0 + (t >> 6) + 4 * k;
+      if (j < M && col < d) pw[((int64_t)s * M + j) * d + col] = acc[k];
+    }
+    if (blockIdx.x == 0 && t < 64 && j0 + t < M) pb[(int64_t)s * M + j0 + t] = bacc;
+  }
+}
+
+__global__ void __launch_bounds__(256) route_dw_reduce_kernel(const float* __restrict__ pw,
+                                                              const float* __restrict__ pb, int slices, int M, int d,
+                                                              float* __restrict__ dW, float* __restrict__ db) {
+  const int64_t n = (int64_t)M * d;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    float s = 0.0f;
+    for (int k = 0; k < slices; ++k) s += pw[(int64_t)k * n + e];
+    dW[e] = s;
+  }
+  if (db && blockIdx.x == 0) {
+    for (int j = threadIdx.x; j < M; j += blockDim.x) {
+      float s = 0.0f;
+      for (int k = 0; k < slices; ++k) s += pb[(int64_t)k * M + j];
+      db[j] = s;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bwd(const DevCtx& c, const BwdArgs& a, bool dq) {
+  if (a.d_h == 128) return dq ? launch_bwd_dh<128, true>(c, a) : launch_bwd_dh<128, false>(c, a);
+  if (a.d_h == 64) return dq ? launch_bwd_dh<64, true>(c, a) : launch_bwd_dh<64, false>(c, a);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_bwd_prep(const DevCtx& c, const void* dout, const void* o, const int32_t* perm, const float* gate,
+                            float w, int64_t N, int H, int d_h, void* dO_hat, float* dsum, float* dgate) {
+  if (N == 0) return cudaSuccess;
+  int64_t blocks = ceil_div(N, 8);
+  const int64_t cap = (int64_t)c.num_sms * 8;
+  if (blocks > cap) blocks = cap;
+  bwd_prep_kernel<<<(unsigned)blocks, 256, 0, c.stream>>>((const uint4*)dout, (const uint4*)o, perm, gate, w, N, H,
+                                                           d_h / 8, (uint4*)dO_hat, dsum, dgate, c.status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mean2(const DevCtx& c, const void* x, const void* y, int64_t n, void* out) {
+  const int64_t n8 = n / 8;
+  if (n8 == 0) return cudaSuccess;
+  int64_t blocks = ceil_div(n8, 256);
+  const int64_t cap = (int64_t)c.num_sms * 8;
+  if (blocks > cap) blocks = cap;
+  mean2_kernel<<<(unsigned)blocks, 256, 0, c.stream>>>((const uint4*)x, (const uint4*)y, n8, (uint4*)out);
+  return cudaGetLastError();
+}
+
+size_t route_bwd_ws_bytes(int64_t N, int d, int M) {
+  return align_up((size_t)N * M * 4, 256) + align_up((size_t)kRouteSlices * M * d * 4, 256) +
+         align_up((size_t)kRouteSlices * M * 4, 256);
+}
+
+cudaError_t launch_route_bwd(const DevCtx& c, const void* x, const void* W, const float* b, bool bf16, int64_t N,
+                             int d, int M, const int32_t* gid, const float* dgate, void* dx, float* dW, float* db,
+                             uint8_t* ws) {
+  float* dr = reinterpret_cast<float*>(ws);
+  float* pw = reinterpret_cast<float*>(ws + align_up((size_t)N * M * 4, 256));
+  float* pb = reinterpret_cast<float*>(ws + align_up((size_t)N * M * 4, 256) +
+                                       align_up((size_t)kRouteSlices * M * d * 4, 256));
+  const size_t smem = (size_t)kRbWarps * M * 4;
+  if (N > 0) {
+    int64_t blocks = ceil_div(N, kRbWarps);
+    const int64_t cap = (int64_t)c.num_sms * 8;
+    if (blocks > cap) blocks = cap;
+    if (bf16) {
+      auto k = route_bwd_kernel<__nv_bfloat16>;
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return cudaErrorInvalidValue;
+      k<<<(unsigned)blocks, kRbWarps * 32, smem, c.stream>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)W, b,
+                                                             gid, dgate, N, d, M, dr, (__nv_bfloat16*)dx, c.status);
+    } else {
+      auto k = route_bwd_kernel<float>;
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return cudaErrorInvalidValue;
+      k<<<(unsigned)blocks, kRbWarps * 32, smem, c.stream>>>((const float*)x, (const float*)W, b, gid, dgate, N, d,
+                                                             M, dr, (float*)dx, c.status);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t per = ceil_div(N > 0 ? N : 1, kRouteSlices);
+  dim3 grid((unsigned)ceil_div(d, 64), kRouteSlices);
+  if (bf16)
+    route_dw_kernel<__nv_bfloat16><<<grid, 256, 0, c.stream>>>((const __nv_bfloat16*)x, dr, N, d, M, per, pw, pb);
+  else
+    route_dw_kernel<float><<<grid, 256, 0, c.stream>>>((const float*)x, dr, N, d, M, per, pw, pb);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  int64_t blocks = ceil_div((int64_t)M * d, 256);
+  if (blocks > 1024) blocks = 1024;
+  route_dw_reduce_kernel<<<(unsigned)blocks, 256, 0, c.stream>>>(pw, pb, kRouteSlices, M, d, dW, db);
+  return cudaGetLastError();
+}
+
+}  // namespace moga

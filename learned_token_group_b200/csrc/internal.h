@@ -48,8 +48,10 @@ cudaError_t launch_scatter(const DevCtx& c, const int32_t* group_id, const int32
 // ------------------------------------------------------------------ attention
 // Window-order permutation of the STGA grid.
 cudaError_t launch_window_perm(const DevCtx& c, int T, int Hg, int Wg, const int* window, int32_t* perm_w);
-// Sorted segment table (largest group first) for the grouped attention.
-cudaError_t launch_seg_table(const DevCtx& c, const int32_t* offsets, int M, int H, int64_t N, int32_t* table);
+// Sorted segment table (largest group first) for the grouped attention; a
+// work unit is tiles_per_unit 128-row tiles of one (group, head).
+cudaError_t launch_seg_table(const DevCtx& c, const int32_t* offsets, int M, int H, int64_t N, int32_t* table,
+                             int tiles_per_unit = 2);
 
 // Q/K/V rows gathered by perm into head-major [H][N][d_h] buffers.
 cudaError_t launch_gather(const DevCtx& c, const void* q, const void* k, const void* v, const int32_t* perm,
@@ -91,8 +93,52 @@ struct AttnArgs {
   int nseg;               // groups: M ; windows: number of windows ; mode 2: table capacity (windows)
   int T, Hg, Wg, wt, wh, ww;
   int debug_withhold_first_k;  // test hook: the producer skips each CTA's first K tile
+  // modes 0 and 1 (nullable): natural-log log-sum-exp of each query row's
+  // scaled scores, [H][N] fp32 at segment positions (the training forward
+  // keeps it for the backward pass)
+  float* lse;
 };
 cudaError_t launch_attention(const DevCtx& c, const AttnArgs& a);
+
+// ------------------------------------------------------------------ training (bwd.cu)
+// Attention backward over groups (mode 0) or STGA windows (mode 1).  q, k, v
+// and dout are head-major copies [H][N][d_h] in segment order; lse and dsum
+// are [H][N] fp32 at segment positions (lse: natural-log log-sum-exp of the
+// scaled scores from the forward; dsum: D = sum_c dO*O).  perm maps a
+// segment position to its token (null: identity).
+struct BwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* dout;
+  const float* lse;
+  const float* dsum;
+  const int32_t* perm;
+  void* out1;  // dV (dK/dV pass) or dQ (dQ pass): bf16 [N, H, d_h] by token
+  void* out2;  // dK (dK/dV pass)
+  int64_t N;
+  int H;
+  int d_h;
+  int accumulate;  // 0: store; 1: add into the outputs
+  int mode;
+  const int32_t* table;  // groups: the segment table with one 128-row tile per unit
+  int nseg;
+  int T, Hg, Wg, wt, wh, ww;
+};
+// dq = false: dK and dV (keys stationary); dq = true: dQ (queries stationary).
+cudaError_t launch_attn_bwd(const DevCtx& c, const BwdArgs& a, bool dq);
+// dO_hat = w * gate * dout gathered by perm (head-major), D, and (when dgate
+// is given) the gate gradient sum_h D / gate per token.
+cudaError_t launch_bwd_prep(const DevCtx& c, const void* dout, const void* o, const int32_t* perm, const float* gate,
+                            float w, int64_t N, int H, int d_h, void* dO_hat, float* dsum, float* dgate);
+// out = (x + y) / 2 over n bf16 values (n a multiple of 8).
+cudaError_t launch_mean2(const DevCtx& c, const void* x, const void* y, int64_t n, void* out);
+// Router backward through the gate: dx (dtype of x), dW_r fp32 [M, d], db fp32 [M] (nullable).
+constexpr int kRouteSlices = 16;
+size_t route_bwd_ws_bytes(int64_t N, int d, int M);
+cudaError_t launch_route_bwd(const DevCtx& c, const void* x, const void* W, const float* b, bool bf16, int64_t N,
+                             int d, int M, const int32_t* gid, const float* dgate, void* dx, float* dW, float* db,
+                             uint8_t* ws);
 
 // ------------------------------------------------------------------ shot windows
 // Window table of shot-aware STGA (int32, device):

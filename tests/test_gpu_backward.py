@@ -1,0 +1,181 @@
+"""Training path on the GPU against the oracle: the forward that keeps the
+log-sum-exp (moga_layer_train) and the block's gradients (moga_layer_backward).
+
+"MoGA: Mixture-of-Groups Attention for End-to-End Long Video Generation"
+(paper-graph-ui summary), section 3.4, "MoGA Router" and "Grouped Attention":
+the hard assignment is held fixed; the router learns through the gate of
+Eq. 5, q, k, v through each branch's attention.
+
+Tolerances (bf16 operands, fp32 accumulation; the arithmetic behind them):
+* lse: fp32 scores of bf16 inputs and an fp32 sum, |err| <= LSE_ABS.
+* dq, dk, dv (bf16): P, dS and dO enter the tensor core as bf16 (relative
+  rounding 2^-9 each) and the result is rounded to bf16 once per branch
+  (twice with STGA): about sqrt(3) * 2^-9 ~ 3.4e-3 of the norm for
+  independent roundings, so GRAD_REL_L2 = 1e-2 leaves a factor of three; no
+  element may be off by more than GRAD_MAX_REL of the tensor's largest
+  magnitude (a few ulps of bf16 at that magnitude).
+* dx, dW_r, db_r: the gate gradient sums dout * o over H * d_h products of
+  bf16 values (o rounded to bf16), then the router's fp32 arithmetic:
+  ROUTER_REL_L2 of the tensor's norm.
+"""
+import numpy as np
+import pytest
+import torch
+
+import learned_token_group_b200 as moga
+import oracle
+from parity import check_route, compare_out, np_cpu
+from workloads import custom, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+LSE_ABS = 2e-3
+GRAD_REL_L2 = 1e-2
+GRAD_MAX_REL = 2e-2
+ROUTER_REL_L2 = 1e-2
+
+
+def _run(wl, seed, with_bias=True):
+    inp = make_inputs(wl, seed=seed, device="cuda")
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(seed + 7)
+    b_r = (0.1 * torch.randn(wl.M, generator=gen, device="cuda")) if with_bias else None
+    dout = torch.randn((wl.N, wl.H, wl.d_h), generator=gen, device="cuda").to(torch.bfloat16)
+    sv = moga.layer_train(inp["x"], inp["W_r"], b_r, inp["q"], inp["k"], inp["v"], wl.M, wl.grid, wl.window)
+    g = moga.layer_backward(dout, sv, inp["x"], inp["W_r"], b_r, inp["q"], inp["k"], inp["v"], wl.M, wl.grid,
+                            wl.window)
+    moga.sync_status(sv["ws"])
+    moga.sync_status(g["ws"])
+    return inp, b_r, dout, sv, g
+
+
+def _rel(a, b):
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def _check_grads(g, ref, what=""):
+    errs = {}
+    for name in ("dq", "dk", "dv"):
+        a = np_cpu(g[name]).astype(np.float64)
+        b = ref[name]
+        assert np.isfinite(a).all(), f"{what}{name}: non-finite"
+        rel = _rel(a, b)
+        mx = float(np.abs(a - b).max() / max(np.abs(b).max(), 1e-30))
+        errs[name] = (rel, mx)
+        assert rel <= GRAD_REL_L2, f"{what}{name}: rel-L2 {rel:.3e}"
+        assert mx <= GRAD_MAX_REL, f"{what}{name}: max error {mx:.3e} of max |ref|"
+    for name in ("dx", "dW_r", "db_r"):
+        if g[name] is None:
+            continue
+        a = np_cpu(g[name]).astype(np.float64)
+        assert np.isfinite(a).all(), f"{what}{name}: non-finite"
+        rel = _rel(a, ref[name])
+        errs[name] = (rel,)
+        assert rel <= ROUTER_REL_L2, f"{what}{name}: rel-L2 {rel:.3e}"
+    return errs
+
+
+def _check_forward(wl, inp, sv, b_r):
+    x, W, q, k, v = (np_cpu(inp[n]) for n in ("x", "W_r", "q", "k", "v"))
+    b = None if b_r is None else np_cpu(b_r)
+    gid, _ = check_route({n: sv[n] for n in ("group_id", "gate", "perm", "offsets")}, inp["x"], inp["W_r"], b_r,
+                         wl.M, 1e-4 if wl.x_dtype == "bf16" else 1e-5)
+    ref = oracle.moga_layer(x, W, b, q, k, v, wl.M, grid=wl.grid, window=wl.window)
+    compare_out(sv["o_moga"], ref["moga"], groups=gid, what="o_moga")
+    if wl.window is not None:
+        compare_out(sv["o_stga"], ref["stga"], what="o_stga")
+    compare_out(sv["out"], ref["out"], what="out")
+    # log-sum-exp at sorted positions (groups) and window positions (STGA)
+    lse = np_cpu(sv["lse_moga"])
+    perm = np_cpu(sv["perm"]).astype(np.int64)
+    off = np_cpu(sv["offsets"]).astype(np.int64)
+    worst = 0.0
+    for m in range(wl.M):
+        idx = perm[off[m]:off[m + 1]]
+        for h in range(wl.H):
+            r = oracle.attention_lse(q[idx, h].astype(np.float64), k[idx, h].astype(np.float64))
+            worst = max(worst, float(np.abs(lse[h, off[m]:off[m + 1]] - r).max()) if idx.size else 0.0)
+    assert worst <= LSE_ABS, f"lse_moga error {worst:.3e}"
+    if wl.window is not None:
+        lse_s = np_cpu(sv["lse_stga"])
+        pos = 0
+        for idx in oracle.stga_windows(*wl.grid, wl.window):
+            for h in range(wl.H):
+                r = oracle.attention_lse(q[idx, h].astype(np.float64), k[idx, h].astype(np.float64))
+                assert np.abs(lse_s[h, pos:pos + idx.size] - r).max() <= LSE_ABS
+            pos += idx.size
+    return gid
+
+
+def _reference(wl, inp, b_r, dout):
+    x, W, q, k, v = (np_cpu(inp[n]) for n in ("x", "W_r", "q", "k", "v"))
+    return oracle.moga_layer_backward(x, W, None if b_r is None else np_cpu(b_r), q, k, v, wl.M, np_cpu(dout),
+                                      grid=wl.grid, window=wl.window)
+
+
+CASES = [
+    # groups only, ragged tiles, d_h 128
+    (custom(700, H=2, d_h=128, d=64, M=3), 1),
+    # groups + STGA on a small grid, d_h 64
+    (custom(360, H=2, d_h=64, d=64, M=4, grid=(3, 10, 12), window=(3, 8, 8)), 2),
+    # the 480p latent grid, clustered tokens: groups of thousands of tokens
+    (custom(9360, H=2, d_h=128, d=256, M=5, x_kind="clustered", grid=(6, 30, 52), window=(3, 8, 8)), 3),
+    # fp32 router input (the tiny configuration's dtype)
+    (custom(1024, H=1, d_h=64, d=64, M=4, x_dtype="f32"), 4),
+    # windows larger than two tiles (whole frames)
+    (custom(3120, H=1, d_h=128, d=64, M=2, grid=(2, 30, 52), window=(1, 30, 52)), 5),
+]
+
+
+@pytest.mark.parametrize("wl,seed", CASES, ids=[f"{c[0].N}_{c[0].d_h}_{c[0].window}" for c in CASES])
+def test_backward(wl, seed):
+    inp, b_r, dout, sv, g = _run(wl, seed)
+    gid = _check_forward(wl, inp, sv, b_r)
+    _, _, margin = oracle.route(np_cpu(inp["x"]), np_cpu(inp["W_r"]), np_cpu(b_r))
+    assert (gid == oracle.route(np_cpu(inp["x"]), np_cpu(inp["W_r"]), np_cpu(b_r))[0]).all(), \
+        "a token's group differs from the oracle's; pick inputs without near-ties"
+    ref = _reference(wl, inp, b_r, dout)
+    errs = _check_grads(g, ref)
+    print(wl.N, wl.d_h, wl.window, {k_: tuple(f"{e:.2e}" for e in v_) for k_, v_ in errs.items()})
+
+
+def test_backward_without_bias():
+    wl = custom(500, H=1, d_h=128, d=64, M=3)
+    inp, b_r, dout, sv, g = _run(wl, 11, with_bias=False)
+    assert g["db_r"] is None
+    ref = _reference(wl, inp, None, dout)
+    _check_grads(g, ref)
+
+
+def test_backward_one_group_router_silent():
+    # one group: the gate is identically 1, so the router gets no gradient
+    wl = custom(300, H=1, d_h=64, d=64, M=1)
+    inp, b_r, dout, sv, g = _run(wl, 12)
+    assert float(g["dW_r"].abs().max()) < 1e-6 and float(g["db_r"].abs().max()) < 1e-6
+    assert float(g["dx"].float().abs().max()) < 1e-6
+    ref = _reference(wl, inp, b_r, dout)
+    _check_grads(g, ref)
+
+
+def test_autograd_function_matches_calls():
+    wl = custom(360, H=2, d_h=64, d=64, M=4, grid=(3, 10, 12), window=(3, 8, 8))
+    inp, b_r, dout, sv, g = _run(wl, 2)
+    leaves = {n: inp[n].clone().requires_grad_(True) for n in ("x", "W_r", "q", "k", "v")}
+    b = b_r.clone().requires_grad_(True)
+    out = moga.MogaFunction.apply(leaves["x"], leaves["W_r"], b, leaves["q"], leaves["k"], leaves["v"], wl.M,
+                                  wl.grid, wl.window)
+    out.backward(dout)
+    torch.cuda.synchronize()
+    assert torch.equal(out, sv["out"])
+    for n, gn in (("x", "dx"), ("q", "dq"), ("k", "dk"), ("v", "dv")):
+        assert torch.equal(leaves[n].grad, g[gn]), n
+    assert torch.equal(leaves["W_r"].grad.float(), g["dW_r"].to(leaves["W_r"].dtype).float())
+    assert torch.equal(b.grad, g["db_r"])
+
+
+def test_backward_is_deterministic():
+    wl = custom(9360, H=2, d_h=128, d=256, M=5, x_kind="clustered", grid=(6, 30, 52), window=(3, 8, 8))
+    _, _, _, _, g1 = _run(wl, 3)
+    _, _, _, _, g2 = _run(wl, 3)
+    for n in ("dx", "dW_r", "db_r", "dq", "dk", "dv"):
+        assert torch.equal(g1[n], g2[n]), n
