@@ -477,6 +477,37 @@ def run_ours(args, wl, rank, world, dist):
         widened["per_frame_branch_tflops"] = 4.0 * wl.grid[0] * L * L * wl.H * wl.d_h / (ms_f * 1e-3) / 1e12
         moga.sync_status(ws_f)
         del out_f, ws_f
+        # training: the forward that keeps the log-sum-exp, then the backward
+        # pass (gradients of q, k, v, x, W_r, b_r) of the same block
+        gen_t = torch.Generator(device=dev)
+        gen_t.manual_seed(args.seed + 99)
+        dout = torch.randn((wl.N, wl.H, wl.d_h), generator=gen_t, device=dev).to(torch.bfloat16)
+        targs = (inp["x"], inp["W_r"], inp["b_r"], inp["q"], inp["k"], inp["v"], wl.M, wl.grid, wl.window)
+        tr = moga.layer_train(*targs)
+        gr = moga.layer_backward(dout, tr, *targs)
+        torch.cuda.synchronize()
+        ev2 = torch.cuda.Event(enable_timing=True)
+        t_fwd = t_bwd = 0.0
+        for _ in range(args.steps):
+            ev0.record(stream)
+            moga.layer_train(*targs, res=tr)
+            ev1.record(stream)
+            moga.layer_backward(dout, tr, *targs, grads=gr)
+            ev2.record(stream)
+            torch.cuda.synchronize()
+            t_fwd += ev0.elapsed_time(ev1)
+            t_bwd += ev1.elapsed_time(ev2)
+        moga.sync_status(tr["ws"])
+        moga.sync_status(gr["ws"])
+        t_fwd /= args.steps
+        t_bwd /= args.steps
+        widened["train_forward_ms"] = t_fwd
+        widened["train_backward_ms"] = t_bwd
+        # algorithmic backward work: five n x n x d_h products per head and
+        # token set (S recomputed, dP, dV, dK, dQ) = 2.5 x the forward's
+        widened["train_backward_attn_tflops"] = 2.5 * (flops_group + flops_stga) / (t_bwd * 1e-3) / 1e12
+        widened["train_step_tokens_per_s"] = wl.N / ((t_fwd + t_bwd) * 1e-3)
+        del tr, gr, dout
         rt = lambda: moga.route(inp["x"], inp["W_r"], inp["b_r"], wl.M, out=r_out, ws=r_ws)
         rs = lambda: moga.route_stats(inp["x"], inp["W_r"], inp["b_r"], wl.M)
         r_out = moga.route(inp["x"], inp["W_r"], inp["b_r"], wl.M)

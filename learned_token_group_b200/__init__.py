@@ -390,10 +390,11 @@ def moga_layer(x, W_r, b_r, q, k, v, M: int, grid=None, window=None, per_frame: 
             "offsets": layer.offsets, "ws": layer.ws}
 
 
-def layer_train(x, W_r, b_r, q, k, v, M: int, grid=None, window=None, ws=None):
+def layer_train(x, W_r, b_r, q, k, v, M: int, grid=None, window=None, ws=None, res=None):
     """Training forward of one block (moga_layer_train in moga.h): returns
     dict(out, o_moga, o_stga, lse_moga, lse_stga, group_id, gate, perm,
-    offsets, ws); everything but out is what ``layer_backward`` needs."""
+    offsets, ws); everything but out is what ``layer_backward`` needs.
+    ``res``: a previous result of the same shapes whose buffers are reused."""
     lib = get_lib()
     N, d = x.shape
     _, H, d_h = q.shape
@@ -404,7 +405,9 @@ def layer_train(x, W_r, b_r, q, k, v, M: int, grid=None, window=None, ws=None):
     w3 = _int3(window) if window is not None else None
     x_dt = {torch.float32: MOGA_F32, torch.bfloat16: MOGA_BF16}[x.dtype]
     mat = lambda: torch.empty((N, H, d_h), dtype=torch.bfloat16, device=dev)
-    r = {"out": mat(), "o_moga": mat(), "o_stga": mat() if window is not None else None,
+    if res is not None:
+        ws = res["ws"] if ws is None else ws
+    r = dict(res) if res is not None else {"out": mat(), "o_moga": mat(), "o_stga": mat() if window is not None else None,
          "lse_moga": torch.empty((H, N), dtype=torch.float32, device=dev),
          "lse_stga": torch.empty((H, N), dtype=torch.float32, device=dev) if window is not None else None,
          "group_id": torch.empty(N, dtype=torch.int32, device=dev),
@@ -423,10 +426,11 @@ def layer_train(x, W_r, b_r, q, k, v, M: int, grid=None, window=None, ws=None):
     return r
 
 
-def layer_backward(dout, saved, x, W_r, b_r, q, k, v, M: int, grid=None, window=None, ws=None):
+def layer_backward(dout, saved, x, W_r, b_r, q, k, v, M: int, grid=None, window=None, ws=None, grads=None):
     """Gradients of one block (moga_layer_backward in moga.h) from dout and
     the dict ``layer_train`` returned: dict(dx, dW_r, db_r, dq, dk, dv, ws).
-    db_r is None when b_r is None."""
+    db_r is None when b_r is None.  ``grads``: a previous result of the same
+    shapes whose buffers are reused."""
     lib = get_lib()
     N, d = x.shape
     _, H, d_h = q.shape
@@ -435,7 +439,10 @@ def layer_backward(dout, saved, x, W_r, b_r, q, k, v, M: int, grid=None, window=
     grid3 = tuple(int(g) for g in grid) if grid is not None else (0, 0, 0)
     w3 = _int3(window) if window is not None else None
     x_dt = {torch.float32: MOGA_F32, torch.bfloat16: MOGA_BF16}[x.dtype]
-    g = {"dx": torch.empty_like(x), "dW_r": torch.empty((M, d), dtype=torch.float32, device=dev),
+    if grads is not None:
+        ws = grads["ws"] if ws is None else ws
+    g = dict(grads) if grads is not None else {"dx": torch.empty_like(x),
+         "dW_r": torch.empty((M, d), dtype=torch.float32, device=dev),
          "db_r": torch.empty(M, dtype=torch.float32, device=dev) if b_r is not None else None,
          "dq": torch.empty_like(q), "dk": torch.empty_like(q), "dv": torch.empty_like(q)}
     need = lib.moga_layer_backward_workspace_size(N, d, H, d_h, M)

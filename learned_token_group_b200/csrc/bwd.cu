@@ -33,6 +33,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include "internal.h"
 #include "ptx.cuh"
 #include "windows.cuh"
@@ -110,15 +112,16 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P::kBar);
   uint64_t* x_full = bars + 0;
   uint64_t* x_empty = bars + 1;
-  uint64_t* y_full = bars + 2;    // [kYStages]
-  uint64_t* y_empty = bars + 5;   // [kYStages]
-  uint64_t* s_full = bars + 8;    // [2]: S and dP of buffer b computed
-  uint64_t* p_full = bars + 10;   // [2]: P and dS of buffer b written
-  uint64_t* acc_full = bars + 12;
-  uint64_t* acc_empty = bars + 13;
-  uint64_t* done_bar = bars + 14;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 16);
+  uint64_t* y_full = bars + 2;                  // [kYStages]
+  uint64_t* y_empty = y_full + kYStages;        // [kYStages]
+  uint64_t* s_full = y_empty + kYStages;        // [2]: S and dP of buffer b computed
+  uint64_t* p_full = s_full + 2;                // [2]: P and dS of buffer b written
+  uint64_t* acc_full = p_full + 2;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* done_bar = acc_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(done_bar + 2);
+  static_assert(2 + 2 * kYStages + 7 <= 32, "barrier area holds 32 words");
   int* tab = reinterpret_cast<int*>(smem + P::kTable);
   float* vec = reinterpret_cast<float*>(smem + P::kVec);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -674,39 +677,79 @@ route_bwd_kernel(const T* __restrict__ x, const T* __restrict__ W, const float* 
   }
 }
 
-// Partial dW_r and db over one slice of the tokens: block (cx, s) covers
-// columns [64 cx, 64 cx + 64) and tokens of slice s; thread t owns column
-// 64 cx + t % 64 and groups t / 64 + 4 k.  Slices are reduced in a fixed
-// order afterwards, so the result does not depend on scheduling.
+// Partial dW_r and db over one slice of the tokens.  Block (cx, s) covers
+// columns [256 cx, 256 cx + 256) for tokens of slice s: lane l of warp w
+// owns 8 consecutive columns and the groups w, w + 8, w + 16, ... (up to 64
+// per pass), so each token costs a lane one 8-column load of x, a broadcast
+// read of dr per group and 8 FMAs per group.  Four tokens are loaded before
+// their products are formed, keeping loads in flight.  Slices are reduced in
+// a fixed order afterwards, so the result does not depend on scheduling.
 template <typename T>
 __global__ void __launch_bounds__(256)
 route_dw_kernel(const T* __restrict__ x, const float* __restrict__ dr, int64_t N, int d, int M, int64_t per_slice,
                 float* __restrict__ pw, float* __restrict__ pb) {
-  const int t = threadIdx.x;
-  const int col = blockIdx.x * 64 + (t & 63);
+  constexpr int V = Vec<T>::n;       // values per vector load (8 bf16 / 4 fp32)
+  constexpr int kLoads = 8 / V;
+  constexpr int kG = 8;              // groups per warp and pass (64 per pass)
+  constexpr int kU = 4;              // tokens in flight
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int col = (blockIdx.x * 32 + lane) * 8;
+  const bool cv = col < d;           // d is a multiple of 8 (bf16) or 4 (fp32); tail lanes of fp32 handled below
   const int s = blockIdx.y;
   const int64_t i0 = (int64_t)s * per_slice, i1 = min(N, i0 + per_slice);
-  for (int j0 = 0; j0 < M; j0 += 64) {
-    float acc[16];
+  for (int jp = 0; jp < M; jp += 8 * kG) {
+    float acc[kG][8];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) acc[k] = 0.0f;
-    float bacc = 0.0f;
-    for (int64_t i = i0; i < i1; ++i) {
-      const float xv = col < d ? (float)x[i * d + col] : 0.0f;
-      const float* di = dr + i * M + j0;
+    for (int g = 0; g < kG; ++g)
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const int j = (t >> 6) + 4 * k;
-        if (j0 + j < M) acc[k] = fmaf(di[j], xv, acc[k]);
+      for (int e = 0; e < 8; ++e) acc[g][e] = 0.0f;
+    float bacc[kG];
+#pragma unroll
+    for (int g = 0; g < kG; ++g) bacc[g] = 0.0f;
+    for (int64_t ib = i0; ib < i1; ib += kU) {
+      float xv[kU][8];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int64_t i = ib + u;
+#pragma unroll
+        for (int l = 0; l < kLoads; ++l) {
+          const int c = col + l * V;
+          if (i < i1 && c + V <= d)
+            Vec<T>::load(x + i * d + c, &xv[u][l * V]);
+          else
+#pragma unroll
+            for (int e = 0; e < V; ++e) xv[u][l * V + e] = 0.0f;
+        }
       }
-      if (blockIdx.x == 0 && t < 64 && j0 + t < M) bacc += di[t];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int64_t i = ib + u;
+        if (i >= i1) break;
+        const float* di = dr + i * M;
+#pragma unroll
+        for (int g = 0; g < kG; ++g) {
+          const int j = jp + w + 8 * g;
+          if (j < M) {
+            const float r = di[j];
+            bacc[g] += r;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(r, xv[u][e], acc[g][e]);
+          }
+        }
+      }
     }
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int j = j0 + (t >> 6) + 4 * k;
-      if (j < M && col < d) pw[((int64_t)s * M + j) * d + col] = acc[k];
+    for (int g = 0; g < kG; ++g) {
+      const int j = jp + w + 8 * g;
+      if (j >= M) continue;
+      float* dst = pw + ((int64_t)s * M + j) * d + col;
+      if (cv) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (col + e < d) dst[e] = acc[g][e];
+      }
+      if (blockIdx.x == 0 && lane == 0) pb[(int64_t)s * M + j] = bacc[g];
     }
-    if (blockIdx.x == 0 && t < 64 && j0 + t < M) pb[(int64_t)s * M + j0 + t] = bacc;
   }
 }
 
@@ -757,9 +800,16 @@ cudaError_t launch_mean2(const DevCtx& c, const void* x, const void* y, int64_t 
   return cudaGetLastError();
 }
 
+// Token slices of the dW_r partial sums: at most kRouteSlices, and at most
+// 64 MiB of partials.
+static int route_max_slices(int d, int M) {
+  const int64_t per = (int64_t)M * d * 4;
+  return (int)std::max<int64_t>(1, std::min<int64_t>(kRouteSlices, ((int64_t)64 << 20) / per));
+}
+
 size_t route_bwd_ws_bytes(int64_t N, int d, int M) {
-  return align_up((size_t)N * M * 4, 256) + align_up((size_t)kRouteSlices * M * d * 4, 256) +
-         align_up((size_t)kRouteSlices * M * 4, 256);
+  const size_t S = (size_t)route_max_slices(d, M);
+  return align_up((size_t)N * M * 4, 256) + align_up(S * M * d * 4, 256) + align_up(S * M * 4, 256);
 }
 
 cudaError_t launch_route_bwd(const DevCtx& c, const void* x, const void* W, const float* b, bool bf16, int64_t N,
@@ -767,8 +817,9 @@ cudaError_t launch_route_bwd(const DevCtx& c, const void* x, const void* W, cons
                              uint8_t* ws) {
   float* dr = reinterpret_cast<float*>(ws);
   float* pw = reinterpret_cast<float*>(ws + align_up((size_t)N * M * 4, 256));
+  const int smax = route_max_slices(d, M);
   float* pb = reinterpret_cast<float*>(ws + align_up((size_t)N * M * 4, 256) +
-                                       align_up((size_t)kRouteSlices * M * d * 4, 256));
+                                       align_up((size_t)smax * M * d * 4, 256));
   const size_t smem = (size_t)kRbWarps * M * 4;
   if (N > 0) {
     int64_t blocks = ceil_div(N, kRbWarps);
@@ -790,8 +841,11 @@ cudaError_t launch_route_bwd(const DevCtx& c, const void* x, const void* W, cons
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  const int64_t per = ceil_div(N > 0 ? N : 1, kRouteSlices);
-  dim3 grid((unsigned)ceil_div(d, 64), kRouteSlices);
+  // about two blocks per SM: column tiles of 256 times token slices
+  const int64_t cx = ceil_div(d, 256);
+  const int slices = (int)std::min<int64_t>(smax, std::max<int64_t>(1, 2 * c.num_sms / cx));
+  const int64_t per = ceil_div(N > 0 ? N : 1, slices);
+  dim3 grid((unsigned)cx, (unsigned)slices);
   if (bf16)
     route_dw_kernel<__nv_bfloat16><<<grid, 256, 0, c.stream>>>((const __nv_bfloat16*)x, dr, N, d, M, per, pw, pb);
   else
@@ -800,7 +854,7 @@ cudaError_t launch_route_bwd(const DevCtx& c, const void* x, const void* W, cons
   if (e != cudaSuccess) return e;
   int64_t blocks = ceil_div((int64_t)M * d, 256);
   if (blocks > 1024) blocks = 1024;
-  route_dw_reduce_kernel<<<(unsigned)blocks, 256, 0, c.stream>>>(pw, pb, kRouteSlices, M, d, dW, db);
+  route_dw_reduce_kernel<<<(unsigned)blocks, 256, 0, c.stream>>>(pw, pb, slices, M, d, dW, db);
   return cudaGetLastError();
 }
 

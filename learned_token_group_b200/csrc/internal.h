@@ -134,7 +134,7 @@ cudaError_t launch_bwd_prep(const DevCtx& c, const void* dout, const void* o, co
 // out = (x + y) / 2 over n bf16 values (n a multiple of 8).
 cudaError_t launch_mean2(const DevCtx& c, const void* x, const void* y, int64_t n, void* out);
 // Router backward through the gate: dx (dtype of x), dW_r fp32 [M, d], db fp32 [M] (nullable).
-constexpr int kRouteSlices = 16;
+constexpr int kRouteSlices = 64;  // upper bound on token slices of the dW_r partial sums
 size_t route_bwd_ws_bytes(int64_t N, int d, int M);
 cudaError_t launch_route_bwd(const DevCtx& c, const void* x, const void* W, const float* b, bool bf16, int64_t N,
                              int d, int M, const int32_t* gid, const float* dgate, void* dx, float* dW, float* db,

@@ -221,3 +221,56 @@ def test_layer_shots_validation(lib):
     assert f(*small) == WORKSPACE
     assert lib.moga_layer_shots_workspace_size(9360, 2, 128, 4, 6, 30, 52, w, 2, 2, 2, 1) >= \
         lib.moga_layer_shots_workspace_size(9360, 2, 128, 4, 6, 30, 52, w, 2, 2, 2, 0) > 0
+
+
+def test_train_validation(lib):
+    w = (ctypes.c_int * 3)(3, 8, 8)
+    f = lib.moga_layer_train
+    Q = 0x1000010  # a second aligned fake pointer, distinct from P
+    R = 0x1000020
+    args = [P, P, None, 1, P, P, P, 360, 64, 2, 128, 4, 3, 10, 12, w, P, Q, R, P, P, P, P, P, P, P, BIG, None]
+    bad = list(args)
+    bad[17] = P                                       # o_moga must differ from out when STGA is on
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[18] = None                                    # o_stga missing with a window
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[19] = None                                    # lse_moga missing
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[10] = 96                                      # unsupported head dim
+    assert f(*bad) == UNSUPPORTED
+    small = list(args)
+    small[26] = 64
+    assert f(*small) == WORKSPACE
+    assert lib.moga_layer_train_workspace_size(360, 2, 128, 4, 3, 10, 12, w) == \
+        lib.moga_layer_workspace_size(360, 2, 128, 4, 3, 10, 12, w)
+
+
+def test_backward_validation(lib):
+    w = (ctypes.c_int * 3)(3, 8, 8)
+    f = lib.moga_layer_backward
+    args = [P, P, P, None, 1, P, P, P, 360, 64, 2, 128, 4, 3, 10, 12, w, P, P, P, P, P, P, P, P,
+            P, P, None, P, P, P, P, BIG, None]
+    bad = list(args)
+    bad[0] = None                                     # dout missing
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[26] = None                                    # dW_r missing
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[18] = None                                    # o_stga missing with a window
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[13] = 4                                       # grid must cover N
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[12] = 0                                       # M >= 1
+    assert f(*bad) == INVALID
+    small = list(args)
+    small[32] = 4096
+    assert f(*small) == WORKSPACE
+    need = lib.moga_layer_backward_workspace_size(360, 64, 2, 128, 4)
+    assert need >= 4 * 360 * 2 * 128 * 2                 # head-major q, k, v and dO copies
+    assert lib.moga_layer_backward_workspace_size(360, 64, 2, 96, 4) == 0
