@@ -618,10 +618,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       // S_x = Q_x K^T (both K-major in smem, 128B swizzle); qc / kch: byte
       // stride between the 64-column chunks of the query / key tile.
       auto issue_s = [&](int x, uint32_t qa, int qc, uint32_t ka, int kch) {
+        const uint64_t qd = sdesc_sw128(qa, 16, 1024), kd = sdesc_sw128(ka, 16, 1024);
+        const uint32_t ts = tS(x);
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
           const uint32_t qo = (kk >> 2) * qc + (kk & 3) * 32, ko = (kk >> 2) * kch + (kk & 3) * 32;
-          umma_bf16(tS(x), sdesc_sw128(qa + qo, 16, 1024), sdesc_sw128(ka + ko, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          umma_bf16(ts, sdesc_add(qd, qo), sdesc_add(kd, ko), idS, kk > 0 ? 1u : 0u);
         }
       };
       // O_x += P_x V (P in TMEM over S_x, V MN-major in smem, vch between its
@@ -629,11 +631,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       // the rest hold masked keys (P = 0) and, in a compact tile, no rows at
       // all.  Full tiles issue all eight without a test on the issue path.
       auto issue_pv = [&](int x, uint32_t va, int vch, int nk, bool acc) {
+        const uint64_t vd = sdesc_sw128(va, vch, 1024);
+        const uint32_t to = tO(x), ts = tS(x);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
           if (!kSmall || kk < nk)
-            umma_bf16_ts(tO(x), tS(x) + kk * 8, sdesc_sw128(va + kk * 2048, vch, 1024), idO,
-                         (acc || kk > 0) ? 1u : 0u);
+            umma_bf16_ts(to, ts + kk * 8, sdesc_add(vd, kk * 2048), idO, (acc || kk > 0) ? 1u : 0u);
       };
       // K/V tile j of a unit: a ring of kStages slots, or (small windows) slot j.
       auto kslot = [&](int j) { return kSmall ? j : (int)(kc % kStages); };

@@ -17,19 +17,22 @@
 //
 // attn_bwd_kernel<DH, kDQ> is one persistent kernel shape for both halves:
 // a CTA holds a 128-row "X" tile of one (segment, head) and streams the
-// segment's 64-row "Y" tiles past it.
+// segment's 128-row "Y" tiles past it.
 //   kDQ = false: X = (K, V) rows, Y = (Q, dO) rows:  S^T = K Q^T,
 //                dP^T = V dO^T, then dV += P^T dO and dK += dS^T Q;
 //   kDQ = true:  X = (Q, dO) rows, Y = (K, V) rows:  S = Q K^T, dP = dO V^T,
 //                then dQ += dS K.
 // Warp 0 loads tiles with TMA (and, for dK/dV, the per-column lse and D),
-// warp 1 issues tcgen05.mma, warps 4-11 (two warpgroups, each owning 32 of
-// the 64 Y columns of every TMEM lane) turn S and dP into bf16 P and dS in
-// TMEM, which the accumulating products read as their A operand.  Two S/dP
-// buffers alternate, so the tensor core computes tile i+1's S and tile i's
-// accumulations while the warpgroups work on tile i.  TMEM columns: buffer b
-// holds S at [128b, 128b+64) and dP at [128b+64, 128b+128); accumulators
-// start at 256 (dV then dK, or dQ).
+// warp 1 issues tcgen05.mma, warps 4-11 (two warpgroups, each owning 64 of
+// the 128 Y columns of every TMEM lane) turn S and dP into bf16 P and dS in
+// TMEM, which the accumulating products read as their A operand.  TMEM
+// columns: S at [0, 128), dP at [128, 256), accumulators from 256 (dV then
+// dK, or dQ): one S/dP buffer, so a tile's softmax is not overlapped with the
+// next tile's S and dP.  With d_h = 128 two 128-wide buffers and the dK, dV
+// accumulators do not fit the 512 columns; 128-row Y tiles are still the
+// faster choice, because an M=128 MMA reads its whole A slice from shared
+// memory for every instruction, and N = 128 halves those bytes per
+// multiply-add against N = 64 (shared-memory bandwidth bounds those products).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -43,22 +46,22 @@ namespace moga {
 namespace {
 
 constexpr int kBwdThreads = 384;
-constexpr int kYRows = 64;
-constexpr int kYStages = 3;
+constexpr int kYRows = 128;
+constexpr int kYStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int DH>
 struct BPlan {
   static constexpr int kChunks = DH / 64;
   static constexpr int kXBytes = kTile * DH * 2;    // 128-row bf16 tile
-  static constexpr int kYBytes = kYRows * DH * 2;   // 64-row bf16 tile
+  static constexpr int kYBytes = kYRows * DH * 2;   // 128-row bf16 tile
   static constexpr int kXChunk = kTile * 128;       // bytes of one 64-column chunk of an X tile
   static constexpr int kYChunk = kYRows * 128;      // the same for a Y tile
   static constexpr int kX1 = 0;
   static constexpr int kX2 = kXBytes;
   static constexpr int kY0 = 2 * kXBytes;           // ring of kYStages x (Y1, Y2)
   static constexpr int kYStage = 2 * kYBytes;
-  static constexpr int kVec = kY0 + kYStages * kYStage;  // ring of kYStages x (-lse*log2e [64], D [64]) fp32
+  static constexpr int kVec = kY0 + kYStages * kYStage;  // ring of kYStages x (-lse*log2e [128], D [128]) fp32
   static constexpr int kBar = kVec + kYStages * 2 * kYRows * 4;
   static constexpr int kTable = kBar + 256;
   static size_t bytes(int table_ints) { return (size_t)kTable + (size_t)table_ints * 4 + 1024; }
@@ -114,9 +117,9 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
   uint64_t* x_empty = bars + 1;
   uint64_t* y_full = bars + 2;                  // [kYStages]
   uint64_t* y_empty = y_full + kYStages;        // [kYStages]
-  uint64_t* s_full = y_empty + kYStages;        // [2]: S and dP of buffer b computed
-  uint64_t* p_full = s_full + 2;                // [2]: P and dS of buffer b written
-  uint64_t* acc_full = p_full + 2;
+  uint64_t* s_full = y_empty + kYStages;        // S and dP computed
+  uint64_t* p_full = s_full + 1;                // P and dS written
+  uint64_t* acc_full = p_full + 1;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* done_bar = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
@@ -133,10 +136,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
       mbar_init(&y_full[s], kDQ ? 1 : 2);  // dK/dV: the TMA bytes and the lse/D vectors
       mbar_init(&y_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 256);
-    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 256);
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 256);
     mbar_init(done_bar, 1);
@@ -164,10 +165,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
   tc_fence_after();
   const int total = a.mode == 0 ? tab[a.nseg] : a.nseg * dec.upw * a.H;
   const uint32_t tmem = *tmem_slot;
-  auto tS = [tmem](int b) { return tmem + (uint32_t)(b * 128); };        // S (then P over its first columns)
-  auto tD = [tmem](int b) { return tmem + (uint32_t)(b * 128 + 64); };   // dP (then dS)
-  const uint32_t tAccA = tmem + 256u;                                      // dV, or dQ
-  const uint32_t tAccB = tmem + 256u + (uint32_t)DH;                       // dK
+  const uint32_t tS = tmem;                          // S (then P, packed, over part of it)
+  const uint32_t tD = tmem + 128u;                   // dP (then dS)
+  const uint32_t tAccA = tmem + 256u;                // dV, or dQ
+  const uint32_t tAccB = tmem + 256u + (uint32_t)DH; // dK
   WaitCtx wc{abort_flag, status, wait_ns};
   const int64_t N = a.N;
 
@@ -249,63 +250,69 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
       uint32_t uc = 0, yc = 0;
       bool ok = true;
       // S (or S^T) = X1 Y1^T and dP (or dP^T) = X2 Y2^T, both operands K-major.
-      auto issue_s = [&](int b, int s) {
-        const uint32_t y1 = smem_u32(smem + P::kY0 + s * P::kYStage), y2 = y1 + P::kYBytes;
+      const uint64_t x1d = sdesc_sw128(x1, 16, 1024), x2d = sdesc_sw128(x2, 16, 1024);
+      auto issue_s = [&](int s) {
+        const uint32_t y1 = smem_u32(smem + P::kY0 + s * P::kYStage);
+        const uint64_t y1d = sdesc_sw128(y1, 16, 1024), y2d = sdesc_sw128(y1 + P::kYBytes, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
           const uint32_t xo = (kk >> 2) * P::kXChunk + (kk & 3) * 32, yo = (kk >> 2) * P::kYChunk + (kk & 3) * 32;
-          umma_bf16(tS(b), sdesc_sw128(x1 + xo, 16, 1024), sdesc_sw128(y1 + yo, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          umma_bf16(tS, sdesc_add(x1d, xo), sdesc_add(y1d, yo), idS, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
           const uint32_t xo = (kk >> 2) * P::kXChunk + (kk & 3) * 32, yo = (kk >> 2) * P::kYChunk + (kk & 3) * 32;
-          umma_bf16(tD(b), sdesc_sw128(x2 + xo, 16, 1024), sdesc_sw128(y2 + yo, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          umma_bf16(tD, sdesc_add(x2d, xo), sdesc_add(y2d, yo), idS, kk > 0 ? 1u : 0u);
         }
       };
-      // Accumulations over the 64 Y rows (four 16-row steps); P / dS of the
-      // step's rows sit in TMEM where the owning warpgroup wrote them
-      // (columns [32w, 32w + 16) of its S / dP region for Y rows [32w, 32w + 32)).
-      auto issue_acc = [&](int b, int s, bool acc) {
-        const uint32_t y1 = smem_u32(smem + P::kY0 + s * P::kYStage), y2 = y1 + P::kYBytes;
+      // Accumulations over the 128 Y rows (eight 16-row steps).  Warpgroup w
+      // wrote P / dS of Y rows [64w, 64w + 64) as packed bf16 into columns
+      // [64w, 64w + 32) of the S / dP region, so step kk's 16 rows start at
+      // column 64 (kk / 4) + 8 (kk % 4).
+      auto issue_acc = [&](int s, bool acc) {
+        const uint32_t y1 = smem_u32(smem + P::kY0 + s * P::kYStage);
+        const uint64_t y1d = sdesc_sw128(y1, P::kYChunk, 1024), y2d = sdesc_sw128(y1 + P::kYBytes, P::kYChunk, 1024);
 #pragma unroll
         for (int kk = 0; kk < kYRows / 16; ++kk) {
-          const uint32_t pc = 32u * (kk >> 1) + 8u * (kk & 1);
+          const uint32_t pc = 64u * (kk >> 2) + 8u * (kk & 3);
           const uint32_t en = (acc || kk > 0) ? 1u : 0u;
           if (kDQ) {
-            umma_bf16_ts(tAccA, tD(b) + pc, sdesc_sw128(y1 + kk * 2048, P::kYChunk, 1024), idA, en);  // dQ += dS K
+            umma_bf16_ts(tAccA, tD + pc, sdesc_add(y1d, kk * 2048), idA, en);  // dQ += dS K
           } else {
-            umma_bf16_ts(tAccA, tS(b) + pc, sdesc_sw128(y2 + kk * 2048, P::kYChunk, 1024), idA, en);  // dV += P^T dO
-            umma_bf16_ts(tAccB, tD(b) + pc, sdesc_sw128(y1 + kk * 2048, P::kYChunk, 1024), idA, en);  // dK += dS^T Q
+            umma_bf16_ts(tAccA, tS + pc, sdesc_add(y2d, kk * 2048), idA, en);  // dV += P^T dO
+            umma_bf16_ts(tAccB, tD + pc, sdesc_add(y1d, kk * 2048), idA, en);  // dK += dS^T Q
           }
         }
+      };
+      // One S/dP buffer: tile i's S and dP are issued after tile i-1's
+      // accumulations (which read its P and dS from the same columns), and
+      // only once the softmax warps have released tile i-1.
+      auto finish_tile = [&](uint32_t t, bool first, bool last_of_unit) {
+        const int st = (int)(t % kYStages);
+        if (!mbar_wait(p_full, t & 1, wc, 5, t)) return false;
+        if (first && uc > 0 && !mbar_wait(acc_empty, (uc - 1) & 1, wc, 6, uc)) return false;
+        tc_fence_after();
+        issue_acc(st, !first);
+        umma_commit(&y_empty[st]);
+        if (last_of_unit) umma_commit(acc_full);
+        return true;
       };
       for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
         const BUnit u = dec(idx);
         if (u.x0 >= u.len) continue;
         const int ny = (u.len + kYRows - 1) / kYRows;
         if (!mbar_wait(x_full, uc & 1, wc, 3, uc)) break;
-        for (int i = 0; i <= ny && ok; ++i) {
-          if (i < ny) {
-            const int s = (int)(yc % kYStages), b = (int)(yc & 1);
-            if (!mbar_wait(&y_full[s], (yc / kYStages) & 1, wc, 4, yc)) { ok = false; break; }
-            tc_fence_after();
-            issue_s(b, s);
-            umma_commit(&s_full[b]);
-            if (i + 1 == ny) umma_commit(x_empty);
-            ++yc;
-          }
-          if (i > 0) {
-            // tile yc - 1 - (i < ny): the previous Y tile of this unit
-            const uint32_t t = yc - 1 - (i < ny ? 1u : 0u);
-            const int s = (int)(t % kYStages), b = (int)(t & 1);
-            if (!mbar_wait(&p_full[b], (t >> 1) & 1, wc, 5, t)) { ok = false; break; }
-            if (i == 1 && uc > 0 && !mbar_wait(acc_empty, (uc - 1) & 1, wc, 6, uc)) { ok = false; break; }
-            tc_fence_after();
-            issue_acc(b, s, i > 1);
-            umma_commit(&y_empty[s]);
-            if (i == ny) umma_commit(acc_full);
-          }
+        for (int i = 0; i < ny; ++i) {
+          const int s = (int)(yc % kYStages);
+          if (i > 0 && !finish_tile(yc - 1, i == 1, false)) { ok = false; break; }
+          if (!mbar_wait(&y_full[s], (yc / kYStages) & 1, wc, 4, yc)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(s);
+          umma_commit(s_full);
+          if (i + 1 == ny) umma_commit(x_empty);
+          ++yc;
         }
+        if (!ok || !finish_tile(yc - 1, ny == 1, true)) break;
         ++uc;
       }
       umma_commit(done_bar);
@@ -315,7 +322,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
     }
   } else if (warp >= 4) {
     // ---------------------------------------------------------------- P, dS and the epilogue
-    const int wg = (warp - 4) >> 2;   // Y columns [32 wg, 32 wg + 32) of every tile
+    const int wg = (warp - 4) >> 2;   // Y columns [64 wg, 64 wg + 64) of every tile
     const int sub = warp & 3;         // TMEM sub-partition of this warp
     const int row = sub * 32 + lane;  // X row = TMEM lane
     const uint32_t lb = (uint32_t)(sub * 32) << 16;
@@ -341,49 +348,52 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
       }
       const int src = live ? (a.perm ? a.perm[u.start + r] : u.start + r) : 0;
       for (int i = 0; i < ny; ++i, ++yc) {
-        const int b = (int)(yc & 1), s = (int)(yc % kYStages);
-        if (!mbar_wait(&s_full[b], (yc >> 1) & 1, wc, 7 + wg, yc)) { ok = false; break; }
+        const int s = (int)(yc % kYStages);
+        if (!mbar_wait(s_full, yc & 1, wc, 7 + wg, yc)) { ok = false; break; }
         tc_fence_after();
-        float sv[32], dv[32];
-        tmem_ld32(tS(b) + lb + 32 * wg, sv);
-        tmem_ld32(tD(b) + lb + 32 * wg, dv);
-        tmem_ld_wait();
-        uint32_t pk[16], dk[16];
-        if (kDQ) {
-          const int valid = u.len - i * kYRows - 32 * wg;  // keys of these columns inside the segment
+        // the vectors are plain shared-memory stores of the load warp: wait
+        // on the stage's own barrier too (its phase is still this tile's,
+        // since the stage is refilled only after this tile's P and dS)
+        if (!kDQ && !mbar_wait(&y_full[s], (yc / kYStages) & 1, wc, 11 + wg, yc)) { ok = false; break; }
+        // Y columns [64 wg, 64 wg + 64) in two halves of 32; the packed P / dS
+        // of half hf go to columns 64 wg + 16 hf, which this warpgroup has
+        // already read.
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float p0 = fast_exp2(fmaf(sv[2 * e], scale_log2, nl_row));
-            float p1 = fast_exp2(fmaf(sv[2 * e + 1], scale_log2, nl_row));
-            p0 = 2 * e < valid ? p0 : 0.0f;
-            p1 = 2 * e + 1 < valid ? p1 : 0.0f;
-            pk[e] = pack_bf16x2(p0 * (dv[2 * e] - d_row), p1 * (dv[2 * e + 1] - d_row));
-          }
-        } else {
-          // the vectors are plain shared-memory stores of the load warp: wait
-          // on the stage's own barrier too (its phase is still this tile's,
-          // since the stage is refilled only after this tile's P and dS)
-          if (!mbar_wait(&y_full[s], (yc / kYStages) & 1, wc, 11 + wg, yc)) { ok = false; break; }
-          const float* nl = vec + s * 2 * kYRows + 32 * wg;
-          const float* dd = nl + kYRows;
+        for (int hf = 0; hf < 2; ++hf) {
+          const int c0 = 64 * wg + 32 * hf;
+          float sv[32], dv[32];
+          tmem_ld32(tS + lb + c0, sv);
+          tmem_ld32(tD + lb + c0, dv);
+          tmem_ld_wait();
+          uint32_t pk[16], dk[16];
+          if (kDQ) {
+            const int valid = u.len - i * kYRows - c0;  // keys of these columns inside the segment
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = fast_exp2(fmaf(sv[2 * e], scale_log2, nl[2 * e]));
-            const float p1 = fast_exp2(fmaf(sv[2 * e + 1], scale_log2, nl[2 * e + 1]));
-            pk[e] = pack_bf16x2(p0, p1);
-            dk[e] = pack_bf16x2(p0 * (dv[2 * e] - dd[2 * e]), p1 * (dv[2 * e + 1] - dd[2 * e + 1]));
+            for (int e = 0; e < 16; ++e) {
+              float p0 = fast_exp2(fmaf(sv[2 * e], scale_log2, nl_row));
+              float p1 = fast_exp2(fmaf(sv[2 * e + 1], scale_log2, nl_row));
+              p0 = 2 * e < valid ? p0 : 0.0f;
+              p1 = 2 * e + 1 < valid ? p1 : 0.0f;
+              pk[e] = pack_bf16x2(p0 * (dv[2 * e] - d_row), p1 * (dv[2 * e + 1] - d_row));
+            }
+            tmem_st16u(tD + lb + 64 * wg + 16 * hf, pk);
+          } else {
+            const float* nl = vec + s * 2 * kYRows + c0;
+            const float* dd = nl + kYRows;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float p0 = fast_exp2(fmaf(sv[2 * e], scale_log2, nl[2 * e]));
+              const float p1 = fast_exp2(fmaf(sv[2 * e + 1], scale_log2, nl[2 * e + 1]));
+              pk[e] = pack_bf16x2(p0, p1);
+              dk[e] = pack_bf16x2(p0 * (dv[2 * e] - dd[2 * e]), p1 * (dv[2 * e + 1] - dd[2 * e + 1]));
+            }
+            tmem_st16u(tS + lb + 64 * wg + 16 * hf, pk);
+            tmem_st16u(tD + lb + 64 * wg + 16 * hf, dk);
           }
-        }
-        // dQ needs dS only (over dP); dK/dV need P (over S) and dS (over dP)
-        if (kDQ) {
-          tmem_st16u(tD(b) + lb + 32 * wg, pk);
-        } else {
-          tmem_st16u(tS(b) + lb + 32 * wg, pk);
-          tmem_st16u(tD(b) + lb + 32 * wg, dk);
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&p_full[b]);
+        mbar_arrive(p_full);
       }
       if (!ok) break;
       // ------------------------------------------------ epilogue

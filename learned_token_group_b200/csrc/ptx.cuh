@@ -180,6 +180,15 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
+// The same descriptor for an operand byte_off bytes further on.  The start
+// address field (bits 0-13) holds the shared-memory address >> 4, so for a
+// 16-byte multiple that stays inside shared memory (below 256 KB) the move is
+// one add with no carry out of the field: sdesc_add(sdesc_sw128(a, l, s), o)
+// equals sdesc_sw128(a + o, l, s).  Issue loops build each base descriptor
+// once and step with constant offsets, which keeps the single issuing thread's
+// dependent integer work per MMA to one add.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t d, uint32_t byte_off) { return d + (uint64_t)(byte_off >> 4); }
+
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |

@@ -161,14 +161,13 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
           tc_fence_after();
           const uint32_t xa = smem_u32(ring + (size_t)s * stage_bytes);
           const uint32_t wa = xa + x_bytes;
+          const uint64_t xd = sdesc_sw128(xa, 16, 1024), wd = sdesc_sw128(wa, 16, 1024);
 #pragma unroll
           for (int c = 0; c < kRouteChunks; ++c) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = sdesc_sw128(xa + c * (kTile * 128) + kk * 32, 16, 1024);
-              const uint64_t bd = sdesc_sw128(wa + c * (mpad * 128) + kk * 32, 16, 1024);
-              umma_bf16(dt, ad, bd, idesc, (kc | c | kk) != 0);
-            }
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16(dt, sdesc_add(xd, c * (kTile * 128) + kk * 32), sdesc_add(wd, c * (mpad * 128) + kk * 32),
+                        idesc, (kc | c | kk) != 0);
           }
           umma_commit(&empty[s]);
         }
