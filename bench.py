@@ -617,6 +617,56 @@ def run_ours(args, wl, rank, world, dist):
     print(json.dumps(line), flush=True)
 
 
+def run_train(args, wl, rank, world, dist):
+    """--train: the training step of the block (moga_layer_train, then
+    moga_layer_backward with a seeded dout) as the timed step; one JSON line
+    with the forward and backward device times.  For hardware-counter
+    captures of the training kernels and for training throughput."""
+    import learned_token_group_b200 as moga
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = make_inputs(wl, seed=args.seed + rank, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(args.seed + 99 + rank)
+    dout = torch.randn((wl.N, wl.H, wl.d_h), generator=gen, device=dev).to(torch.bfloat16)
+    targs = (inp["x"], inp["W_r"], inp["b_r"], inp["q"], inp["k"], inp["v"], wl.M, wl.grid, wl.window)
+    tr = moga.layer_train(*targs)
+    gr = moga.layer_backward(dout, tr, *targs)
+    for _ in range(max(args.warmup - 1, 0)):
+        moga.layer_train(*targs, res=tr)
+        moga.layer_backward(dout, tr, *targs, grads=gr)
+    moga.sync_status(gr["ws"])
+    counts = np.diff(tr["offsets"].cpu().numpy().astype(np.int64))
+    flops = 4.0 * float((counts.astype(np.float64) ** 2).sum()) * wl.d_h * wl.H + _stga_flops(wl)
+    stream = torch.cuda.current_stream(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    t_fwd = t_bwd = 0.0
+    with ClockSampler(dev.index) as clk:
+        for _ in range(args.steps):
+            if dist is not None:
+                dist.barrier()
+            torch.cuda.synchronize()
+            ev[0].record(stream)
+            moga.layer_train(*targs, res=tr)
+            ev[1].record(stream)
+            moga.layer_backward(dout, tr, *targs, grads=gr)
+            ev[2].record(stream)
+            torch.cuda.synchronize()
+            t_fwd += ev[0].elapsed_time(ev[1])
+            t_bwd += ev[1].elapsed_time(ev[2])
+    moga.sync_status(gr["ws"])
+    t_fwd = max_over_ranks(t_fwd / args.steps, dist, dev)
+    t_bwd = max_over_ranks(t_bwd / args.steps, dist, dev)
+    if rank == 0:
+        print(json.dumps({"metric": "MoGA layer training step (forward + backward) tokens/s",
+                          "value": wl.N * world / ((t_fwd + t_bwd) * 1e-3), "unit": "tokens/s", "n_gpus": world,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_fwd + t_bwd,
+                          "train_forward_ms": t_fwd, "train_backward_ms": t_bwd,
+                          "backward_attn_tflops": 2.5 * flops / (t_bwd * 1e-3) / 1e12,
+                          "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+                          "config": _cfg(wl, world), "clocks": clk.summary()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -629,6 +679,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the widened-row timings")
     ap.add_argument("--lean", action="store_true",
                     help="warm-up and timed steps only (for hardware-counter captures)")
+    ap.add_argument("--train", action="store_true",
+                    help="time the training step (forward keeping the log-sum-exp, then the backward pass)")
     args = ap.parse_args()
     wl = WORKLOADS[args.config]
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -644,7 +696,10 @@ def main():
         dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
         dist = dist_mod
     try:
-        run_ours(args, wl, rank, world, dist)
+        if args.train:
+            run_train(args, wl, rank, world, dist)
+        else:
+            run_ours(args, wl, rank, world, dist)
     finally:
         if dist is not None:
             dist.destroy_process_group()

@@ -687,77 +687,81 @@ route_bwd_kernel(const T* __restrict__ x, const T* __restrict__ W, const float* 
   }
 }
 
-// Partial dW_r and db over one slice of the tokens.  Block (cx, s) covers
-// columns [256 cx, 256 cx + 256) for tokens of slice s: lane l of warp w
-// owns 8 consecutive columns and the groups w, w + 8, w + 16, ... (up to 64
-// per pass), so each token costs a lane one 8-column load of x, a broadcast
-// read of dr per group and 8 FMAs per group.  Four tokens are loaded before
-// their products are formed, keeping loads in flight.  Slices are reduced in
-// a fixed order afterwards, so the result does not depend on scheduling.
+// Partial dW_r and db over one slice of the tokens (a split-K reduction of
+// dW_r = dr^T x).  Block (cx, s) covers columns [256 cx, 256 cx + 256) for
+// the tokens of slice s, 32 tokens at a time: the block stages the chunk's x
+// (as fp32) and dr in shared memory with wide loads, then lane l of warp w
+// accumulates columns 256 cx + 8 l .. + 8 for the groups w, w + 8, ... (64
+// groups per pass).  Slices are summed in a fixed order afterwards, so the
+// result does not depend on scheduling.
+constexpr int kDwTok = 32;
+constexpr int kDwCols = 256;
+constexpr int kDwGroups = 64;  // groups per pass
 template <typename T>
 __global__ void __launch_bounds__(256)
 route_dw_kernel(const T* __restrict__ x, const float* __restrict__ dr, int64_t N, int d, int M, int64_t per_slice,
                 float* __restrict__ pw, float* __restrict__ pb) {
-  constexpr int V = Vec<T>::n;       // values per vector load (8 bf16 / 4 fp32)
-  constexpr int kLoads = 8 / V;
-  constexpr int kG = 8;              // groups per warp and pass (64 per pass)
-  constexpr int kU = 4;              // tokens in flight
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int col = (blockIdx.x * 32 + lane) * 8;
-  const bool cv = col < d;           // d is a multiple of 8 (bf16) or 4 (fp32); tail lanes of fp32 handled below
+  constexpr int V = Vec<T>::n;  // values per vector load (8 bf16 / 4 fp32)
+  __shared__ __align__(16) float xs[kDwTok][kDwCols];
+  __shared__ float ds[kDwTok][kDwGroups];
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  const int c0 = blockIdx.x * kDwCols;
   const int s = blockIdx.y;
   const int64_t i0 = (int64_t)s * per_slice, i1 = min(N, i0 + per_slice);
-  for (int jp = 0; jp < M; jp += 8 * kG) {
-    float acc[kG][8];
+  constexpr int kVecPerRow = kDwCols / V;
+  for (int jp = 0; jp < M; jp += kDwGroups) {
+    float acc[8][8];
 #pragma unroll
-    for (int g = 0; g < kG; ++g)
+    for (int g = 0; g < 8; ++g)
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[g][e] = 0.0f;
-    float bacc[kG];
+    float bacc[8];
 #pragma unroll
-    for (int g = 0; g < kG; ++g) bacc[g] = 0.0f;
-    for (int64_t ib = i0; ib < i1; ib += kU) {
-      float xv[kU][8];
+    for (int g = 0; g < 8; ++g) bacc[g] = 0.0f;
+    for (int64_t ib = i0; ib < i1; ib += kDwTok) {
+      __syncthreads();  // the previous chunk has been consumed
+      for (int v = t; v < kDwTok * kVecPerRow; v += 256) {
+        const int r = v / kVecPerRow, cv = v - r * kVecPerRow;
+        const int64_t i = ib + r;
+        const int c = c0 + cv * V;
+        float tmp[V];
+        if (i < i1 && c + V <= d)
+          Vec<T>::load(x + i * d + c, tmp);
+        else
 #pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int64_t i = ib + u;
+          for (int e = 0; e < V; ++e) tmp[e] = 0.0f;
 #pragma unroll
-        for (int l = 0; l < kLoads; ++l) {
-          const int c = col + l * V;
-          if (i < i1 && c + V <= d)
-            Vec<T>::load(x + i * d + c, &xv[u][l * V]);
-          else
-#pragma unroll
-            for (int e = 0; e < V; ++e) xv[u][l * V + e] = 0.0f;
-        }
+        for (int e = 0; e < V; ++e) xs[r][cv * V + e] = tmp[e];
       }
+      for (int v = t; v < kDwTok * kDwGroups; v += 256) {
+        const int r = v / kDwGroups, j = v - r * kDwGroups;
+        const int64_t i = ib + r;
+        ds[r][j] = (i < i1 && jp + j < M) ? dr[i * M + jp + j] : 0.0f;
+      }
+      __syncthreads();
+#pragma unroll 4
+      for (int r = 0; r < kDwTok; ++r) {
+        const float4 xa = *reinterpret_cast<const float4*>(&xs[r][lane * 8]);
+        const float4 xb = *reinterpret_cast<const float4*>(&xs[r][lane * 8 + 4]);
+        const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
 #pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int64_t i = ib + u;
-        if (i >= i1) break;
-        const float* di = dr + i * M;
+        for (int g = 0; g < 8; ++g) {
+          const float rj = ds[r][w + 8 * g];
+          bacc[g] += rj;
 #pragma unroll
-        for (int g = 0; g < kG; ++g) {
-          const int j = jp + w + 8 * g;
-          if (j < M) {
-            const float r = di[j];
-            bacc[g] += r;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(r, xv[u][e], acc[g][e]);
-          }
+          for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(rj, xv[e], acc[g][e]);
         }
       }
     }
 #pragma unroll
-    for (int g = 0; g < kG; ++g) {
+    for (int g = 0; g < 8; ++g) {
       const int j = jp + w + 8 * g;
       if (j >= M) continue;
+      const int col = c0 + lane * 8;
       float* dst = pw + ((int64_t)s * M + j) * d + col;
-      if (cv) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          if (col + e < d) dst[e] = acc[g][e];
-      }
+      for (int e = 0; e < 8; ++e)
+        if (col + e < d) dst[e] = acc[g][e];
       if (blockIdx.x == 0 && lane == 0) pb[(int64_t)s * M + j] = bacc[g];
     }
   }
@@ -851,8 +855,8 @@ cudaError_t launch_route_bwd(const DevCtx& c, const void* x, const void* W, cons
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  // about two blocks per SM: column tiles of 256 times token slices
-  const int64_t cx = ceil_div(d, 256);
+  // about two blocks per SM: column tiles times token slices
+  const int64_t cx = ceil_div(d, kDwCols);
   const int slices = (int)std::min<int64_t>(smax, std::max<int64_t>(1, 2 * c.num_sms / cx));
   const int64_t per = ceil_div(N > 0 ? N : 1, slices);
   dim3 grid((unsigned)cx, (unsigned)slices);

@@ -77,6 +77,10 @@ WORKLOADS = {
     # device footprint stays near 2 GB, for hardware-counter captures.
     "profile_187k_h4": Workload("profile_187k_h4", 187200, 4, 128, 1536, 16, "bf16", "clustered",
                                 (120, 30, 52), (3, 8, 8)),
+    # the same with 2 heads, for full captures of the training kernels
+    # (gathered q/k/v/dO copies of 96 MB each; about 1.5 GB on the device)
+    "profile_187k_h2": Workload("profile_187k_h2", 187200, 2, 128, 1536, 16, "bf16", "clustered",
+                                (120, 30, 52), (3, 8, 8)),
 }
 
 _FORCED = (1, 2, 3, 5, 8, 13, 21, 34)   # sizes of the forced small groups (skew)
