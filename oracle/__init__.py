@@ -63,7 +63,7 @@ __all__ = [
     "route", "balance_stats", "counting_sort", "attention_rows", "group_attention",
     "stga_windows", "stga_attention", "frame_attention", "moga_layer",
     "shot_windows", "stga_shot_attention", "attention_lse", "attention_rows_backward",
-    "moga_layer_backward",
+    "moga_layer_backward", "attention_dq_rows",
 ]
 
 _ROW_BLOCK = 16384
@@ -444,3 +444,22 @@ def moga_layer_backward(x, W_r, b_r, q, k, v, M: int, dout, grid=None, window=No
     dr = (dgate * gate)[:, None] * (onehot - p)
     return {"dx": dr @ W, "dW_r": dr.T @ X, "db_r": dr.sum(axis=0),
             "dq": dq, "dk": dk, "dv": dv, "dgate": dgate}
+
+
+def attention_dq_rows(Q_rows: np.ndarray, K: np.ndarray, V: np.ndarray, dO_rows: np.ndarray):
+    """dQ of selected query rows of one head, each row on its own (the rows of
+    ``attention_rows_backward`` computed without the other queries).
+
+    For a query row q with scores s = q K^T / sqrt(d_h), p = softmax(s),
+    o = p V and its output gradient g:  dp = g V^T,
+    ds = p * (dp - sum(p * dp)),  dq = ds K / sqrt(d_h).
+    Returns (dq [r, d_h], o [r, d_h]).
+    """
+    c = 1.0 / math.sqrt(K.shape[1])
+    S = (Q_rows @ K.T) * c
+    S = S - S.max(axis=1, keepdims=True)
+    P = np.exp(S)
+    P = P / P.sum(axis=1, keepdims=True)
+    dP = dO_rows @ V.T
+    dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+    return (dS @ K) * c, P @ V

@@ -179,3 +179,95 @@ def test_backward_is_deterministic():
     _, _, _, _, g2 = _run(wl, 3)
     for n in ("dx", "dW_r", "db_r", "dq", "dk", "dv"):
         assert torch.equal(g1[n], g2[n]), n
+
+
+def test_backward_full_size_sampled():
+    """video_187k (187,200 tokens, 12 heads, M = 16, STGA 3x8x8) in the
+    launch configuration `bench.py --train` times, checked on samples the
+    oracle computes exactly: dq of sampled query rows of every group (each row
+    against its whole group, plus its STGA window), dk and dv of every token
+    of the small groups (whole-group backward, plus each token's window), and
+    dx of sampled tokens (their gate gradient over all 12 heads).  Group
+    membership is the GPU's assignment, which the routing check above pins
+    (the backward holds the assignment fixed)."""
+    from workloads import WORKLOADS
+    wl = WORKLOADS["video_187k"]
+    inp, b_r, dout, sv, g = _run(wl, 0, with_bias=False)
+    route_res = {n: sv[n] for n in ("group_id", "gate", "perm", "offsets")}
+    gid, _ = check_route(route_res, inp["x"], inp["W_r"], None, wl.M, 1e-4)
+    x64 = np_cpu(inp["x"]).astype(np.float64)
+    W64 = np_cpu(inp["W_r"]).astype(np.float64)
+    r = x64 @ W64.T
+    p = np.exp(r - r.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    gate = p[np.arange(wl.N), gid]
+    w = 0.5
+    rng = np.random.default_rng(5)
+    heads = [0, wl.H - 1]
+    windows = oracle.stga_windows(*wl.grid, wl.window)
+    win_of = np.empty(wl.N, dtype=np.int64)
+    for wi, idx in enumerate(windows):
+        win_of[idx] = wi
+    rows_of = lambda t, idx, h: np_cpu(t[torch.as_tensor(idx, device="cuda"), h]).astype(np.float64)
+    win_cache = {}
+
+    def window_grads(wi, h):
+        key = (wi, h)
+        if key not in win_cache:
+            idx = windows[wi]
+            win_cache[key] = (idx,) + oracle.attention_rows_backward(
+                rows_of(inp["q"], idx, h), rows_of(inp["k"], idx, h), rows_of(inp["v"], idx, h),
+                w * rows_of(dout, idx, h))[:3]
+        return win_cache[key]
+
+    got_q, ref_q, got_kv, ref_kv = [], [], [], []
+    sizes = np.bincount(gid, minlength=wl.M)
+    for m in range(wl.M):
+        idx = np.nonzero(gid == m)[0]
+        if idx.size == 0:
+            continue
+        rows = np.sort(rng.choice(idx, size=min(16, idx.size), replace=False))
+        for h in heads:
+            K, V = rows_of(inp["k"], idx, h), rows_of(inp["v"], idx, h)
+            dOr = w * gate[rows][:, None] * rows_of(dout, rows, h)
+            dq = oracle.attention_dq_rows(rows_of(inp["q"], rows, h), K, V, dOr)[0]
+            for a, t in enumerate(rows):
+                widx, wq, _, _ = window_grads(win_of[t], h)
+                dq[a] += wq[np.searchsorted(widx, t)]
+            ref_q.append(dq)
+            got_q.append(np_cpu(g["dq"][torch.as_tensor(rows, device="cuda"), h]).astype(np.float64))
+            if 100 <= sizes[m] <= 3000:   # small groups: dk, dv of every token
+                Q = rows_of(inp["q"], idx, h)
+                dO = w * gate[idx][:, None] * rows_of(dout, idx, h)
+                _, dk, dv, _ = oracle.attention_rows_backward(Q, K, V, dO)
+                for a, t in enumerate(idx):
+                    widx, _, wk, wv = window_grads(win_of[t], h)
+                    j = np.searchsorted(widx, t)
+                    dk[a] += wk[j]
+                    dv[a] += wv[j]
+                tt = torch.as_tensor(idx, device="cuda")
+                ref_kv.append(np.concatenate([dk, dv], axis=1))
+                got_kv.append(np.concatenate([np_cpu(g["dk"][tt, h]), np_cpu(g["dv"][tt, h])], axis=1))
+    assert got_kv, "no group of 100-3000 tokens to check dk and dv on"
+    for what, got, ref in (("dq", got_q, ref_q), ("dk|dv", got_kv, ref_kv)):
+        a, b = np.concatenate(got), np.concatenate(ref)
+        rel = _rel(a, b)
+        mx = float(np.abs(a - b).max() / np.abs(b).max())
+        assert rel <= GRAD_REL_L2 and mx <= GRAD_MAX_REL, f"{what}: rel-L2 {rel:.3e}, max {mx:.3e}"
+    # dx of sampled tokens of three groups: the gate gradient sums all heads
+    got_x, ref_x = [], []
+    for m in np.argsort(sizes)[-3:]:
+        idx = np.nonzero(gid == m)[0]
+        rows = np.sort(rng.choice(idx, size=8, replace=False))
+        dgate = np.zeros(rows.size)
+        for h in range(wl.H):
+            K, V = rows_of(inp["k"], idx, h), rows_of(inp["v"], idx, h)
+            A = oracle.attention_rows(rows_of(inp["q"], rows, h), K, V)
+            dgate += w * (rows_of(dout, rows, h) * A).sum(axis=1)
+        onehot = np.zeros((rows.size, wl.M))
+        onehot[np.arange(rows.size), gid[rows]] = 1.0
+        dr = (dgate * gate[rows])[:, None] * (onehot - p[rows])
+        ref_x.append(dr @ W64)
+        got_x.append(np_cpu(g["dx"][torch.as_tensor(rows, device="cuda")]).astype(np.float64))
+    rel = _rel(np.concatenate(got_x), np.concatenate(ref_x))
+    assert rel <= ROUTER_REL_L2, f"dx: rel-L2 {rel:.3e}"

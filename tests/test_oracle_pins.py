@@ -537,12 +537,28 @@ def check_attention_lse(o):
     assert np.allclose(o.attention_lse(q, K), ref, rtol=0, atol=1e-12)
 
 
+def check_dq_rows(o):
+    """Row-wise dQ equals the dQ rows of the whole-set backward, and torch
+    autograd of Eq. 1 (float64) for those rows."""
+    rng = np.random.default_rng(70)
+    Q, K, V, dO = (rng.normal(size=(40, 8)) for _ in range(4))
+    rows = np.array([0, 7, 39])
+    dq, out = o.attention_dq_rows(Q[rows], K, V, dO[rows])
+    full = o.attention_rows_backward(Q, K, V, dO)
+    assert np.allclose(dq, full[0][rows], rtol=1e-12, atol=1e-12)
+    assert np.allclose(out, full[3][rows], rtol=1e-12, atol=1e-12)
+    tq = torch.tensor(Q[rows], requires_grad=True)
+    o_t = torch.softmax(tq @ torch.tensor(K).T / math.sqrt(8), dim=1) @ torch.tensor(V)
+    (o_t * torch.tensor(dO[rows])).sum().backward()
+    assert np.allclose(dq, tq.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
 CHECKS = [check_route_closed_form, check_route_ties_and_M1, check_route_brute, check_counting_sort,
           check_full_attention_when_M1, check_group_equals_subset_attention, check_special_cases,
           check_brute_force_tiny, check_permutation_equivariance, check_stga, check_layer_combine,
           check_golden, check_three_branch_mean, check_balance_stats, check_shot_stga,
           check_backward_finite_differences, check_backward_dense_autograd, check_backward_special_cases,
-          check_attention_lse]
+          check_attention_lse, check_dq_rows]
 
 
 @pytest.mark.parametrize("check", CHECKS, ids=[c.__name__ for c in CHECKS])
