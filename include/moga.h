@@ -289,6 +289,34 @@ moga_status moga_layer_backward(const void* dout, const void* x, const void* W_r
                                 float* dW_r, float* db_r, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
                                 void* stream);
 
+/* moga_layer_train_ex / moga_layer_backward_ex: the same pair with the
+ * per-frame branch of the "Spatial-Temporal Group Attention (STGA)" section
+ * as a third branch (per_frame = 1: attention among all Hg*Wg tokens of each
+ * latent frame; T, Hg, Wg are then required even when window == NULL).
+ * out is the plain mean of the branches that are on, and each branch's share
+ * of dout in the backward is dout divided by their number.  o_frame (bf16
+ * [N, H, d_h]) and lse_frame (fp32 [H, N], token order) are the per-frame
+ * branch's output and log-sum-exp, unused when per_frame = 0.  Everything
+ * else as moga_layer_train / moga_layer_backward (which are these calls with
+ * per_frame = 0).
+ * Workspace: moga_layer_train_ex_workspace_size(...) / moga_layer_backward_workspace_size(...). */
+size_t moga_layer_train_ex_workspace_size(int64_t N, int H, int d_h, int M, int T, int Hg, int Wg,
+                                          const int* window, int per_frame);
+moga_status moga_layer_train_ex(const void* x, const void* W_r, const float* b_r, moga_dtype x_dt, const void* q,
+                                const void* k, const void* v, int64_t N, int d, int H, int d_h, int M, int T, int Hg,
+                                int Wg, const int* window, int per_frame, void* out, void* o_moga, void* o_stga,
+                                void* o_frame, float* lse_moga, float* lse_stga, float* lse_frame, int32_t* group_id,
+                                float* gate, int32_t* perm, int32_t* offsets, void* ws, size_t ws_bytes,
+                                void* stream);
+moga_status moga_layer_backward_ex(const void* dout, const void* x, const void* W_r, const float* b_r,
+                                   moga_dtype x_dt, const void* q, const void* k, const void* v, int64_t N, int d,
+                                   int H, int d_h, int M, int T, int Hg, int Wg, const int* window, int per_frame,
+                                   const void* o_moga, const void* o_stga, const void* o_frame, const float* lse_moga,
+                                   const float* lse_stga, const float* lse_frame, const int32_t* group_id,
+                                   const float* gate, const int32_t* perm, const int32_t* offsets, void* dx,
+                                   float* dW_r, float* db_r, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                                   void* stream);
+
 /* moga_layer_ex: the visual block with a choice of branches, as in the pages'
  * "Spatial-Temporal Group Attention (STGA)" section (each token's output is
  * the mean of its MoGA group, its STGA window and its per-frame group):

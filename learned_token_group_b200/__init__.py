@@ -88,6 +88,11 @@ def get_lib():
         "moga_layer_train": (_I, [_P, _P, _P, _I, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _I, _P,
                                   _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
         "moga_layer_backward_workspace_size": (_SZ, [_I64, _I, _I, _I, _I]),
+        "moga_layer_train_ex_workspace_size": (_SZ, [_I64, _I, _I, _I, _I, _I, _I, _P, _I]),
+        "moga_layer_train_ex": (_I, [_P, _P, _P, _I, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _I, _P, _I,
+                                     _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+        "moga_layer_backward_ex": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _I, _P, _I,
+                                        _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
         "moga_layer_backward": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _I, _P,
                                      _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     }
@@ -390,11 +395,13 @@ def moga_layer(x, W_r, b_r, q, k, v, M: int, grid=None, window=None, per_frame: 
             "offsets": layer.offsets, "ws": layer.ws}
 
 
-def layer_train(x, W_r, b_r, q, k, v, M: int, grid=None, window=None, ws=None, res=None):
-    """Training forward of one block (moga_layer_train in moga.h): returns
-    dict(out, o_moga, o_stga, lse_moga, lse_stga, group_id, gate, perm,
-    offsets, ws); everything but out is what ``layer_backward`` needs.
-    ``res``: a previous result of the same shapes whose buffers are reused."""
+def layer_train(x, W_r, b_r, q, k, v, M: int, grid=None, window=None, ws=None, res=None, per_frame: bool = False):
+    """Training forward of one block (moga_layer_train_ex in moga.h): returns
+    dict(out, o_moga, o_stga, o_frame, lse_moga, lse_stga, lse_frame,
+    group_id, gate, perm, offsets, ws); everything but out is what
+    ``layer_backward`` needs.  per_frame adds the per-frame branch (out is the
+    mean of the branches).  ``res``: a previous result of the same shapes
+    whose buffers are reused."""
     lib = get_lib()
     N, d = x.shape
     _, H, d_h = q.shape
@@ -407,21 +414,24 @@ def layer_train(x, W_r, b_r, q, k, v, M: int, grid=None, window=None, ws=None, r
     mat = lambda: torch.empty((N, H, d_h), dtype=torch.bfloat16, device=dev)
     if res is not None:
         ws = res["ws"] if ws is None else ws
+    vec = lambda: torch.empty((H, N), dtype=torch.float32, device=dev)
     r = dict(res) if res is not None else {"out": mat(), "o_moga": mat(), "o_stga": mat() if window is not None else None,
-         "lse_moga": torch.empty((H, N), dtype=torch.float32, device=dev),
-         "lse_stga": torch.empty((H, N), dtype=torch.float32, device=dev) if window is not None else None,
+         "o_frame": mat() if per_frame else None,
+         "lse_moga": vec(), "lse_stga": vec() if window is not None else None, "lse_frame": vec() if per_frame else None,
          "group_id": torch.empty(N, dtype=torch.int32, device=dev),
          "gate": torch.empty(N, dtype=torch.float32, device=dev),
          "perm": torch.empty(N, dtype=torch.int32, device=dev),
          "offsets": torch.empty(M + 1, dtype=torch.int32, device=dev)}
-    need = lib.moga_layer_train_workspace_size(N, H, d_h, M, *grid3, w3)
+    need = lib.moga_layer_train_ex_workspace_size(N, H, d_h, M, *grid3, w3, int(bool(per_frame)))
     if ws is None or ws.numel() < need:
         ws = workspace(need, dev)
-    st = lib.moga_layer_train(_ptr(x), _ptr(W_r), _ptr(b_r), x_dt, _ptr(q), _ptr(k), _ptr(v), N, d, H, d_h, M,
-                              *grid3, w3, _ptr(r["out"]), _ptr(r["o_moga"]), _ptr(r["o_stga"]),
-                              _ptr(r["lse_moga"]), _ptr(r["lse_stga"]), _ptr(r["group_id"]), _ptr(r["gate"]),
-                              _ptr(r["perm"]), _ptr(r["offsets"]), _ptr(ws), ws.numel(), _stream(dev))
-    _check(st, "moga_layer_train")
+    st = lib.moga_layer_train_ex(_ptr(x), _ptr(W_r), _ptr(b_r), x_dt, _ptr(q), _ptr(k), _ptr(v), N, d, H, d_h, M,
+                                 *grid3, w3, int(bool(per_frame)), _ptr(r["out"]), _ptr(r["o_moga"]),
+                                 _ptr(r["o_stga"]), _ptr(r["o_frame"]), _ptr(r["lse_moga"]), _ptr(r["lse_stga"]),
+                                 _ptr(r["lse_frame"]), _ptr(r["group_id"]), _ptr(r["gate"]), _ptr(r["perm"]),
+                                 _ptr(r["offsets"]), _ptr(ws), ws.numel(), _stream(dev))
+    _check(st, "moga_layer_train_ex")
+    r["per_frame"] = bool(per_frame)
     r["ws"] = ws
     return r
 
@@ -449,12 +459,15 @@ def layer_backward(dout, saved, x, W_r, b_r, q, k, v, M: int, grid=None, window=
     if ws is None or ws.numel() < need:
         ws = workspace(need, dev)
     s = saved
-    st = lib.moga_layer_backward(_ptr(dout), _ptr(x), _ptr(W_r), _ptr(b_r), x_dt, _ptr(q), _ptr(k), _ptr(v), N, d,
-                                 H, d_h, M, *grid3, w3, _ptr(s["o_moga"]), _ptr(s["o_stga"]), _ptr(s["lse_moga"]),
-                                 _ptr(s["lse_stga"]), _ptr(s["group_id"]), _ptr(s["gate"]), _ptr(s["perm"]),
-                                 _ptr(s["offsets"]), _ptr(g["dx"]), _ptr(g["dW_r"]), _ptr(g["db_r"]),
-                                 _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(ws), ws.numel(), _stream(dev))
-    _check(st, "moga_layer_backward")
+    pf = int(bool(s.get("per_frame", False)))
+    st = lib.moga_layer_backward_ex(_ptr(dout), _ptr(x), _ptr(W_r), _ptr(b_r), x_dt, _ptr(q), _ptr(k), _ptr(v), N,
+                                    d, H, d_h, M, *grid3, w3, pf, _ptr(s["o_moga"]), _ptr(s["o_stga"]),
+                                    _ptr(s.get("o_frame")), _ptr(s["lse_moga"]), _ptr(s["lse_stga"]),
+                                    _ptr(s.get("lse_frame")), _ptr(s["group_id"]), _ptr(s["gate"]),
+                                    _ptr(s["perm"]), _ptr(s["offsets"]), _ptr(g["dx"]), _ptr(g["dW_r"]),
+                                    _ptr(g["db_r"]), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(ws),
+                                    ws.numel(), _stream(dev))
+    _check(st, "moga_layer_backward_ex")
     g["ws"] = ws
     return g
 
@@ -466,13 +479,13 @@ class MogaFunction(torch.autograd.Function):
     reach the router through the gate only."""
 
     @staticmethod
-    def forward(ctx, x, W_r, b_r, q, k, v, M, grid=None, window=None):
+    def forward(ctx, x, W_r, b_r, q, k, v, M, grid=None, window=None, per_frame=False):
         r = layer_train(x.contiguous(), W_r.contiguous(), b_r, q.contiguous(), k.contiguous(), v.contiguous(), M,
-                        grid, window)
+                        grid, window, per_frame=per_frame)
         ctx.save_for_backward(x, W_r, q, k, v)
         ctx.b_r = b_r
-        ctx.saved = {n: r[n] for n in ("o_moga", "o_stga", "lse_moga", "lse_stga", "group_id", "gate", "perm",
-                                       "offsets")}
+        ctx.saved = {n: r[n] for n in ("o_moga", "o_stga", "o_frame", "lse_moga", "lse_stga", "lse_frame",
+                                       "group_id", "gate", "perm", "offsets", "per_frame")}
         ctx.args = (M, grid, window)
         return r["out"]
 
@@ -483,7 +496,7 @@ class MogaFunction(torch.autograd.Function):
         g = layer_backward(dout.contiguous().to(torch.bfloat16), ctx.saved, x, W_r, ctx.b_r, q, k, v, M, grid,
                            window)
         db = g["db_r"] if ctx.b_r is not None else None
-        return g["dx"], g["dW_r"].to(W_r.dtype), db, g["dq"], g["dk"], g["dv"], None, None, None
+        return g["dx"], g["dW_r"].to(W_r.dtype), db, g["dq"], g["dk"], g["dv"], None, None, None, None
 
 
 def _host_tensor(t: torch.Tensor, name: str, dtype, shape):

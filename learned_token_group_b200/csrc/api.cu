@@ -825,29 +825,48 @@ moga_status moga_layer(const void* x, const void* W_r, const float* b_r, moga_dt
   return MOGA_OK;
 }
 
-size_t moga_layer_train_workspace_size(int64_t N, int H, int d_h, int M, int T, int Hg, int Wg, const int* window) {
-  return moga_layer_workspace_size(N, H, d_h, M, T, Hg, Wg, window);
+size_t moga_layer_train_ex_workspace_size(int64_t N, int H, int d_h, int M, int T, int Hg, int Wg,
+                                          const int* window, int per_frame) {
+  if (per_frame != 0 && per_frame != 1) return 0;
+  if (!per_frame) return moga_layer_workspace_size(N, H, d_h, M, T, Hg, Wg, window);
+  return moga_layer_ex_workspace_size(N, H, d_h, M, (window ? 1 : 0) | 2);
 }
 
-moga_status moga_layer_train(const void* x, const void* W_r, const float* b_r, moga_dtype x_dt, const void* q,
-                             const void* k, const void* v, int64_t N, int d, int H, int d_h, int M, int T, int Hg,
-                             int Wg, const int* window, void* out, void* o_moga, void* o_stga, float* lse_moga,
-                             float* lse_stga, int32_t* group_id, float* gate, int32_t* perm, int32_t* offsets,
-                             void* ws, size_t ws_bytes, void* stream) {
+size_t moga_layer_train_workspace_size(int64_t N, int H, int d_h, int M, int T, int Hg, int Wg, const int* window) {
+  return moga_layer_train_ex_workspace_size(N, H, d_h, M, T, Hg, Wg, window, 0);
+}
+
+moga_status moga_layer_train_ex(const void* x, const void* W_r, const float* b_r, moga_dtype x_dt, const void* q,
+                                const void* k, const void* v, int64_t N, int d, int H, int d_h, int M, int T, int Hg,
+                                int Wg, const int* window, int per_frame, void* out, void* o_moga, void* o_stga,
+                                void* o_frame, float* lse_moga, float* lse_stga, float* lse_frame, int32_t* group_id,
+                                float* gate, int32_t* perm, int32_t* offsets, void* ws, size_t ws_bytes,
+                                void* stream) {
+  if (per_frame != 0 && per_frame != 1) return MOGA_ERR_INVALID_ARG;
   moga_status st = check_route_args(x, W_r, b_r, x_dt, N, d, M, group_id, gate, perm, offsets, offsets);
   if (st != MOGA_OK) return st;
   if ((st = check_qkv(q, k, v, out)) != MOGA_OK) return st;
   if ((st = check_attn_shape(N, H, d_h)) != MOGA_OK) return st;
   if (!o_moga || !aligned16(o_moga) || (N > 0 && (!lse_moga || !aligned4(lse_moga)))) return MOGA_ERR_INVALID_ARG;
-  if (window) {
+  const int frame_window[3] = {1, Hg, Wg};
+  if (window || per_frame) {
     int64_t n = 0;
-    if ((st = check_window(T, Hg, Wg, window, &n)) != MOGA_OK) return st;
+    if ((st = check_window(T, Hg, Wg, window ? window : frame_window, &n)) != MOGA_OK) return st;
     if (n != N) return MOGA_ERR_INVALID_ARG;
+    if (out == o_moga) return MOGA_ERR_INVALID_ARG;
+  }
+  if (window) {
     if (!o_stga || !aligned16(o_stga) || (N > 0 && (!lse_stga || !aligned4(lse_stga)))) return MOGA_ERR_INVALID_ARG;
-    if (out == o_moga || out == o_stga || o_moga == o_stga) return MOGA_ERR_INVALID_ARG;
+    if (out == o_stga || o_moga == o_stga) return MOGA_ERR_INVALID_ARG;
+  }
+  if (per_frame) {
+    if (!o_frame || !aligned16(o_frame) || (N > 0 && (!lse_frame || !aligned4(lse_frame))))
+      return MOGA_ERR_INVALID_ARG;
+    if (out == o_frame || o_moga == o_frame || (window && o_stga == o_frame)) return MOGA_ERR_INVALID_ARG;
   }
   if (!ws || !aligned16(ws)) return MOGA_ERR_INVALID_ARG;
-  if (ws_bytes < moga_layer_train_workspace_size(N, H, d_h, M, T, Hg, Wg, window)) return MOGA_ERR_WORKSPACE;
+  if (ws_bytes < moga_layer_train_ex_workspace_size(N, H, d_h, M, T, Hg, Wg, window, per_frame))
+    return MOGA_ERR_WORKSPACE;
   DevCtx c;
   if (!make_ctx(&c, ws, stream)) return MOGA_ERR_CUDA;
   uint8_t* w = (uint8_t*)ws;
@@ -858,9 +877,17 @@ moga_status moga_layer_train(const void* x, const void* W_r, const float* b_r, m
   if ((st = group_attn_body(c, q, k, v, perm, offsets, gate, N, H, d_h, M, 1.0f, o_moga, w, lse_moga)) != MOGA_OK)
     return st;
   const int64_t n = N * H * d_h;
-  if (window) {
-    if ((st = stga_body(c, q, k, v, T, Hg, Wg, window, H, d_h, 0, o_stga, w, 1.0f, lse_stga)) != MOGA_OK) return st;
-    if (launch_mean2(c, o_moga, o_stga, n, out) != cudaSuccess) return MOGA_ERR_CUDA;
+  if (window &&
+      (st = stga_body(c, q, k, v, T, Hg, Wg, window, H, d_h, 0, o_stga, w, 1.0f, lse_stga)) != MOGA_OK)
+    return st;
+  if (per_frame &&
+      (st = stga_body(c, q, k, v, T, Hg, Wg, frame_window, H, d_h, 0, o_frame, w, 1.0f, lse_frame)) != MOGA_OK)
+    return st;
+  if (window || per_frame) {
+    // out = the plain mean of the branches that are on
+    const void* b2 = window ? o_stga : o_frame;
+    const void* b3 = (window && per_frame) ? o_frame : nullptr;
+    if (launch_mean(c, o_moga, b2, b3, n, out) != cudaSuccess) return MOGA_ERR_CUDA;
     count(1);
   } else if (out != o_moga) {
     if (cudaMemcpyAsync(out, o_moga, (size_t)n * 2, cudaMemcpyDeviceToDevice, c.stream) != cudaSuccess)
@@ -869,18 +896,30 @@ moga_status moga_layer_train(const void* x, const void* W_r, const float* b_r, m
   return MOGA_OK;
 }
 
+moga_status moga_layer_train(const void* x, const void* W_r, const float* b_r, moga_dtype x_dt, const void* q,
+                             const void* k, const void* v, int64_t N, int d, int H, int d_h, int M, int T, int Hg,
+                             int Wg, const int* window, void* out, void* o_moga, void* o_stga, float* lse_moga,
+                             float* lse_stga, int32_t* group_id, float* gate, int32_t* perm, int32_t* offsets,
+                             void* ws, size_t ws_bytes, void* stream) {
+  return moga_layer_train_ex(x, W_r, b_r, x_dt, q, k, v, N, d, H, d_h, M, T, Hg, Wg, window, 0, out, o_moga, o_stga,
+                             nullptr, lse_moga, lse_stga, nullptr, group_id, gate, perm, offsets, ws, ws_bytes,
+                             stream);
+}
+
 size_t moga_layer_backward_workspace_size(int64_t N, int d, int H, int d_h, int M) {
   if (N < 0 || d < 1 || H < 1 || M < 1 || M > 1024 || (d_h != 64 && d_h != 128)) return 0;
   return bwd_ws(N, d, H, d_h, M).total;
 }
 
-moga_status moga_layer_backward(const void* dout, const void* x, const void* W_r, const float* b_r, moga_dtype x_dt,
-                                const void* q, const void* k, const void* v, int64_t N, int d, int H, int d_h, int M,
-                                int T, int Hg, int Wg, const int* window, const void* o_moga, const void* o_stga,
-                                const float* lse_moga, const float* lse_stga, const int32_t* group_id,
-                                const float* gate, const int32_t* perm, const int32_t* offsets, void* dx,
-                                float* dW_r, float* db_r, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
-                                void* stream) {
+moga_status moga_layer_backward_ex(const void* dout, const void* x, const void* W_r, const float* b_r,
+                                   moga_dtype x_dt, const void* q, const void* k, const void* v, int64_t N, int d,
+                                   int H, int d_h, int M, int T, int Hg, int Wg, const int* window, int per_frame,
+                                   const void* o_moga, const void* o_stga, const void* o_frame, const float* lse_moga,
+                                   const float* lse_stga, const float* lse_frame, const int32_t* group_id,
+                                   const float* gate, const int32_t* perm, const int32_t* offsets, void* dx,
+                                   float* dW_r, float* db_r, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  if (per_frame != 0 && per_frame != 1) return MOGA_ERR_INVALID_ARG;
   // the routing results are inputs here; the forward's checks cover them
   moga_status st = check_route_args(x, W_r, b_r, x_dt, N, d, M, group_id, gate, perm, offsets, offsets);
   if (st != MOGA_OK) return st;
@@ -889,12 +928,16 @@ moga_status moga_layer_backward(const void* dout, const void* x, const void* W_r
   if ((st = check_qkv(dq, dk, dv, o_moga)) != MOGA_OK) return st;
   if (!dW_r || !aligned4(dW_r) || (db_r && !aligned4(db_r))) return MOGA_ERR_INVALID_ARG;
   if (N > 0 && (!dx || !aligned16(dx) || !lse_moga || !aligned4(lse_moga))) return MOGA_ERR_INVALID_ARG;
-  if (window) {
+  const int frame_window[3] = {1, Hg, Wg};
+  if (window || per_frame) {
     int64_t n = 0;
-    if ((st = check_window(T, Hg, Wg, window, &n)) != MOGA_OK) return st;
+    if ((st = check_window(T, Hg, Wg, window ? window : frame_window, &n)) != MOGA_OK) return st;
     if (n != N) return MOGA_ERR_INVALID_ARG;
-    if (!o_stga || !aligned16(o_stga) || (N > 0 && (!lse_stga || !aligned4(lse_stga)))) return MOGA_ERR_INVALID_ARG;
   }
+  if (window && (!o_stga || !aligned16(o_stga) || (N > 0 && (!lse_stga || !aligned4(lse_stga)))))
+    return MOGA_ERR_INVALID_ARG;
+  if (per_frame && (!o_frame || !aligned16(o_frame) || (N > 0 && (!lse_frame || !aligned4(lse_frame)))))
+    return MOGA_ERR_INVALID_ARG;
   if (!ws || !aligned16(ws)) return MOGA_ERR_INVALID_ARG;
   if (ws_bytes < moga_layer_backward_workspace_size(N, d, H, d_h, M)) return MOGA_ERR_WORKSPACE;
   DevCtx c;
@@ -906,18 +949,34 @@ moga_status moga_layer_backward(const void* dout, const void* x, const void* W_r
     if (e == cudaSuccess && db_r) e = cudaMemsetAsync(db_r, 0, (size_t)M * 4, c.stream);
     return from_cuda(e);
   }
-  const float wgt = window ? 0.5f : 1.0f;
+  // each branch's share of dout: one over the number of branches
+  const float wgt = 1.0f / (float)(1 + (window ? 1 : 0) + per_frame);
   if ((st = attn_bwd_branch(c, bw, w, 0, dout, o_moga, lse_moga, q, k, v, perm, offsets, gate, wgt, N, H, d_h, M,
                             T, Hg, Wg, window, 0, dq, dk, dv)) != MOGA_OK)
     return st;
   if (window && (st = attn_bwd_branch(c, bw, w, 1, dout, o_stga, lse_stga, q, k, v, nullptr, nullptr, nullptr, wgt,
                                       N, H, d_h, M, T, Hg, Wg, window, 1, dq, dk, dv)) != MOGA_OK)
     return st;
+  if (per_frame && (st = attn_bwd_branch(c, bw, w, 1, dout, o_frame, lse_frame, q, k, v, nullptr, nullptr, nullptr,
+                                         wgt, N, H, d_h, M, T, Hg, Wg, frame_window, 1, dq, dk, dv)) != MOGA_OK)
+    return st;
   if (launch_route_bwd(c, x, W_r, b_r, x_dt == MOGA_BF16, N, d, M, group_id,
                        reinterpret_cast<const float*>(w + bw.dgate), dx, dW_r, db_r, w + bw.route) != cudaSuccess)
     return MOGA_ERR_CUDA;
   count(3);
   return MOGA_OK;
+}
+
+moga_status moga_layer_backward(const void* dout, const void* x, const void* W_r, const float* b_r, moga_dtype x_dt,
+                                const void* q, const void* k, const void* v, int64_t N, int d, int H, int d_h, int M,
+                                int T, int Hg, int Wg, const int* window, const void* o_moga, const void* o_stga,
+                                const float* lse_moga, const float* lse_stga, const int32_t* group_id,
+                                const float* gate, const int32_t* perm, const int32_t* offsets, void* dx,
+                                float* dW_r, float* db_r, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                                void* stream) {
+  return moga_layer_backward_ex(dout, x, W_r, b_r, x_dt, q, k, v, N, d, H, d_h, M, T, Hg, Wg, window, 0, o_moga,
+                                o_stga, nullptr, lse_moga, lse_stga, nullptr, group_id, gate, perm, offsets, dx, dW_r,
+                                db_r, dq, dk, dv, ws, ws_bytes, stream);
 }
 
 size_t moga_layer_ex_workspace_size(int64_t N, int H, int d_h, int M, int branches) {

@@ -543,18 +543,21 @@ bwd_prep_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ o, con
   }
 }
 
-// out = 0.5 * (a + b), bf16, n8 groups of 8 values
-__global__ void __launch_bounds__(256) mean2_kernel(const uint4* __restrict__ x, const uint4* __restrict__ y,
-                                                    int64_t n8, uint4* __restrict__ out) {
+// out = (x + y (+ z)) / (2 or 3), bf16, n8 groups of 8 values (z nullable)
+__global__ void __launch_bounds__(256) mean_kernel(const uint4* __restrict__ x, const uint4* __restrict__ y,
+                                                   const uint4* __restrict__ z, int64_t n8, uint4* __restrict__ out) {
+  const float inv = z ? (1.0f / 3.0f) : 0.5f;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
     const uint4 a = x[i], b = y[i];
+    const uint4 c = z ? z[i] : make_uint4(0, 0, 0, 0);
     const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
     const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+    const __nv_bfloat162* c2 = reinterpret_cast<const __nv_bfloat162*>(&c);
     uint32_t pk[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float2 fa = __bfloat1622float2(a2[e]), fb = __bfloat1622float2(b2[e]);
-      pk[e] = pack_bf16x2(0.5f * (fa.x + fb.x), 0.5f * (fa.y + fb.y));
+      const float2 fa = __bfloat1622float2(a2[e]), fb = __bfloat1622float2(b2[e]), fc = __bfloat1622float2(c2[e]);
+      pk[e] = pack_bf16x2(inv * (fa.x + fb.x + fc.x), inv * (fa.y + fb.y + fc.y));
     }
     out[i] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
   }
@@ -804,13 +807,14 @@ cudaError_t launch_bwd_prep(const DevCtx& c, const void* dout, const void* o, co
   return cudaGetLastError();
 }
 
-cudaError_t launch_mean2(const DevCtx& c, const void* x, const void* y, int64_t n, void* out) {
+cudaError_t launch_mean(const DevCtx& c, const void* x, const void* y, const void* z, int64_t n, void* out) {
   const int64_t n8 = n / 8;
   if (n8 == 0) return cudaSuccess;
   int64_t blocks = ceil_div(n8, 256);
   const int64_t cap = (int64_t)c.num_sms * 8;
   if (blocks > cap) blocks = cap;
-  mean2_kernel<<<(unsigned)blocks, 256, 0, c.stream>>>((const uint4*)x, (const uint4*)y, n8, (uint4*)out);
+  mean_kernel<<<(unsigned)blocks, 256, 0, c.stream>>>((const uint4*)x, (const uint4*)y, (const uint4*)z, n8,
+                                                      (uint4*)out);
   return cudaGetLastError();
 }
 

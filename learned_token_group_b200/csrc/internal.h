@@ -131,8 +131,8 @@ cudaError_t launch_attn_bwd(const DevCtx& c, const BwdArgs& a, bool dq);
 // is given) the gate gradient sum_h D / gate per token.
 cudaError_t launch_bwd_prep(const DevCtx& c, const void* dout, const void* o, const int32_t* perm, const float* gate,
                             float w, int64_t N, int H, int d_h, void* dO_hat, float* dsum, float* dgate);
-// out = (x + y) / 2 over n bf16 values (n a multiple of 8).
-cudaError_t launch_mean2(const DevCtx& c, const void* x, const void* y, int64_t n, void* out);
+// out = (x + y + z) / 3, or (x + y) / 2 when z is null, over n bf16 values (n a multiple of 8).
+cudaError_t launch_mean(const DevCtx& c, const void* x, const void* y, const void* z, int64_t n, void* out);
 // Router backward through the gate: dx (dtype of x), dW_r fp32 [M, d], db fp32 [M] (nullable).
 constexpr int kRouteSlices = 64;  // upper bound on token slices of the dW_r partial sums
 size_t route_bwd_ws_bytes(int64_t N, int d, int M);

@@ -274,3 +274,35 @@ def test_backward_validation(lib):
     need = lib.moga_layer_backward_workspace_size(360, 64, 2, 128, 4)
     assert need >= 4 * 360 * 2 * 128 * 2                 # head-major q, k, v and dO copies
     assert lib.moga_layer_backward_workspace_size(360, 64, 2, 96, 4) == 0
+
+
+def test_train_ex_validation(lib):
+    w = (ctypes.c_int * 3)(3, 8, 8)
+    f = lib.moga_layer_train_ex
+    Q, R, S = 0x1000010, 0x1000020, 0x1000030
+    args = [P, P, None, 1, P, P, P, 360, 64, 2, 128, 4, 3, 10, 12, w, 1, P, Q, R, S, P, P, P, P, P, P, P, P, BIG,
+            None]
+    bad = list(args)
+    bad[16] = 2                                       # per_frame must be 0 or 1
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[20] = None                                    # o_frame missing with per_frame
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[20] = R                                       # o_frame must differ from o_stga
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[15] = None
+    bad[12] = 4                                       # per-frame alone still needs a grid covering N
+    assert f(*bad) == INVALID
+    assert lib.moga_layer_train_ex_workspace_size(360, 2, 128, 4, 3, 10, 12, w, 1) >= \
+        lib.moga_layer_train_ex_workspace_size(360, 2, 128, 4, 3, 10, 12, w, 0) > 0
+    g = lib.moga_layer_backward_ex
+    gargs = [P, P, P, None, 1, P, P, P, 360, 64, 2, 128, 4, 3, 10, 12, w, 1, P, P, P, P, P, P, P, P, P, P,
+             P, P, None, P, P, P, P, BIG, None]
+    bad = list(gargs)
+    bad[17] = 3
+    assert g(*bad) == INVALID
+    bad = list(gargs)
+    bad[20] = None                                    # o_frame missing with per_frame
+    assert g(*bad) == INVALID

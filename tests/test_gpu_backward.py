@@ -271,3 +271,30 @@ def test_backward_full_size_sampled():
         got_x.append(np_cpu(g["dx"][torch.as_tensor(rows, device="cuda")]).astype(np.float64))
     rel = _rel(np.concatenate(got_x), np.concatenate(ref_x))
     assert rel <= ROUTER_REL_L2, f"dx: rel-L2 {rel:.3e}"
+
+
+@pytest.mark.parametrize("wl,window", [
+    (custom(360, H=2, d_h=64, d=64, M=4, grid=(3, 10, 12), window=(3, 8, 8)), (3, 8, 8)),
+    (custom(3120, H=1, d_h=128, d=64, M=3, grid=(2, 30, 52), window=(3, 8, 8)), (3, 8, 8)),
+    (custom(360, H=2, d_h=128, d=64, M=4, grid=(3, 10, 12)), None),     # MoGA + per-frame only
+])
+def test_backward_three_branches(wl, window):
+    """The block with the per-frame branch (moga_layer_train_ex /
+    moga_layer_backward_ex): out is the mean of the branches that are on and
+    each branch's share of dout is dout divided by their number."""
+    inp = make_inputs(wl, seed=21, device="cuda")
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(22)
+    b_r = 0.1 * torch.randn(wl.M, generator=gen, device="cuda")
+    dout = torch.randn((wl.N, wl.H, wl.d_h), generator=gen, device="cuda").to(torch.bfloat16)
+    args = (inp["x"], inp["W_r"], b_r, inp["q"], inp["k"], inp["v"], wl.M, wl.grid, window)
+    sv = moga.layer_train(*args, per_frame=True)
+    g = moga.layer_backward(dout, sv, *args)
+    moga.sync_status(g["ws"])
+    x, W, q, k, v = (np_cpu(inp[n]) for n in ("x", "W_r", "q", "k", "v"))
+    ref = oracle.moga_layer(x, W, np_cpu(b_r), q, k, v, wl.M, grid=wl.grid, window=window, per_frame=True)
+    compare_out(sv["o_frame"], ref["frame"], what="o_frame")
+    compare_out(sv["out"], ref["out"], what="out")
+    gref = oracle.moga_layer_backward(x, W, np_cpu(b_r), q, k, v, wl.M, np_cpu(dout), grid=wl.grid, window=window,
+                                      per_frame=True)
+    _check_grads(g, gref)

@@ -444,7 +444,8 @@ def _fd_problem(seed, M=3, window=(1, 2, 3), per_frame=True, bias=True):
 def check_backward_finite_differences(o):
     """Every gradient of L = sum(dout * out) against central differences of
     the (separately pinned) forward, on sampled coordinates of every input."""
-    for seed, kw in ((30, {}), (31, {"window": None, "per_frame": False}), (32, {"per_frame": False})):
+    for seed, kw in ((30, {}), (31, {"window": None, "per_frame": False}), (32, {"per_frame": False}),
+                     (33, {"window": None})):
         pr = _fd_problem(seed, **kw)
         fwd_args = {k_: pr[k_] for k_ in ("x", "W_r", "b_r", "q", "k", "v")}
         M, grid, window, pf, dout = pr["M"], pr["grid"], pr["window"], pr["per_frame"], pr["dout"]
