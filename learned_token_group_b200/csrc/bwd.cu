@@ -117,8 +117,9 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
   uint64_t* x_empty = bars + 1;
   uint64_t* y_full = bars + 2;                  // [kYStages]
   uint64_t* y_empty = y_full + kYStages;        // [kYStages]
-  uint64_t* s_full = y_empty + kYStages;        // S and dP computed
-  uint64_t* p_full = s_full + 1;                // P and dS written
+  uint64_t* s_full = y_empty + kYStages;        // S computed
+  uint64_t* d_full = s_full + 1;                // dP computed
+  uint64_t* p_full = d_full + 1;                // P and dS written
   uint64_t* acc_full = p_full + 1;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* done_bar = acc_empty + 1;
@@ -137,6 +138,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
       mbar_init(&y_empty[s], 1);
     }
     mbar_init(s_full, 1);
+    mbar_init(d_full, 1);
     mbar_init(p_full, 256);
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 256);
@@ -251,6 +253,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
       bool ok = true;
       // S (or S^T) = X1 Y1^T and dP (or dP^T) = X2 Y2^T, both operands K-major.
       const uint64_t x1d = sdesc_sw128(x1, 16, 1024), x2d = sdesc_sw128(x2, 16, 1024);
+      // S first, with its own commit, so that the softmax warps compute P
+      // while the tensor core computes dP.
       auto issue_s = [&](int s) {
         const uint32_t y1 = smem_u32(smem + P::kY0 + s * P::kYStage);
         const uint64_t y1d = sdesc_sw128(y1, 16, 1024), y2d = sdesc_sw128(y1 + P::kYBytes, 16, 1024);
@@ -259,11 +263,13 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
           const uint32_t xo = (kk >> 2) * P::kXChunk + (kk & 3) * 32, yo = (kk >> 2) * P::kYChunk + (kk & 3) * 32;
           umma_bf16(tS, sdesc_add(x1d, xo), sdesc_add(y1d, yo), idS, kk > 0 ? 1u : 0u);
         }
+        umma_commit(s_full);
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
           const uint32_t xo = (kk >> 2) * P::kXChunk + (kk & 3) * 32, yo = (kk >> 2) * P::kYChunk + (kk & 3) * 32;
           umma_bf16(tD, sdesc_add(x2d, xo), sdesc_add(y2d, yo), idS, kk > 0 ? 1u : 0u);
         }
+        umma_commit(d_full);
       };
       // Accumulations over the 128 Y rows (eight 16-row steps).  Warpgroup w
       // wrote P / dS of Y rows [64w, 64w + 64) as packed bf16 into columns
@@ -308,7 +314,6 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
           if (!mbar_wait(&y_full[s], (yc / kYStages) & 1, wc, 4, yc)) { ok = false; break; }
           tc_fence_after();
           issue_s(s);
-          umma_commit(s_full);
           if (i + 1 == ny) umma_commit(x_empty);
           ++yc;
         }
@@ -355,41 +360,58 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
         // on the stage's own barrier too (its phase is still this tile's,
         // since the stage is refilled only after this tile's P and dS)
         if (!kDQ && !mbar_wait(&y_full[s], (yc / kYStages) & 1, wc, 11 + wg, yc)) { ok = false; break; }
-        // Y columns [64 wg, 64 wg + 64) in two halves of 32; the packed P / dS
-        // of half hf go to columns 64 wg + 16 hf, which this warpgroup has
-        // already read.
+        // Y columns [64 wg, 64 wg + 64): P from S as soon as S is in (the
+        // tensor core is still computing dP), then dS once dP is in.  The
+        // packed P / dS of half hf go to columns 64 wg + 16 hf, which this
+        // warpgroup has already read.
+        float pv[64];
+        {
+          float sv[64];
+          tmem_ld32(tS + lb + 64 * wg, sv);
+          tmem_ld32(tS + lb + 64 * wg + 32, sv + 32);
+          tmem_ld_wait();
+          if (kDQ) {
+            const int valid = u.len - i * kYRows - 64 * wg;  // keys of these columns inside the segment
+#pragma unroll
+            for (int e = 0; e < 64; ++e) {
+              const float pe = fast_exp2(fmaf(sv[e], scale_log2, nl_row));
+              pv[e] = e < valid ? pe : 0.0f;
+            }
+          } else {
+            const float* nl = vec + s * 2 * kYRows + 64 * wg;
+#pragma unroll
+            for (int e = 0; e < 64; ++e) pv[e] = fast_exp2(fmaf(sv[e], scale_log2, nl[e]));
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pv[32 * hf + 2 * e], pv[32 * hf + 2 * e + 1]);
+              tmem_st16u(tS + lb + 64 * wg + 16 * hf, pk);
+            }
+          }
+        }
+        if (!mbar_wait(d_full, yc & 1, wc, 13 + wg, yc)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           const int c0 = 64 * wg + 32 * hf;
-          float sv[32], dv[32];
-          tmem_ld32(tS + lb + c0, sv);
+          float dv[32];
           tmem_ld32(tD + lb + c0, dv);
           tmem_ld_wait();
-          uint32_t pk[16], dk[16];
+          uint32_t dk[16];
           if (kDQ) {
-            const int valid = u.len - i * kYRows - c0;  // keys of these columns inside the segment
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float p0 = fast_exp2(fmaf(sv[2 * e], scale_log2, nl_row));
-              float p1 = fast_exp2(fmaf(sv[2 * e + 1], scale_log2, nl_row));
-              p0 = 2 * e < valid ? p0 : 0.0f;
-              p1 = 2 * e + 1 < valid ? p1 : 0.0f;
-              pk[e] = pack_bf16x2(p0 * (dv[2 * e] - d_row), p1 * (dv[2 * e + 1] - d_row));
-            }
-            tmem_st16u(tD + lb + 64 * wg + 16 * hf, pk);
+            for (int e = 0; e < 16; ++e)
+              dk[e] = pack_bf16x2(pv[32 * hf + 2 * e] * (dv[2 * e] - d_row),
+                                  pv[32 * hf + 2 * e + 1] * (dv[2 * e + 1] - d_row));
           } else {
-            const float* nl = vec + s * 2 * kYRows + c0;
-            const float* dd = nl + kYRows;
+            const float* dd = vec + s * 2 * kYRows + kYRows + c0;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float p0 = fast_exp2(fmaf(sv[2 * e], scale_log2, nl[2 * e]));
-              const float p1 = fast_exp2(fmaf(sv[2 * e + 1], scale_log2, nl[2 * e + 1]));
-              pk[e] = pack_bf16x2(p0, p1);
-              dk[e] = pack_bf16x2(p0 * (dv[2 * e] - dd[2 * e]), p1 * (dv[2 * e + 1] - dd[2 * e + 1]));
-            }
-            tmem_st16u(tS + lb + 64 * wg + 16 * hf, pk);
-            tmem_st16u(tD + lb + 64 * wg + 16 * hf, dk);
+            for (int e = 0; e < 16; ++e)
+              dk[e] = pack_bf16x2(pv[32 * hf + 2 * e] * (dv[2 * e] - dd[2 * e]),
+                                  pv[32 * hf + 2 * e + 1] * (dv[2 * e + 1] - dd[2 * e + 1]));
           }
+          tmem_st16u(tD + lb + 64 * wg + 16 * hf, dk);
         }
         tmem_st_wait();
         tc_fence_before();
