@@ -298,7 +298,13 @@ moga_status moga_layer_backward(const void* dout, const void* x, const void* W_r
  * [N, H, d_h]) and lse_frame (fp32 [H, N], token order) are the per-frame
  * branch's output and log-sum-exp, unused when per_frame = 0.  Everything
  * else as moga_layer_train / moga_layer_backward (which are these calls with
- * per_frame = 0).
+ * per_frame = 0 and balance_alpha = 0).
+ * balance_alpha (finite): adds the group balancing loss of the "Group
+ * Balancing Loss" section, alpha * M * sum_i F_i P_i with F_i the share of
+ * tokens routed to group i (from offsets; an argmax count, so it carries no
+ * gradient) and P_i the mean over tokens of p(i|x), to the loss whose router
+ * gradient is returned: dr_ij += alpha * M / N * p_ij * (F_j - sum_k F_k p_ik).
+ * 0 leaves it out.
  * Workspace: moga_layer_train_ex_workspace_size(...) / moga_layer_backward_workspace_size(...). */
 size_t moga_layer_train_ex_workspace_size(int64_t N, int H, int d_h, int M, int T, int Hg, int Wg,
                                           const int* window, int per_frame);
@@ -311,7 +317,8 @@ moga_status moga_layer_train_ex(const void* x, const void* W_r, const float* b_r
 moga_status moga_layer_backward_ex(const void* dout, const void* x, const void* W_r, const float* b_r,
                                    moga_dtype x_dt, const void* q, const void* k, const void* v, int64_t N, int d,
                                    int H, int d_h, int M, int T, int Hg, int Wg, const int* window, int per_frame,
-                                   const void* o_moga, const void* o_stga, const void* o_frame, const float* lse_moga,
+                                   float balance_alpha, const void* o_moga, const void* o_stga, const void* o_frame,
+                                   const float* lse_moga,
                                    const float* lse_stga, const float* lse_frame, const int32_t* group_id,
                                    const float* gate, const int32_t* perm, const int32_t* offsets, void* dx,
                                    float* dW_r, float* db_r, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,

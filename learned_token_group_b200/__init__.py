@@ -91,7 +91,7 @@ def get_lib():
         "moga_layer_train_ex_workspace_size": (_SZ, [_I64, _I, _I, _I, _I, _I, _I, _P, _I]),
         "moga_layer_train_ex": (_I, [_P, _P, _P, _I, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _I, _P, _I,
                                      _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
-        "moga_layer_backward_ex": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _I, _P, _I,
+        "moga_layer_backward_ex": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _I, _P, _I, _F,
                                         _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
         "moga_layer_backward": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _I, _P,
                                      _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -436,11 +436,13 @@ def layer_train(x, W_r, b_r, q, k, v, M: int, grid=None, window=None, ws=None, r
     return r
 
 
-def layer_backward(dout, saved, x, W_r, b_r, q, k, v, M: int, grid=None, window=None, ws=None, grads=None):
-    """Gradients of one block (moga_layer_backward in moga.h) from dout and
+def layer_backward(dout, saved, x, W_r, b_r, q, k, v, M: int, grid=None, window=None, ws=None, grads=None,
+                   balance_alpha: float = 0.0):
+    """Gradients of one block (moga_layer_backward_ex in moga.h) from dout and
     the dict ``layer_train`` returned: dict(dx, dW_r, db_r, dq, dk, dv, ws).
-    db_r is None when b_r is None.  ``grads``: a previous result of the same
-    shapes whose buffers are reused."""
+    db_r is None when b_r is None.  balance_alpha adds the group balancing
+    loss alpha * M * sum_i F_i P_i to the router's gradient.  ``grads``: a
+    previous result of the same shapes whose buffers are reused."""
     lib = get_lib()
     N, d = x.shape
     _, H, d_h = q.shape
@@ -461,7 +463,8 @@ def layer_backward(dout, saved, x, W_r, b_r, q, k, v, M: int, grid=None, window=
     s = saved
     pf = int(bool(s.get("per_frame", False)))
     st = lib.moga_layer_backward_ex(_ptr(dout), _ptr(x), _ptr(W_r), _ptr(b_r), x_dt, _ptr(q), _ptr(k), _ptr(v), N,
-                                    d, H, d_h, M, *grid3, w3, pf, _ptr(s["o_moga"]), _ptr(s["o_stga"]),
+                                    d, H, d_h, M, *grid3, w3, pf, float(balance_alpha), _ptr(s["o_moga"]),
+                                    _ptr(s["o_stga"]),
                                     _ptr(s.get("o_frame")), _ptr(s["lse_moga"]), _ptr(s["lse_stga"]),
                                     _ptr(s.get("lse_frame")), _ptr(s["group_id"]), _ptr(s["gate"]),
                                     _ptr(s["perm"]), _ptr(s["offsets"]), _ptr(g["dx"]), _ptr(g["dW_r"]),
@@ -474,29 +477,31 @@ def layer_backward(dout, saved, x, W_r, b_r, q, k, v, M: int, grid=None, window=
 
 class MogaFunction(torch.autograd.Function):
     """The block as an autograd function: out = MogaFunction.apply(x, W_r,
-    b_r, q, k, v, M, grid, window).  Forward runs ``layer_train``, backward
-    ``layer_backward``; the group assignment is held fixed, so gradients
-    reach the router through the gate only."""
+    b_r, q, k, v, M, grid, window, per_frame, balance_alpha).  Forward runs
+    ``layer_train``, backward ``layer_backward``; the group assignment is held
+    fixed, so gradients reach the router through the gate (and, with
+    balance_alpha, through the group balancing loss, which the caller adds to
+    its loss as alpha * M * sum_i F_i P_i)."""
 
     @staticmethod
-    def forward(ctx, x, W_r, b_r, q, k, v, M, grid=None, window=None, per_frame=False):
+    def forward(ctx, x, W_r, b_r, q, k, v, M, grid=None, window=None, per_frame=False, balance_alpha=0.0):
         r = layer_train(x.contiguous(), W_r.contiguous(), b_r, q.contiguous(), k.contiguous(), v.contiguous(), M,
                         grid, window, per_frame=per_frame)
         ctx.save_for_backward(x, W_r, q, k, v)
         ctx.b_r = b_r
         ctx.saved = {n: r[n] for n in ("o_moga", "o_stga", "o_frame", "lse_moga", "lse_stga", "lse_frame",
                                        "group_id", "gate", "perm", "offsets", "per_frame")}
-        ctx.args = (M, grid, window)
+        ctx.args = (M, grid, window, balance_alpha)
         return r["out"]
 
     @staticmethod
     def backward(ctx, dout):
         x, W_r, q, k, v = ctx.saved_tensors
-        M, grid, window = ctx.args
+        M, grid, window, alpha = ctx.args
         g = layer_backward(dout.contiguous().to(torch.bfloat16), ctx.saved, x, W_r, ctx.b_r, q, k, v, M, grid,
-                           window)
+                           window, balance_alpha=alpha)
         db = g["db_r"] if ctx.b_r is not None else None
-        return g["dx"], g["dW_r"].to(W_r.dtype), db, g["dq"], g["dk"], g["dv"], None, None, None, None
+        return g["dx"], g["dW_r"].to(W_r.dtype), db, g["dq"], g["dk"], g["dv"], None, None, None, None, None
 
 
 def _host_tensor(t: torch.Tensor, name: str, dtype, shape):

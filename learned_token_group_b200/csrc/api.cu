@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cmath>
 #include <mutex>
 
 #include "../../include/moga.h"
@@ -914,12 +915,15 @@ size_t moga_layer_backward_workspace_size(int64_t N, int d, int H, int d_h, int 
 moga_status moga_layer_backward_ex(const void* dout, const void* x, const void* W_r, const float* b_r,
                                    moga_dtype x_dt, const void* q, const void* k, const void* v, int64_t N, int d,
                                    int H, int d_h, int M, int T, int Hg, int Wg, const int* window, int per_frame,
-                                   const void* o_moga, const void* o_stga, const void* o_frame, const float* lse_moga,
+                                   float balance_alpha, const void* o_moga, const void* o_stga, const void* o_frame,
+                                   const float* lse_moga,
                                    const float* lse_stga, const float* lse_frame, const int32_t* group_id,
                                    const float* gate, const int32_t* perm, const int32_t* offsets, void* dx,
                                    float* dW_r, float* db_r, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
                                    void* stream) {
   if (per_frame != 0 && per_frame != 1) return MOGA_ERR_INVALID_ARG;
+  if (!std::isfinite(balance_alpha))
+    return MOGA_ERR_INVALID_ARG;
   // the routing results are inputs here; the forward's checks cover them
   moga_status st = check_route_args(x, W_r, b_r, x_dt, N, d, M, group_id, gate, perm, offsets, offsets);
   if (st != MOGA_OK) return st;
@@ -961,7 +965,8 @@ moga_status moga_layer_backward_ex(const void* dout, const void* x, const void* 
                                          wgt, N, H, d_h, M, T, Hg, Wg, frame_window, 1, dq, dk, dv)) != MOGA_OK)
     return st;
   if (launch_route_bwd(c, x, W_r, b_r, x_dt == MOGA_BF16, N, d, M, group_id,
-                       reinterpret_cast<const float*>(w + bw.dgate), dx, dW_r, db_r, w + bw.route) != cudaSuccess)
+                       reinterpret_cast<const float*>(w + bw.dgate), offsets, balance_alpha, dx, dW_r, db_r,
+                       w + bw.route) != cudaSuccess)
     return MOGA_ERR_CUDA;
   count(3);
   return MOGA_OK;
@@ -974,9 +979,9 @@ moga_status moga_layer_backward(const void* dout, const void* x, const void* W_r
                                 const float* gate, const int32_t* perm, const int32_t* offsets, void* dx,
                                 float* dW_r, float* db_r, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
                                 void* stream) {
-  return moga_layer_backward_ex(dout, x, W_r, b_r, x_dt, q, k, v, N, d, H, d_h, M, T, Hg, Wg, window, 0, o_moga,
-                                o_stga, nullptr, lse_moga, lse_stga, nullptr, group_id, gate, perm, offsets, dx, dW_r,
-                                db_r, dq, dk, dv, ws, ws_bytes, stream);
+  return moga_layer_backward_ex(dout, x, W_r, b_r, x_dt, q, k, v, N, d, H, d_h, M, T, Hg, Wg, window, 0, 0.0f,
+                                o_moga, o_stga, nullptr, lse_moga, lse_stga, nullptr, group_id, gate, perm, offsets,
+                                dx, dW_r, db_r, dq, dk, dv, ws, ws_bytes, stream);
 }
 
 size_t moga_layer_ex_workspace_size(int64_t N, int H, int d_h, int M, int branches) {

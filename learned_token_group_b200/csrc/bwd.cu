@@ -588,7 +588,11 @@ __global__ void __launch_bounds__(256) mean_kernel(const uint4* __restrict__ x, 
 // ------------------------------------------------------------------ router backward
 // Eqs. 2-3 ("MoGA Router") differentiated through the gate:
 //   r = x W_r^T + b,  p = softmax(r),  gate = p_g (g = the forward's group id),
-//   dr_j = dgate * p_g * ([j == g] - p_j),
+//   dr_j = dgate * p_g * ([j == g] - p_j)
+//        + bcoef * p_j * (F_j - sum_k F_k p_k)   (the group balancing loss of
+//          Eq. 6, alpha * M * sum_i F_i P_i with P_i the mean of p(i|x) over
+//          the N tokens: bcoef = alpha * M / N; F_i, the share of tokens routed
+//          to i, comes from the forward's offsets and carries no gradient),
 //   dx = dr W_r,  dW_r = dr^T x,  db = sum over tokens of dr.
 template <typename T>
 struct Vec;
@@ -634,11 +638,17 @@ constexpr int kRbGroups = 16;  // logits accumulated per pass over a row of x
 template <typename T>
 __global__ void __launch_bounds__(kRbWarps * 32)
 route_bwd_kernel(const T* __restrict__ x, const T* __restrict__ W, const float* __restrict__ b,
-                 const int32_t* __restrict__ gid, const float* __restrict__ dgate, int64_t N, int d, int M,
-                 float* __restrict__ dr, T* __restrict__ dx, int* status) {
+                 const int32_t* __restrict__ gid, const float* __restrict__ dgate, const int32_t* __restrict__ offsets,
+                 float bcoef, int64_t N, int d, int M, float* __restrict__ dr, T* __restrict__ dx, int* status) {
   extern __shared__ float rb_smem[];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   float* lg = rb_smem + wid * M;  // this warp's logits, then dr
+  float* F = rb_smem + kRbWarps * M;  // share of tokens per group (balancing loss)
+  if (bcoef != 0.0f) {
+    const float invN = 1.0f / (float)N;
+    for (int j = threadIdx.x; j < M; j += blockDim.x) F[j] = (float)(offsets[j + 1] - offsets[j]) * invN;
+  }
+  __syncthreads();
   constexpr int V = Vec<T>::n;
   const int nv = d / V;
   for (int64_t i = (int64_t)blockIdx.x * kRbWarps + wid; i < N; i += (int64_t)gridDim.x * kRbWarps) {
@@ -687,10 +697,16 @@ route_bwd_kernel(const T* __restrict__ x, const T* __restrict__ W, const float* 
     for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
     const float pg = expf(lg[g] - mx) / z;
     const float k = dgate[i] * pg;
+    float fs = 0.0f;  // sum_k F_k p_k
+    if (bcoef != 0.0f) {
+      for (int j = lane; j < M; j += 32) fs += F[j] * expf(lg[j] - mx) / z;
+      for (int off = 16; off > 0; off >>= 1) fs += __shfl_xor_sync(0xffffffffu, fs, off);
+    }
     __syncwarp();
     for (int j = lane; j < M; j += 32) {
       const float pj = expf(lg[j] - mx) / z;
-      const float v = k * ((j == g ? 1.0f : 0.0f) - pj);
+      float v = k * ((j == g ? 1.0f : 0.0f) - pj);
+      if (bcoef != 0.0f) v += bcoef * pj * (F[j] - fs);
       lg[j] = v;
       dr[i * M + j] = v;
     }
@@ -853,14 +869,15 @@ size_t route_bwd_ws_bytes(int64_t N, int d, int M) {
 }
 
 cudaError_t launch_route_bwd(const DevCtx& c, const void* x, const void* W, const float* b, bool bf16, int64_t N,
-                             int d, int M, const int32_t* gid, const float* dgate, void* dx, float* dW, float* db,
-                             uint8_t* ws) {
+                             int d, int M, const int32_t* gid, const float* dgate, const int32_t* offsets,
+                             float balance_alpha, void* dx, float* dW, float* db, uint8_t* ws) {
+  const float bcoef = N > 0 ? balance_alpha * (float)M / (float)N : 0.0f;
   float* dr = reinterpret_cast<float*>(ws);
   float* pw = reinterpret_cast<float*>(ws + align_up((size_t)N * M * 4, 256));
   const int smax = route_max_slices(d, M);
   float* pb = reinterpret_cast<float*>(ws + align_up((size_t)N * M * 4, 256) +
                                        align_up((size_t)smax * M * d * 4, 256));
-  const size_t smem = (size_t)kRbWarps * M * 4;
+  const size_t smem = (size_t)(kRbWarps + 1) * M * 4;
   if (N > 0) {
     int64_t blocks = ceil_div(N, kRbWarps);
     const int64_t cap = (int64_t)c.num_sms * 8;
@@ -870,13 +887,14 @@ cudaError_t launch_route_bwd(const DevCtx& c, const void* x, const void* W, cons
       if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return cudaErrorInvalidValue;
       k<<<(unsigned)blocks, kRbWarps * 32, smem, c.stream>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)W, b,
-                                                             gid, dgate, N, d, M, dr, (__nv_bfloat16*)dx, c.status);
+                                                             gid, dgate, offsets, bcoef, N, d, M, dr,
+                                                             (__nv_bfloat16*)dx, c.status);
     } else {
       auto k = route_bwd_kernel<float>;
       if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return cudaErrorInvalidValue;
-      k<<<(unsigned)blocks, kRbWarps * 32, smem, c.stream>>>((const float*)x, (const float*)W, b, gid, dgate, N, d,
-                                                             M, dr, (float*)dx, c.status);
+      k<<<(unsigned)blocks, kRbWarps * 32, smem, c.stream>>>((const float*)x, (const float*)W, b, gid, dgate,
+                                                             offsets, bcoef, N, d, M, dr, (float*)dx, c.status);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -133,12 +133,14 @@ cudaError_t launch_bwd_prep(const DevCtx& c, const void* dout, const void* o, co
                             float w, int64_t N, int H, int d_h, void* dO_hat, float* dsum, float* dgate);
 // out = (x + y + z) / 3, or (x + y) / 2 when z is null, over n bf16 values (n a multiple of 8).
 cudaError_t launch_mean(const DevCtx& c, const void* x, const void* y, const void* z, int64_t n, void* out);
-// Router backward through the gate: dx (dtype of x), dW_r fp32 [M, d], db fp32 [M] (nullable).
+// Router backward through the gate (plus, when balance_alpha != 0, the group
+// balancing loss alpha * M * sum_i F_i P_i with F from offsets): dx (dtype of
+// x), dW_r fp32 [M, d], db fp32 [M] (nullable).
 constexpr int kRouteSlices = 64;  // upper bound on token slices of the dW_r partial sums
 size_t route_bwd_ws_bytes(int64_t N, int d, int M);
 cudaError_t launch_route_bwd(const DevCtx& c, const void* x, const void* W, const float* b, bool bf16, int64_t N,
-                             int d, int M, const int32_t* gid, const float* dgate, void* dx, float* dW, float* db,
-                             uint8_t* ws);
+                             int d, int M, const int32_t* gid, const float* dgate, const int32_t* offsets,
+                             float balance_alpha, void* dx, float* dW, float* db, uint8_t* ws);
 
 // ------------------------------------------------------------------ shot windows
 // Window table of shot-aware STGA (int32, device):

@@ -388,8 +388,11 @@ def attention_rows_backward(Q: np.ndarray, K: np.ndarray, V: np.ndarray, dO: np.
 
 
 def moga_layer_backward(x, W_r, b_r, q, k, v, M: int, dout, grid=None, window=None,
-                        per_frame: bool = False):
-    """Gradients of L = sum(dout * out) for the block of ``moga_layer``.
+                        per_frame: bool = False, balance_alpha: float = 0.0):
+    """Gradients of L = sum(dout * out) + alpha * M * sum_i F_i P_i for the
+    block of ``moga_layer`` (the second term is the group balancing loss of
+    Eq. 6 in the reading of ``balance_stats``; F_i, a count of argmax
+    assignments, is piecewise constant and carries no gradient).
 
     out = mean over the branches that are on of: MoGA (Eq. 5: gate * SA within
     the token's group), STGA (SA within each window), per-frame (SA within each
@@ -397,7 +400,8 @@ def moga_layer_backward(x, W_r, b_r, q, k, v, M: int, dout, grid=None, window=No
     group assignment is held fixed (see the module notes); the gate
     p = softmax(x W_r^T + b)_g carries the router's gradient:
       dgate_i = sum_{h,c} w * dout[i,h,c] * SA_i[h,c];
-      dr_ij   = dgate_i * p_ig * ([j == g] - p_ij)      (softmax Jacobian);
+      dr_ij   = dgate_i * p_ig * ([j == g] - p_ij)      (softmax Jacobian)
+              + alpha * M / N * p_ij * (F_j - sum_k F_k p_ik)   (balancing loss);
       dW_r = dr^T x;  db_r = sum_i dr_i;  dx = dr W_r   (the router's part of dx).
     Returns a dict of float64 arrays dx [N, d], dW_r [M, d], db_r [M],
     dq, dk, dv [N, H, d_h], plus dgate [N].
@@ -442,6 +446,9 @@ def moga_layer_backward(x, W_r, b_r, q, k, v, M: int, dout, grid=None, window=No
     onehot = np.zeros((N, M))
     onehot[np.arange(N), g] = 1.0
     dr = (dgate * gate)[:, None] * (onehot - p)
+    if balance_alpha:
+        F = np.bincount(g, minlength=M) / N
+        dr += (balance_alpha * M / N) * p * (F[None, :] - (p @ F)[:, None])
     return {"dx": dr @ W, "dW_r": dr.T @ X, "db_r": dr.sum(axis=0),
             "dq": dq, "dk": dk, "dv": dv, "dgate": dgate}
 

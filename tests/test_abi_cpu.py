@@ -298,11 +298,14 @@ def test_train_ex_validation(lib):
     assert lib.moga_layer_train_ex_workspace_size(360, 2, 128, 4, 3, 10, 12, w, 1) >= \
         lib.moga_layer_train_ex_workspace_size(360, 2, 128, 4, 3, 10, 12, w, 0) > 0
     g = lib.moga_layer_backward_ex
-    gargs = [P, P, P, None, 1, P, P, P, 360, 64, 2, 128, 4, 3, 10, 12, w, 1, P, P, P, P, P, P, P, P, P, P,
+    gargs = [P, P, P, None, 1, P, P, P, 360, 64, 2, 128, 4, 3, 10, 12, w, 1, 0.0, P, P, P, P, P, P, P, P, P, P,
              P, P, None, P, P, P, P, BIG, None]
     bad = list(gargs)
     bad[17] = 3
     assert g(*bad) == INVALID
     bad = list(gargs)
-    bad[20] = None                                    # o_frame missing with per_frame
+    bad[21] = None                                    # o_frame missing with per_frame
+    assert g(*bad) == INVALID
+    bad = list(gargs)
+    bad[18] = float("nan")                            # balance_alpha must be finite
     assert g(*bad) == INVALID

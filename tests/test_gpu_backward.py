@@ -298,3 +298,30 @@ def test_backward_three_branches(wl, window):
     gref = oracle.moga_layer_backward(x, W, np_cpu(b_r), q, k, v, wl.M, np_cpu(dout), grid=wl.grid, window=window,
                                       per_frame=True)
     _check_grads(g, gref)
+
+
+def test_backward_with_balancing_loss():
+    """balance_alpha adds the group balancing loss (alpha * M * sum_i F_i P_i,
+    "Group Balancing Loss") to the router's gradient; q, k, v are unaffected."""
+    wl = custom(700, H=2, d_h=128, d=64, M=5, x_kind="clustered")
+    inp, b_r, dout, sv, g0 = _run(wl, 31)
+    args = (inp["x"], inp["W_r"], b_r, inp["q"], inp["k"], inp["v"], wl.M, wl.grid, wl.window)
+    g = moga.layer_backward(dout, sv, *args, balance_alpha=0.1)
+    moga.sync_status(g["ws"])
+    for n in ("dq", "dk", "dv"):
+        assert torch.equal(g[n], g0[n]), n
+    x, W, q, k, v = (np_cpu(inp[n]) for n in ("x", "W_r", "q", "k", "v"))
+    ref = oracle.moga_layer_backward(x, W, np_cpu(b_r), q, k, v, wl.M, np_cpu(dout), balance_alpha=0.1)
+    _check_grads(g, ref)
+    # with dout = 0 the balancing term is the router's whole gradient (and
+    # q, k, v get none), so the term is compared on its own
+    zero = torch.zeros_like(dout)
+    gz = moga.layer_backward(zero, sv, *args, balance_alpha=0.5)
+    moga.sync_status(gz["ws"])
+    refz = oracle.moga_layer_backward(x, W, np_cpu(b_r), q, k, v, wl.M, np_cpu(zero), balance_alpha=0.5)
+    assert np.abs(refz["dW_r"]).max() > 0
+    for n in ("dq", "dk", "dv"):
+        assert float(gz[n].float().abs().max()) == 0.0, n
+    for n in ("dx", "dW_r", "db_r"):
+        rel = _rel(np_cpu(gz[n]).astype(np.float64), refz[n])
+        assert rel <= ROUTER_REL_L2, f"{n}: rel-L2 {rel:.3e}"

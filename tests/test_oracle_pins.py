@@ -480,6 +480,40 @@ def check_backward_finite_differences(o):
                 assert abs(num - ana) <= 1e-6 * (1 + abs(num)), (seed, gname, int(c), num, ana)
 
 
+def check_balance_loss_gradient(o):
+    """The balancing-loss term of the router gradient against central
+    differences of alpha * M * sum_i F_i P_i computed with ``balance_stats``
+    (F held at the unperturbed assignment)."""
+    rng = np.random.default_rng(80)
+    N, d, M, alpha = 30, 6, 4, 0.7
+    x = rng.normal(size=(N, d))
+    W = rng.normal(size=(M, d))
+    b = rng.normal(size=M)
+    q, k, v = (rng.normal(size=(N, 1, 4)) for _ in range(3))
+    zero = np.zeros((N, 1, 4))
+    g = o.moga_layer_backward(x, W, b, q, k, v, M, zero, balance_alpha=alpha)
+    F0, _, _ = o.balance_stats(x, W, b)
+
+    def loss(xx, WW, bb):
+        _, P, _ = o.balance_stats(xx, WW, bb)
+        return alpha * M * float(np.sum(F0 * P))
+
+    eps = 1e-6
+    for name, arr, gname in (("x", x, "dx"), ("W_r", W, "dW_r"), ("b_r", b, "db_r")):
+        flat = arr.reshape(-1)
+        for c in rng.choice(flat.size, size=min(flat.size, 10), replace=False):
+            pl, mi = flat.copy(), flat.copy()
+            pl[c] += eps
+            mi[c] -= eps
+            args_p = {"x": x, "W_r": W, "b_r": b}
+            args_m = dict(args_p)
+            args_p[name] = pl.reshape(arr.shape)
+            args_m[name] = mi.reshape(arr.shape)
+            num = (loss(args_p["x"], args_p["W_r"], args_p["b_r"]) - loss(args_m["x"], args_m["W_r"], args_m["b_r"])) / (2 * eps)
+            ana = g[gname].reshape(-1)[c]
+            assert abs(num - ana) <= 1e-7 * (1 + abs(num)), (gname, int(c), num, ana)
+
+
 def check_backward_dense_autograd(o):
     """The same gradients from torch autograd (float64) through a dense
     formulation: every branch as N x N attention with a membership mask."""
@@ -559,7 +593,7 @@ CHECKS = [check_route_closed_form, check_route_ties_and_M1, check_route_brute, c
           check_brute_force_tiny, check_permutation_equivariance, check_stga, check_layer_combine,
           check_golden, check_three_branch_mean, check_balance_stats, check_shot_stga,
           check_backward_finite_differences, check_backward_dense_autograd, check_backward_special_cases,
-          check_attention_lse, check_dq_rows]
+          check_attention_lse, check_dq_rows, check_balance_loss_gradient]
 
 
 @pytest.mark.parametrize("check", CHECKS, ids=[c.__name__ for c in CHECKS])
@@ -653,6 +687,15 @@ def _bwd_router_sign(*a, **kw):                     # gradient ascent on the rou
     return g
 
 
+def _bwd_balance_sign(*a, **kw):                   # the balancing term added with the wrong sign
+    alpha = kw.get("balance_alpha", 0.0)
+    if not alpha:
+        return _ORIG_LBWD(*a, **kw)
+    g0 = _ORIG_LBWD(*a, **dict(kw, balance_alpha=0.0))
+    g1 = _ORIG_LBWD(*a, **kw)
+    return {n: (2 * g0[n] - g1[n]) if n in ("dx", "dW_r", "db_r") else g1[n] for n in g1}
+
+
 def _lse_no_scale(q_rows, K):
     s = q_rows @ K.T
     m = s.max(axis=1)
@@ -682,6 +725,7 @@ MUTANTS = {
     "bwd_dk_untransposed": ("attention_rows_backward", _bwd_dk_untransposed),
     "bwd_router_sign_flipped": ("moga_layer_backward", _bwd_router_sign),
     "lse_without_scale": ("attention_lse", _lse_no_scale),
+    "balance_gradient_sign_flipped": ("moga_layer_backward", _bwd_balance_sign),
 }
 
 
