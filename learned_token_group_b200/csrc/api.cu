@@ -533,6 +533,19 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t o
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_window(CUtensorMap* map, const void* base, uint64_t d_h, uint64_t H, uint64_t Wg, uint64_t rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {d_h, H, Wg, rows};
+  cuuint64_t strides[3] = {d_h * 2, H * d_h * 2, Wg * H * d_h * 2};
+  cuuint32_t box[4] = {64, 1, 8, 8};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool make_tmap_tokens(CUtensorMap* map, const void* base, uint64_t d_h, uint64_t H, uint64_t N) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;

@@ -239,6 +239,7 @@ struct Plan {
 struct Unit {
   int h, start, len, q0;  // query segment; q0: first row of tile A in it (tile B starts at q0 + 128)
   int kvs, kvl;           // key/value segment (the query segment except for shot windows)
+  int seg;                // STGA windows: the window's index (else -1)
 };
 
 // kShots: the decoder of the in-place kernel, which also serves shot windows
@@ -270,6 +271,7 @@ struct Decoder {
       u.q0 = (local - u.h * npair) * 2 * kTile;
       u.kvs = u.start;
       u.kvl = u.len;
+      u.seg = -1;
     } else if (!kShots || mode == 1) {
       // Units in place go window by window with the heads innermost, so the
       // CTAs running at once read whole token rows of q, k, v (all heads)
@@ -289,6 +291,7 @@ struct Decoder {
       u.q0 = qp * 2 * kTile;
       u.kvs = u.start;
       u.kvl = u.len;
+      u.seg = seg;
     } else {
       // shot windows: binary search of the unit prefix in the global table
       const int nwin = gtab[0];
@@ -306,6 +309,7 @@ struct Decoder {
       u.kvl = e[3];
       u.h = local % heads;
       u.q0 = (local / heads) * 2 * kTile;
+      u.seg = -1;
     }
     return u;
   }
@@ -546,12 +550,50 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       fence_proxy_async_smem();
       __syncwarp();
     }
+    // STGA windows of 8x8 tokens whose frames lie inside the grid are loaded
+    // with 4-D TMA boxes instead: one box per frame and 64-column chunk is
+    // the frame's 64 rows in the window's token order, so frames 0-1 fill
+    // the 128-row tile and frame 2 the compact 64-row tile.  Clipped edge
+    // windows (and other window shapes) keep the row copies.  pend[] holds
+    // the phase of a barrier's last use when that use was a TMA load, for the
+    // drain at exit.
+    int pend[2] = {-1, -1};
+    auto tma_window = [&](const Unit& u, int& t0, int& h0, int& w0) -> bool {
+      if (!kSmall || a.mode != 1 || a.wh != 8 || a.ww != 8 || a.wt > 3 || u.seg < 0) return false;
+      const int nbh = (a.Hg + 7) / 8, nbw = (a.Wg + 7) / 8;
+      const int tb = u.seg / (nbh * nbw), hb = (u.seg / nbw) % nbh, wb = u.seg % nbw;
+      t0 = tb * a.wt;
+      h0 = hb * 8;
+      w0 = wb * 8;
+      return t0 + a.wt <= a.T && h0 + 8 <= a.Hg && w0 + 8 <= a.Wg;
+    };
+    constexpr uint32_t kBoxBytes = 64 * 128;  // one frame's 64 rows of one 64-column chunk
     for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
       const Unit u = dec(idx);
       if (u.q0 >= u.len) continue;
       const bool hb = u.q0 + kTile < u.len;
       const int nkv = (u.kvl + kTile - 1) / kTile;
       const int seg_end = u.start + u.len, kv_end = u.kvs + u.kvl;
+      int t0 = 0, h0 = 0, w0 = 0;
+      const bool twin = tma_window(u, t0, h0, w0);
+      if (li == 0 && twin) {
+        const int qb = (int)(ucnt & 1);
+        const uint32_t qph = ucnt >> 1;
+        if (!warp_wait(&q_empty[qb], (qph & 1) ^ 1, 1, ucnt)) { ok = false; break; }
+        if (lane == 0) {
+          mbar_expect_tx(&q_full[qb], (uint32_t)(a.wt * P::kChunks) * kBoxBytes);
+          for (int f = 0; f < a.wt; ++f)
+#pragma unroll
+            for (int c = 0; c < P::kChunks; ++c) {
+              uint8_t* dst = f < 2 ? smem + P::kSQA + qb * P::kTileBytes + c * P::kChunkFull + f * kBoxBytes
+                                   : smem + P::kSQB + qb * P::kHalfBytes + c * P::kChunkHalf;
+              tma_load_4d(&tq, &q_full[qb], dst, c * 64, u.h, w0, (t0 + f) * a.Hg + h0);
+            }
+        }
+        pend[qb] = (int)qph;
+        ++ucnt;
+        continue;
+      }
       if (li == 0) {
         int ra[4], rb[4];
         fetch_rows(a.perm, u.start + u.q0, seg_end, u.h, ra);
@@ -570,6 +612,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         }
         finish();
         if (lane == 0) mbar_arrive(&q_full[qb]);
+        if (kSmall) pend[qb] = -1;
         ++ucnt;
         continue;
       }
@@ -579,7 +622,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         // slot and phase: a ring of kStages tiles, or (small windows) tile j in slot j
         const int s = kSmall ? j : (int)(t % kStages);
         const uint32_t ph = kSmall ? (j ? sc1 : sc0) : t / kStages;
-        fetch_rows(kvperm, u.kvs + j * kTile, kv_end, u.h, tr);
+        if (!twin) fetch_rows(kvperm, u.kvs + j * kTile, kv_end, u.h, tr);
         if (!warp_wait(is_v ? &v_empty[s] : &k_empty[s], (ph & 1) ^ 1, is_v ? 3 : 2, t)) {
           ok = false;
           break;
@@ -587,6 +630,24 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         // Test hook: the first K tile never arrives, so the MMA warp's
         // bounded wait runs out and the kernel reports a timeout.
         if (!is_v && t == 0 && a.debug_withhold_first_k) { ok = false; break; }
+        if (kSmall && twin) {
+          // tile j holds frames [2j, min(2j + 2, wt))
+          const int f0 = 2 * j, f1 = min(a.wt, 2 * j + 2);
+          uint64_t* bar = is_v ? &v_full[s] : &k_full[s];
+          if (lane == 0) {
+            mbar_expect_tx(bar, (uint32_t)((f1 - f0) * P::kChunks) * kBoxBytes);
+            for (int f = f0; f < f1; ++f)
+#pragma unroll
+              for (int c = 0; c < P::kChunks; ++c) {
+                uint8_t* dst = j ? smem + (is_v ? P::kSV1 : P::kSK1) + c * P::kChunkHalf
+                                 : smem + (is_v ? P::kSV0 : P::kSK0) + c * P::kChunkFull + (f - f0) * kBoxBytes;
+                tma_load_4d(is_v ? &tv : &tk, bar, dst, c * 64, u.h, w0, (t0 + f) * a.Hg + h0);
+              }
+          }
+          pend[j] = (int)ph;
+          if (j) ++sc1; else ++sc0;
+          continue;
+        }
         uint8_t* dst;
         int chunk = P::kChunkFull;
         if constexpr (kSmall) {
@@ -603,9 +664,18 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         copy_tile(is_v ? a.v : a.k, dst, tr, toks, u.kvl - j * kTile, chunk);
         finish();
         if (lane == 0) mbar_arrive(is_v ? &v_full[s] : &k_full[s]);
+        if (kSmall) pend[j] = -1;
       }
     }
-    // Every copy was waited for before its arrive, so nothing is in flight.
+    // Row copies were waited for before their arrive; TMA loads still in
+    // flight (after an abort) are drained here, one barrier's last use each.
+    if (kSmall && lane == 0) {
+      volatile int zero = 0;
+      WaitCtx dc{&zero, nullptr, 100000000ull};
+      uint64_t* fb = li == 0 ? q_full : li == 1 ? k_full : v_full;
+      for (int b = 0; b < 2; ++b)
+        if (pend[b] >= 0) mbar_wait(&fb[b], (uint32_t)pend[b] & 1, dc);
+    }
   }
   if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -903,9 +973,16 @@ cudaError_t launch_attention_dh(const DevCtx& c, const AttnArgs& a) {
   // with 128-row boxes.  The in-place kernel copies rows itself and does not
   // read the maps.
   const uint32_t box_rows = (uint32_t)kTile;
+  const bool small_plan =
+      a.direct && a.mode == 1 && (int64_t)a.wt * a.wh * a.ww <= kTile + 64 && kSmallWindows;
   if (a.contiguous) {  // the caller's [N, H, d_h] tensors, read in place
     if (!make_tmap_tokens(&mq, a.q, DH, a.H, a.N) || !make_tmap_tokens(&mk, a.k, DH, a.H, a.N) ||
         !make_tmap_tokens(&mv, a.v, DH, a.H, a.N))
+      return cudaErrorInvalidValue;
+  } else if (small_plan) {  // 8x8 windows read in place by frame boxes
+    const uint64_t grid_rows = (uint64_t)a.T * a.Hg;
+    if (!make_tmap_window(&mq, a.q, DH, a.H, a.Wg, grid_rows) || !make_tmap_window(&mk, a.k, DH, a.H, a.Wg, grid_rows) ||
+        !make_tmap_window(&mv, a.v, DH, a.H, a.Wg, grid_rows))
       return cudaErrorInvalidValue;
   } else {
     if (!make_tmap_2d(&mq, a.q, DH, rows, DH * 2, box_rows)) return cudaErrorInvalidValue;
@@ -917,7 +994,7 @@ cudaError_t launch_attention_dh(const DevCtx& c, const AttnArgs& a) {
   const size_t smem = P::bytes(table_ints);
   // windows of at most 192 tokens fit the small-window plan (query tile B and
   // the second K/V tiles of at most 64 rows)
-  const bool small = a.direct && a.mode == 1 && (int64_t)a.wt * a.wh * a.ww <= kTile + 64 && kSmallWindows;
+  const bool small = small_plan;
   auto kern = a.direct ? (small ? attn_kernel<DH, true, true, true> : attn_kernel<DH, true, true, false>)
                        : (a.mode == 2 ? attn_kernel<DH, false, true, false> : attn_kernel<DH, false, false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
