@@ -28,7 +28,8 @@
 // TMEM, which the accumulating products read as their A operand.  TMEM
 // columns: S at [0, 128), dP at [128, 256), accumulators from 256 (dV then
 // dK, or dQ): one S/dP buffer, so a tile's softmax is not overlapped with the
-// next tile's S and dP.  With d_h = 128 two 128-wide buffers and the dK, dV
+// next tile's S and dP (S and dP are committed separately, so P is computed
+// while dP is still in flight).  With d_h = 128 two 128-wide buffers and the dK, dV
 // accumulators do not fit the 512 columns; 128-row Y tiles are still the
 // faster choice, because an M=128 MMA reads its whole A slice from shared
 // memory for every instruction, and N = 128 halves those bytes per
@@ -125,7 +126,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
   uint64_t* done_bar = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(done_bar + 2);
-  static_assert(2 + 2 * kYStages + 7 <= 32, "barrier area holds 32 words");
+  static_assert(2 + 2 * kYStages + 8 <= 32, "barrier area holds 32 words");
   int* tab = reinterpret_cast<int*>(smem + P::kTable);
   float* vec = reinterpret_cast<float*>(smem + P::kVec);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -483,7 +484,7 @@ cudaError_t launch_bwd_dh(const DevCtx& c, const BwdArgs& a) {
   using P = BPlan<DH>;
   CUtensorMap m1, m2, m3, m4;
   const uint64_t rows = (uint64_t)a.N * (uint64_t)a.H;
-  // X: 128-row boxes; Y: 64-row boxes (all [H][N][d_h] head-major copies)
+  // X and Y: 128-row boxes (all [H][N][d_h] head-major copies)
   const void* xs1 = kDQ ? a.q : a.k;
   const void* xs2 = kDQ ? a.dout : a.v;
   const void* ys1 = kDQ ? a.k : a.q;
