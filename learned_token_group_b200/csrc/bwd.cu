@@ -118,15 +118,15 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
   uint64_t* x_empty = bars + 1;
   uint64_t* y_full = bars + 2;                  // [kYStages]
   uint64_t* y_empty = y_full + kYStages;        // [kYStages]
-  uint64_t* s_full = y_empty + kYStages;        // S computed
-  uint64_t* d_full = s_full + 1;                // dP computed
+  uint64_t* s_full = y_empty + kYStages;        // [2]: S computed (buffer b; dK/dV use buffer 0)
+  uint64_t* d_full = s_full + 2;                // dP computed
   uint64_t* p_full = d_full + 1;                // P and dS written
   uint64_t* acc_full = p_full + 1;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* done_bar = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(done_bar + 2);
-  static_assert(2 + 2 * kYStages + 8 <= 32, "barrier area holds 32 words");
+  static_assert(2 + 2 * kYStages + 9 <= 32, "barrier area holds 32 words");
   int* tab = reinterpret_cast<int*>(smem + P::kTable);
   float* vec = reinterpret_cast<float*>(smem + P::kVec);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -138,7 +138,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
       mbar_init(&y_full[s], kDQ ? 1 : 2);  // dK/dV: the TMA bytes and the lse/D vectors
       mbar_init(&y_empty[s], 1);
     }
-    mbar_init(s_full, 1);
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
     mbar_init(d_full, 1);
     mbar_init(p_full, 256);
     mbar_init(acc_full, 1);
@@ -172,6 +173,9 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
   const uint32_t tD = tmem + 128u;                   // dP (then dS)
   const uint32_t tAccA = tmem + 256u;                // dV, or dQ
   const uint32_t tAccB = tmem + 256u + (uint32_t)DH; // dK
+  // dQ: the columns dK would use hold a second S buffer, so tile i+1's S is
+  // computed while the warpgroups finish tile i
+  auto tSb = [&](uint32_t yc_) { return (kDQ && (yc_ & 1u)) ? tmem + 384u : tS; };
   WaitCtx wc{abort_flag, status, wait_ns};
   const int64_t N = a.N;
 
@@ -254,17 +258,20 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
       bool ok = true;
       // S (or S^T) = X1 Y1^T and dP (or dP^T) = X2 Y2^T, both operands K-major.
       const uint64_t x1d = sdesc_sw128(x1, 16, 1024), x2d = sdesc_sw128(x2, 16, 1024);
-      // S first, with its own commit, so that the softmax warps compute P
-      // while the tensor core computes dP.
-      auto issue_s = [&](int s) {
-        const uint32_t y1 = smem_u32(smem + P::kY0 + s * P::kYStage);
-        const uint64_t y1d = sdesc_sw128(y1, 16, 1024), y2d = sdesc_sw128(y1 + P::kYBytes, 16, 1024);
+      // S and dP with their own commits, so that the softmax warps compute
+      // P while the tensor core computes dP.
+      auto issue_sonly = [&](int s, uint32_t ycs) {
+        const uint64_t y1d = sdesc_sw128(smem_u32(smem + P::kY0 + s * P::kYStage), 16, 1024);
+        const uint32_t ts = tSb(ycs);
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
           const uint32_t xo = (kk >> 2) * P::kXChunk + (kk & 3) * 32, yo = (kk >> 2) * P::kYChunk + (kk & 3) * 32;
-          umma_bf16(tS, sdesc_add(x1d, xo), sdesc_add(y1d, yo), idS, kk > 0 ? 1u : 0u);
+          umma_bf16(ts, sdesc_add(x1d, xo), sdesc_add(y1d, yo), idS, kk > 0 ? 1u : 0u);
         }
-        umma_commit(s_full);
+        umma_commit(&s_full[ycs & (kDQ ? 1u : 0u)]);
+      };
+      auto issue_dp = [&](int s) {
+        const uint64_t y2d = sdesc_sw128(smem_u32(smem + P::kY0 + s * P::kYStage) + P::kYBytes, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
           const uint32_t xo = (kk >> 2) * P::kXChunk + (kk & 3) * 32, yo = (kk >> 2) * P::kYChunk + (kk & 3) * 32;
@@ -309,14 +316,42 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
         if (u.x0 >= u.len) continue;
         const int ny = (u.len + kYRows - 1) / kYRows;
         if (!mbar_wait(x_full, uc & 1, wc, 3, uc)) break;
-        for (int i = 0; i < ny; ++i) {
-          const int s = (int)(yc % kYStages);
-          if (i > 0 && !finish_tile(yc - 1, i == 1, false)) { ok = false; break; }
-          if (!mbar_wait(&y_full[s], (yc / kYStages) & 1, wc, 4, yc)) { ok = false; break; }
+        if (kDQ) {
+          // Two S buffers: tile i's S was issued one tile ahead, so the order
+          // per tile is dQ(i-1), dP(i), S(i+1).  S(i+1) reuses the buffer of
+          // tile i-1, which the warpgroups released (P and dS written) before
+          // dQ(i-1) was issued.
+          const int s0 = (int)(yc % kYStages);
+          if (!mbar_wait(&y_full[s0], (yc / kYStages) & 1, wc, 4, yc)) break;
           tc_fence_after();
-          issue_s(s);
-          if (i + 1 == ny) umma_commit(x_empty);
-          ++yc;
+          issue_sonly(s0, yc);
+          for (int i = 0; i < ny; ++i) {
+            const int s = (int)(yc % kYStages);
+            if (i > 0 && !finish_tile(yc - 1, i == 1, false)) { ok = false; break; }
+            tc_fence_after();
+            issue_dp(s);
+            if (i + 1 == ny) {
+              umma_commit(x_empty);
+            } else {
+              const uint32_t y1 = yc + 1;
+              const int s1 = (int)(y1 % kYStages);
+              if (!mbar_wait(&y_full[s1], (y1 / kYStages) & 1, wc, 4, y1)) { ok = false; break; }
+              tc_fence_after();
+              issue_sonly(s1, y1);
+            }
+            ++yc;
+          }
+        } else {
+          for (int i = 0; i < ny; ++i) {
+            const int s = (int)(yc % kYStages);
+            if (i > 0 && !finish_tile(yc - 1, i == 1, false)) { ok = false; break; }
+            if (!mbar_wait(&y_full[s], (yc / kYStages) & 1, wc, 4, yc)) { ok = false; break; }
+            tc_fence_after();
+            issue_sonly(s, yc);
+            issue_dp(s);
+            if (i + 1 == ny) umma_commit(x_empty);
+            ++yc;
+          }
         }
         if (!ok || !finish_tile(yc - 1, ny == 1, true)) break;
         ++uc;
@@ -355,7 +390,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
       const int src = live ? (a.perm ? a.perm[u.start + r] : u.start + r) : 0;
       for (int i = 0; i < ny; ++i, ++yc) {
         const int s = (int)(yc % kYStages);
-        if (!mbar_wait(s_full, yc & 1, wc, 7 + wg, yc)) { ok = false; break; }
+        // dQ: S buffer yc & 1 (its phase advances every other tile); dK/dV: buffer 0
+        const bool ok_s = kDQ ? mbar_wait(&s_full[yc & 1], (yc >> 1) & 1, wc, 7 + wg, yc)
+                              : mbar_wait(&s_full[0], yc & 1, wc, 7 + wg, yc);
+        if (!ok_s) { ok = false; break; }
         tc_fence_after();
         // the vectors are plain shared-memory stores of the load warp: wait
         // on the stage's own barrier too (its phase is still this tile's,
@@ -368,8 +406,9 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
         float pv[64];
         {
           float sv[64];
-          tmem_ld32(tS + lb + 64 * wg, sv);
-          tmem_ld32(tS + lb + 64 * wg + 32, sv + 32);
+          const uint32_t ts = tSb(yc);
+          tmem_ld32(ts + lb + 64 * wg, sv);
+          tmem_ld32(ts + lb + 64 * wg + 32, sv + 32);
           tmem_ld_wait();
           if (kDQ) {
             const int valid = u.len - i * kYRows - 64 * wg;  // keys of these columns inside the segment
