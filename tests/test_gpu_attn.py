@@ -42,6 +42,10 @@ GROUP_CASES = [
     (1500, 3, 128, 1, None),                          # M = 1: full attention
     (700, 2, 128, 7, [0, 1, 127, 128, 129, 0, 315]),   # empty, singleton, tile edges
     (2600, 1, 128, 3, [2048, 1, 551]),                # many KV tiles + ragged tail
+    # segment ends around a unit of two 128-row query tiles: one row into the
+    # third tile, a unit and a half, one row past it, two full units, one row
+    # over, a single short tile
+    (2100, 2, 128, 6, [257, 384, 385, 512, 513, 49]),
 ]
 
 
