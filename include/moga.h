@@ -96,6 +96,8 @@ moga_status moga_route(const void* x, const void* W_r, const float* b_r, moga_dt
  * counts only valid tokens) and moga_sync_status() reports
  * MOGA_ERR_DEVICE_CHECK.  Used when routing happened elsewhere (e.g. on other
  * ranks of a sequence-parallel group).
+ * Limits: 1 <= M <= 1024 (the same group limit as moga_route) and
+ * 0 <= N < 2^31; anything else returns MOGA_ERR_INVALID_ARG before any launch.
  * Workspace: moga_sort_workspace_size(N, M) bytes. */
 size_t moga_sort_workspace_size(int64_t N, int M);
 moga_status moga_sort(const int32_t* group_id, int64_t N, int M, int32_t* perm, int32_t* offsets,

@@ -622,7 +622,9 @@ size_t moga_sort_workspace_size(int64_t N, int M) {
 
 moga_status moga_sort(const int32_t* group_id, int64_t N, int M, int32_t* perm, int32_t* offsets,
                       int32_t* max_seqlen, void* ws, size_t ws_bytes, void* stream) {
-  if (N < 0 || N >= ((int64_t)1 << 31) || M < 1 || M > 65536) return MOGA_ERR_INVALID_ARG;
+  // scan_kernel keeps one shared-memory slot per group in 1024-entry arrays
+  // and sums each group with one of its 1024 threads, so M is capped there.
+  if (N < 0 || N >= ((int64_t)1 << 31) || M < 1 || M > 1024) return MOGA_ERR_INVALID_ARG;
   if (!offsets || !max_seqlen || !aligned4(offsets) || !aligned4(max_seqlen)) return MOGA_ERR_INVALID_ARG;
   if (N > 0 && (!group_id || !perm || !aligned4(group_id) || !aligned4(perm))) return MOGA_ERR_INVALID_ARG;
   if (!ws || !aligned16(ws)) return MOGA_ERR_INVALID_ARG;

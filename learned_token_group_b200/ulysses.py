@@ -82,12 +82,15 @@ def ulysses_layer(x: torch.Tensor, W_r: torch.Tensor, b_r: Optional[torch.Tensor
     for the shard, equal to the single-device block's rows of these tokens.
 
     x [n, d], q/k/v [n, H, d_h] with n = N / P consecutive tokens and H a
-    multiple of P; grid (T, Hg, Wg) describes all N tokens.
+    multiple of P; grid (T, Hg, Wg) describes all N tokens.  1 <= M <= 1024,
+    the group limit of the library's routing and counting sort.
     """
     world = dist.get_world_size(group)
     n, H, _ = q.shape
     if H % world:
         raise ValueError(f"{H} heads do not split over {world} ranks")
+    if not 1 <= M <= 1024:
+        raise ValueError(f"M = {M} groups: routing and sorting take 1 to 1024")
     ops = ops or CudaOps
     gid_local, gate_local = ops.route(x, W_r, b_r, M)
     gid = all_gather_1d(gid_local, world, group)

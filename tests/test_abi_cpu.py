@@ -68,6 +68,19 @@ def test_route_validation(lib):
     assert _route(lib, wsb=16) == WORKSPACE
 
 
+def test_sort_validation(lib):
+    """moga_sort's scan keeps one shared-memory slot per group in 1024-entry
+    arrays, so group counts above 1024 are refused before any launch."""
+    f = lib.moga_sort
+    assert f(P, 1000, 1025, P, P, P, P, BIG, None) == INVALID
+    assert f(P, 1000, 2000, P, P, P, P, BIG, None) == INVALID
+    assert f(P, 1000, 65536, P, P, P, P, BIG, None) == INVALID
+    assert f(P, 1000, 0, P, P, P, P, BIG, None) == INVALID
+    assert f(P, -1, 4, P, P, P, P, BIG, None) == INVALID
+    assert f(None, 1000, 4, P, P, P, P, BIG, None) == INVALID
+    assert f(P, 1000, 4, P, P, P, P, 16, None) == WORKSPACE
+
+
 def _ga(lib, q=P, perm=P, N=1000, H=2, d_h=128, M=4, ws=P, wsb=BIG):
     return lib.moga_group_attn(q, q, q, perm, perm, None, N, H, d_h, M, 1.0, q, ws, wsb, None)
 
