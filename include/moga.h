@@ -131,16 +131,24 @@ moga_status moga_route_ex(const void* x, const void* W_r, const float* b_r, moga
  * - It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  * - The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture on the device.
+ *   before any stream capture on the device.  The address is kept per device
+ *   and context, so a call after a device reset looks it up again.
  * - Every call shares the one array and it keeps the last call's contents;
  *   the call clears what must start at zero.  Calls that overlap on the GPU
  *   (different streams, or different host threads, on one device) race on
  *   the array: order them on one stream.
- * - Device-side wait timeouts of this call are not reported (there is no
- *   workspace status word to read back). */
+ * - Device-side conditions (a bounded wait that ran out, ids out of range)
+ *   go to a status word at the head of the array; read them with
+ *   moga_route_noalloc_status. */
 moga_status moga_route_noalloc(const void* x, const void* W_r, const float* b_r, moga_dtype dt, int64_t N, int d,
                                int M, int32_t* group_id, float* gate, int32_t* perm, int32_t* offsets,
                                int32_t* max_seqlen, void* stream);
+
+/* moga_route_noalloc_status: synchronises the stream, then reads and clears
+ * the device status word of moga_route_noalloc's scratch on the current
+ * device (MOGA_OK, MOGA_ERR_TIMEOUT or MOGA_ERR_DEVICE_CHECK, as
+ * moga_sync_status does for a workspace).  Allocates nothing. */
+moga_status moga_route_noalloc_status(void* stream);
 
 /* ---------------------------------------------------------------- grouped attention
  * moga_group_attn: Algorithm 1 steps 2 (gather Q/K/V into group order), 3

@@ -71,6 +71,7 @@ def get_lib():
                                _P, _P, _P, _P, _P, _P, _SZ, _P]),
         "moga_kernel_launches": (ctypes.c_uint64, []),
         "moga_route_noalloc": (_I, [_P, _P, _P, _I, _I64, _I, _I, _P, _P, _P, _P, _P, _P]),
+        "moga_route_noalloc_status": (_I, [_P]),
         "moga_set_timing_events": (_I, [_I, _P, _P]),
         "moga_debug_inject": (_I, [_I]),
         "stga_shot_attn_workspace_size": (_SZ, [_I, _I, _I, _P, _I, _I, _I, _I, _I]),

@@ -66,17 +66,43 @@ constexpr int64_t kNoAllocCells = (int64_t)1 << 18;  // max ceil(N/128) * M
 constexpr size_t kNoAllocBytes = 256 + 2 * (size_t)kNoAllocCells * 4;
 static __device__ __align__(256) uint8_t g_route_scratch[kNoAllocBytes];
 
+// The driver's cuCtxGetCurrent, resolved at run time like the tensor-map encoder.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
 // Device address of g_route_scratch for the current device, looked up once per
-// device (the first call on a device does it; see moga.h).
+// device and context (the first call on a device does it; see moga.h).  The
+// context is part of the key: after a device reset the runtime loads the
+// module again in a new context, where the array may sit elsewhere.
 uint8_t* noalloc_scratch(int dev) {
   static std::mutex mu;
   static uint8_t* addr[64] = {};
+  static CUcontext ctx_of[64] = {};
   if (dev < 0 || dev >= 64) return nullptr;
+  const CtxGetCurrentFn get = ctx_get_current();
+  if (!get) return nullptr;
+  // null while this thread has no current context yet; the lookup below then
+  // makes the device's primary context current
+  CUcontext ctx = nullptr;
+  if (get(&ctx) != CUDA_SUCCESS) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  if (!addr[dev] || !ctx || ctx_of[dev] != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    if (get(&ctx) != CUDA_SUCCESS) return nullptr;
     addr[dev] = static_cast<uint8_t*>(p);
+    ctx_of[dev] = ctx;
   }
   return addr[dev];
 }
@@ -1049,6 +1075,14 @@ moga_status moga_layer_ex(const void* x, const void* W_r, const float* b_r, moga
   if ((branches & 2) && (st = stga_body(c, q, k, v, T, Hg, Wg, frame_window, H, d_h, 1, out, w, scale)) != MOGA_OK)
     return st;
   return MOGA_OK;
+}
+
+moga_status moga_route_noalloc_status(void* stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOGA_ERR_CUDA;
+  uint8_t* scratch = noalloc_scratch(dev);
+  if (!scratch) return MOGA_ERR_CUDA;
+  return moga_sync_status(scratch, stream);
 }
 
 moga_status moga_sync_status(void* ws, void* stream) {

@@ -85,3 +85,39 @@ def groups_to_perm(gid, M):
     perm = np.argsort(gid, kind="stable").astype(np.int32)
     offsets = np.concatenate([[0], np.cumsum(np.bincount(gid, minlength=M))]).astype(np.int32)
     return perm, offsets
+
+
+def sample_rows(gid, M, grid, window, rng, per_group=256, stga_rows=1024):
+    """Seeded row sample for full-size parity checks.
+
+    Every row of the two smallest non-empty groups, ``per_group`` random rows
+    of every other group (all of them when the group is smaller), and, with a
+    window, ``stga_rows`` tokens spread evenly over the window kinds the grid
+    has: whole windows, and windows clipped in rows, in columns, in both, and
+    (when T is not a multiple of the temporal extent) in time.  Each sampled
+    row is later compared in full: its whole group / window is attended.
+    """
+    gid = np.asarray(gid)
+    rows = []
+    counts = np.bincount(gid, minlength=M)
+    nonempty = [int(m) for m in np.argsort(counts, kind="stable") if counts[m] > 0]
+    for m in nonempty[:2]:
+        rows.append(np.nonzero(gid == m)[0])
+    for m in nonempty[2:]:
+        idx = np.nonzero(gid == m)[0]
+        rows.append(rng.choice(idx, size=min(per_group, idx.size), replace=False))
+    if window is not None and stga_rows:
+        T, Hg, Wg = grid
+        wt, wh, ww = window
+        tok = np.arange(T * Hg * Wg)
+        t, h, w = tok // (Hg * Wg), (tok // Wg) % Hg, tok % Wg
+        ct = (t // wt) * wt + wt > T
+        ch = (h // wh) * wh + wh > Hg
+        cw = (w // ww) * ww + ww > Wg
+        kind = ct.astype(np.int64) * 4 + ch * 2 + cw
+        kinds = np.unique(kind)
+        per = max(1, stga_rows // kinds.size)
+        for kd in kinds:
+            idx = np.nonzero(kind == kd)[0]
+            rows.append(rng.choice(idx, size=min(per, idx.size), replace=False))
+    return np.unique(np.concatenate(rows))

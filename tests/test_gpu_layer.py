@@ -6,7 +6,9 @@ Algorithm 1), STGA, and the mean of the two branches.
 
 Small workloads are compared on every output row.  At full size the oracle
 computes a seeded sample of rows exactly (each sampled row still sees its whole
-group / window), in the launch configuration the benchmark times.
+group / window), in the launch configuration the benchmark times: every row of
+the two smallest non-empty groups, 256 rows of every other group and 1,024
+STGA rows spread over whole and clipped windows, on all heads.
 """
 import numpy as np
 import pytest
@@ -14,7 +16,7 @@ import torch
 
 import learned_token_group_b200 as moga
 import oracle
-from parity import GATE_TOL_BF16, GATE_TOL_F32, check_route, compare_out, np_cpu
+from parity import GATE_TOL_BF16, GATE_TOL_F32, check_route, compare_out, np_cpu, sample_rows
 from workloads import WORKLOADS, custom, make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -26,25 +28,6 @@ def _layer(wl, seed):
                           wl.window)
     moga.sync_status(res["ws"])
     return inp, res
-
-
-def _sample_rows(gid, M, grid, window, rng, per_group=48):
-    rows = []
-    counts = np.bincount(gid, minlength=M)
-    nonempty = [m for m in np.argsort(counts) if counts[m] > 0]
-    for m in nonempty[:2]:                      # the two smallest groups in full (if small)
-        idx = np.nonzero(gid == m)[0]
-        rows.append(idx[:256])
-    for m in nonempty:
-        idx = np.nonzero(gid == m)[0]
-        rows.append(rng.choice(idx, size=min(per_group, idx.size), replace=False))
-    if window is not None:                      # tokens of edge (clipped) windows
-        T, Hg, Wg = grid
-        t = rng.integers(0, T, size=64)
-        h = np.where(rng.random(64) < 0.5, Hg - 1, rng.integers(0, Hg, size=64))
-        w = np.where(rng.random(64) < 0.5, Wg - 1, rng.integers(0, Wg, size=64))
-        rows.append((t * Hg + h) * Wg + w)
-    return np.unique(np.concatenate(rows))
 
 
 SMALL = [
@@ -76,8 +59,11 @@ def test_layer_workload(name):
     inp, res = _layer(wl, seed=0)
     gid, info = check_route(res, inp["x"], inp["W_r"], inp["b_r"], wl.M, GATE_TOL_BF16)
     rng = np.random.default_rng(123)
-    rows = _sample_rows(gid, wl.M, wl.grid, wl.window, rng, per_group=48 if wl.N < 500000 else 16)
-    heads = [0, wl.H - 1] if wl.H <= 12 else [0, wl.H // 2, wl.H - 1]
+    # every row of the two smallest groups, 256 rows of every other group and
+    # 1,024 STGA rows over all window kinds (whole and clipped), on every head
+    # (at 580k the oracle needs about 3 s of host time per head)
+    rows = sample_rows(gid, wl.M, wl.grid, wl.window, rng, per_group=256, stga_rows=1024)
+    heads = list(range(wl.H))
     gate = np_cpu(res["gate"]).astype(np.float64)
     # the oracle reads only the rows/heads it needs, straight from the seeded inputs
     q, k, v = inp["q"], inp["k"], inp["v"]
@@ -134,7 +120,7 @@ def test_layer_three_branches_wan_sampled():
                           wl.window, per_frame=True)
     moga.sync_status(res["ws"])
     gid, _ = check_route(res, inp["x"], inp["W_r"], inp["b_r"], wl.M, GATE_TOL_BF16)
-    rows = _sample_rows(gid, wl.M, wl.grid, wl.window, np.random.default_rng(5), per_group=24)
+    rows = sample_rows(gid, wl.M, wl.grid, wl.window, np.random.default_rng(5), per_group=64, stga_rows=256)
     heads = [0, wl.H - 1]
     gate = np_cpu(res["gate"]).astype(np.float64)
     q, k, v = inp["q"], inp["k"], inp["v"]

@@ -3,9 +3,11 @@ sequence-parallel block on one GPU.
 
 moga_sort must reproduce the oracle's stable counting sort bit for bit and
 report ids outside [0, M).  The sequence-parallel path (ulysses_layer) with a
-single rank over NCCL exchanges nothing, so it must equal moga_layer bit for
-bit: same routing, same sort, same kernels in the same order.  Its two-rank
-exchange is checked on the CPU (tests/test_multirank_cpu.py).
+single rank over NCCL exchanges nothing: its routing and output are compared
+with the oracle (group ids with the near-tie rule, gate, and per group the
+block output), and it must also equal moga_layer bit for bit (same routing,
+same sort, same kernels in the same order).  Its two-rank exchange is checked
+on the CPU (tests/test_multirank_cpu.py).
 """
 import datetime
 import os
@@ -18,7 +20,7 @@ import torch.distributed as dist
 
 import learned_token_group_b200 as moga
 import oracle
-from parity import np_cpu
+from parity import GATE_TOL_BF16, MARGIN, compare_out, np_cpu
 from workloads import custom, make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -72,5 +74,17 @@ def test_sequence_parallel_single_rank_equals_layer(window):
     ref = moga.moga_layer(inp["x"], inp["W_r"], inp["b_r"], inp["q"], inp["k"], inp["v"], wl.M,
                           grid if window else None, window)
     moga.sync_status(ref["ws"])
+    # against the oracle
+    ref_gid, ref_gate, margin = oracle.route(np_cpu(inp["x"]), np_cpu(inp["W_r"]), None)
+    g = np_cpu(gid).astype(np.int64)
+    assert not ((g != ref_gid) & (margin >= MARGIN)).any()
+    same = g == ref_gid
+    assert np.abs(np_cpu(gate)[same] - ref_gate[same]).max() <= GATE_TOL_BF16
+    q, k, v = (np_cpu(inp[n]) for n in "qkv")
+    want = oracle.group_attention(q, k, v, g, np_cpu(gate).astype(np.float64), wl.M)
+    if window:
+        want = 0.5 * (want + oracle.stga_attention(q, k, v, *grid, window))
+    compare_out(out, want, groups=g)
+    # and bit for bit against the single-device block
     assert torch.equal(gid, ref["group_id"]) and torch.equal(gate, ref["gate"])
     assert torch.equal(out, ref["out"])

@@ -4,8 +4,11 @@ Some callers cannot call cudaMalloc themselves (their framework's allocator
 owns the GPU, or they replay a fixed launch sequence).  moga_route_noalloc
 gives them the router and counting sort with the library's own fixed device
 scratch instead of a caller workspace.  This test calls it through the C ABI
-and checks it against moga_route on consecutive calls of different sizes, so
-that contents left behind by one call cannot leak into the next.  It lives in
+and checks it on consecutive calls of different sizes, so that contents left
+behind by one call cannot leak into the next: against the oracle (group ids
+with the near-tie rule, gate, and perm/offsets bit-exact against the oracle's
+counting sort), against moga_route, and through moga_route_noalloc_status,
+which must report no device-side condition.  It lives in
 its own file, collected last, and passes alone or after the other tests.
 """
 import ctypes
@@ -15,7 +18,7 @@ import pytest
 import torch
 
 import learned_token_group_b200 as moga
-from parity import GATE_TOL_BF16, GATE_TOL_F32, np_cpu
+from parity import GATE_TOL_BF16, GATE_TOL_F32, check_route, np_cpu
 from workloads import WORKLOADS, custom, make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -58,10 +61,12 @@ def test_noalloc_matches_route_on_consecutive_calls():
         inp = make_inputs(wl, seed=seed, device="cuda", with_qkv=False)
         ref = moga.route(inp["x"], inp["W_r"], inp["b_r"], wl.M)
         got = _noalloc(inp, wl.M)
-        torch.cuda.synchronize()
+        stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        assert moga.get_lib().moga_route_noalloc_status(stream) == 0
+        tol = GATE_TOL_F32 if wl.x_dtype == "f32" else GATE_TOL_BF16
+        check_route(got, inp["x"], inp["W_r"], inp["b_r"], wl.M, tol)
         for key in ("group_id", "perm", "offsets", "max_seqlen"):
             assert np.array_equal(np_cpu(got[key]), np_cpu(ref[key])), f"{wl.name}: {key} differs"
-        tol = GATE_TOL_F32 if wl.x_dtype == "f32" else GATE_TOL_BF16
         assert np.abs(np_cpu(got["gate"]) - np_cpu(ref["gate"])).max() <= tol
 
 
