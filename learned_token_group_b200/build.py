@@ -15,7 +15,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["api.cu", "route.cu", "attn.cu", "shot.cu", "pipe.cu", "bwd.cu"]
+SOURCES = ["api.cu", "route.cu", "attn.cu", "stga.cu", "shot.cu", "pipe.cu", "bwd.cu"]
 HEADERS = ["ptx.cuh", "internal.h", "windows.cuh"]
 LIB = os.path.join(HERE, "libmoga.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

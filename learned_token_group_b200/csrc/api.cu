@@ -18,6 +18,12 @@ namespace {
 std::atomic<uint64_t> g_wait_ns{4000000000ull};
 std::atomic<uint64_t> g_launches{0};
 std::atomic<int> g_debug_inject{0};
+// 1: STGA windows of at most 192 tokens run stga_kernel (whole-window TMA
+// boxes); 0: the in-place rows of attn_kernel.
+#ifndef MOGA_STGA_BOX
+#define MOGA_STGA_BOX 1
+#endif
+constexpr bool kStgaBox = MOGA_STGA_BOX != 0;
 constexpr int kNumStages = 6;
 std::atomic<void*> g_ev_begin[kNumStages];
 std::atomic<void*> g_ev_end[kNumStages];
@@ -274,8 +280,12 @@ moga_status stga_body(const DevCtx& c, const void* q, const void* k, const void*
   const bool contiguous = !direct && window[1] >= Hg && window[2] >= Wg;
   const AttnWs w = attn_ws(N, H, d_h, 0, true, !direct);
   int32_t* permw = reinterpret_cast<int32_t*>(ws + w.permw);
+  // Small windows are loaded as whole TMA boxes (stga.cu) and need no
+  // permutation, except for the training forward, whose log-sum-exp rows
+  // (and the backward pass after it) follow the window order.
+  const bool box = kStgaBox && stga_box_supported(d_h, window);
   mark(MOGA_STAGE_STGA_PREP, true, c.stream);
-  if (!contiguous) {
+  if (!contiguous && (!box || lse)) {
     if (launch_window_perm(c, T, Hg, Wg, window, permw) != cudaSuccess) return MOGA_ERR_CUDA;
     count(1);
   }
@@ -315,7 +325,17 @@ moga_status stga_body(const DevCtx& c, const void* q, const void* k, const void*
   a.lse = lse;
   a.debug_withhold_first_k = g_debug_inject.load(std::memory_order_relaxed) == 1;
   mark(MOGA_STAGE_STGA_ATTN, true, c.stream);
-  const cudaError_t e = launch_attention(c, a);
+  bool handled = false;
+  cudaError_t e = box ? launch_stga_box(c, a, &handled) : cudaSuccess;
+  if (e == cudaSuccess && !handled) {
+    if (box && !lse && !contiguous) {
+      // the box kernel declined (tensor map not encodable): the general
+      // kernel reads rows by the window permutation
+      if (launch_window_perm(c, T, Hg, Wg, window, permw) != cudaSuccess) return MOGA_ERR_CUDA;
+      count(1);
+    }
+    e = launch_attention(c, a);
+  }
   mark(MOGA_STAGE_STGA_ATTN, false, c.stream);
   count(1);
   return from_cuda(e);
@@ -567,6 +587,22 @@ bool make_tmap_window(CUtensorMap* map, const void* base, uint64_t d_h, uint64_t
   cuuint32_t box[4] = {64, 1, 8, 8};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_box5(CUtensorMap* map, const void* base, uint64_t d_h, uint64_t H, uint64_t Wg, uint64_t Hg,
+                    uint64_t T, const int* window) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[5] = {d_h, H, Wg, Hg, T};
+  cuuint64_t strides[4] = {d_h * 2, H * d_h * 2, Wg * H * d_h * 2, Hg * Wg * H * d_h * 2};
+  cuuint32_t box[5] = {64, 1, (cuuint32_t)window[2], (cuuint32_t)window[1], (cuuint32_t)window[0]};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  for (int i = 2; i < 5; ++i)
+    if (box[i] < 1 || box[i] > 256) return false;
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;

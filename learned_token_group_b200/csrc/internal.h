@@ -99,6 +99,11 @@ struct AttnArgs {
   float* lse;
 };
 cudaError_t launch_attention(const DevCtx& c, const AttnArgs& a);
+// STGA windows of at most 192 tokens (d_h 64 or 128), every window loaded as
+// one 5-D TMA box per 64-column chunk (stga.cu).  *handled = false when the
+// arguments do not fit it (the caller then runs launch_attention).
+bool stga_box_supported(int d_h, const int* window);
+cudaError_t launch_stga_box(const DevCtx& c, const AttnArgs& a, bool* handled);
 
 // ------------------------------------------------------------------ training (bwd.cu)
 // Attention backward over groups (mode 0) or STGA windows (mode 1).  q, k, v
@@ -187,5 +192,12 @@ bool make_tmap_tokens(CUtensorMap* map, const void* base, uint64_t d_h, uint64_t
 // grid row x 8 grid rows and 128-byte swizzle: one box is the 64 rows (grid
 // row-major) of one frame of an 8x8 STGA window, for one head.
 bool make_tmap_window(CUtensorMap* map, const void* base, uint64_t d_h, uint64_t H, uint64_t Wg, uint64_t rows);
+// Encodes a 5-D bf16 tensor map over the (d_h, H, Wg, Hg, T) view of a
+// [T*Hg*Wg, H, d_h] tensor with a box of 64 columns x 1 head x window[2] x
+// window[1] x window[0] and 128-byte swizzle: one box is one STGA window of
+// one head in the window's own (frame, row, column) order, with zeros where
+// it leaves the grid.
+bool make_tmap_box5(CUtensorMap* map, const void* base, uint64_t d_h, uint64_t H, uint64_t Wg, uint64_t Hg,
+                    uint64_t T, const int* window);
 
 }  // namespace moga

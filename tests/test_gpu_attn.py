@@ -112,6 +112,15 @@ STGA_CASES = [
     ((2, 30, 52), (1, 30, 52), 2, 128),  # per-frame attention, 1560 tokens (ragged tail)
     ((5, 30, 52), (2, 30, 52), 1, 64),   # two frames per window, last window clipped
     ((3, 7, 9), (2, 20, 20), 2, 64),     # wider than the frame, shorter than the clip
+    # windows of up to 192 tokens loaded as whole boxes: every clip kind, box
+    # sizes that use one or two query tiles, a second tile with one live warp
+    ((5, 10, 12), (3, 8, 8), 3, 128),    # T not a multiple of wt: clipped in time too
+    ((4, 30, 52), (3, 8, 8), 1, 64),     # d_h 64 on the 480p grid
+    ((2, 9, 20), (2, 4, 8), 2, 128),     # 64-token boxes
+    ((3, 16, 40), (1, 8, 16), 2, 128),   # 128-token boxes: one query tile
+    ((3, 13, 23), (3, 6, 10), 2, 128),   # 180-token boxes, clipped in rows and columns
+    ((2, 25, 25), (1, 12, 12), 2, 128),  # 144 tokens: the second tile's last warp holds no row
+    ((3, 5, 6), (3, 8, 8), 2, 128),      # box larger than the grid in rows and columns
 ]
 
 
