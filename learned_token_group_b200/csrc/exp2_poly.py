@@ -5,7 +5,7 @@ instead of the MUFU unit: t = n + f with n = round(t) and f in [-1/2, 1/2]
 (Cody-Waite style range reduction with one rounding step), 2^t = 2^n * p(f),
 where p is a degree-3 polynomial fitted to 2^f in the minimax sense for
 RELATIVE error by Lawson's iteratively re-weighted least squares on Chebyshev
-points.  Run this file to reproduce the constants in attn.cu.
+points.  Run this file to reproduce the constants in ptx.cuh (exp2_poly_x2).
 """
 import numpy as np
 
