@@ -833,50 +833,16 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             if (c >= valid) sr[c] = -INFINITY;
         }
         // row max as a tree: 8 independent chains of 3-input maxima
-        auto row_max = [&]() {
-          float m8[8];
+        float m8[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float m = fmax3(sr[16 * i], sr[16 * i + 1], sr[16 * i + 2]);
+        for (int i = 0; i < 8; ++i) {
+          float m = fmax3(sr[16 * i], sr[16 * i + 1], sr[16 * i + 2]);
 #pragma unroll
-            for (int k = 3; k + 1 < 16; k += 2) m = fmax3(m, sr[16 * i + k], sr[16 * i + k + 1]);
-            m8[i] = fmaxf(m, sr[16 * i + 15]);
-          }
-          return fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
-        };
-        // P = 2^(S*scale - m) for the whole row, summed into four packed
-        // partial sums and written back over S as packed bf16 (two keys per
-        // TMEM column); pairs of keys go through the packed fp32x2 FMA/ADD
-        // units.  Masked keys are -inf, so their P is 0.
-        const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
-        auto exp_row = [&](uint64_t nm2, uint64_t& s0, uint64_t& s1, uint64_t& s2, uint64_t& s3) {
-#pragma unroll
-          for (int c = 0; c < kTile / 32; ++c) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const uint64_t t2 = f2_fma(f2_pack(sr[c * 32 + 2 * e], sr[c * 32 + 2 * e + 1]), sc2, nm2);
-              float p0, p1;
-              if (kExp2PolyEvery > 0 && e % (kExp2PolyEvery > 0 ? kExp2PolyEvery : 1) == kExp2PolyEvery - 1) {
-                f2_unpack(exp2_poly_x2(t2), p0, p1);
-              } else {
-                float t0, t1;
-                f2_unpack(t2, t0, t1);
-                p0 = fast_exp2(t0);
-                p1 = fast_exp2(t1);
-              }
-              const uint64_t pp = f2_pack(p0, p1);
-              switch (e & 3) {
-                case 0: s0 = f2_add(s0, pp); break;
-                case 1: s1 = f2_add(s1, pp); break;
-                case 2: s2 = f2_add(s2, pp); break;
-                default: s3 = f2_add(s3, pp); break;
-              }
-              pk[e] = pack_bf16x2(p0, p1);
-            }
-            tmem_st16u(tSx + c * 16, pk);
-          }
-        };
+          for (int k = 3; k + 1 < 16; k += 2) m = fmax3(m, sr[16 * i + k], sr[16 * i + k + 1]);
+          m8[i] = fmaxf(m, sr[16 * i + 15]);
+        }
+        const float mx = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
+        const float m_new = fmaxf(m_run, mx * scale_log2);
         // O_x was last written by the previous P V product, which completed
         // before this S (the MMA thread issued it first).  The running max is
         // moved (and O rescaled) only when it grows by more than 2^8; P and l
@@ -884,51 +850,50 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         float alpha = 1.0f;
         bool rescale = false;
         if (j == 0) {
-          m_run = row_max() * scale_log2;
-          exp_row(f2_pack(-m_run, -m_run), la, lb, lc, ld);
+          m_run = m_new;
         } else {
-          // Later key tiles: the exponentials start at once with the running
-          // max, and the row max is taken beside them (it only checks that
-          // max afterwards), so it is off the chain from S to P.  A row
-          // whose max grew by more than 2^8 (rare once a few tiles are in)
-          // moves its running max by a whole number of octaves, scales l and
-          // O by that exact power of two, and the warp computes P again: keys
-          // 0-63 from registers, keys 64-127 read again from TMEM, where P
-          // (columns 0-63) has not overwritten them.  Without such a move the
-          // arithmetic is that of taking the max first.
-          const uint64_t z2 = f2_pack(0.f, 0.f);
-          uint64_t ta = z2, tb = z2, tc = z2, td = z2;  // this tile's sum of P
-          exp_row(f2_pack(-m_run, -m_run), ta, tb, tc, td);
-          const float m_new = row_max() * scale_log2;
           const bool need = m_new > m_run + 8.0f;
           rescale = __any_sync(0xffffffffu, need);
-          if (rescale) {
-            if (need) {
-              const int up = (int)ceilf(m_new - m_run);  // whole octaves, >= 9
-              alpha = up > 126 ? 0.0f : __int_as_float((127 - up) << 23);
-              const uint64_t a2 = f2_pack(alpha, alpha);
-              la = f2_mul(la, a2);
-              lb = f2_mul(lb, a2);
-              lc = f2_mul(lc, a2);
-              ld = f2_mul(ld, a2);
-              m_run += (float)up;
-            }
-            tmem_st_wait();  // the first P lands before it is overwritten
-            tmem_ld32(tSx + 64, sr + 64);
-            tmem_ld32(tSx + 96, sr + 96);
-            tmem_ld_wait();
-            if (valid < kTile) {
-#pragma unroll
-              for (int c = 64; c < kTile; ++c)
-                if (c >= valid) sr[c] = -INFINITY;
-            }
-            ta = tb = tc = td = z2;
-            exp_row(f2_pack(-m_run, -m_run), ta, tb, tc, td);
+          if (need) {
+            alpha = fast_exp2(m_run - m_new);
+            const uint64_t a2 = f2_pack(alpha, alpha);
+            la = f2_mul(la, a2);
+            lb = f2_mul(lb, a2);
+            lc = f2_mul(lc, a2);
+            ld = f2_mul(ld, a2);
+            m_run = m_new;
           }
-          la = f2_add(la, ta);
-          lb = f2_add(lb, tb);
-          lc = f2_add(lc, tc);
-          ld = f2_add(ld, td);
+        }
+        // P = 2^(S*scale - m), summed into l and written back over S as packed
+        // bf16 (two keys per TMEM column); pairs of keys go through the packed
+        // fp32x2 FMA/ADD units.  Masked keys are -inf, so their P is 0.
+        const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
+        const uint64_t nm2 = f2_pack(-m_run, -m_run);
+#pragma unroll
+        for (int c = 0; c < kTile / 32; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const uint64_t t2 = f2_fma(f2_pack(sr[c * 32 + 2 * e], sr[c * 32 + 2 * e + 1]), sc2, nm2);
+            float p0, p1;
+            if (kExp2PolyEvery > 0 && e % (kExp2PolyEvery > 0 ? kExp2PolyEvery : 1) == kExp2PolyEvery - 1) {
+              f2_unpack(exp2_poly_x2(t2), p0, p1);
+            } else {
+              float t0, t1;
+              f2_unpack(t2, t0, t1);
+              p0 = fast_exp2(t0);
+              p1 = fast_exp2(t1);
+            }
+            const uint64_t pp = f2_pack(p0, p1);
+            switch (e & 3) {
+              case 0: la = f2_add(la, pp); break;
+              case 1: lb = f2_add(lb, pp); break;
+              case 2: lc = f2_add(lc, pp); break;
+              default: ld = f2_add(ld, pp); break;
+            }
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16u(tSx + c * 16, pk);
         }
         if (rescale) {
 #pragma unroll
