@@ -414,13 +414,17 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       // One 128-row tile of head h starting at segment position pos: a row of
       // the gathered head-major copy (rows = rows per head), or, for
       // contiguous segments, 128 consecutive tokens read in place.
-      auto load_tile = [&](const CUtensorMap* map, uint64_t* bar, uint8_t* dst, int h, int64_t rows, int pos) {
+      // K/V tiles are read again by every query pair of their (group, head):
+      // keep them in L2; query tiles are read once
+      const uint64_t pol_keep = l2_policy_evict_last(), pol_once = l2_policy_evict_first();
+      auto load_tile = [&](const CUtensorMap* map, uint64_t* bar, uint8_t* dst, int h, int64_t rows, int pos,
+                           uint64_t pol) {
 #pragma unroll
         for (int c = 0; c < P::kChunks; ++c) {
           if (a.contiguous)
             tma_load_3d(map, bar, dst + c * 16384, c * 64, h, pos);
           else
-            tma_load_2d(map, bar, dst + c * 16384, c * 64, (int)((int64_t)h * rows + pos));
+            tma_load_2d_hint(map, bar, dst + c * 16384, c * 64, (int)((int64_t)h * rows + pos), pol);
         }
       };
       for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
@@ -430,8 +434,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         const int nkv = (u.kvl + kTile - 1) / kTile;
         if (!mbar_wait(q_empty, (ucnt & 1) ^ 1, wc, 1, ucnt)) break;
         mbar_expect_tx(q_full, (hb ? 2 : 1) * P::kTileBytes);
-        load_tile(&tq, q_full, smem + P::kQA, u.h, N, u.start + u.q0);
-        if (hb) load_tile(&tq, q_full, smem + P::kQB, u.h, N, u.start + u.q0 + kTile);
+        load_tile(&tq, q_full, smem + P::kQA, u.h, N, u.start + u.q0, pol_once);
+        if (hb) load_tile(&tq, q_full, smem + P::kQB, u.h, N, u.start + u.q0 + kTile, pol_once);
         ++ucnt;
         for (int j = 0; j < nkv; ++j) {
           const int posk = u.kvs + j * kTile;
@@ -445,12 +449,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             break;
           }
           mbar_expect_tx(&k_full[ks], P::kTileBytes);
-          load_tile(&tk, &k_full[ks], smem + P::kK0 + ks * P::kTileBytes, u.h, kv_rows, posk);
+          load_tile(&tk, &k_full[ks], smem + P::kK0 + ks * P::kTileBytes, u.h, kv_rows, posk, pol_keep);
           ++kc;
           const int vs = vc % kStages;
           if (!mbar_wait(&v_empty[vs], ((vc / kStages) & 1) ^ 1, wc, 3, vc)) { ok = false; break; }
           mbar_expect_tx(&v_full[vs], P::kTileBytes);
-          load_tile(&tv, &v_full[vs], smem + P::kV0 + vs * P::kTileBytes, u.h, kv_rows, posk);
+          load_tile(&tv, &v_full[vs], smem + P::kV0 + vs * P::kTileBytes, u.h, kv_rows, posk, pol_keep);
           ++vc;
         }
       }
@@ -924,6 +928,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       // log-sum-exp of the scaled scores: S*scale = log2(e)^-1 (m + log2 l)
       if (a.lse && live) a.lse[(int64_t)u.h * N + u.start + r] = (m_run + log2f(l_lo + l_hi)) * 0.6931471805599453f;
       const float gt = (live && a.gate) ? a.gate[src] : 1.0f;
+      // output rows are written once: mark them first out of L2, so the K/V
+      // tiles that other CTAs still read stay
+      const uint64_t pol_out = l2_policy_evict_first();
       const float inv = a.out_scale * gt / (l_lo + l_hi);
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) + ((int64_t)src * a.H + u.h) * (int64_t)DH;
 #pragma unroll
@@ -948,7 +955,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             if (a.accumulate)
               red_add_bf16x8(dst + q4, pk);
             else
-              dst[q4] = pk;
+              st_global_hint(dst + q4, pk, pol_out);
           }
         }
       }

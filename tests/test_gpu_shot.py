@@ -67,11 +67,15 @@ def test_shot_stga_accumulate_and_scale():
     compare_out(out, ref)
 
 
-@pytest.mark.parametrize("window,plain", [((3, 8, 8), (3, 8, 8)),       # read in place on both sides
-                                          ((0, 30, 52), (6, 30, 52))])   # gathered copies, tiled loads
-def test_one_shot_equals_plain_stga(window, plain):
+@pytest.mark.parametrize("window,plain,bitwise", [((3, 8, 8), (3, 8, 8), False),       # different kernels
+                                                  ((0, 30, 52), (6, 30, 52), True)])   # same tiled kernel
+def test_one_shot_equals_plain_stga(window, plain, bitwise):
     """With a single shot there is nothing to augment: the result is the
-    plain STGA branch (same window order, same tiles)."""
+    plain STGA branch.  Whole-shot windows and plain whole-clip windows run
+    the same kernel over the same tiles, so they agree bit for bit.  For
+    3x8x8 windows plain STGA runs the whole-window box kernel (one softmax
+    step over 192 keys) while shot windows are copied by rows (two key
+    tiles), so the two are compared with the oracle instead."""
     grid = (6, 30, 52)
     q, k, v = _qkv(9360, 2, 128, seed=9)
     ss = torch.tensor([0, 6], dtype=torch.int32, device="cuda")
@@ -79,7 +83,12 @@ def test_one_shot_equals_plain_stga(window, plain):
     moga.sync_status(ws)
     b = moga.stga_window_attn(q, k, v, grid, plain)
     torch.cuda.synchronize()
-    assert torch.equal(a, b)
+    if bitwise:
+        assert torch.equal(a, b)
+    else:
+        ref = oracle.stga_attention(np_cpu(q), np_cpu(k), np_cpu(v), *grid, plain)
+        compare_out(a, ref)
+        compare_out(b, ref)
 
 
 def test_bad_shot_boundaries_are_reported():
