@@ -18,12 +18,6 @@ namespace {
 std::atomic<uint64_t> g_wait_ns{4000000000ull};
 std::atomic<uint64_t> g_launches{0};
 std::atomic<int> g_debug_inject{0};
-// 1: STGA windows of at most 192 tokens run stga_kernel (whole-window TMA
-// boxes); 0: the in-place rows of attn_kernel.
-#ifndef MOGA_STGA_BOX
-#define MOGA_STGA_BOX 1
-#endif
-constexpr bool kStgaBox = MOGA_STGA_BOX != 0;
 constexpr int kNumStages = 6;
 std::atomic<void*> g_ev_begin[kNumStages];
 std::atomic<void*> g_ev_end[kNumStages];
@@ -283,7 +277,7 @@ moga_status stga_body(const DevCtx& c, const void* q, const void* k, const void*
   // Small windows are loaded as whole TMA boxes (stga.cu) and need no
   // permutation, except for the training forward, whose log-sum-exp rows
   // (and the backward pass after it) follow the window order.
-  const bool box = kStgaBox && stga_box_supported(d_h, window);
+  const bool box = stga_box_supported(d_h, window);
   mark(MOGA_STAGE_STGA_PREP, true, c.stream);
   if (!contiguous && (!box || lse)) {
     if (launch_window_perm(c, T, Hg, Wg, window, permw) != cudaSuccess) return MOGA_ERR_CUDA;
@@ -574,19 +568,6 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t o
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-bool make_tmap_window(CUtensorMap* map, const void* base, uint64_t d_h, uint64_t H, uint64_t Wg, uint64_t rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[4] = {d_h, H, Wg, rows};
-  cuuint64_t strides[3] = {d_h * 2, H * d_h * 2, Wg * H * d_h * 2};
-  cuuint32_t box[4] = {64, 1, 8, 8};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;

@@ -12,8 +12,11 @@
 //                   at a time, streaming the segment's K/V tiles once for both.
 //                   Loads: grouped attention (and large windows) read 128-row
 //                   tiles of a gathered head-major copy with 2-D TMA (warp 0);
-//                   windows of up to 256 tokens are copied straight from
-//                   q, k, v by token index with cp.async by warps 0, 2 and 3.
+//                   whole-frame windows read 128 consecutive tokens in place
+//                   with 3-D TMA; STGA windows of 193 to 256 tokens and short
+//                   shot windows are copied straight from q, k, v by token
+//                   index with cp.async by warps 0, 2 and 3.  (STGA windows of
+//                   up to 192 tokens run stga_kernel, stga.cu.)
 //                   Warp 1 issues tcgen05.mma in the order
 //                   PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so the tensor core
 //                   works on one tile while the other tile's softmax runs;
@@ -36,13 +39,6 @@
 namespace moga {
 
 namespace {
-
-// Windows of at most 192 tokens use the small-window plan (double-buffered
-// query tiles, compact half tiles); 0 sends them through the general plan.
-#ifndef MOGA_STGA_SMALL
-#define MOGA_STGA_SMALL 1
-#endif
-constexpr bool kSmallWindows = MOGA_STGA_SMALL != 0;
 
 // One key pair in every kExp2PolyEvery goes through the FMA-pipe polynomial
 // instead of MUFU ex2 (0 disables), balancing the two units in the softmax.
@@ -216,22 +212,7 @@ struct Plan {
   static constexpr int kBar = kV0 + kStages * kTileBytes;
   static constexpr int kTable = kBar + 256;
   static size_t bytes(int table_ints) { return (size_t)kTable + (size_t)table_ints * 4 + 1024; }
-  // Small windows (at most 192 tokens, read in place): query tile B and the
-  // second K and V tiles hold at most 64 rows and are stored compactly (64
-  // rows per 64-column chunk), which frees room for a second pair of query
-  // tiles.  Compact query tiles come first and full ones follow, so a
-  // 128-row operand read of a compact tile stays in shared memory; its rows
-  // past 64 only reach query rows that are dropped or keys that are masked.
-  static constexpr int kChunkFull = kTile * 128;               // bytes of one 64-column chunk, 128 rows
-  static constexpr int kChunkHalf = 64 * 128;                  // the same for 64 rows
-  static constexpr int kHalfBytes = kChunks * kChunkHalf;
-  static constexpr int kSQB = 0;                                // [2] compact query tiles B
-  static constexpr int kSQA = 2 * kHalfBytes;                   // [2] query tiles A
-  static constexpr int kSK0 = kSQA + 2 * kTileBytes;            // K tile 0, then compact K tile 1
-  static constexpr int kSK1 = kSK0 + kTileBytes;
-  static constexpr int kSV0 = kSK1 + kHalfBytes;                // V tile 0, then compact V tile 1
-  static constexpr int kSV1 = kSV0 + kTileBytes;
-  static_assert(kSV1 + kHalfBytes <= kBar, "small-window plan must fit the standard one");
+  static constexpr int kChunkFull = kTile * 128;  // bytes of one 64-column chunk, 128 rows
 };
 
 // A work unit is a pair of consecutive 128-row query tiles (A, B) of one
@@ -319,10 +300,7 @@ struct Decoder {
 // otherwise 128-row tiles of a gathered head-major copy (2-D tiled TMA).
 // kShots: the unit decoder also reads shot-window tables (mode 2); the
 // grouped-attention instantiation leaves it out.
-// kSmall: in place, windows of at most 192 tokens (see Plan): compact tiles,
-// K/V tile j always in slot j, and two query buffers used in turn, so the
-// next window's queries load while this one computes.
-template <int DH, bool kDirect, bool kShots, bool kSmall>
+template <int DH, bool kDirect, bool kShots>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
             const __grid_constant__ CUtensorMap tv, const AttnArgs a, int* status, unsigned long long wait_ns) {
@@ -331,8 +309,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P::kBar);
-  uint64_t* q_full = bars + 0;    // [2] (the second pair only for small windows)
-  uint64_t* q_empty = bars + 2;   // [2]
+  uint64_t* q_full = bars + 0;    // query tiles A, B loaded (slot 0; slot 1 spare)
+  uint64_t* q_empty = bars + 2;   // query tiles free again (slot 0; slot 1 spare)
   uint64_t* k_full = bars + 4;    // [kStages]
   uint64_t* k_empty = bars + 6;   // [kStages]
   uint64_t* v_full = bars + 8;    // [kStages]
@@ -490,7 +468,6 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     int* toks = tab + li * 2 * kTile;  // this loader's token rows (two tiles for Q)
     const int H = a.H;
     uint32_t ucnt = 0, t = 0;
-    uint32_t sc0 = 0, sc1 = 0;  // small windows: uses of K/V slot 0 and 1 by this loader
     bool ok = true;
     // Row indices of tile rows [pos0, pos0 + 128), four per lane: token * H + h,
     // or -1 (zero-filled) for a token out of range or a row past the segment
@@ -538,95 +515,40 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
     };
     {
       // Rows past a segment's end are never copied, so the K and V rings
-      // (and, for small windows, the query buffers) start as zeros: every
-      // row the tensor core reads is then finite (a masked key's P is 0, and
-      // 0 times a finite V row adds nothing).
-      int off, bytes;
-      if constexpr (kSmall) {
-        off = li == 0 ? P::kSQB : li == 1 ? P::kSK0 : P::kSV0;
-        bytes = li == 0 ? P::kSK0 : P::kTileBytes + P::kHalfBytes;
-      } else {
-        off = li == 1 ? P::kK0 : P::kV0;
-        bytes = li == 0 ? 0 : kStages * P::kTileBytes;
-      }
+      // start as zeros: every row the tensor core reads is then finite (a
+      // masked key's P is 0, and 0 times a finite V row adds nothing).
+      const int off = li == 1 ? P::kK0 : P::kV0;
+      const int bytes = li == 0 ? 0 : kStages * P::kTileBytes;
       uint4* ring = reinterpret_cast<uint4*>(smem + off);
       for (int i = lane; i < bytes / 16; i += 32) ring[i] = make_uint4(0, 0, 0, 0);
       fence_proxy_async_smem();
       __syncwarp();
     }
-    // STGA windows of 8x8 tokens whose frames lie inside the grid are loaded
-    // with 4-D TMA boxes instead: one box per frame and 64-column chunk is
-    // the frame's 64 rows in the window's token order, so frames 0-1 fill
-    // the 128-row tile and frame 2 the compact 64-row tile.  Clipped edge
-    // windows (and other window shapes) keep the row copies.  pend[] holds
-    // the phase of a barrier's last use when that use was a TMA load, for the
-    // drain at exit.
-    int pend[2] = {-1, -1};
-    auto tma_window = [&](const Unit& u, int& t0, int& h0, int& w0) -> bool {
-      if (!kSmall || a.mode != 1 || a.wh != 8 || a.ww != 8 || a.wt > 3 || u.seg < 0) return false;
-      const int nbh = (a.Hg + 7) / 8, nbw = (a.Wg + 7) / 8;
-      const int tb = u.seg / (nbh * nbw), hb = (u.seg / nbw) % nbh, wb = u.seg % nbw;
-      t0 = tb * a.wt;
-      h0 = hb * 8;
-      w0 = wb * 8;
-      return t0 + a.wt <= a.T && h0 + 8 <= a.Hg && w0 + 8 <= a.Wg;
-    };
-    constexpr uint32_t kBoxBytes = 64 * 128;  // one frame's 64 rows of one 64-column chunk
     for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
       const Unit u = dec(idx);
       if (u.q0 >= u.len) continue;
       const bool hb = u.q0 + kTile < u.len;
       const int nkv = (u.kvl + kTile - 1) / kTile;
       const int seg_end = u.start + u.len, kv_end = u.kvs + u.kvl;
-      int t0 = 0, h0 = 0, w0 = 0;
-      const bool twin = tma_window(u, t0, h0, w0);
-      if (li == 0 && twin) {
-        const int qb = (int)(ucnt & 1);
-        const uint32_t qph = ucnt >> 1;
-        if (!warp_wait(&q_empty[qb], (qph & 1) ^ 1, 1, ucnt)) { ok = false; break; }
-        if (lane == 0) {
-          mbar_expect_tx(&q_full[qb], (uint32_t)(a.wt * P::kChunks) * kBoxBytes);
-          for (int f = 0; f < a.wt; ++f)
-#pragma unroll
-            for (int c = 0; c < P::kChunks; ++c) {
-              uint8_t* dst = f < 2 ? smem + P::kSQA + qb * P::kTileBytes + c * P::kChunkFull + f * kBoxBytes
-                                   : smem + P::kSQB + qb * P::kHalfBytes + c * P::kChunkHalf;
-              tma_load_4d(&tq, &q_full[qb], dst, c * 64, u.h, w0, (t0 + f) * a.Hg + h0);
-            }
-        }
-        pend[qb] = (int)qph;
-        ++ucnt;
-        continue;
-      }
       if (li == 0) {
         int ra[4], rb[4];
         fetch_rows(a.perm, u.start + u.q0, seg_end, u.h, ra);
         if (hb) fetch_rows(a.perm, u.start + u.q0 + kTile, seg_end, u.h, rb);
-        // small windows: query buffers alternate by unit, each with its own barriers
-        const int qb = kSmall ? (int)(ucnt & 1) : 0;
-        const uint32_t qph = kSmall ? (ucnt >> 1) : ucnt;
-        if (!warp_wait(&q_empty[qb], (qph & 1) ^ 1, 1, ucnt)) { ok = false; break; }
-        if constexpr (kSmall) {
-          copy_tile(a.q, smem + P::kSQA + qb * P::kTileBytes, ra, toks, u.len - u.q0, P::kChunkFull);
-          if (hb) copy_tile(a.q, smem + P::kSQB + qb * P::kHalfBytes, rb, toks + kTile, u.len - u.q0 - kTile,
-                            P::kChunkHalf);
-        } else {
-          copy_tile(a.q, smem + P::kQA, ra, toks, u.len - u.q0, P::kChunkFull);
-          if (hb) copy_tile(a.q, smem + P::kQB, rb, toks + kTile, u.len - u.q0 - kTile, P::kChunkFull);
-        }
+        if (!warp_wait(q_empty, (ucnt & 1) ^ 1, 1, ucnt)) { ok = false; break; }
+        copy_tile(a.q, smem + P::kQA, ra, toks, u.len - u.q0, P::kChunkFull);
+        if (hb) copy_tile(a.q, smem + P::kQB, rb, toks + kTile, u.len - u.q0 - kTile, P::kChunkFull);
         finish();
-        if (lane == 0) mbar_arrive(&q_full[qb]);
-        if (kSmall) pend[qb] = -1;
+        if (lane == 0) mbar_arrive(q_full);
         ++ucnt;
         continue;
       }
       const bool is_v = li == 2;
       for (int j = 0; j < nkv; ++j, ++t) {
         int tr[4];
-        // slot and phase: a ring of kStages tiles, or (small windows) tile j in slot j
-        const int s = kSmall ? j : (int)(t % kStages);
-        const uint32_t ph = kSmall ? (j ? sc1 : sc0) : t / kStages;
-        if (!twin) fetch_rows(kvperm, u.kvs + j * kTile, kv_end, u.h, tr);
+        // slot and phase in the ring of kStages tiles
+        const int s = (int)(t % kStages);
+        const uint32_t ph = t / kStages;
+        fetch_rows(kvperm, u.kvs + j * kTile, kv_end, u.h, tr);
         if (!warp_wait(is_v ? &v_empty[s] : &k_empty[s], (ph & 1) ^ 1, is_v ? 3 : 2, t)) {
           ok = false;
           break;
@@ -634,52 +556,13 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         // Test hook: the first K tile never arrives, so the MMA warp's
         // bounded wait runs out and the kernel reports a timeout.
         if (!is_v && t == 0 && a.debug_withhold_first_k) { ok = false; break; }
-        if (kSmall && twin) {
-          // tile j holds frames [2j, min(2j + 2, wt))
-          const int f0 = 2 * j, f1 = min(a.wt, 2 * j + 2);
-          uint64_t* bar = is_v ? &v_full[s] : &k_full[s];
-          if (lane == 0) {
-            mbar_expect_tx(bar, (uint32_t)((f1 - f0) * P::kChunks) * kBoxBytes);
-            for (int f = f0; f < f1; ++f)
-#pragma unroll
-              for (int c = 0; c < P::kChunks; ++c) {
-                uint8_t* dst = j ? smem + (is_v ? P::kSV1 : P::kSK1) + c * P::kChunkHalf
-                                 : smem + (is_v ? P::kSV0 : P::kSK0) + c * P::kChunkFull + (f - f0) * kBoxBytes;
-                tma_load_4d(is_v ? &tv : &tk, bar, dst, c * 64, u.h, w0, (t0 + f) * a.Hg + h0);
-              }
-          }
-          pend[j] = (int)ph;
-          if (j) ++sc1; else ++sc0;
-          continue;
-        }
-        uint8_t* dst;
-        int chunk = P::kChunkFull;
-        if constexpr (kSmall) {
-          dst = smem + (is_v ? (j ? P::kSV1 : P::kSV0) : (j ? P::kSK1 : P::kSK0));
-          if (j) {
-            chunk = P::kChunkHalf;
-            ++sc1;
-          } else {
-            ++sc0;
-          }
-        } else {
-          dst = smem + (is_v ? P::kV0 : P::kK0) + s * P::kTileBytes;
-        }
-        copy_tile(is_v ? a.v : a.k, dst, tr, toks, u.kvl - j * kTile, chunk);
+        uint8_t* dst = smem + (is_v ? P::kV0 : P::kK0) + s * P::kTileBytes;
+        copy_tile(is_v ? a.v : a.k, dst, tr, toks, u.kvl - j * kTile, P::kChunkFull);
         finish();
         if (lane == 0) mbar_arrive(is_v ? &v_full[s] : &k_full[s]);
-        if (kSmall) pend[j] = -1;
       }
     }
-    // Row copies were waited for before their arrive; TMA loads still in
-    // flight (after an abort) are drained here, one barrier's last use each.
-    if (kSmall && lane == 0) {
-      volatile int zero = 0;
-      WaitCtx dc{&zero, nullptr, 100000000ull};
-      uint64_t* fb = li == 0 ? q_full : li == 1 ? k_full : v_full;
-      for (int b = 0; b < 2; ++b)
-        if (pend[b] >= 0) mbar_wait(&fb[b], (uint32_t)pend[b] & 1, dc);
-    }
+    // Row copies were waited for before their arrive, so nothing is in flight here.
   }
   if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -687,7 +570,6 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
       constexpr uint32_t idS = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idO = idesc_bf16(128, DH, false, true);
       uint32_t ucnt = 0, kc = 0, vc = 0, pc0 = 0, pc1 = 0;
-      uint32_t kc0 = 0, kc1 = 0, vc0 = 0, vc1 = 0;  // small windows: uses of K/V slot 0 and 1
       bool ok = true;
       // S_x = Q_x K^T (both K-major in smem, 128B swizzle); qc / kch: byte
       // stride between the 64-column chunks of the query / key tile.
@@ -700,68 +582,51 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
           umma_bf16(ts, sdesc_add(qd, qo), sdesc_add(kd, ko), idS, kk > 0 ? 1u : 0u);
         }
       };
-      // O_x += P_x V (P in TMEM over S_x, V MN-major in smem, vch between its
-      // 64-column chunks).  Small windows issue only the first nk 16-key steps:
-      // the rest hold masked keys (P = 0) and, in a compact tile, no rows at
-      // all.  Full tiles issue all eight without a test on the issue path.
-      auto issue_pv = [&](int x, uint32_t va, int vch, int nk, bool acc) {
-        const uint64_t vd = sdesc_sw128(va, vch, 1024);
+      // O_x += P_x V (P in TMEM over S_x, V MN-major in smem, its 64-column
+      // chunks kChunkFull bytes apart).
+      auto issue_pv = [&](int x, uint32_t va, bool acc) {
+        const uint64_t vd = sdesc_sw128(va, P::kChunkFull, 1024);
         const uint32_t to = tO(x), ts = tS(x);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          if (!kSmall || kk < nk)
-            umma_bf16_ts(to, ts + kk * 8, sdesc_add(vd, kk * 2048), idO, (acc || kk > 0) ? 1u : 0u);
+          umma_bf16_ts(to, ts + kk * 8, sdesc_add(vd, kk * 2048), idO, (acc || kk > 0) ? 1u : 0u);
       };
-      // K/V tile j of a unit: a ring of kStages slots, or (small windows) slot j.
-      auto kslot = [&](int j) { return kSmall ? j : (int)(kc % kStages); };
-      auto vslot = [&](int j) { return kSmall ? j : (int)(vc % kStages); };
-      auto kphase = [&](int j) { return kSmall ? (j ? kc1 : kc0) : kc / kStages; };
-      auto vphase = [&](int j) { return kSmall ? (j ? vc1 : vc0) : vc / kStages; };
-      auto kaddr = [&](int sl) {
-        return smem_u32(smem + (kSmall ? (sl ? P::kSK1 : P::kSK0) : P::kK0 + sl * P::kTileBytes));
-      };
-      auto vaddr = [&](int sl) {
-        return smem_u32(smem + (kSmall ? (sl ? P::kSV1 : P::kSV0) : P::kV0 + sl * P::kTileBytes));
-      };
-      auto chunk_of = [&](int sl) { return (kSmall && sl) ? P::kChunkHalf : P::kChunkFull; };
+      // K/V tiles sit in a ring of kStages slots.
+      auto kaddr = [&](int sl) { return smem_u32(smem + P::kK0 + sl * P::kTileBytes); };
+      auto vaddr = [&](int sl) { return smem_u32(smem + P::kV0 + sl * P::kTileBytes); };
+      const uint32_t qa_addr = smem_u32(smem + P::kQA), qb_addr = smem_u32(smem + P::kQB);
       for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
         const Unit u = dec(idx);
         if (u.q0 >= u.len) continue;
         const bool hb = u.q0 + kTile < u.len;
         const int nkv = (u.kvl + kTile - 1) / kTile;
-        const int qb = kSmall ? (int)(ucnt & 1) : 0;
-        const uint32_t qph = kSmall ? (ucnt >> 1) : ucnt;
-        if (!mbar_wait(&q_full[qb], qph & 1, wc, 4, ucnt)) break;
+        if (!mbar_wait(q_full, ucnt & 1, wc, 4, ucnt)) break;
         ++ucnt;
-        const uint32_t qa_addr = smem_u32(smem + (kSmall ? P::kSQA + qb * P::kTileBytes : P::kQA));
-        const uint32_t qb_addr = smem_u32(smem + (kSmall ? P::kSQB + qb * P::kHalfBytes : P::kQB));
-        const int qb_chunk = kSmall ? P::kChunkHalf : P::kChunkFull;
-        int ks = kslot(0);
-        if (!mbar_wait(&k_full[ks], kphase(0) & 1, wc, 5, kc)) break;
+        int ks = (int)(kc % kStages);
+        if (!mbar_wait(&k_full[ks], (kc / kStages) & 1, wc, 5, kc)) break;
         tc_fence_after();
-        issue_s(0, qa_addr, P::kChunkFull, kaddr(ks), chunk_of(ks));
+        issue_s(0, qa_addr, P::kChunkFull, kaddr(ks), P::kChunkFull);
         umma_commit(&s_full[0]);
         if (hb) {
-          issue_s(1, qb_addr, qb_chunk, kaddr(ks), chunk_of(ks));
+          issue_s(1, qb_addr, P::kChunkFull, kaddr(ks), P::kChunkFull);
           umma_commit(&s_full[1]);
         }
         umma_commit(&k_empty[ks]);
-        if (kSmall) ++kc0; else ++kc;
-        if (nkv == 1) umma_commit(&q_empty[qb]);
+        ++kc;
+        if (nkv == 1) umma_commit(q_empty);
         for (int j = 0; j < nkv; ++j) {
-          const int vs = vslot(j);
+          const int vs = (int)(vc % kStages);
           const bool more = j + 1 < nkv;
-          const int nk = (min(kTile, u.kvl - j * kTile) + 15) / 16;
-          if (!mbar_wait(&v_full[vs], vphase(j) & 1, wc, 7, vc)) { ok = false; break; }
+          if (!mbar_wait(&v_full[vs], (vc / kStages) & 1, wc, 7, vc)) { ok = false; break; }
           if (!mbar_wait(&p_full[0], pc0 & 1, wc, 13, pc0)) { ok = false; break; }
           ++pc0;
           tc_fence_after();
-          issue_pv(0, vaddr(vs), chunk_of(vs), nk, j > 0);
-          ks = kslot(j + 1);
+          issue_pv(0, vaddr(vs), j > 0);
+          ks = (int)(kc % kStages);
           if (more) {
-            if (!mbar_wait(&k_full[ks], kphase(j + 1) & 1, wc, 8, kc)) { ok = false; break; }
+            if (!mbar_wait(&k_full[ks], (kc / kStages) & 1, wc, 8, kc)) { ok = false; break; }
             tc_fence_after();
-            issue_s(0, qa_addr, P::kChunkFull, kaddr(ks), chunk_of(ks));
+            issue_s(0, qa_addr, P::kChunkFull, kaddr(ks), P::kChunkFull);
             umma_commit(&s_full[0]);
           } else {
             umma_commit(&o_full[0]);
@@ -770,20 +635,20 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
             if (!mbar_wait(&p_full[1], pc1 & 1, wc, 29, pc1)) { ok = false; break; }
             ++pc1;
             tc_fence_after();
-            issue_pv(1, vaddr(vs), chunk_of(vs), nk, j > 0);
+            issue_pv(1, vaddr(vs), j > 0);
             if (more) {
-              issue_s(1, qb_addr, qb_chunk, kaddr(ks), chunk_of(ks));
+              issue_s(1, qb_addr, P::kChunkFull, kaddr(ks), P::kChunkFull);
               umma_commit(&s_full[1]);
             } else {
               umma_commit(&o_full[1]);
             }
           }
           umma_commit(&v_empty[vs]);
-          if (kSmall) { if (j) ++vc1; else ++vc0; } else { ++vc; }
+          ++vc;
           if (more) {
             umma_commit(&k_empty[ks]);
-            if (kSmall) ++kc1; else ++kc;  // tile j + 1 of a small window is tile 1
-            if (j + 2 == nkv) umma_commit(&q_empty[qb]);  // the unit's last S products are issued
+            ++kc;
+            if (j + 2 == nkv) umma_commit(q_empty);  // the unit's last S products are issued
           }
         }
       }
@@ -980,16 +845,9 @@ cudaError_t launch_attention_dh(const DevCtx& c, const AttnArgs& a) {
   // with 128-row boxes.  The in-place kernel copies rows itself and does not
   // read the maps.
   const uint32_t box_rows = (uint32_t)kTile;
-  const bool small_plan =
-      a.direct && a.mode == 1 && (int64_t)a.wt * a.wh * a.ww <= kTile + 64 && kSmallWindows;
   if (a.contiguous) {  // the caller's [N, H, d_h] tensors, read in place
     if (!make_tmap_tokens(&mq, a.q, DH, a.H, a.N) || !make_tmap_tokens(&mk, a.k, DH, a.H, a.N) ||
         !make_tmap_tokens(&mv, a.v, DH, a.H, a.N))
-      return cudaErrorInvalidValue;
-  } else if (small_plan) {  // 8x8 windows read in place by frame boxes
-    const uint64_t grid_rows = (uint64_t)a.T * a.Hg;
-    if (!make_tmap_window(&mq, a.q, DH, a.H, a.Wg, grid_rows) || !make_tmap_window(&mk, a.k, DH, a.H, a.Wg, grid_rows) ||
-        !make_tmap_window(&mv, a.v, DH, a.H, a.Wg, grid_rows))
       return cudaErrorInvalidValue;
   } else {
     if (!make_tmap_2d(&mq, a.q, DH, rows, DH * 2, box_rows)) return cudaErrorInvalidValue;
@@ -999,11 +857,8 @@ cudaError_t launch_attention_dh(const DevCtx& c, const AttnArgs& a) {
   // groups: the segment table; in place: the loaders' token rows (2 tiles each)
   const int table_ints = a.mode == 0 ? 3 * a.nseg + 1 : (a.direct ? 6 * kTile : 0);
   const size_t smem = P::bytes(table_ints);
-  // windows of at most 192 tokens fit the small-window plan (query tile B and
-  // the second K/V tiles of at most 64 rows)
-  const bool small = small_plan;
-  auto kern = a.direct ? (small ? attn_kernel<DH, true, true, true> : attn_kernel<DH, true, true, false>)
-                       : (a.mode == 2 ? attn_kernel<DH, false, true, false> : attn_kernel<DH, false, false, false>);
+  auto kern = a.direct ? attn_kernel<DH, true, true>
+                       : (a.mode == 2 ? attn_kernel<DH, false, true> : attn_kernel<DH, false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int grid = c.num_sms;

@@ -187,11 +187,6 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t o
 // with a box of 64 columns x 1 head x 128 tokens and 128-byte swizzle: one
 // box is a 128-row operand tile of one head, read in place.
 bool make_tmap_tokens(CUtensorMap* map, const void* base, uint64_t d_h, uint64_t H, uint64_t N);
-// Encodes a 4-D bf16 tensor map over the (T*Hg, Wg, H, d_h) view of a
-// [T*Hg*Wg, H, d_h] tensor with a box of 64 columns x 1 head x 8 tokens of a
-// grid row x 8 grid rows and 128-byte swizzle: one box is the 64 rows (grid
-// row-major) of one frame of an 8x8 STGA window, for one head.
-bool make_tmap_window(CUtensorMap* map, const void* base, uint64_t d_h, uint64_t H, uint64_t Wg, uint64_t rows);
 // Encodes a 5-D bf16 tensor map over the (d_h, H, Wg, Hg, T) view of a
 // [T*Hg*Wg, H, d_h] tensor with a box of 64 columns x 1 head x window[2] x
 // window[1] x window[0] and 128-byte swizzle: one box is one STGA window of

@@ -85,10 +85,10 @@ def test_bad_perm_reported():
 
 @pytest.mark.parametrize("window", [(3, 8, 8), (2, 10, 12), (2, 30, 52)])
 def test_window_kernels_time_out_cleanly(window):
-    """The same hook on the STGA kernels: small-window plan (3x8x8), general
-    in-place plan (240-token windows) and the tiled copy (whole frames).  Each
-    loader gives up, the bounded waits run out, the status says so, and the
-    next call matches the oracle."""
+    """The same hook on the STGA kernels: the whole-window box kernel (3x8x8),
+    the general in-place plan (240-token windows) and the tiled loads of whole
+    frames.  Each producer gives up, the bounded waits run out, the status
+    says so, and the next call matches the oracle."""
     lib = moga.get_lib()
     grid = (4, 30, 52)
     N = 4 * 30 * 52
