@@ -39,6 +39,10 @@
  * - Arguments are validated before any device work is enqueued; an invalid
  *   argument returns MOGA_ERR_INVALID_ARG (or MOGA_ERR_UNSUPPORTED /
  *   MOGA_ERR_WORKSPACE) and touches nothing.
+ * - N = 0 (no tokens) is legal wherever N is an argument: per-token buffers
+ *   (x, q, k, v, out, group_id, gate, perm, and the gradient and branch
+ *   outputs of the training calls) may then be NULL, offsets is set to zeros
+ *   and nothing else is written.
  * - The library keeps no state between calls apart from cached kernel
  *   attributes, so distinct workspaces may be used from distinct threads.
  */

@@ -430,8 +430,9 @@ moga_status check_route_args(const void* x, const void* W_r, const float* b_r, m
   return MOGA_OK;
 }
 
-moga_status check_qkv(const void* q, const void* k, const void* v, const void* out) {
-  if (!q || !k || !v || !out) return MOGA_ERR_INVALID_ARG;
+// q, k, v and out may be NULL only when there are no tokens (n == 0).
+moga_status check_qkv(const void* q, const void* k, const void* v, const void* out, int64_t n = 1) {
+  if (n > 0 && (!q || !k || !v || !out)) return MOGA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return MOGA_ERR_INVALID_ARG;
   return MOGA_OK;
 }
@@ -737,7 +738,7 @@ size_t moga_group_attn_workspace_size(int64_t N, int H, int d_h, int M) {
 moga_status moga_group_attn(const void* q, const void* k, const void* v, const int32_t* perm,
                             const int32_t* offsets, const float* gate, int64_t N, int H, int d_h, int M,
                             float out_scale, void* out, void* ws, size_t ws_bytes, void* stream) {
-  moga_status st = check_qkv(q, k, v, out);
+  moga_status st = check_qkv(q, k, v, out, N);
   if (st != MOGA_OK) return st;
   if (!perm || !offsets || !aligned4(perm) || !aligned4(offsets) || (gate && !aligned4(gate)))
     return MOGA_ERR_INVALID_ARG;
@@ -861,7 +862,7 @@ moga_status moga_layer(const void* x, const void* W_r, const float* b_r, moga_dt
                        int32_t* offsets, void* ws, size_t ws_bytes, void* stream) {
   moga_status st = check_route_args(x, W_r, b_r, x_dt, N, d, M, group_id, gate, perm, offsets, offsets);
   if (st != MOGA_OK) return st;
-  if ((st = check_qkv(q, k, v, out)) != MOGA_OK) return st;
+  if ((st = check_qkv(q, k, v, out, N)) != MOGA_OK) return st;
   if ((st = check_attn_shape(N, H, d_h)) != MOGA_OK) return st;
   if (window) {
     int64_t n = 0;
@@ -904,9 +905,10 @@ moga_status moga_layer_train_ex(const void* x, const void* W_r, const float* b_r
   if (per_frame != 0 && per_frame != 1) return MOGA_ERR_INVALID_ARG;
   moga_status st = check_route_args(x, W_r, b_r, x_dt, N, d, M, group_id, gate, perm, offsets, offsets);
   if (st != MOGA_OK) return st;
-  if ((st = check_qkv(q, k, v, out)) != MOGA_OK) return st;
+  if ((st = check_qkv(q, k, v, out, N)) != MOGA_OK) return st;
   if ((st = check_attn_shape(N, H, d_h)) != MOGA_OK) return st;
-  if (!o_moga || !aligned16(o_moga) || (N > 0 && (!lse_moga || !aligned4(lse_moga)))) return MOGA_ERR_INVALID_ARG;
+  if ((N > 0 && !o_moga) || !aligned16(o_moga) || (N > 0 && (!lse_moga || !aligned4(lse_moga))))
+    return MOGA_ERR_INVALID_ARG;
   const int frame_window[3] = {1, Hg, Wg};
   if (window || per_frame) {
     int64_t n = 0;
@@ -985,9 +987,9 @@ moga_status moga_layer_backward_ex(const void* dout, const void* x, const void* 
   // the routing results are inputs here; the forward's checks cover them
   moga_status st = check_route_args(x, W_r, b_r, x_dt, N, d, M, group_id, gate, perm, offsets, offsets);
   if (st != MOGA_OK) return st;
-  if ((st = check_qkv(q, k, v, dout)) != MOGA_OK) return st;
+  if ((st = check_qkv(q, k, v, dout, N)) != MOGA_OK) return st;
   if ((st = check_attn_shape(N, H, d_h)) != MOGA_OK) return st;
-  if ((st = check_qkv(dq, dk, dv, o_moga)) != MOGA_OK) return st;
+  if ((st = check_qkv(dq, dk, dv, o_moga, N)) != MOGA_OK) return st;
   if (!dW_r || !aligned4(dW_r) || (db_r && !aligned4(db_r))) return MOGA_ERR_INVALID_ARG;
   if (N > 0 && (!dx || !aligned16(dx) || !lse_moga || !aligned4(lse_moga))) return MOGA_ERR_INVALID_ARG;
   const int frame_window[3] = {1, Hg, Wg};
@@ -1061,7 +1063,7 @@ moga_status moga_layer_ex(const void* x, const void* W_r, const float* b_r, moga
   if (branches < 0 || branches > 3) return MOGA_ERR_INVALID_ARG;
   moga_status st = check_route_args(x, W_r, b_r, x_dt, N, d, M, group_id, gate, perm, offsets, offsets);
   if (st != MOGA_OK) return st;
-  if ((st = check_qkv(q, k, v, out)) != MOGA_OK) return st;
+  if ((st = check_qkv(q, k, v, out, N)) != MOGA_OK) return st;
   if ((st = check_attn_shape(N, H, d_h)) != MOGA_OK) return st;
   const int frame_window[3] = {1, Hg, Wg};
   if (branches & 1) {

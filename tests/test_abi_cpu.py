@@ -108,6 +108,18 @@ def test_stga_validation(lib):
     assert f(P, P, P, 3, 8, 16, w, 2, 128, 0, P, P, 100, None) == WORKSPACE
 
 
+def test_empty_input_takes_null_token_buffers(lib):
+    """N = 0: the per-token pointers may be NULL; argument checks pass and
+    nothing is dereferenced (a NULL workspace still fails first, so this
+    runs without a GPU)."""
+    f = lib.moga_layer
+    args = [None, P, None, 1, None, None, None, 0, 256, 2, 128, 4, 0, 0, 0, None, None, None, None, None, P, None,
+            BIG, None]
+    assert f(*args) == INVALID                        # the workspace is still required
+    assert lib.moga_group_attn(None, None, None, None, P, None, 0, 2, 128, 4, 1.0, None, None, BIG, None) == INVALID
+    assert lib.moga_group_attn(None, None, None, None, P, None, 1, 2, 128, 4, 1.0, None, P, BIG, None) == INVALID
+
+
 def test_layer_validation(lib):
     w = (ctypes.c_int * 3)(3, 8, 8)
     f = lib.moga_layer

@@ -46,6 +46,9 @@ GROUP_CASES = [
     # third tile, a unit and a half, one row past it, two full units, one row
     # over, a single short tile
     (2100, 2, 128, 6, [257, 384, 385, 512, 513, 49]),
+    # the largest group count the library takes: 1024 groups of a few tokens
+    # (some empty), one short tile each
+    (6000, 2, 128, 1024, None),
 ]
 
 

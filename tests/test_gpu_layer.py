@@ -30,6 +30,29 @@ def _layer(wl, seed):
     return inp, res
 
 
+def test_layer_empty_input():
+    """N = 0 tokens: nothing to route or attend; the call succeeds, the
+    offsets are all zero and nothing is written."""
+    wl = custom(64, H=2, d_h=128, d=128, M=5, name="empty")
+    inp = make_inputs(wl, seed=1, device="cuda")
+    cut = {k: (v[:0] if k in ("x", "q", "k", "v") else v) for k, v in inp.items()}
+    res = moga.moga_layer(cut["x"], cut["W_r"], cut["b_r"], cut["q"], cut["k"], cut["v"], wl.M)
+    moga.sync_status(res["ws"])
+    assert res["out"].shape == (0, 2, 128)
+    assert np.array_equal(np_cpu(res["offsets"]), np.zeros(wl.M + 1, dtype=np.int32))
+
+
+def test_layer_max_groups():
+    """The largest group count (M = 1024, the SIMT router): every token's
+    group and gate against the oracle, and every row of the output."""
+    wl = custom(4096, H=2, d_h=128, d=256, M=1024, x_kind="clustered", name="m1024")
+    inp, res = _layer(wl, seed=3)
+    gid, info = check_route(res, inp["x"], inp["W_r"], inp["b_r"], wl.M, GATE_TOL_BF16)
+    gate = np_cpu(res["gate"]).astype(np.float64)
+    q, k, v = (np_cpu(inp[n]) for n in "qkv")
+    compare_out(res["out"], oracle.group_attention(q, k, v, gid, gate, wl.M), groups=gid)
+
+
 SMALL = [
     WORKLOADS["tiny"],
     custom(384, H=2, d_h=128, d=256, M=4, x_kind="clustered", grid=(3, 8, 16), window=(3, 8, 8), name="small_stga"),
