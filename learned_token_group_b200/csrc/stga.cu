@@ -1,4 +1,4 @@
-// STGA window attention for small windows ("MoGA: Mixture-of-Groups Attention
+// STGA window attention for windows of up to 192 tokens ("MoGA: Mixture-of-Groups Attention
 // for End-to-End Long Video Generation", §3.4 "Spatial-Temporal Group
 // Attention (STGA)"): full softmax attention inside every non-overlapping
 // (wt, wh, ww) box of the (T, Hg, Wg) latent grid, boxes anchored at the
