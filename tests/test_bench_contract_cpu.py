@@ -31,6 +31,10 @@ def test_reference_line_has_contract_keys():
     assert d["steps"] == 1 and d["warmup"] == 0 and d["n_gpus"] == 1
     assert d["higher_is_better"] is True and d["scaling"] == "weak"
     assert d["value"] > 0 and d["ms_per_step"] > 0
+    # a step is one bounded sample (its measured wall time); the layer time
+    # the sample extrapolates to is reported beside it
+    assert d["layer_ms_extrapolated"] > 0
+    assert abs(d["value"] - d["config"]["N"] / (d["layer_ms_extrapolated"] * 1e-3)) <= 1e-6 * d["value"]
     assert d["config"]["workload"] == "tiny"
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
