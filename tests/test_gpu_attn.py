@@ -124,6 +124,8 @@ STGA_CASES = [
     ((3, 13, 23), (3, 6, 10), 2, 128),   # 180-token boxes, clipped in rows and columns
     ((2, 25, 25), (1, 12, 12), 2, 128),  # 144 tokens: the second tile's last warp holds no row
     ((3, 5, 6), (3, 8, 8), 2, 128),      # box larger than the grid in rows and columns
+    ((2, 8, 8), (3, 8, 8), 2, 128),      # fewer frames than the window's extent
+    ((1, 1, 1), (3, 8, 8), 3, 64),       # a single token
 ]
 
 

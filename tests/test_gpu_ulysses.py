@@ -26,7 +26,7 @@ from workloads import custom, make_inputs
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("N,M", [(0, 4), (1, 3), (127, 2), (1000, 7), (4097, 64), (20000, 300)])
+@pytest.mark.parametrize("N,M", [(0, 4), (1, 3), (127, 2), (1000, 7), (4097, 64), (20000, 300), (5000, 1024)])
 def test_sort_matches_oracle(N, M):
     rng = np.random.default_rng(N + M)
     gid = rng.integers(0, M, size=N).astype(np.int32)
