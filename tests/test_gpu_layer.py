@@ -136,15 +136,19 @@ def test_layer_three_branches(wl):
     compare_out(res["out"], ref, groups=gid)
 
 
-def test_layer_three_branches_wan_sampled():
-    wl = WORKLOADS["wan_32k"]
+@pytest.mark.parametrize("name,heads_all", [("wan_32k", False), ("video_187k", True)])
+def test_layer_three_branches_sampled(name, heads_all):
+    """The three-branch block at full size, in the launch configuration of
+    the bench's widened row: sampled rows of every group and of every window
+    kind, compared in full (whole group, window and frame attended)."""
+    wl = WORKLOADS[name]
     inp = make_inputs(wl, seed=3, device="cuda")
     res = moga.moga_layer(inp["x"], inp["W_r"], inp["b_r"], inp["q"], inp["k"], inp["v"], wl.M, wl.grid,
                           wl.window, per_frame=True)
     moga.sync_status(res["ws"])
     gid, _ = check_route(res, inp["x"], inp["W_r"], inp["b_r"], wl.M, GATE_TOL_BF16)
     rows = sample_rows(gid, wl.M, wl.grid, wl.window, np.random.default_rng(5), per_group=64, stga_rows=256)
-    heads = [0, wl.H - 1]
+    heads = list(range(wl.H)) if heads_all else [0, wl.H - 1]
     gate = np_cpu(res["gate"]).astype(np.float64)
     q, k, v = inp["q"], inp["k"], inp["v"]
     ref = (oracle.group_attention(q, k, v, gid, gate, wl.M, rows=rows, heads=heads)
