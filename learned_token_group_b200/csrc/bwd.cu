@@ -25,15 +25,19 @@
 // Warp 0 loads tiles with TMA (and, for dK/dV, the per-column lse and D),
 // warp 1 issues tcgen05.mma, warps 4-11 (two warpgroups, each owning 64 of
 // the 128 Y columns of every TMEM lane) turn S and dP into bf16 P and dS in
-// TMEM, which the accumulating products read as their A operand.  TMEM
-// columns: S at [0, 128), dP at [128, 256), accumulators from 256 (dV then
-// dK, or dQ): one S/dP buffer, so a tile's softmax is not overlapped with the
-// next tile's S and dP (S and dP are committed separately, so P is computed
-// while dP is still in flight).  With d_h = 128 two 128-wide buffers and the dK, dV
-// accumulators do not fit the 512 columns; 128-row Y tiles are still the
-// faster choice, because an M=128 MMA reads its whole A slice from shared
-// memory for every instruction, and N = 128 halves those bytes per
-// multiply-add against N = 64 (shared-memory bandwidth bounds those products).
+// TMEM, which the accumulating products read as their A operand.
+// S and dP each take a 128-column TMEM buffer.  The warpgroups read both
+// into registers and write the packed bf16 operands (P and dS, or dS alone)
+// into the S buffer, 64 columns at most, so the dP buffer is free as soon as
+// dP is read: the next tile's S goes there, and the tensor core computes it
+// (and, for dQ, the next dP) while the warpgroups finish this tile.  dK/dV
+// alternate two buffers (dV and dK fill the other 256 columns); dQ rotates
+// three (dQ takes 128).  Y1 (Q or K) sits in a three-slot ring, since the
+// closing product reads it a tile after S did; Y2 (dO or V) in two slots.
+// 128-row Y tiles are the faster choice, because an M=128 MMA reads its
+// whole A slice from shared memory for every instruction, and N = 128
+// halves those bytes per multiply-add against N = 64 (shared-memory
+// bandwidth bounds those products).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -48,24 +52,31 @@ namespace {
 
 constexpr int kBwdThreads = 384;
 constexpr int kYRows = 128;
-constexpr int kYStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int DH>
+template <int DH, bool kDQ>
 struct BPlan {
   static constexpr int kChunks = DH / 64;
   static constexpr int kXBytes = kTile * DH * 2;    // 128-row bf16 tile
   static constexpr int kYBytes = kYRows * DH * 2;   // 128-row bf16 tile
   static constexpr int kXChunk = kTile * 128;       // bytes of one 64-column chunk of an X tile
   static constexpr int kYChunk = kYRows * 128;      // the same for a Y tile
+  // Y1 and Y2 tiles sit in rings of their own.  Y1 (Q, or K for dQ) is
+  // read by S in its tile's turn and by the product that closes the tile
+  // (dK += dS^T Q, or dQ += dS K) during the next tile's, so its ring has
+  // three slots; Y2 (dO, or V) is first read by dP, later in its tile's
+  // turn, and two slots keep it ahead.
+  static constexpr int kS1 = 3;
+  static constexpr int kS2 = 2;
   static constexpr int kX1 = 0;
   static constexpr int kX2 = kXBytes;
-  static constexpr int kY0 = 2 * kXBytes;           // ring of kYStages x (Y1, Y2)
-  static constexpr int kYStage = 2 * kYBytes;
-  static constexpr int kVec = kY0 + kYStages * kYStage;  // ring of kYStages x (-lse*log2e [128], D [128]) fp32
-  static constexpr int kBar = kVec + kYStages * 2 * kYRows * 4;
+  static constexpr int kY1 = 2 * kXBytes;
+  static constexpr int kY2 = kY1 + kS1 * kYBytes;
+  // dK/dV: -lse*log2(e) of the Y rows per Y1 slot and D per Y2 slot (fp32)
+  static constexpr int kVec1 = kY2 + kS2 * kYBytes;
+  static constexpr int kVec2 = kVec1 + (kDQ ? 0 : kS1 * kYRows * 4);
+  static constexpr int kBar = kVec2 + (kDQ ? 0 : kS2 * kYRows * 4);
   static constexpr int kTable = kBar + 256;
-  static size_t bytes(int table_ints) { return (size_t)kTable + (size_t)table_ints * 4 + 1024; }
 };
 
 struct BUnit {
@@ -75,7 +86,7 @@ struct BUnit {
 struct BDecoder {
   int mode;        // 0 groups (table), 1 windows (geometry)
   int nseg;
-  const int* tab;  // shared copy of [unit_prefix (M+1) | seg_start (M) | seg_len (M)]
+  const int* tab;  // [unit_prefix (M+1) | seg_start (M) | seg_len (M)]: a shared copy, or global
   WinGeom g;
   int upw;         // windows: X tiles per window
   __device__ __forceinline__ BUnit operator()(int idx) const {
@@ -104,46 +115,62 @@ struct BDecoder {
   }
 };
 
+// tab_smem: copy the segment table into shared memory (it fits); pad: bytes
+// allocated beyond the plan, for aligning the tiles to 1024 B.
 template <int DH, bool kDQ>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__ CUtensorMap tx2,
                 const __grid_constant__ CUtensorMap ty1, const __grid_constant__ CUtensorMap ty2, const BwdArgs a,
-                int* status, unsigned long long wait_ns) {
-  using P = BPlan<DH>;
+                int tab_smem, int pad, int* status, unsigned long long wait_ns) {
+  using P = BPlan<DH, kDQ>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
-  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const uint32_t off = ((raw + 1023u) & ~1023u) - raw;
+  if (off > (uint32_t)pad) {  // no room to align the swizzled tiles: the whole CTA returns at once
+    if (threadIdx.x == 0 && status) atomicOr(status, DEV_RANGE);
+    return;
+  }
+  uint8_t* smem = smem_raw + off;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P::kBar);
   uint64_t* x_full = bars + 0;
   uint64_t* x_empty = bars + 1;
-  uint64_t* y_full = bars + 2;                  // [kYStages]
-  uint64_t* y_empty = y_full + kYStages;        // [kYStages]
-  uint64_t* s_full = y_empty + kYStages;        // [2]: S computed (buffer b; dK/dV use buffer 0)
-  uint64_t* d_full = s_full + 2;                // dP computed
+  uint64_t* y1_full = bars + 2;                 // [kS1]
+  uint64_t* y1_empty = y1_full + P::kS1;        // [kS1]
+  uint64_t* y2_full = y1_empty + P::kS1;        // [kS2]
+  uint64_t* y2_empty = y2_full + P::kS2;        // [kS2]
+  uint64_t* s_full = y2_empty + P::kS2;         // S computed
+  uint64_t* d_full = s_full + 1;                // dP computed
   uint64_t* p_full = d_full + 1;                // P and dS written
   uint64_t* acc_full = p_full + 1;
   uint64_t* acc_empty = acc_full + 1;
-  uint64_t* done_bar = acc_empty + 1;
+  uint64_t* dp_free = acc_empty + 1;            // the warpgroups have read dP
+  uint64_t* done_bar = dp_free + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(done_bar + 2);
-  static_assert(2 + 2 * kYStages + 9 <= 32, "barrier area holds 32 words");
+  static_assert(2 + 2 * (P::kS1 + P::kS2) + 9 <= 32, "barrier area holds 32 words");
   int* tab = reinterpret_cast<int*>(smem + P::kTable);
-  float* vec = reinterpret_cast<float*>(smem + P::kVec);
+  float* vec1 = reinterpret_cast<float*>(smem + P::kVec1);
+  float* vec2 = reinterpret_cast<float*>(smem + P::kVec2);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     mbar_init(x_full, 1);
     mbar_init(x_empty, 1);
-    for (int s = 0; s < kYStages; ++s) {
-      mbar_init(&y_full[s], kDQ ? 1 : 2);  // dK/dV: the TMA bytes and the lse/D vectors
-      mbar_init(&y_empty[s], 1);
+    // dK/dV: the TMA bytes and the lse (Y1) or D (Y2) vector
+    for (int s = 0; s < P::kS1; ++s) {
+      mbar_init(&y1_full[s], kDQ ? 1 : 2);
+      mbar_init(&y1_empty[s], 1);
     }
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
+    for (int s = 0; s < P::kS2; ++s) {
+      mbar_init(&y2_full[s], kDQ ? 1 : 2);
+      mbar_init(&y2_empty[s], 1);
+    }
+    mbar_init(s_full, 1);
     mbar_init(d_full, 1);
     mbar_init(p_full, 256);
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 256);
+    mbar_init(dp_free, 256);
     mbar_init(done_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -151,11 +178,14 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
   BDecoder dec;
   dec.mode = a.mode;
   dec.nseg = a.nseg;
-  dec.tab = tab;
+  dec.tab = a.table;
   dec.upw = 1;
   if (a.mode == 0) {
-    const int n = 3 * a.nseg + 1;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) tab[i] = a.table[i];
+    if (tab_smem) {
+      const int n = 3 * a.nseg + 1;
+      for (int i = threadIdx.x; i < n; i += blockDim.x) tab[i] = a.table[i];
+      dec.tab = tab;
+    }
   } else {
     dec.g = WinGeom{a.T, a.Hg, a.Wg, a.wt, a.wh, a.ww, (a.Hg + a.wh - 1) / a.wh, (a.Wg + a.ww - 1) / a.ww};
     dec.upw = (a.wt * a.wh * a.ww + kTile - 1) / kTile;
@@ -167,21 +197,33 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const int total = a.mode == 0 ? tab[a.nseg] : a.nseg * dec.upw * a.H;
+  const int total = a.mode == 0 ? dec.tab[a.nseg] : a.nseg * dec.upw * a.H;
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem;                          // S (then P, packed, over part of it)
-  const uint32_t tD = tmem + 128u;                   // dP (then dS)
   const uint32_t tAccA = tmem + 256u;                // dV, or dQ
   const uint32_t tAccB = tmem + 256u + (uint32_t)DH; // dK
-  // dQ: the columns dK would use hold a second S buffer, so tile i+1's S is
-  // computed while the warpgroups finish tile i
-  auto tSb = [&](uint32_t yc_) { return (kDQ && (yc_ & 1u)) ? tmem + 384u : tS; };
+  // TMEM buffers of Y tile yc (a CTA-wide tile counter).  S goes to one
+  // 128-column buffer and dP to another; the warpgroups read both into
+  // registers and write the packed bf16 operands of the closing products
+  // (dK/dV: P, then dS 32 columns further; dQ: dS) into the S buffer.  So
+  // the dP buffer is free once dP is read, and the next tile's S and dP are
+  // computed while this tile's dS and products proceed.
+  //   dK/dV: two buffers (0, 128; dV and dK fill the rest) swap roles:
+  //          S(yc) in buffer yc % 2, dP(yc) in the other, which held the
+  //          previous tile's S (its P and dS are read before dP(yc) is
+  //          issued).
+  //   dQ:    three buffers (0, 128, 384; dQ at 256) rotate: S(yc) in buffer
+  //          yc % 3, where dP(yc - 1) was, and dP(yc) in buffer (yc + 1) % 3,
+  //          where S(yc - 2) was (its dS is read by dQ(yc - 2), issued
+  //          before dP(yc)).
+  auto tbuf = [&](uint32_t b) { return tmem + (b == 2u ? 384u : 128u * b); };
+  auto tSb = [&](uint32_t yc_) { return kDQ ? tbuf(yc_ % 3u) : tmem + 128u * (yc_ & 1u); };
+  auto tDb = [&](uint32_t yc_) { return kDQ ? tbuf((yc_ + 1u) % 3u) : tmem + 128u * ((yc_ & 1u) ^ 1u); };
   WaitCtx wc{abort_flag, status, wait_ns};
   const int64_t N = a.N;
 
   if (warp == 0) {
     // ---------------------------------------------------------------- loads
-    uint32_t uc = 0, yc = 0;
+    uint32_t uc = 0, n1 = 0, n2 = 0;  // X tiles, Y1 and Y2 tiles issued
     bool ok = true;
     auto wwait = [&](uint64_t* bar, uint32_t parity, int site, uint32_t count) {
       int w = 1;
@@ -194,6 +236,28 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
       tma_prefetch_desc(&ty1);
       tma_prefetch_desc(&ty2);
     }
+    // dK/dV: this lane's share of a Y tile's -lse*log2(e) and D, read one
+    // tile ahead so that their latency hides behind the rings' waits.  Rows
+    // past the segment get -inf and 0, so their P and dS are exactly 0.
+    float lv[kYRows / 32], dv[kYRows / 32];
+    auto fetch = [&](const BUnit& u, int i) {
+#pragma unroll
+      for (int q = 0; q < kYRows / 32; ++q) {
+        const int pos = i * kYRows + lane + 32 * q;
+        const bool valid = pos < u.len;
+        const int64_t gi = (int64_t)u.h * N + u.start + pos;
+        lv[q] = valid ? -a.lse[gi] * kLog2e : -INFINITY;
+        dv[q] = valid ? a.dsum[gi] : 0.0f;
+      }
+    };
+    // plain shared-memory stores of a vector, then the slot's second arrival
+    auto put = [&](float* v, const float* r, uint64_t* bar) {
+#pragma unroll
+      for (int q = 0; q < kYRows / 32; ++q) v[lane + 32 * q] = r[q];
+      __threadfence_block();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
+    };
     for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
       const BUnit u = dec(idx);
       if (u.x0 >= u.len) continue;
@@ -209,35 +273,32 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
         }
       }
       ++uc;
+      if (!kDQ) fetch(u, 0);
       for (int i = 0; i < ny; ++i) {
-        const int s = (int)(yc % kYStages);
-        if (!wwait(&y_empty[s], ((yc / kYStages) & 1) ^ 1, 2, yc)) { ok = false; break; }
+        const int row = (int)((int64_t)u.h * N + u.start + i * kYRows);
+        const int s1 = (int)(n1 % P::kS1);
+        if (!wwait(&y1_empty[s1], ((n1 / P::kS1) & 1) ^ 1, 2, n1)) { ok = false; break; }
         if (lane == 0) {
-          const int row = (int)((int64_t)u.h * N + u.start + i * kYRows);
-          uint8_t* y1 = smem + P::kY0 + s * P::kYStage;
-          mbar_expect_tx(&y_full[s], 2 * P::kYBytes);
+          uint8_t* y = smem + P::kY1 + s1 * P::kYBytes;
+          mbar_expect_tx(&y1_full[s1], P::kYBytes);
 #pragma unroll
-          for (int c = 0; c < P::kChunks; ++c) {
-            tma_load_2d(&ty1, &y_full[s], y1 + c * P::kYChunk, c * 64, row);
-            tma_load_2d(&ty2, &y_full[s], y1 + P::kYBytes + c * P::kYChunk, c * 64, row);
-          }
+          for (int c = 0; c < P::kChunks; ++c) tma_load_2d(&ty1, &y1_full[s1], y + c * P::kYChunk, c * 64, row);
+        }
+        if (!kDQ) put(vec1 + s1 * kYRows, lv, &y1_full[s1]);
+        ++n1;
+        const int s2 = (int)(n2 % P::kS2);
+        if (!wwait(&y2_empty[s2], ((n2 / P::kS2) & 1) ^ 1, 16, n2)) { ok = false; break; }
+        if (lane == 0) {
+          uint8_t* y = smem + P::kY2 + s2 * P::kYBytes;
+          mbar_expect_tx(&y2_full[s2], P::kYBytes);
+#pragma unroll
+          for (int c = 0; c < P::kChunks; ++c) tma_load_2d(&ty2, &y2_full[s2], y + c * P::kYChunk, c * 64, row);
         }
         if (!kDQ) {
-          // per Y row (query): -lse * log2(e) and D; rows past the segment
-          // get -inf and 0, so their P and dS are exactly 0
-          float* v = vec + s * 2 * kYRows;
-          for (int c = lane; c < kYRows; c += 32) {
-            const int pos = i * kYRows + c;
-            const bool valid = pos < u.len;
-            const int64_t gi = (int64_t)u.h * N + u.start + pos;
-            v[c] = valid ? -a.lse[gi] * kLog2e : -INFINITY;
-            v[kYRows + c] = valid ? a.dsum[gi] : 0.0f;
-          }
-          __threadfence_block();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&y_full[s]);
+          put(vec2 + s2 * kYRows, dv, &y2_full[s2]);
+          if (i + 1 < ny) fetch(u, i + 1);
         }
-        ++yc;
+        ++n2;
       }
     }
     // Drain every load this warp issued before the CTA exits.
@@ -245,8 +306,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
       volatile int zero = 0;
       WaitCtx dc{&zero, nullptr, 100000000ull};
       if (uc > 0) mbar_wait(x_full, (uc - 1) & 1, dc);
-      for (int s = 0; s < kYStages; ++s)
-        if ((uint32_t)s < yc) mbar_wait(&y_full[s], ((yc - 1 - ((yc - 1 - s) % kYStages)) / kYStages) & 1, dc);
+      for (int s = 0; s < P::kS1; ++s)
+        if ((uint32_t)s < n1) mbar_wait(&y1_full[s], ((n1 - 1 - ((n1 - 1 - s) % P::kS1)) / P::kS1) & 1, dc);
+      for (int s = 0; s < P::kS2; ++s)
+        if ((uint32_t)s < n2) mbar_wait(&y2_full[s], ((n2 - 1 - ((n2 - 1 - s) % P::kS2)) / P::kS2) & 1, dc);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -260,98 +323,86 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
       const uint64_t x1d = sdesc_sw128(x1, 16, 1024), x2d = sdesc_sw128(x2, 16, 1024);
       // S and dP with their own commits, so that the softmax warps compute
       // P while the tensor core computes dP.
-      auto issue_sonly = [&](int s, uint32_t ycs) {
-        const uint64_t y1d = sdesc_sw128(smem_u32(smem + P::kY0 + s * P::kYStage), 16, 1024);
+      auto issue_sonly = [&](uint32_t ycs) {
+        const uint64_t y1d = sdesc_sw128(smem_u32(smem + P::kY1 + (ycs % P::kS1) * P::kYBytes), 16, 1024);
         const uint32_t ts = tSb(ycs);
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
           const uint32_t xo = (kk >> 2) * P::kXChunk + (kk & 3) * 32, yo = (kk >> 2) * P::kYChunk + (kk & 3) * 32;
           umma_bf16(ts, sdesc_add(x1d, xo), sdesc_add(y1d, yo), idS, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&s_full[ycs & (kDQ ? 1u : 0u)]);
+        umma_commit(s_full);
       };
-      auto issue_dp = [&](int s) {
-        const uint64_t y2d = sdesc_sw128(smem_u32(smem + P::kY0 + s * P::kYStage) + P::kYBytes, 16, 1024);
+      auto issue_dp = [&](uint32_t ycs) {
+        const uint64_t y2d = sdesc_sw128(smem_u32(smem + P::kY2 + (ycs % P::kS2) * P::kYBytes), 16, 1024);
+        const uint32_t td = tDb(ycs);
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
           const uint32_t xo = (kk >> 2) * P::kXChunk + (kk & 3) * 32, yo = (kk >> 2) * P::kYChunk + (kk & 3) * 32;
-          umma_bf16(tD, sdesc_add(x2d, xo), sdesc_add(y2d, yo), idS, kk > 0 ? 1u : 0u);
+          umma_bf16(td, sdesc_add(x2d, xo), sdesc_add(y2d, yo), idS, kk > 0 ? 1u : 0u);
         }
         umma_commit(d_full);
       };
       // Accumulations over the 128 Y rows (eight 16-row steps).  Warpgroup w
-      // wrote P / dS of Y rows [64w, 64w + 64) as packed bf16 into columns
-      // [64w, 64w + 32) of the S / dP region, so step kk's 16 rows start at
-      // column 64 (kk / 4) + 8 (kk % 4).
-      auto issue_acc = [&](int s, bool acc) {
-        const uint32_t y1 = smem_u32(smem + P::kY0 + s * P::kYStage);
-        const uint64_t y1d = sdesc_sw128(y1, P::kYChunk, 1024), y2d = sdesc_sw128(y1 + P::kYBytes, P::kYChunk, 1024);
+      // wrote P / dS of Y rows [64w, 64w + 64) as packed bf16 into the S
+      // buffer, 32 columns from 64w (dK/dV: P there, dS 32 columns further),
+      // so step kk's 16 rows start at column 64 (kk / 4) + 8 (kk % 4).
+      auto issue_acc = [&](uint32_t ycs, bool acc) {
+        const uint64_t y1d = sdesc_sw128(smem_u32(smem + P::kY1 + (ycs % P::kS1) * P::kYBytes), P::kYChunk, 1024);
+        const uint64_t y2d = sdesc_sw128(smem_u32(smem + P::kY2 + (ycs % P::kS2) * P::kYBytes), P::kYChunk, 1024);
+        const uint32_t ts = tSb(ycs);
 #pragma unroll
         for (int kk = 0; kk < kYRows / 16; ++kk) {
           const uint32_t pc = 64u * (kk >> 2) + 8u * (kk & 3);
           const uint32_t en = (acc || kk > 0) ? 1u : 0u;
           if (kDQ) {
-            umma_bf16_ts(tAccA, tD + pc, sdesc_add(y1d, kk * 2048), idA, en);  // dQ += dS K
+            umma_bf16_ts(tAccA, ts + pc, sdesc_add(y1d, kk * 2048), idA, en);  // dQ += dS K
           } else {
-            umma_bf16_ts(tAccA, tS + pc, sdesc_add(y2d, kk * 2048), idA, en);  // dV += P^T dO
-            umma_bf16_ts(tAccB, tD + pc, sdesc_add(y1d, kk * 2048), idA, en);  // dK += dS^T Q
+            umma_bf16_ts(tAccA, ts + pc, sdesc_add(y2d, kk * 2048), idA, en);       // dV += P^T dO
+            umma_bf16_ts(tAccB, ts + 32 + pc, sdesc_add(y1d, kk * 2048), idA, en);  // dK += dS^T Q
           }
         }
       };
-      // One S/dP buffer: tile i's S and dP are issued after tile i-1's
-      // accumulations (which read its P and dS from the same columns), and
-      // only once the softmax warps have released tile i-1.
+      // Tile t's accumulations, once the warpgroups have written its P and
+      // dS (and, for a unit's first tile, read out the previous unit's
+      // accumulators); they are the last readers of its Y1 tile (and, for
+      // dK/dV, of its Y2 tile).
       auto finish_tile = [&](uint32_t t, bool first, bool last_of_unit) {
-        const int st = (int)(t % kYStages);
         if (!mbar_wait(p_full, t & 1, wc, 5, t)) return false;
         if (first && uc > 0 && !mbar_wait(acc_empty, (uc - 1) & 1, wc, 6, uc)) return false;
         tc_fence_after();
-        issue_acc(st, !first);
-        umma_commit(&y_empty[st]);
+        issue_acc(t, !first);
+        umma_commit(&y1_empty[t % P::kS1]);
+        if (!kDQ) umma_commit(&y2_empty[t % P::kS2]);
         if (last_of_unit) umma_commit(acc_full);
         return true;
       };
+      auto wait_y1 = [&](uint32_t t) { return mbar_wait(&y1_full[t % P::kS1], (t / P::kS1) & 1, wc, 4, t); };
+      auto wait_y2 = [&](uint32_t t) { return mbar_wait(&y2_full[t % P::kS2], (t / P::kS2) & 1, wc, 17, t); };
       for (int idx = blockIdx.x; idx < total && ok; idx += gridDim.x) {
         const BUnit u = dec(idx);
         if (u.x0 >= u.len) continue;
         const int ny = (u.len + kYRows - 1) / kYRows;
         if (!mbar_wait(x_full, uc & 1, wc, 3, uc)) break;
-        if (kDQ) {
-          // Two S buffers: tile i's S was issued one tile ahead, so the order
-          // per tile is dQ(i-1), dP(i), S(i+1).  S(i+1) reuses the buffer of
-          // tile i-1, which the warpgroups released (P and dS written) before
-          // dQ(i-1) was issued.
-          const int s0 = (int)(yc % kYStages);
-          if (!mbar_wait(&y_full[s0], (yc / kYStages) & 1, wc, 4, yc)) break;
+        // S(i) goes where dP(i-1) was, once the warpgroups have read it.
+        // dK/dV: S(i), the products of tile i-1, dP(i), which goes where
+        // those products read P and dS of tile i-1 just before.  dQ: S(i),
+        // dP(i), where dQ(i-2) read dS, then dQ(i-1); V is read by dP alone
+        // and released right after it.  (The tensor pipe runs in issue
+        // order.)
+        for (int i = 0; i < ny; ++i) {
+          if (!wait_y1(yc)) { ok = false; break; }
+          if (yc > 0 && !mbar_wait(dp_free, (yc - 1) & 1, wc, 15, yc)) { ok = false; break; }
           tc_fence_after();
-          issue_sonly(s0, yc);
-          for (int i = 0; i < ny; ++i) {
-            const int s = (int)(yc % kYStages);
-            if (i > 0 && !finish_tile(yc - 1, i == 1, false)) { ok = false; break; }
-            tc_fence_after();
-            issue_dp(s);
-            if (i + 1 == ny) {
-              umma_commit(x_empty);
-            } else {
-              const uint32_t y1 = yc + 1;
-              const int s1 = (int)(y1 % kYStages);
-              if (!mbar_wait(&y_full[s1], (y1 / kYStages) & 1, wc, 4, y1)) { ok = false; break; }
-              tc_fence_after();
-              issue_sonly(s1, y1);
-            }
-            ++yc;
-          }
-        } else {
-          for (int i = 0; i < ny; ++i) {
-            const int s = (int)(yc % kYStages);
-            if (i > 0 && !finish_tile(yc - 1, i == 1, false)) { ok = false; break; }
-            if (!mbar_wait(&y_full[s], (yc / kYStages) & 1, wc, 4, yc)) { ok = false; break; }
-            tc_fence_after();
-            issue_sonly(s, yc);
-            issue_dp(s);
-            if (i + 1 == ny) umma_commit(x_empty);
-            ++yc;
-          }
+          issue_sonly(yc);
+          if (!kDQ && i > 0 && !finish_tile(yc - 1, i == 1, false)) { ok = false; break; }
+          if (!wait_y2(yc)) { ok = false; break; }
+          tc_fence_after();
+          issue_dp(yc);
+          if (kDQ) umma_commit(&y2_empty[yc % P::kS2]);
+          if (i + 1 == ny) umma_commit(x_empty);
+          if (kDQ && i > 0 && !finish_tile(yc - 1, i == 1, false)) { ok = false; break; }
+          ++yc;
         }
         if (!ok || !finish_tile(yc - 1, ny == 1, true)) break;
         ++uc;
@@ -389,24 +440,22 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
       }
       const int src = live ? (a.perm ? a.perm[u.start + r] : u.start + r) : 0;
       for (int i = 0; i < ny; ++i, ++yc) {
-        const int s = (int)(yc % kYStages);
-        // dQ: S buffer yc & 1 (its phase advances every other tile); dK/dV: buffer 0
-        const bool ok_s = kDQ ? mbar_wait(&s_full[yc & 1], (yc >> 1) & 1, wc, 7 + wg, yc)
-                              : mbar_wait(&s_full[0], yc & 1, wc, 7 + wg, yc);
-        if (!ok_s) { ok = false; break; }
+        const int s1 = (int)(yc % P::kS1), s2 = (int)(yc % P::kS2);
+        if (!mbar_wait(s_full, yc & 1, wc, 7 + wg, yc)) { ok = false; break; }
         tc_fence_after();
         // the vectors are plain shared-memory stores of the load warp: wait
-        // on the stage's own barrier too (its phase is still this tile's,
-        // since the stage is refilled only after this tile's P and dS)
-        if (!kDQ && !mbar_wait(&y_full[s], (yc / kYStages) & 1, wc, 11 + wg, yc)) { ok = false; break; }
+        // on the slot's own barrier too (its phase is still this tile's,
+        // since the slot is refilled only after this tile's P and dS)
+        if (!kDQ && !mbar_wait(&y1_full[s1], (yc / P::kS1) & 1, wc, 11 + wg, yc)) { ok = false; break; }
         // Y columns [64 wg, 64 wg + 64): P from S as soon as S is in (the
         // tensor core is still computing dP), then dS once dP is in.  The
-        // packed P / dS of half hf go to columns 64 wg + 16 hf, which this
+        // packed P (dK/dV) and dS of half hf go to S-buffer columns
+        // 64 wg + 16 hf and, for dK/dV's dS, 32 further: columns this
         // warpgroup has already read.
+        const uint32_t ts = tSb(yc), td = tDb(yc);
         float pv[64];
         {
           float sv[64];
-          const uint32_t ts = tSb(yc);
           tmem_ld32(ts + lb + 64 * wg, sv);
           tmem_ld32(ts + lb + 64 * wg + 32, sv + 32);
           tmem_ld_wait();
@@ -418,7 +467,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
               pv[e] = e < valid ? pe : 0.0f;
             }
           } else {
-            const float* nl = vec + s * 2 * kYRows + 64 * wg;
+            const float* nl = vec1 + s1 * kYRows + 64 * wg;
 #pragma unroll
             for (int e = 0; e < 64; ++e) pv[e] = fast_exp2(fmaf(sv[e], scale_log2, nl[e]));
 #pragma unroll
@@ -426,32 +475,35 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
               uint32_t pk[16];
 #pragma unroll
               for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pv[32 * hf + 2 * e], pv[32 * hf + 2 * e + 1]);
-              tmem_st16u(tS + lb + 64 * wg + 16 * hf, pk);
+              tmem_st16u(ts + lb + 64 * wg + 16 * hf, pk);
             }
           }
         }
         if (!mbar_wait(d_full, yc & 1, wc, 13 + wg, yc)) { ok = false; break; }
         tc_fence_after();
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int c0 = 64 * wg + 32 * hf;
-          float dv[32];
-          tmem_ld32(tD + lb + c0, dv);
+        {
+          // all of dP is read first, so its buffer is released for the next
+          // tile's S before dS is computed
+          float dv[64];
+          tmem_ld32(td + lb + 64 * wg, dv);
+          tmem_ld32(td + lb + 64 * wg + 32, dv + 32);
           tmem_ld_wait();
-          uint32_t dk[16];
-          if (kDQ) {
+          tc_fence_before();
+          mbar_arrive(dp_free);
+          // D per Y row (dK/dV: from the Y2 slot's vector), or of this X row (dQ)
+          const float* dd = vec2 + s2 * kYRows + 64 * wg;
+          if (!kDQ && !mbar_wait(&y2_full[s2], (yc / P::kS2) & 1, wc, 18 + wg, yc)) { ok = false; break; }
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              dk[e] = pack_bf16x2(pv[32 * hf + 2 * e] * (dv[2 * e] - d_row),
-                                  pv[32 * hf + 2 * e + 1] * (dv[2 * e + 1] - d_row));
-          } else {
-            const float* dd = vec + s * 2 * kYRows + kYRows + c0;
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t dk[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              dk[e] = pack_bf16x2(pv[32 * hf + 2 * e] * (dv[2 * e] - dd[2 * e]),
-                                  pv[32 * hf + 2 * e + 1] * (dv[2 * e + 1] - dd[2 * e + 1]));
+            for (int e = 0; e < 16; ++e) {
+              const int c = 32 * hf + 2 * e;
+              dk[e] = kDQ ? pack_bf16x2(pv[c] * (dv[c] - d_row), pv[c + 1] * (dv[c + 1] - d_row))
+                          : pack_bf16x2(pv[c] * (dv[c] - dd[c]), pv[c + 1] * (dv[c + 1] - dd[c + 1]));
+            }
+            tmem_st16u(ts + lb + 64 * wg + (kDQ ? 0 : 32) + 16 * hf, dk);
           }
-          tmem_st16u(tD + lb + 64 * wg + 16 * hf, dk);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -520,7 +572,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
 
 template <int DH, bool kDQ>
 cudaError_t launch_bwd_dh(const DevCtx& c, const BwdArgs& a) {
-  using P = BPlan<DH>;
+  using P = BPlan<DH, kDQ>;
   CUtensorMap m1, m2, m3, m4;
   const uint64_t rows = (uint64_t)a.N * (uint64_t)a.H;
   // X and Y: 128-row boxes (all [H][N][d_h] head-major copies)
@@ -531,10 +583,19 @@ cudaError_t launch_bwd_dh(const DevCtx& c, const BwdArgs& a) {
   if (!make_tmap_2d(&m1, xs1, DH, rows, DH * 2, kTile) || !make_tmap_2d(&m2, xs2, DH, rows, DH * 2, kTile) ||
       !make_tmap_2d(&m3, ys1, DH, rows, DH * 2, kYRows) || !make_tmap_2d(&m4, ys2, DH, rows, DH * 2, kYRows))
     return cudaErrorInvalidValue;
-  const int table_ints = a.mode == 0 ? 3 * a.nseg + 1 : 0;
-  const size_t smem = P::bytes(table_ints);
+  int max_smem = 0;
+  cudaError_t e = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, c.device);
+  if (e != cudaSuccess) return e;
+  // The segment table goes to shared memory when it fits beside the tiles
+  // (the kernel reads it from global memory otherwise); up to 1 KB more
+  // aligns the tiles to 1024 B, and the kernel checks that it got enough.
+  const size_t table_bytes = a.mode == 0 ? (size_t)(3 * a.nseg + 1) * 4 : 0;
+  const bool tab_smem = P::kTable + table_bytes <= (size_t)max_smem;
+  const size_t need = P::kTable + (tab_smem ? table_bytes : 0);
+  if (need > (size_t)max_smem) return cudaErrorInvalidValue;
+  const size_t smem = std::min(need + 1024, (size_t)max_smem);
   auto kern = attn_bwd_kernel<DH, kDQ>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int grid = c.num_sms;
   if (a.mode == 1) {
@@ -542,7 +603,8 @@ cudaError_t launch_bwd_dh(const DevCtx& c, const BwdArgs& a) {
     if (total < grid) grid = (int)total;
   }
   if (grid < 1) return cudaSuccess;
-  kern<<<grid, kBwdThreads, smem, c.stream>>>(m1, m2, m3, m4, a, c.status, (unsigned long long)c.wait_ns);
+  kern<<<grid, kBwdThreads, smem, c.stream>>>(m1, m2, m3, m4, a, tab_smem ? 1 : 0, (int)(smem - need), c.status,
+                                              (unsigned long long)c.wait_ns);
   return cudaGetLastError();
 }
 
