@@ -29,10 +29,10 @@
 // S and dP each take a 128-column TMEM buffer.  The warpgroups read both
 // into registers and write the packed bf16 operands (P and dS, or dS alone)
 // into the S buffer, 64 columns at most, so the dP buffer is free as soon as
-// dP is read: the next tile's S goes there, and the tensor core computes it
-// (and, for dQ, the next dP) while the warpgroups finish this tile.  dK/dV
-// alternate two buffers (dV and dK fill the other 256 columns); dQ rotates
-// three (dQ takes 128).  Y1 (Q or K) sits in a three-slot ring, since the
+// dP is read.  dK/dV alternate two buffers (dV and dK fill the other 256
+// columns): the next tile's S goes where dP was and is computed while the
+// warpgroups finish this tile.  dQ keeps dP in one buffer and alternates S
+// between two, issuing S a whole tile ahead (dQ takes the last 128).  Y1 (Q or K) sits in a three-slot ring, since the
 // closing product reads it a tile after S did; Y2 (dO or V) in two slots.
 // 128-row Y tiles are the faster choice, because an M=128 MMA reads its
 // whole A slice from shared memory for every instruction, and N = 128
@@ -138,16 +138,20 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
   uint64_t* y1_empty = y1_full + P::kS1;        // [kS1]
   uint64_t* y2_full = y1_empty + P::kS1;        // [kS2]
   uint64_t* y2_empty = y2_full + P::kS2;        // [kS2]
-  uint64_t* s_full = y2_empty + P::kS2;         // S computed
-  uint64_t* d_full = s_full + 1;                // dP computed
-  uint64_t* p_full = d_full + 1;                // P and dS written
-  uint64_t* acc_full = p_full + 1;
+  uint64_t* s_full = y2_empty + P::kS2;         // [2]: S computed (dQ: S(t) on s_full[t % 2])
+  uint64_t* d_full = s_full + 2;                // dP computed
+  // [2]: P and dS of tile t written, on p_full[t % 2].  Two barriers,
+  // because the dQ pass issues dP(t + 1) before it waits for tile t, so the
+  // warpgroups may finish tile t + 1 before that wait begins; the next phase
+  // of the same barrier needs dP(t + 2), which comes after it.
+  uint64_t* p_full = d_full + 1;
+  uint64_t* acc_full = p_full + 2;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* dp_free = acc_empty + 1;            // the warpgroups have read dP
   uint64_t* done_bar = dp_free + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(done_bar + 2);
-  static_assert(2 + 2 * (P::kS1 + P::kS2) + 9 <= 32, "barrier area holds 32 words");
+  static_assert(2 + 2 * (P::kS1 + P::kS2) + 11 <= 32, "barrier area holds 32 words");
   int* tab = reinterpret_cast<int*>(smem + P::kTable);
   float* vec1 = reinterpret_cast<float*>(smem + P::kVec1);
   float* vec2 = reinterpret_cast<float*>(smem + P::kVec2);
@@ -165,9 +169,11 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
       mbar_init(&y2_full[s], kDQ ? 1 : 2);
       mbar_init(&y2_empty[s], 1);
     }
-    mbar_init(s_full, 1);
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
     mbar_init(d_full, 1);
-    mbar_init(p_full, 256);
+    mbar_init(&p_full[0], 256);
+    mbar_init(&p_full[1], 256);
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 256);
     mbar_init(dp_free, 256);
@@ -205,19 +211,17 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
   // 128-column buffer and dP to another; the warpgroups read both into
   // registers and write the packed bf16 operands of the closing products
   // (dK/dV: P, then dS 32 columns further; dQ: dS) into the S buffer.  So
-  // the dP buffer is free once dP is read, and the next tile's S and dP are
-  // computed while this tile's dS and products proceed.
+  // the dP buffer is free once dP is read.
   //   dK/dV: two buffers (0, 128; dV and dK fill the rest) swap roles:
   //          S(yc) in buffer yc % 2, dP(yc) in the other, which held the
   //          previous tile's S (its P and dS are read before dP(yc) is
-  //          issued).
-  //   dQ:    three buffers (0, 128, 384; dQ at 256) rotate: S(yc) in buffer
-  //          yc % 3, where dP(yc - 1) was, and dP(yc) in buffer (yc + 1) % 3,
-  //          where S(yc - 2) was (its dS is read by dQ(yc - 2), issued
-  //          before dP(yc)).
-  auto tbuf = [&](uint32_t b) { return tmem + (b == 2u ? 384u : 128u * b); };
-  auto tSb = [&](uint32_t yc_) { return kDQ ? tbuf(yc_ % 3u) : tmem + 128u * (yc_ & 1u); };
-  auto tDb = [&](uint32_t yc_) { return kDQ ? tbuf((yc_ + 1u) % 3u) : tmem + 128u * ((yc_ & 1u) ^ 1u); };
+  //          issued); S(yc + 1) is computed while the warpgroups finish yc.
+  //   dQ:    S alternates between 0 and 384, dP stays at 128 (dQ at 256).
+  //          S(yc + 1) is issued right after dQ(yc - 1) has read dS from
+  //          its buffer, a whole tile ahead, and dP(yc + 1) once dP(yc) is
+  //          read.
+  auto tSb = [&](uint32_t yc_) { return kDQ ? tmem + ((yc_ & 1u) ? 384u : 0u) : tmem + 128u * (yc_ & 1u); };
+  auto tDb = [&](uint32_t yc_) { return kDQ ? tmem + 128u : tmem + 128u * ((yc_ & 1u) ^ 1u); };
   WaitCtx wc{abort_flag, status, wait_ns};
   const int64_t N = a.N;
 
@@ -331,7 +335,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
           const uint32_t xo = (kk >> 2) * P::kXChunk + (kk & 3) * 32, yo = (kk >> 2) * P::kYChunk + (kk & 3) * 32;
           umma_bf16(ts, sdesc_add(x1d, xo), sdesc_add(y1d, yo), idS, kk > 0 ? 1u : 0u);
         }
-        umma_commit(s_full);
+        umma_commit(&s_full[kDQ ? (ycs & 1u) : 0u]);
       };
       auto issue_dp = [&](uint32_t ycs) {
         const uint64_t y2d = sdesc_sw128(smem_u32(smem + P::kY2 + (ycs % P::kS2) * P::kYBytes), 16, 1024);
@@ -368,7 +372,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
       // accumulators); they are the last readers of its Y1 tile (and, for
       // dK/dV, of its Y2 tile).
       auto finish_tile = [&](uint32_t t, bool first, bool last_of_unit) {
-        if (!mbar_wait(p_full, t & 1, wc, 5, t)) return false;
+        if (!mbar_wait(&p_full[t & 1], (t >> 1) & 1, wc, 5, t)) return false;
         if (first && uc > 0 && !mbar_wait(acc_empty, (uc - 1) & 1, wc, 6, uc)) return false;
         tc_fence_after();
         issue_acc(t, !first);
@@ -384,25 +388,46 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
         if (u.x0 >= u.len) continue;
         const int ny = (u.len + kYRows - 1) / kYRows;
         if (!mbar_wait(x_full, uc & 1, wc, 3, uc)) break;
-        // S(i) goes where dP(i-1) was, once the warpgroups have read it.
-        // dK/dV: S(i), the products of tile i-1, dP(i), which goes where
-        // those products read P and dS of tile i-1 just before.  dQ: S(i),
-        // dP(i), where dQ(i-2) read dS, then dQ(i-1); V is read by dP alone
-        // and released right after it.  (The tensor pipe runs in issue
-        // order.)
-        for (int i = 0; i < ny; ++i) {
-          if (!wait_y1(yc)) { ok = false; break; }
-          if (yc > 0 && !mbar_wait(dp_free, (yc - 1) & 1, wc, 15, yc)) { ok = false; break; }
+        if (kDQ) {
+          // Order per tile: dP(i), dQ(i-1), S(i+1).  dP(i) goes where dP(i-1)
+          // was, once the warpgroups have read it; S(i+1) where S(i-1) was,
+          // after dQ(i-1) read its dS (the tensor pipe runs in issue order).
+          // V is read by dP alone and released right after it.
+          if (!wait_y1(yc)) break;
           tc_fence_after();
           issue_sonly(yc);
-          if (!kDQ && i > 0 && !finish_tile(yc - 1, i == 1, false)) { ok = false; break; }
-          if (!wait_y2(yc)) { ok = false; break; }
-          tc_fence_after();
-          issue_dp(yc);
-          if (kDQ) umma_commit(&y2_empty[yc % P::kS2]);
-          if (i + 1 == ny) umma_commit(x_empty);
-          if (kDQ && i > 0 && !finish_tile(yc - 1, i == 1, false)) { ok = false; break; }
-          ++yc;
+          for (int i = 0; i < ny; ++i) {
+            if (!wait_y2(yc)) { ok = false; break; }
+            if (yc > 0 && !mbar_wait(dp_free, (yc - 1) & 1, wc, 15, yc)) { ok = false; break; }
+            tc_fence_after();
+            issue_dp(yc);
+            umma_commit(&y2_empty[yc % P::kS2]);
+            if (i + 1 == ny) umma_commit(x_empty);
+            if (i > 0 && !finish_tile(yc - 1, i == 1, false)) { ok = false; break; }
+            if (i + 1 < ny) {
+              if (!wait_y1(yc + 1)) { ok = false; break; }
+              tc_fence_after();
+              issue_sonly(yc + 1);
+            }
+            ++yc;
+          }
+        } else {
+          // Order per tile: S(i), dV/dK(i-1), dP(i).  S(i) goes where dP(i-1)
+          // was, once the warpgroups have read it; dP(i) where dV/dK(i-1)
+          // read P and dS of tile i-1 just before (the tensor pipe runs in
+          // issue order).
+          for (int i = 0; i < ny; ++i) {
+            if (!wait_y1(yc)) { ok = false; break; }
+            if (yc > 0 && !mbar_wait(dp_free, (yc - 1) & 1, wc, 15, yc)) { ok = false; break; }
+            tc_fence_after();
+            issue_sonly(yc);
+            if (i > 0 && !finish_tile(yc - 1, i == 1, false)) { ok = false; break; }
+            if (!wait_y2(yc)) { ok = false; break; }
+            tc_fence_after();
+            issue_dp(yc);
+            if (i + 1 == ny) umma_commit(x_empty);
+            ++yc;
+          }
         }
         if (!ok || !finish_tile(yc - 1, ny == 1, true)) break;
         ++uc;
@@ -441,7 +466,11 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
       const int src = live ? (a.perm ? a.perm[u.start + r] : u.start + r) : 0;
       for (int i = 0; i < ny; ++i, ++yc) {
         const int s1 = (int)(yc % P::kS1), s2 = (int)(yc % P::kS2);
-        if (!mbar_wait(s_full, yc & 1, wc, 7 + wg, yc)) { ok = false; break; }
+        // dQ: S(t) on s_full[t % 2], whose phase advances every other tile
+        // (S runs a tile ahead); dK/dV: s_full[0]
+        const bool ok_s = kDQ ? mbar_wait(&s_full[yc & 1], (yc >> 1) & 1, wc, 7 + wg, yc)
+                              : mbar_wait(&s_full[0], yc & 1, wc, 7 + wg, yc);
+        if (!ok_s) { ok = false; break; }
         tc_fence_after();
         // the vectors are plain shared-memory stores of the load warp: wait
         // on the slot's own barrier too (its phase is still this tile's,
@@ -507,7 +536,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(p_full);
+        mbar_arrive(&p_full[yc & 1]);
       }
       if (!ok) break;
       // ------------------------------------------------ epilogue
