@@ -762,179 +762,148 @@ struct Vec<float> {
   __device__ static void store(float* p, const float* v) { *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]); }
 };
 
-constexpr int kRbWarps = 8;
-constexpr int kRbGroups = 16;  // logits accumulated per pass over a row of x
-
-// One warp per token: logits, softmax, dr (kept in dr [N, M] for dW_r) and dx.
-template <typename T>
-__global__ void __launch_bounds__(kRbWarps * 32)
-route_bwd_kernel(const T* __restrict__ x, const T* __restrict__ W, const float* __restrict__ b,
-                 const int32_t* __restrict__ gid, const float* __restrict__ dgate, const int32_t* __restrict__ offsets,
-                 float bcoef, int64_t N, int d, int M, float* __restrict__ dr, T* __restrict__ dx, int* status) {
-  extern __shared__ float rb_smem[];
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  float* lg = rb_smem + wid * M;  // this warp's logits, then dr
-  float* F = rb_smem + kRbWarps * M;  // share of tokens per group (balancing loss)
-  if (bcoef != 0.0f) {
-    const float invN = 1.0f / (float)N;
-    for (int j = threadIdx.x; j < M; j += blockDim.x) F[j] = (float)(offsets[j + 1] - offsets[j]) * invN;
+// Router backward from the router's own logits (fp32 [N][M], recomputed by
+// the forward router kernels, so they equal the forward's bit for bit).
+// dr[i][j] = d(out)/d(r_ij) with p = softmax(r_i) and g = the token's group:
+//   dgate_i * p_g * ([j == g] - p_j)  +  bcoef * p_j * (F_j - sum_k F_k p_k)
+// (the gate's gradient, and the balancing loss's when bcoef != 0; F_j is the
+// share of tokens routed to j).  Written in place over the logits.
+__global__ void __launch_bounds__(256)
+route_dr_kernel(float* __restrict__ lr, const int32_t* __restrict__ gid, const float* __restrict__ dgate,
+                const int32_t* __restrict__ offsets, float bcoef, int64_t N, int M, int* status) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= N) return;
+  float* r = lr + i * M;
+  const int g = gid[i];
+  if (g < 0 || g >= M) {
+    if (status) atomicOr(status, DEV_RANGE);
+    for (int j = 0; j < M; ++j) r[j] = 0.0f;
+    return;
   }
-  __syncthreads();
-  constexpr int V = Vec<T>::n;
-  const int nv = d / V;
-  for (int64_t i = (int64_t)blockIdx.x * kRbWarps + wid; i < N; i += (int64_t)gridDim.x * kRbWarps) {
-    const T* xr = x + i * d;
-    for (int j0 = 0; j0 < M; j0 += kRbGroups) {
-      float acc[kRbGroups];
-#pragma unroll
-      for (int jj = 0; jj < kRbGroups; ++jj) acc[jj] = 0.0f;
-      for (int cv = lane; cv < nv; cv += 32) {
-        float xv[V];
-        Vec<T>::load(xr + cv * V, xv);
-#pragma unroll
-        for (int jj = 0; jj < kRbGroups; ++jj) {
-          if (j0 + jj < M) {
-            float wv[V];
-            Vec<T>::load(W + (int64_t)(j0 + jj) * d + cv * V, wv);
-#pragma unroll
-            for (int e = 0; e < V; ++e) acc[jj] = fmaf(xv[e], wv[e], acc[jj]);
-          }
-        }
-      }
-#pragma unroll
-      for (int jj = 0; jj < kRbGroups; ++jj) {
-        float s = acc[jj];
-        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-        if (lane == 0 && j0 + jj < M) lg[j0 + jj] = s + (b ? b[j0 + jj] : 0.0f);
-      }
-    }
-    __syncwarp();
-    const int g = gid[i];
-    if (g < 0 || g >= M) {
-      if (lane == 0 && status) atomicOr(status, DEV_RANGE);
-      for (int j = lane; j < M; j += 32) dr[i * M + j] = 0.0f;
-      for (int cv = lane; cv < nv; cv += 32) {
-        float z[V] = {};
-        Vec<T>::store(dx + i * d + cv * V, z);
-      }
-      __syncwarp();
-      continue;
-    }
-    float mx = -INFINITY;
-    for (int j = lane; j < M; j += 32) mx = fmaxf(mx, lg[j]);
-    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    float z = 0.0f;
-    for (int j = lane; j < M; j += 32) z += expf(lg[j] - mx);
-    for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
-    const float pg = expf(lg[g] - mx) / z;
-    const float k = dgate[i] * pg;
-    float fs = 0.0f;  // sum_k F_k p_k
-    if (bcoef != 0.0f) {
-      for (int j = lane; j < M; j += 32) fs += F[j] * expf(lg[j] - mx) / z;
-      for (int off = 16; off > 0; off >>= 1) fs += __shfl_xor_sync(0xffffffffu, fs, off);
-    }
-    __syncwarp();
-    for (int j = lane; j < M; j += 32) {
-      const float pj = expf(lg[j] - mx) / z;
-      float v = k * ((j == g ? 1.0f : 0.0f) - pj);
-      if (bcoef != 0.0f) v += bcoef * pj * (F[j] - fs);
-      lg[j] = v;
-      dr[i * M + j] = v;
-    }
-    __syncwarp();
-    for (int cv = lane; cv < nv; cv += 32) {
-      float o[V];
-#pragma unroll
-      for (int e = 0; e < V; ++e) o[e] = 0.0f;
-      for (int j = 0; j < M; ++j) {
-        const float rj = lg[j];
-        float wv[V];
-        Vec<T>::load(W + (int64_t)j * d + cv * V, wv);
-#pragma unroll
-        for (int e = 0; e < V; ++e) o[e] = fmaf(rj, wv[e], o[e]);
-      }
-      Vec<T>::store(dx + i * d + cv * V, o);
-    }
-    __syncwarp();
+  float mx = -INFINITY;
+  for (int j = 0; j < M; ++j) mx = fmaxf(mx, r[j]);
+  float z = 0.0f;
+  for (int j = 0; j < M; ++j) z += expf(r[j] - mx);
+  const float inv = 1.0f / z;
+  const float k = dgate[i] * expf(r[g] - mx) * inv;
+  float fs = 0.0f;
+  const float invN = 1.0f / (float)N;
+  if (bcoef != 0.0f)
+    for (int j = 0; j < M; ++j) fs += (float)(offsets[j + 1] - offsets[j]) * invN * expf(r[j] - mx) * inv;
+  for (int j = 0; j < M; ++j) {
+    const float pj = expf(r[j] - mx) * inv;
+    float v = k * ((j == g ? 1.0f : 0.0f) - pj);
+    if (bcoef != 0.0f) v += bcoef * pj * ((float)(offsets[j + 1] - offsets[j]) * invN - fs);
+    r[j] = v;
   }
 }
 
-// Partial dW_r and db over one slice of the tokens (a split-K reduction of
-// dW_r = dr^T x).  Block (cx, s) covers columns [256 cx, 256 cx + 256) for
-// the tokens of slice s, 32 tokens at a time: the block stages the chunk's x
-// (as fp32) and dr in shared memory with wide loads, then lane l of warp w
-// accumulates columns 256 cx + 8 l .. + 8 for the groups w, w + 8, ... (64
-// groups per pass).  Slices are summed in a fixed order afterwards, so the
-// result does not depend on scheduling.
-constexpr int kDwTok = 32;
-constexpr int kDwCols = 256;
-constexpr int kDwGroups = 64;  // groups per pass
+// dx = dr W_r.  A thread owns Vec<T>::n columns and kDxTok tokens per pass,
+// so each row of W_r it loads serves kDxTok tokens; dr is read warp-uniformly
+// (the same address across the warp).
+constexpr int kDxTok = 8;
 template <typename T>
 __global__ void __launch_bounds__(256)
+route_dx_kernel(const T* __restrict__ W, const float* __restrict__ dr, int64_t N, int d, int M, T* __restrict__ dx) {
+  constexpr int V = Vec<T>::n;
+  const int c = (blockIdx.x * blockDim.x + threadIdx.x) * V;
+  if (c >= d) return;  // d is a multiple of V
+  for (int64_t t0 = (int64_t)blockIdx.y * kDxTok; t0 < N; t0 += (int64_t)gridDim.y * kDxTok) {
+    float acc[kDxTok][V];
+#pragma unroll
+    for (int tk = 0; tk < kDxTok; ++tk)
+#pragma unroll
+      for (int e = 0; e < V; ++e) acc[tk][e] = 0.0f;
+    const int nt = (int)(N - t0 < kDxTok ? N - t0 : kDxTok);
+    for (int j = 0; j < M; ++j) {
+      float w[V];
+      Vec<T>::load(W + (int64_t)j * d + c, w);
+#pragma unroll
+      for (int tk = 0; tk < kDxTok; ++tk) {
+        const float r = tk < nt ? __ldg(dr + (t0 + tk) * M + j) : 0.0f;
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[tk][e] = fmaf(r, w[e], acc[tk][e]);
+      }
+    }
+#pragma unroll
+    for (int tk = 0; tk < kDxTok; ++tk)
+      if (tk < nt) Vec<T>::store(dx + (t0 + tk) * d + c, acc[tk]);
+  }
+}
+
+// Partial dW_r = dr^T x and db = sum dr over one slice of the tokens (a
+// split-K reduction).  Block (cx, s): each thread owns Vec<T>::n columns of
+// x and accumulates them against 16 groups at a time, for the tokens of
+// slice s, in chunks of kDwChunk tokens whose dr the block stages in shared
+// memory; kDwUnroll rows of x are loaded before they are used, so several
+// loads per thread are in flight.  Slices are summed in a fixed order
+// afterwards, so the result does not depend on scheduling.
+constexpr int kDwGroups = 16;
+constexpr int kDwUnroll = 8;
+constexpr int kDwThreads = 64;
+constexpr int kDwChunk = 64;
+template <typename T>
+__global__ void __launch_bounds__(kDwThreads)
 route_dw_kernel(const T* __restrict__ x, const float* __restrict__ dr, int64_t N, int d, int M, int64_t per_slice,
                 float* __restrict__ pw, float* __restrict__ pb) {
-  constexpr int V = Vec<T>::n;  // values per vector load (8 bf16 / 4 fp32)
-  __shared__ __align__(16) float xs[kDwTok][kDwCols];
-  __shared__ float ds[kDwTok][kDwGroups];
-  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-  const int c0 = blockIdx.x * kDwCols;
+  constexpr int V = Vec<T>::n;
+  __shared__ float drs[kDwChunk][kDwGroups];
+  const int c = (blockIdx.x * kDwThreads + threadIdx.x) * V;
   const int s = blockIdx.y;
   const int64_t i0 = (int64_t)s * per_slice, i1 = min(N, i0 + per_slice);
-  constexpr int kVecPerRow = kDwCols / V;
-  for (int jp = 0; jp < M; jp += kDwGroups) {
-    float acc[8][8];
+  const bool col_ok = c < d;  // d is a multiple of V
+  const bool bias_lane = blockIdx.x == 0 && threadIdx.x == 0;
+  for (int j0 = 0; j0 < M; j0 += kDwGroups) {
+    float acc[kDwGroups][V];
+    float bacc[kDwGroups];
 #pragma unroll
-    for (int g = 0; g < 8; ++g)
+    for (int g = 0; g < kDwGroups; ++g) {
+      bacc[g] = 0.0f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[g][e] = 0.0f;
-    float bacc[8];
-#pragma unroll
-    for (int g = 0; g < 8; ++g) bacc[g] = 0.0f;
-    for (int64_t ib = i0; ib < i1; ib += kDwTok) {
+      for (int e = 0; e < V; ++e) acc[g][e] = 0.0f;
+    }
+    for (int64_t cb = i0; cb < i1; cb += kDwChunk) {
+      const int nc = (int)(i1 - cb < kDwChunk ? i1 - cb : kDwChunk);
       __syncthreads();  // the previous chunk has been consumed
-      for (int v = t; v < kDwTok * kVecPerRow; v += 256) {
-        const int r = v / kVecPerRow, cv = v - r * kVecPerRow;
-        const int64_t i = ib + r;
-        const int c = c0 + cv * V;
-        float tmp[V];
-        if (i < i1 && c + V <= d)
-          Vec<T>::load(x + i * d + c, tmp);
-        else
-#pragma unroll
-          for (int e = 0; e < V; ++e) tmp[e] = 0.0f;
-#pragma unroll
-        for (int e = 0; e < V; ++e) xs[r][cv * V + e] = tmp[e];
-      }
-      for (int v = t; v < kDwTok * kDwGroups; v += 256) {
-        const int r = v / kDwGroups, j = v - r * kDwGroups;
-        const int64_t i = ib + r;
-        ds[r][j] = (i < i1 && jp + j < M) ? dr[i * M + jp + j] : 0.0f;
+      for (int e = threadIdx.x; e < kDwChunk * kDwGroups; e += kDwThreads) {
+        const int r = e / kDwGroups, g = e - r * kDwGroups;
+        drs[r][g] = (r < nc && j0 + g < M) ? dr[(cb + r) * M + j0 + g] : 0.0f;
       }
       __syncthreads();
-#pragma unroll 4
-      for (int r = 0; r < kDwTok; ++r) {
-        const float4 xa = *reinterpret_cast<const float4*>(&xs[r][lane * 8]);
-        const float4 xb = *reinterpret_cast<const float4*>(&xs[r][lane * 8 + 4]);
-        const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+      for (int u0 = 0; u0 < nc; u0 += kDwUnroll) {
+        float xv[kDwUnroll][V];
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          const float rj = ds[r][w + 8 * g];
-          bacc[g] += rj;
+        for (int u = 0; u < kDwUnroll; ++u) {
+          if (col_ok && u0 + u < nc)
+            Vec<T>::load(x + (cb + u0 + u) * d + c, xv[u]);
+          else
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(rj, xv[e], acc[g][e]);
+            for (int e = 0; e < V; ++e) xv[u][e] = 0.0f;
+        }
+        // rows past the chunk have x = 0 and dr = 0: they add nothing
+#pragma unroll
+        for (int u = 0; u < kDwUnroll; ++u) {
+          const int rr = (u0 + u) < kDwChunk ? u0 + u : kDwChunk - 1;
+#pragma unroll
+          for (int g = 0; g < kDwGroups; ++g) {
+            const float r = (u0 + u) < nc ? drs[rr][g] : 0.0f;
+            if (bias_lane) bacc[g] += r;
+#pragma unroll
+            for (int e = 0; e < V; ++e) acc[g][e] = fmaf(r, xv[u][e], acc[g][e]);
+          }
         }
       }
     }
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
-      const int j = jp + w + 8 * g;
-      if (j >= M) continue;
-      const int col = c0 + lane * 8;
-      float* dst = pw + ((int64_t)s * M + j) * d + col;
+    for (int g = 0; g < kDwGroups; ++g) {
+      const int j = j0 + g;
+      if (j >= M) break;
+      if (col_ok) {
+        float* dst = pw + ((int64_t)s * M + j) * d + c;
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
-        if (col + e < d) dst[e] = acc[g][e];
-      if (blockIdx.x == 0 && lane == 0) pb[(int64_t)s * M + j] = bacc[g];
+        for (int e = 0; e < V; ++e) dst[e] = acc[g][e];
+      }
+      if (bias_lane) pb[(int64_t)s * M + j] = bacc[g];
     }
   }
 }
@@ -994,53 +963,81 @@ static int route_max_slices(int d, int M) {
   return (int)std::max<int64_t>(1, std::min<int64_t>(kRouteSlices, ((int64_t)64 << 20) / per));
 }
 
-size_t route_bwd_ws_bytes(int64_t N, int d, int M) {
+// Workspace of the router backward: the logits (then dr) [N][M], the
+// router's group ids, gates and histograms (recomputed, not used), and the
+// dW_r / db partial sums.
+struct RouteBwdWs {
+  size_t lr, gid, gate, hist, pw, pb, total;
+};
+static RouteBwdWs route_bwd_ws(int64_t N, int d, int M) {
+  RouteBwdWs w;
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    const size_t o = off;
+    off += align_up(n, 256);
+    return o;
+  };
   const size_t S = (size_t)route_max_slices(d, M);
-  return align_up((size_t)N * M * 4, 256) + align_up(S * M * d * 4, 256) + align_up(S * M * 4, 256);
+  w.lr = take((size_t)N * M * 4);
+  w.gid = take((size_t)N * 4);
+  w.gate = take((size_t)N * 4);
+  w.hist = take((size_t)ceil_div(N, kTile) * M * 4);
+  w.pw = take(S * M * d * 4);
+  w.pb = take(S * M * 4);
+  w.total = off;
+  return w;
 }
+
+size_t route_bwd_ws_bytes(int64_t N, int d, int M) { return route_bwd_ws(N, d, M).total; }
 
 cudaError_t launch_route_bwd(const DevCtx& c, const void* x, const void* W, const float* b, bool bf16, int64_t N,
                              int d, int M, const int32_t* gid, const float* dgate, const int32_t* offsets,
                              float balance_alpha, void* dx, float* dW, float* db, uint8_t* ws) {
   const float bcoef = N > 0 ? balance_alpha * (float)M / (float)N : 0.0f;
-  float* dr = reinterpret_cast<float*>(ws);
-  float* pw = reinterpret_cast<float*>(ws + align_up((size_t)N * M * 4, 256));
-  const int smax = route_max_slices(d, M);
-  float* pb = reinterpret_cast<float*>(ws + align_up((size_t)N * M * 4, 256) +
-                                       align_up((size_t)smax * M * d * 4, 256));
-  const size_t smem = (size_t)(kRbWarps + 1) * M * 4;
+  const RouteBwdWs w = route_bwd_ws(N, d, M);
+  float* lr = reinterpret_cast<float*>(ws + w.lr);
+  float* pw = reinterpret_cast<float*>(ws + w.pw);
+  float* pb = reinterpret_cast<float*>(ws + w.pb);
+  cudaError_t e;
   if (N > 0) {
-    int64_t blocks = ceil_div(N, kRbWarps);
-    const int64_t cap = (int64_t)c.num_sms * 8;
-    if (blocks > cap) blocks = cap;
-    if (bf16) {
-      auto k = route_bwd_kernel<__nv_bfloat16>;
-      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return cudaErrorInvalidValue;
-      k<<<(unsigned)blocks, kRbWarps * 32, smem, c.stream>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)W, b,
-                                                             gid, dgate, offsets, bcoef, N, d, M, dr,
-                                                             (__nv_bfloat16*)dx, c.status);
-    } else {
-      auto k = route_bwd_kernel<float>;
-      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return cudaErrorInvalidValue;
-      k<<<(unsigned)blocks, kRbWarps * 32, smem, c.stream>>>((const float*)x, (const float*)W, b, gid, dgate,
-                                                             offsets, bcoef, N, d, M, dr, (float*)dx, c.status);
-    }
-    cudaError_t e = cudaGetLastError();
+    // the logits, from the same router kernel the forward used
+    int32_t* gid2 = reinterpret_cast<int32_t*>(ws + w.gid);
+    float* gate2 = reinterpret_cast<float*>(ws + w.gate);
+    int32_t* hist = reinterpret_cast<int32_t*>(ws + w.hist);
+    if (bf16 && M <= 256 && d >= 64)
+      e = launch_route_tc(c, x, W, b, N, d, M, gid2, gate2, hist, nullptr, lr);
+    else
+      e = launch_route_simt(c, x, W, b, bf16, N, d, M, gid2, gate2, hist, nullptr, lr);
     if (e != cudaSuccess) return e;
+    route_dr_kernel<<<(unsigned)ceil_div(N, 256), 256, 0, c.stream>>>(lr, gid, dgate, offsets, bcoef, N, M,
+                                                                       c.status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int vec = bf16 ? 8 : 4;
+    const int64_t lanes = ceil_div(d, vec);
+    const int threads = (int)std::min<int64_t>(256, ceil_div(lanes, 32) * 32);
+    const int64_t cxb = ceil_div(lanes, threads);
+    const int64_t ty = std::max<int64_t>(1, std::min<int64_t>(ceil_div(N, kDxTok), (int64_t)c.num_sms * 8 / cxb));
+    dim3 grid((unsigned)cxb, (unsigned)ty);
+    if (bf16)
+      route_dx_kernel<__nv_bfloat16><<<grid, threads, 0, c.stream>>>((const __nv_bfloat16*)W, lr, N, d, M,
+                                                                      (__nv_bfloat16*)dx);
+    else
+      route_dx_kernel<float><<<grid, threads, 0, c.stream>>>((const float*)W, lr, N, d, M, (float*)dx);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  // about two blocks per SM: column tiles times token slices
-  const int64_t cx = ceil_div(d, kDwCols);
-  const int slices = (int)std::min<int64_t>(smax, std::max<int64_t>(1, 2 * c.num_sms / cx));
+  // enough blocks of kDwThreads to keep x's reads in flight: column blocks
+  // times token slices, about eight blocks per SM
+  const int vec = bf16 ? 8 : 4;
+  const int64_t cx = ceil_div(ceil_div(d, vec), kDwThreads);
+  const int slices = (int)std::min<int64_t>(route_max_slices(d, M), std::max<int64_t>(1, 8 * c.num_sms / cx));
   const int64_t per = ceil_div(N > 0 ? N : 1, slices);
   dim3 grid((unsigned)cx, (unsigned)slices);
   if (bf16)
-    route_dw_kernel<__nv_bfloat16><<<grid, 256, 0, c.stream>>>((const __nv_bfloat16*)x, dr, N, d, M, per, pw, pb);
+    route_dw_kernel<__nv_bfloat16><<<grid, kDwThreads, 0, c.stream>>>((const __nv_bfloat16*)x, lr, N, d, M, per, pw,
+                                                                       pb);
   else
-    route_dw_kernel<float><<<grid, 256, 0, c.stream>>>((const float*)x, dr, N, d, M, per, pw, pb);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+    route_dw_kernel<float><<<grid, kDwThreads, 0, c.stream>>>((const float*)x, lr, N, d, M, per, pw, pb);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   int64_t blocks = ceil_div((int64_t)M * d, 256);
   if (blocks > 1024) blocks = 1024;
   route_dw_reduce_kernel<<<(unsigned)blocks, 256, 0, c.stream>>>(pw, pb, slices, M, d, dW, db);

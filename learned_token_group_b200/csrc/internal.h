@@ -29,10 +29,13 @@ struct DevCtx {
 // ------------------------------------------------------------------ routing
 // Router logits + softmax gate + argmax + per-tile group histogram.
 // pstat (nullable): per (tile, warp) sums of p(i|x) over the warp's tokens, [tiles][4][M].
+// logits (nullable): the logits x W_r^T + b_r themselves, fp32 [N][M].
 cudaError_t launch_route_tc(const DevCtx& c, const void* x, const void* W, const float* b, int64_t N, int d,
-                            int M, int32_t* group_id, float* gate, int32_t* hist, float* pstat);
+                            int M, int32_t* group_id, float* gate, int32_t* hist, float* pstat,
+                            float* logits = nullptr);
 cudaError_t launch_route_simt(const DevCtx& c, const void* x, const void* W, const float* b, bool bf16,
-                              int64_t N, int d, int M, int32_t* group_id, float* gate, int32_t* hist, float* pstat);
+                              int64_t N, int d, int M, int32_t* group_id, float* gate, int32_t* hist, float* pstat,
+                              float* logits = nullptr);
 // Exclusive scan of the per-tile histograms -> offsets, max_seqlen, per-tile
 // bases; with pstat also the mean routing probabilities and the balance metric.
 cudaError_t launch_scan(const DevCtx& c, const int32_t* hist, int64_t ntiles, int M, int32_t* base,
@@ -141,7 +144,7 @@ cudaError_t launch_mean(const DevCtx& c, const void* x, const void* y, const voi
 // Router backward through the gate (plus, when balance_alpha != 0, the group
 // balancing loss alpha * M * sum_i F_i P_i with F from offsets): dx (dtype of
 // x), dW_r fp32 [M, d], db fp32 [M] (nullable).
-constexpr int kRouteSlices = 64;  // upper bound on token slices of the dW_r partial sums
+constexpr int kRouteSlices = 512;  // upper bound on token slices of the dW_r partial sums
 size_t route_bwd_ws_bytes(int64_t N, int d, int M);
 cudaError_t launch_route_bwd(const DevCtx& c, const void* x, const void* W, const float* b, bool bf16, int64_t N,
                              int d, int M, const int32_t* gid, const float* dgate, const int32_t* offsets,

@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
 route_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                 const float* __restrict__ bias, int N, int d, int M, int mpad, int stages, int stage_bytes,
                 int32_t* __restrict__ group_id, float* __restrict__ gate, int32_t* __restrict__ hist,
-                float* __restrict__ pstat, int* status, unsigned long long wait_ns) {
+                float* __restrict__ pstat, float* __restrict__ logits, int* status, unsigned long long wait_ns) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -202,6 +202,21 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
           const int col = c0 + j;
           if (col < M) online_softmax_step(v[j] + (bias ? __ldg(bias + col) : 0.f), col, mx, arg, sum);
         }
+        if (logits && (int64_t)t * kTile + row < N) {
+          float* lr = logits + ((int64_t)t * kTile + row) * M + c0;
+          float o[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) o[j] = v[j] + ((bias && c0 + j < M) ? __ldg(bias + c0 + j) : 0.f);
+          if ((M & 3) == 0 && c0 + 16 <= M) {  // rows start 16-byte aligned
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              reinterpret_cast<float4*>(lr)[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (c0 + j < M) lr[j] = o[j];
+          }
+        }
       }
       const int64_t tok = (int64_t)t * kTile + row;
       if (pstat) {
@@ -252,7 +267,7 @@ template <typename T>
 __global__ void __launch_bounds__(128)
 route_simt_kernel(const T* __restrict__ x, const T* __restrict__ W, const float* __restrict__ bias, int N, int d,
                   int M, int32_t* __restrict__ group_id, float* __restrict__ gate, int32_t* __restrict__ hist,
-                  float* __restrict__ pstat) {
+                  float* __restrict__ pstat, float* __restrict__ logits) {
   extern __shared__ float logit_s[];          // [4][M]
   int* hist_s = reinterpret_cast<int*>(logit_s + 4 * M);  // [M]
   float* ps = logit_s + 5 * M;                           // [4][M] per-warp sums of p(i|x)
@@ -275,6 +290,8 @@ route_simt_kernel(const T* __restrict__ x, const T* __restrict__ W, const float*
       if (lane == 0) lg[m] = acc + (bias ? bias[m] : 0.f);
     }
     __syncwarp();
+    if (logits)
+      for (int m = lane; m < M; m += 32) logits[tok * M + m] = lg[m];
     if (lane == 0) {
       float mx = -INFINITY, sum = 0.f;
       int arg = 0;
@@ -395,7 +412,7 @@ scatter_kernel(const int32_t* __restrict__ group_id, const int32_t* __restrict__
 }  // namespace
 
 cudaError_t launch_route_tc(const DevCtx& c, const void* x, const void* W, const float* b, int64_t N, int d,
-                            int M, int32_t* group_id, float* gate, int32_t* hist, float* pstat) {
+                            int M, int32_t* group_id, float* gate, int32_t* hist, float* pstat, float* logits) {
   const RouteSmemPlan p = route_plan(M);
   if (p.mpad > kRouteMaxMPad) return cudaErrorInvalidValue;
   CUtensorMap mx, mw;
@@ -409,13 +426,15 @@ cudaError_t launch_route_tc(const DevCtx& c, const void* x, const void* W, const
   if (e != cudaSuccess) return e;
   const int grid = (int)(ntiles < c.num_sms ? ntiles : c.num_sms);
   route_tc_kernel<<<grid, kRouteThreads, p.total, c.stream>>>(mx, mw, b, (int)N, d, M, p.mpad, p.stages,
-                                                               p.stage_bytes, group_id, gate, hist, pstat, c.status,
+                                                               p.stage_bytes, group_id, gate, hist, pstat, logits,
+                                                               c.status,
                                                                (unsigned long long)c.wait_ns);
   return cudaGetLastError();
 }
 
 cudaError_t launch_route_simt(const DevCtx& c, const void* x, const void* W, const float* b, bool bf16,
-                              int64_t N, int d, int M, int32_t* group_id, float* gate, int32_t* hist, float* pstat) {
+                              int64_t N, int d, int M, int32_t* group_id, float* gate, int32_t* hist, float* pstat,
+                              float* logits) {
   const int64_t ntiles = ceil_div(N, kTile);
   const size_t smem = (size_t)9 * M * sizeof(float);
   if (bf16) {
@@ -423,13 +442,13 @@ cudaError_t launch_route_simt(const DevCtx& c, const void* x, const void* W, con
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<(unsigned)ntiles, 128, smem, c.stream>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)W, b, (int)N, d,
-                                                  M, group_id, gate, hist, pstat);
+                                                  M, group_id, gate, hist, pstat, logits);
   } else {
     auto k = route_simt_kernel<float>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<(unsigned)ntiles, 128, smem, c.stream>>>((const float*)x, (const float*)W, b, (int)N, d, M, group_id,
-                                                  gate, hist, pstat);
+                                                  gate, hist, pstat, logits);
   }
   return cudaGetLastError();
 }
