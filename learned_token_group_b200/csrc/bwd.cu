@@ -496,9 +496,17 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
               pv[e] = e < valid ? pe : 0.0f;
             }
           } else {
-            const float* nl = vec1 + s1 * kYRows + 64 * wg;
+            // the slot's -lse*log2(e), read as 16-byte vectors (one broadcast
+            // wavefront per four keys)
+            const float4* nl = reinterpret_cast<const float4*>(vec1 + s1 * kYRows + 64 * wg);
 #pragma unroll
-            for (int e = 0; e < 64; ++e) pv[e] = fast_exp2(fmaf(sv[e], scale_log2, nl[e]));
+            for (int e4 = 0; e4 < 16; ++e4) {
+              const float4 n = nl[e4];
+              pv[4 * e4 + 0] = fast_exp2(fmaf(sv[4 * e4 + 0], scale_log2, n.x));
+              pv[4 * e4 + 1] = fast_exp2(fmaf(sv[4 * e4 + 1], scale_log2, n.y));
+              pv[4 * e4 + 2] = fast_exp2(fmaf(sv[4 * e4 + 2], scale_log2, n.z));
+              pv[4 * e4 + 3] = fast_exp2(fmaf(sv[4 * e4 + 3], scale_log2, n.w));
+            }
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
               uint32_t pk[16];
@@ -520,16 +528,22 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tx1, const __grid_constant__
           tc_fence_before();
           mbar_arrive(dp_free);
           // D per Y row (dK/dV: from the Y2 slot's vector), or of this X row (dQ)
-          const float* dd = vec2 + s2 * kYRows + 64 * wg;
+          const float4* dd = reinterpret_cast<const float4*>(vec2 + s2 * kYRows + 64 * wg);
           if (!kDQ && !mbar_wait(&y2_full[s2], (yc / P::kS2) & 1, wc, 18 + wg, yc)) { ok = false; break; }
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
             uint32_t dk[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
+            for (int e = 0; e < 16; e += 2) {
               const int c = 32 * hf + 2 * e;
-              dk[e] = kDQ ? pack_bf16x2(pv[c] * (dv[c] - d_row), pv[c + 1] * (dv[c + 1] - d_row))
-                          : pack_bf16x2(pv[c] * (dv[c] - dd[c]), pv[c + 1] * (dv[c + 1] - dd[c + 1]));
+              if (kDQ) {
+                dk[e] = pack_bf16x2(pv[c] * (dv[c] - d_row), pv[c + 1] * (dv[c + 1] - d_row));
+                dk[e + 1] = pack_bf16x2(pv[c + 2] * (dv[c + 2] - d_row), pv[c + 3] * (dv[c + 3] - d_row));
+              } else {
+                const float4 D = dd[c >> 2];
+                dk[e] = pack_bf16x2(pv[c] * (dv[c] - D.x), pv[c + 1] * (dv[c + 1] - D.y));
+                dk[e + 1] = pack_bf16x2(pv[c + 2] * (dv[c + 2] - D.z), pv[c + 3] * (dv[c + 3] - D.w));
+              }
             }
             tmem_st16u(ts + lb + 64 * wg + (kDQ ? 0 : 32) + 16 * hf, dk);
           }
