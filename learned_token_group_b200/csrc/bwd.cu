@@ -42,6 +42,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -626,9 +627,15 @@ cudaError_t launch_bwd_dh(const DevCtx& c, const BwdArgs& a) {
   if (!make_tmap_2d(&m1, xs1, DH, rows, DH * 2, kTile) || !make_tmap_2d(&m2, xs2, DH, rows, DH * 2, kTile) ||
       !make_tmap_2d(&m3, ys1, DH, rows, DH * 2, kYRows) || !make_tmap_2d(&m4, ys2, DH, rows, DH * 2, kYRows))
     return cudaErrorInvalidValue;
-  int max_smem = 0;
-  cudaError_t e = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, c.device);
-  if (e != cudaSuccess) return e;
+  // the device's opt-in shared memory per block, queried once per device
+  static std::atomic<int> cached[64];
+  int max_smem = (c.device >= 0 && c.device < 64) ? cached[c.device].load(std::memory_order_relaxed) : 0;
+  cudaError_t e = cudaSuccess;
+  if (max_smem <= 0) {
+    if ((e = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, c.device)) != cudaSuccess)
+      return e;
+    if (c.device >= 0 && c.device < 64) cached[c.device].store(max_smem, std::memory_order_relaxed);
+  }
   // The segment table goes to shared memory when it fits beside the tiles
   // (the kernel reads it from global memory otherwise); up to 1 KB more
   // aligns the tiles to 1024 B, and the kernel checks that it got enough.

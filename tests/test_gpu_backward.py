@@ -130,6 +130,8 @@ CASES = [
     (custom(1500, H=1, d_h=64, d=128, M=40, x_kind="clustered"), 6),
     # bf16 router input with M > 256: the logits come from the SIMT router
     (custom(1200, H=1, d_h=64, d=64, M=300), 7),
+    # d_h 128 with 40 groups: the dK/dV pass reads its group table from global memory
+    (custom(1600, H=2, d_h=128, d=128, M=40, x_kind="clustered"), 8),
 ]
 
 
