@@ -617,15 +617,17 @@ attn_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUte
         for (int j = 0; j < nkv; ++j) {
           const int vs = (int)(vc % kStages);
           const bool more = j + 1 < nkv;
+          ks = (int)(kc % kStages);
+          // The next K tile is waited for before tile A's P, so that no wait
+          // sits between tile A's P V and its next S (the loads do not depend
+          // on P).
           if (!mbar_wait(&v_full[vs], (vc / kStages) & 1, wc, 7, vc)) { ok = false; break; }
+          if (more && !mbar_wait(&k_full[ks], (kc / kStages) & 1, wc, 8, kc)) { ok = false; break; }
           if (!mbar_wait(&p_full[0], pc0 & 1, wc, 13, pc0)) { ok = false; break; }
           ++pc0;
           tc_fence_after();
           issue_pv(0, vaddr(vs), j > 0);
-          ks = (int)(kc % kStages);
           if (more) {
-            if (!mbar_wait(&k_full[ks], (kc / kStages) & 1, wc, 8, kc)) { ok = false; break; }
-            tc_fence_after();
             issue_s(0, qa_addr, P::kChunkFull, kaddr(ks), P::kChunkFull);
             umma_commit(&s_full[0]);
           } else {
