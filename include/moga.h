@@ -282,7 +282,8 @@ moga_status moga_layer_train(const void* x, const void* W_r, const float* b_r, m
  *               plus w * dout through STGA's (overwritten, not accumulated);
  *   dgate_i   = w * sum_{h,c} dout * o_moga / gate_i;
  *   dr_ij     = dgate_i * p_ig * ([j == g_i] - p_ij) for the router's
- *               softmax p = softmax(x W_r^T + b);
+ *               softmax p = softmax(x W_r^T + b), recomputed by the
+ *               forward's router kernel (the same logits bit for bit);
  *   dx        = dr W_r   (x's dtype, [N, d]: the router's share of dL/dx;
  *               q, k, v are inputs of the block, so the projections that
  *               produce them are the caller's);
